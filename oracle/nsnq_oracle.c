@@ -1,0 +1,283 @@
+/*
+ * nsnq_oracle.c -- plain, slow CPU oracle for NSNQuant KV-cache vector
+ * quantization and decode attention over the quantized cache.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing on the product path may link, load or call
+ * this file; only the test-suite, the smoke check and the benchmark's CPU
+ * baseline leg do. It shares no code, headers, tables or constants with the
+ * CUDA library: it is written from the method's description alone.
+ *
+ * Single-threaded, fp64 throughout, no blocking, fusion or reordering beyond
+ * the definitions. Sources (gist.science "NSNQuant: A Double Normalization
+ * Approach for Calibration-Free Low-Bit Vector Quantization of KV Cache",
+ * Technical Summary):
+ *   - Methodology §1 "Normalize-Shift-Normalize": token-wise normalize to
+ *     norm sqrt(d), channel-wise mean shift, token-wise re-normalize to
+ *     sqrt(d); byproducts (s1, o, s2) reconstruct the tensor.
+ *   - Methodology §2 "Hadamard Transform": the naive (non-randomized)
+ *     Hadamard transform is the one used in the implementation.
+ *   - Methodology §3 "Vector Quantization and Codebook": one global codebook
+ *     built by K-Means on synthetic standard-normal data; each sub-vector is
+ *     replaced by its nearest codeword.
+ *   - Methodology §4 "Implementation Details": attention scores are computed
+ *     from the quantized cache and the NSN byproducts.
+ * Readings where the text is silent (stated once, used everywhere):
+ *   s = ||v|| / sqrt(d) so that v / s has norm sqrt(d); a zero-norm token maps
+ *   to the zero vector and keeps s = 0; H is the orthonormal Sylvester
+ *   Hadamard matrix in natural order, H[i][j] = (-1)^popcount(i & j) / sqrt(d);
+ *   sub-vector j covers coordinates [j*g, (j+1)*g); argmin ties go to the
+ *   lowest index; k-means starts from the first k samples, runs a fixed
+ *   number of Lloyd iterations and an empty cluster keeps its centroid.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_OK 0
+#define ORACLE_ERR_ARG 1
+#define ORACLE_ERR_MEM 2
+
+static int parity_of_and(unsigned i, unsigned j) {
+    unsigned v = i & j;
+    int p = 0;
+    while (v) {
+        p ^= (int)(v & 1u);
+        v >>= 1;
+    }
+    return p;
+}
+
+/* Orthonormal Sylvester Hadamard matrix, natural order (Methodology §2). */
+int oracle_hadamard(int d, double* H) {
+    if (d <= 0 || (d & (d - 1)) != 0 || !H) return ORACLE_ERR_ARG;
+    double s = 1.0 / sqrt((double)d);
+    for (int i = 0; i < d; ++i)
+        for (int j = 0; j < d; ++j)
+            H[(size_t)i * d + j] = parity_of_and((unsigned)i, (unsigned)j) ? -s : s;
+    return ORACLE_OK;
+}
+
+/* out = H v, explicit dense product (not a butterfly). */
+static void hadamard_apply(const double* H, int d, const double* v, double* out) {
+    for (int i = 0; i < d; ++i) {
+        double acc = 0.0;
+        const double* row = H + (size_t)i * d;
+        for (int k = 0; k < d; ++k) acc += row[k] * v[k];
+        out[i] = acc;
+    }
+}
+
+static double sqdist(const double* a, const double* b, int g) {
+    double s = 0.0;
+    for (int r = 0; r < g; ++r) {
+        double e = a[r] - b[r];
+        s += e * e;
+    }
+    return s;
+}
+
+/*
+ * Codebook construction (Methodology §3): Lloyd's k-means on n samples of
+ * dimension g. Start: the first k samples. Each iteration assigns every
+ * sample to its nearest centroid (lowest index on ties) and moves each
+ * centroid to the mean of its samples; an empty cluster keeps its centroid.
+ * C receives k*g values; counts (optional) the final cluster sizes from the
+ * last assignment step.
+ */
+int oracle_kmeans(const double* X, int64_t n, int g, int k, int iters, double* C,
+                  int64_t* counts) {
+    if (!X || !C || n < k || g <= 0 || k <= 0 || iters < 0) return ORACLE_ERR_ARG;
+    double* sums = (double*)calloc((size_t)k * g, sizeof(double));
+    int64_t* cnt = (int64_t*)calloc((size_t)k, sizeof(int64_t));
+    if (!sums || !cnt) {
+        free(sums);
+        free(cnt);
+        return ORACLE_ERR_MEM;
+    }
+    memcpy(C, X, (size_t)k * g * sizeof(double));
+    for (int it = 0; it < iters; ++it) {
+        memset(sums, 0, (size_t)k * g * sizeof(double));
+        memset(cnt, 0, (size_t)k * sizeof(int64_t));
+        for (int64_t i = 0; i < n; ++i) {
+            const double* x = X + (size_t)i * g;
+            int best = 0;
+            double bd = sqdist(x, C, g);
+            for (int c = 1; c < k; ++c) {
+                double dd = sqdist(x, C + (size_t)c * g, g);
+                if (dd < bd) {
+                    bd = dd;
+                    best = c;
+                }
+            }
+            cnt[best] += 1;
+            for (int r = 0; r < g; ++r) sums[(size_t)best * g + r] += x[r];
+        }
+        for (int c = 0; c < k; ++c)
+            if (cnt[c] > 0)
+                for (int r = 0; r < g; ++r)
+                    C[(size_t)c * g + r] = sums[(size_t)c * g + r] / (double)cnt[c];
+    }
+    if (counts) {
+        for (int c = 0; c < k; ++c) counts[c] = iters > 0 ? cnt[c] : 0;
+    }
+    free(sums);
+    free(cnt);
+    return ORACLE_OK;
+}
+
+/* Nearest codeword of one g-dimensional sub-vector (full squared distance,
+ * lowest index on exact ties). */
+static int nearest_codeword(const double* w, const float* C, int K, int g) {
+    double cw[64];
+    int best = 0;
+    double bd = INFINITY;
+    for (int c = 0; c < K; ++c) {
+        for (int r = 0; r < g; ++r) cw[r] = (double)C[(size_t)c * g + r];
+        double dd = sqdist(w, cw, g);
+        if (dd < bd) {
+            bd = dd;
+            best = c;
+        }
+    }
+    return best;
+}
+
+/*
+ * Encode one (batch, kv-head) slice of T tokens (Methodology §1-§3).
+ *   x       [T][d] input activations (exact values of the I/O type)
+ *   C       [K][g] fp32 codebook
+ *   shift_given = 0: o is the channel mean of the normalized tokens;
+ *               = 1: o is taken from o_in (tokens appended to a cache whose
+ *                    shift was computed over the prompt)
+ * Outputs: codes [T][d/g], s1 [T], s2 [T], o_out [d], and optionally
+ * w_out [T][d] (the transformed tokens that were quantized).
+ */
+int oracle_encode_head(const double* x, int64_t T, int d, int g, const float* C, int K,
+                       int shift_given, const double* o_in, uint8_t* codes, double* s1,
+                       double* s2, double* o_out, double* w_out) {
+    if (d <= 0 || (d & (d - 1)) != 0 || g <= 0 || d % g != 0 || g > 64 || K <= 0 || K > 256 ||
+        T < 0 || (shift_given && !o_in) || !C || !o_out)
+        return ORACLE_ERR_ARG;
+    const int J = d / g;
+    const double sqrt_d = sqrt((double)d);
+    double* H = (double*)malloc((size_t)d * d * sizeof(double));
+    double* y = (double*)malloc((size_t)(T > 0 ? T : 1) * d * sizeof(double));
+    double* u = (double*)malloc((size_t)d * sizeof(double));
+    double* w = (double*)malloc((size_t)d * sizeof(double));
+    if (!H || !y || !u || !w) {
+        free(H); free(y); free(u); free(w);
+        return ORACLE_ERR_MEM;
+    }
+    oracle_hadamard(d, H);
+
+    /* Normalize (token-wise): s1 = ||x|| / sqrt(d), y = x / s1. */
+    for (int64_t t = 0; t < T; ++t) {
+        const double* xt = x + (size_t)t * d;
+        double ss = 0.0;
+        for (int c = 0; c < d; ++c) ss += xt[c] * xt[c];
+        double s = sqrt(ss) / sqrt_d;
+        s1[t] = s;
+        for (int c = 0; c < d; ++c) y[(size_t)t * d + c] = s > 0.0 ? xt[c] / s : 0.0;
+    }
+    /* Shift (channel-wise): o = mean over the T tokens, or the given o. */
+    for (int c = 0; c < d; ++c) {
+        if (shift_given) {
+            o_out[c] = o_in[c];
+        } else {
+            double acc = 0.0;
+            for (int64_t t = 0; t < T; ++t) acc += y[(size_t)t * d + c];
+            o_out[c] = T > 0 ? acc / (double)T : 0.0;
+        }
+    }
+    for (int64_t t = 0; t < T; ++t) {
+        double* yt = y + (size_t)t * d;
+        /* z = y - o; Normalize again: s2 = ||z|| / sqrt(d), u = z / s2. */
+        double ss = 0.0;
+        for (int c = 0; c < d; ++c) {
+            yt[c] -= o_out[c];
+            ss += yt[c] * yt[c];
+        }
+        double s = sqrt(ss) / sqrt_d;
+        s2[t] = s;
+        for (int c = 0; c < d; ++c) u[c] = s > 0.0 ? yt[c] / s : 0.0;
+        /* Hadamard (Methodology §2), then nearest codeword per sub-vector. */
+        hadamard_apply(H, d, u, w);
+        if (w_out) memcpy(w_out + (size_t)t * d, w, (size_t)d * sizeof(double));
+        for (int j = 0; j < J; ++j)
+            codes[(size_t)t * J + j] = (uint8_t)nearest_codeword(w + (size_t)j * g, C, K, g);
+    }
+    free(H); free(y); free(u); free(w);
+    return ORACLE_OK;
+}
+
+/*
+ * Dequantize one (batch, kv-head) slice: x_hat = s1 * (s2 * H w_hat + o),
+ * w_hat the concatenated codewords (Methodology §1: the byproducts
+ * reconstruct the tensor). s1, s2, o are the stored fp32 values.
+ */
+int oracle_dequant_head(const uint8_t* codes, const float* s1, const float* s2, const float* o,
+                        int64_t T, int d, int g, const float* C, int K, double* out) {
+    if (d <= 0 || (d & (d - 1)) != 0 || g <= 0 || d % g != 0 || K <= 0 || K > 256 || T < 0)
+        return ORACLE_ERR_ARG;
+    const int J = d / g;
+    double* H = (double*)malloc((size_t)d * d * sizeof(double));
+    double* wh = (double*)malloc((size_t)d * sizeof(double));
+    double* v = (double*)malloc((size_t)d * sizeof(double));
+    if (!H || !wh || !v) {
+        free(H); free(wh); free(v);
+        return ORACLE_ERR_MEM;
+    }
+    oracle_hadamard(d, H);
+    for (int64_t t = 0; t < T; ++t) {
+        for (int j = 0; j < J; ++j) {
+            int c = codes[(size_t)t * J + j];
+            if (c >= K) {
+                free(H); free(wh); free(v);
+                return ORACLE_ERR_ARG;
+            }
+            for (int r = 0; r < g; ++r) wh[j * g + r] = (double)C[(size_t)c * g + r];
+        }
+        hadamard_apply(H, d, wh, v);
+        for (int c = 0; c < d; ++c)
+            out[(size_t)t * d + c] =
+                (double)s1[t] * ((double)s2[t] * v[c] + (double)o[c]);
+    }
+    free(H); free(wh); free(v);
+    return ORACLE_OK;
+}
+
+/*
+ * Decode attention for the G query heads that share one kv-head, computed
+ * directly from the dense dequantized cache (Methodology §4 together with the
+ * standard definition): l_t = scale * q . k_t, p = softmax(l) (max
+ * subtracted), out = sum_t p_t v_t. T = 0 gives a zero output.
+ */
+int oracle_attention_head(const double* q, int G, const double* Kh, const double* Vh, int64_t T,
+                          int d, double scale, double* out) {
+    if (G <= 0 || d <= 0 || T < 0) return ORACLE_ERR_ARG;
+    double* l = (double*)malloc((size_t)(T > 0 ? T : 1) * sizeof(double));
+    if (!l) return ORACLE_ERR_MEM;
+    for (int h = 0; h < G; ++h) {
+        const double* qh = q + (size_t)h * d;
+        double* oh = out + (size_t)h * d;
+        for (int c = 0; c < d; ++c) oh[c] = 0.0;
+        if (T == 0) continue;
+        double m = -INFINITY;
+        for (int64_t t = 0; t < T; ++t) {
+            double acc = 0.0;
+            for (int c = 0; c < d; ++c) acc += qh[c] * Kh[(size_t)t * d + c];
+            l[t] = scale * acc;
+            if (l[t] > m) m = l[t];
+        }
+        double den = 0.0;
+        for (int64_t t = 0; t < T; ++t) {
+            double p = exp(l[t] - m);
+            den += p;
+            for (int c = 0; c < d; ++c) oh[c] += p * Vh[(size_t)t * d + c];
+        }
+        for (int c = 0; c < d; ++c) oh[c] /= den;
+    }
+    free(l);
+    return ORACLE_OK;
+}

@@ -1,0 +1,172 @@
+"""Python face of the CPU oracle (ctypes over oracle/nsnq_oracle.c).
+
+TEST INFRASTRUCTURE ONLY: imported by tests/, by the smoke check and by the
+benchmark's CPU-baseline leg, never by the product package. Everything here is
+argument marshalling and per-slice looping; the arithmetic is in the C file,
+single-threaded fp64.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        dp = ctypes.POINTER(ctypes.c_double)
+        fp = ctypes.POINTER(ctypes.c_float)
+        u8p = ctypes.POINTER(ctypes.c_uint8)
+        i64p = ctypes.POINTER(ctypes.c_int64)
+        L.oracle_hadamard.argtypes = [ctypes.c_int, dp]
+        L.oracle_kmeans.argtypes = [dp, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                    dp, i64p]
+        L.oracle_encode_head.argtypes = [dp, ctypes.c_int64, ctypes.c_int, ctypes.c_int, fp,
+                                         ctypes.c_int, ctypes.c_int, dp, u8p, dp, dp, dp, dp]
+        L.oracle_dequant_head.argtypes = [u8p, fp, fp, fp, ctypes.c_int64, ctypes.c_int,
+                                          ctypes.c_int, fp, ctypes.c_int, dp]
+        L.oracle_attention_head.argtypes = [dp, ctypes.c_int, dp, dp, ctypes.c_int64,
+                                            ctypes.c_int, ctypes.c_double, dp]
+        for f in ("oracle_hadamard", "oracle_kmeans", "oracle_encode_head",
+                  "oracle_dequant_head", "oracle_attention_head"):
+            getattr(L, f).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _p(a: Optional[np.ndarray], ct):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.POINTER(ct))
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise RuntimeError(f"oracle {what} failed with code {rc}")
+
+
+def hadamard(d: int) -> np.ndarray:
+    H = np.empty((d, d), dtype=np.float64)
+    _check(lib().oracle_hadamard(d, _p(H, ctypes.c_double)), "hadamard")
+    return H
+
+
+def kmeans(X: np.ndarray, k: int, iters: int):
+    """Lloyd k-means from the first k samples; returns (fp64 centroids, counts)."""
+    X = np.ascontiguousarray(X, dtype=np.float64)
+    n, g = X.shape
+    C = np.empty((k, g), dtype=np.float64)
+    counts = np.zeros(k, dtype=np.int64)
+    _check(lib().oracle_kmeans(_p(X, ctypes.c_double), n, g, k, iters, _p(C, ctypes.c_double),
+                               _p(counts, ctypes.c_int64)), "kmeans")
+    return C, counts
+
+
+def encode(x: np.ndarray, codebook: np.ndarray, shift: Optional[np.ndarray] = None,
+           want_w: bool = False):
+    """Encode x [B][H][T][d] (exact fp64 values of the I/O type).
+
+    shift None -> the shift is computed per (b, h) over the T tokens;
+    else shift [B][H][d] is used as given.
+    Returns dict with codes uint8 [B][H][T][d/g], s1, s2 fp64 [B][H][T],
+    o fp64 [B][H][d] and (optionally) w fp64 [B][H][T][d].
+    """
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    B, H, T, d = x.shape
+    C = np.ascontiguousarray(codebook, dtype=np.float32)
+    K, g = C.shape
+    J = d // g
+    codes = np.zeros((B, H, T, J), dtype=np.uint8)
+    s1 = np.zeros((B, H, T))
+    s2 = np.zeros((B, H, T))
+    o = np.zeros((B, H, d))
+    w = np.zeros((B, H, T, d)) if want_w else None
+    for b in range(B):
+        for h in range(H):
+            oin = None
+            if shift is not None:
+                oin = np.ascontiguousarray(shift[b, h], dtype=np.float64)
+            ob = np.zeros(d)
+            cb = np.zeros((T, J), dtype=np.uint8)
+            s1b = np.zeros(T)
+            s2b = np.zeros(T)
+            wb = np.zeros((T, d)) if want_w else None
+            _check(lib().oracle_encode_head(
+                _p(np.ascontiguousarray(x[b, h]), ctypes.c_double), T, d, g,
+                _p(C, ctypes.c_float), K, 1 if shift is not None else 0,
+                _p(oin, ctypes.c_double), _p(cb, ctypes.c_uint8), _p(s1b, ctypes.c_double),
+                _p(s2b, ctypes.c_double), _p(ob, ctypes.c_double), _p(wb, ctypes.c_double)),
+                "encode")
+            codes[b, h] = cb
+            s1[b, h] = s1b
+            s2[b, h] = s2b
+            o[b, h] = ob
+            if want_w:
+                w[b, h] = wb
+    return {"codes": codes, "s1": s1, "s2": s2, "o": o, "w": w}
+
+
+def dequant(codes: np.ndarray, s1: np.ndarray, s2: np.ndarray, o: np.ndarray,
+            codebook: np.ndarray) -> np.ndarray:
+    """x_hat [B][H][T][d] fp64 from codes [B][H][T][J] and stored fp32 s1, s2, o."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    B, H, T, J = codes.shape
+    C = np.ascontiguousarray(codebook, dtype=np.float32)
+    K, g = C.shape
+    d = J * g
+    s1 = np.asarray(s1, dtype=np.float32)
+    s2 = np.asarray(s2, dtype=np.float32)
+    o = np.asarray(o, dtype=np.float32)
+    out = np.zeros((B, H, T, d))
+    for b in range(B):
+        for h in range(H):
+            ob = np.zeros((T, d))
+            _check(lib().oracle_dequant_head(
+                _p(np.ascontiguousarray(codes[b, h]), ctypes.c_uint8),
+                _p(np.ascontiguousarray(s1[b, h]), ctypes.c_float),
+                _p(np.ascontiguousarray(s2[b, h]), ctypes.c_float),
+                _p(np.ascontiguousarray(o[b, h]), ctypes.c_float), T, d, g,
+                _p(C, ctypes.c_float), K, _p(ob, ctypes.c_double)), "dequant")
+            out[b, h] = ob
+    return out
+
+
+def attention(q: np.ndarray, Khat: np.ndarray, Vhat: np.ndarray, seq_lens=None,
+              scale: Optional[float] = None) -> np.ndarray:
+    """Decode attention: q [B][Hq][d], Khat/Vhat [B][Hkv][T][d] (dense dequantized),
+    query head h reads kv-head h // (Hq/Hkv); sequence b attends to its first
+    seq_lens[b] tokens. Returns fp64 [B][Hq][d]."""
+    q = np.ascontiguousarray(q, dtype=np.float64)
+    B, Hq, d = q.shape
+    Hkv, T = Khat.shape[1], Khat.shape[2]
+    G = Hq // Hkv
+    scale = 1.0 / np.sqrt(d) if scale is None else float(scale)
+    out = np.zeros((B, Hq, d))
+    for b in range(B):
+        L = T if seq_lens is None else int(seq_lens[b])
+        for kh in range(Hkv):
+            Kb = np.ascontiguousarray(Khat[b, kh, :L], dtype=np.float64)
+            Vb = np.ascontiguousarray(Vhat[b, kh, :L], dtype=np.float64)
+            qb = np.ascontiguousarray(q[b, kh * G:(kh + 1) * G])
+            ob = np.zeros((G, d))
+            _check(lib().oracle_attention_head(
+                _p(qb, ctypes.c_double), G, _p(Kb, ctypes.c_double), _p(Vb, ctypes.c_double),
+                L, d, scale, _p(ob, ctypes.c_double)), "attention")
+            out[b, kh * G:(kh + 1) * G] = ob
+    return out
+
+
+def stored(enc: dict):
+    """The fp32 values an encoder stores for (s1, s2, o)."""
+    return (enc["s1"].astype(np.float32), enc["s2"].astype(np.float32),
+            enc["o"].astype(np.float32))

@@ -1,0 +1,271 @@
+"""Pins for the CPU oracle: each test checks it against something other than
+itself (library routines, closed forms, textbook quantizers, invariants the
+method's definition fixes, brute force on tiny inputs)."""
+import hashlib
+import json
+import os
+
+import numpy as np
+import pytest
+import scipy.linalg
+import scipy.spatial.distance
+import torch
+
+import nsnq_synth as S
+from oracle import oracle as O
+from tests.conftest import GOLDEN
+
+D = 128
+
+
+# ---------------------------------------------------------------- Hadamard --
+@pytest.mark.parametrize("d", [1, 2, 4, 8, 16, 64, 128, 256])
+def test_hadamard_is_scipy_sylvester(d):
+    """NSNQuant Methodology §2 (naive Hadamard): the oracle's matrix equals
+    SciPy's Sylvester construction, normalised to be orthonormal."""
+    H = O.hadamard(d)
+    ref = scipy.linalg.hadamard(d).astype(np.float64) / np.sqrt(d)
+    assert np.array_equal(H, ref)
+    assert np.abs(H @ H - np.eye(d)).max() < 1e-12        # symmetric and H^2 = I
+    v = np.random.default_rng(d).standard_normal(d)
+    assert abs(np.linalg.norm(H @ v) - np.linalg.norm(v)) < 1e-12
+
+
+# ------------------------------------------------------------------ k-means --
+@pytest.mark.parametrize("k,centroids,mse", [
+    # J. Max, "Quantizing for minimum distortion" (1960), Gaussian source:
+    # 2 levels at +-sqrt(2/pi), MSE 1 - 2/pi; 4 levels at +-0.4528, +-1.5104, MSE 0.1175.
+    (2, [-0.7979, 0.7979], 0.3634),
+    (4, [-1.5104, -0.4528, 0.4528, 1.5104], 0.1175),
+])
+def test_kmeans_reaches_lloyd_max(k, centroids, mse):
+    X = S.normal(11, S.STREAM_EXTRA, 0, 1 << 17).reshape(-1, 1)
+    C, counts = O.kmeans(X, k, 300)
+    c = np.sort(C[:, 0])
+    assert np.allclose(c, centroids, rtol=0.015, atol=0.01), c
+    d2 = ((X - C[:, 0][None, :]) ** 2).min(1).mean()
+    assert abs(d2 - mse) < 0.01 * mse + 2e-3, d2
+    assert counts.sum() == X.shape[0]
+
+
+def test_kmeans_matches_sklearn_lloyd():
+    """Same recipe (init = first k samples, 25 Lloyd iterations) through
+    scikit-learn's independent implementation."""
+    from sklearn.cluster import KMeans
+    X = S.codebook_samples(4, 1 << 13, seed=5)
+    C, counts = O.kmeans(X, 64, 25)
+    assert counts.min() > 0  # no empty cluster, so the relocation rules cannot differ
+    km = KMeans(n_clusters=64, init=X[:64].copy(), n_init=1, max_iter=25, tol=0.0,
+                algorithm="lloyd").fit(X)
+    assert np.abs(km.cluster_centers_ - C).max() < 1e-9
+
+
+def test_kmeans_empty_cluster_keeps_centroid():
+    # Two identical seeds: in the first assignment every tie goes to index 0,
+    # so cluster 1 is empty and keeps its value; centroid 0 moves to the mean.
+    X = np.array([[0.0], [0.0], [1.0], [1.2]])
+    C, counts = O.kmeans(X, 2, 1)
+    assert C[1, 0] == 0.0 and counts[1] == 0
+    assert abs(C[0, 0] - 2.2 / 4) < 1e-15
+    # second iteration: the two zeros now prefer centroid 1
+    C, counts = O.kmeans(X, 2, 2)
+    assert list(counts) == [2, 2] and C[1, 0] == 0.0 and abs(C[0, 0] - 1.1) < 1e-15
+
+
+def test_codebook_files_are_the_recipe():
+    meta = json.load(open(os.path.join(GOLDEN, "codebooks.json")))
+    import oracle.make_codebooks as M
+    for g in (8, 4):
+        _, C, _ = M.make(g)
+        sha = hashlib.sha256(C.astype("<f4").tobytes()).hexdigest()
+        assert sha == meta["files"][f"codebook_g{g}.f32"]["sha256"]
+
+
+@pytest.mark.parametrize("g,lo,hi", [
+    # held-out distortion per coordinate lies between the Gaussian Shannon bound
+    # 2^(-2R) and the scalar Lloyd-Max quantizer at the same rate R = 8/g bits.
+    (8, 0.25, 0.3634),
+    (4, 0.0625, 0.1175),
+])
+def test_codebook_distortion_between_bounds(codebooks, g, lo, hi):
+    C = codebooks[g].astype(np.float64)
+    X = S.normal(21, S.STREAM_EXTRA, 0, 20000 * g).reshape(-1, g)
+    d2 = scipy.spatial.distance.cdist(X, C, "sqeuclidean").min(1).mean() / g
+    assert lo < d2 < hi, d2
+
+
+# ----------------------------------------------------------- NSN + encode --
+def _tiny_keys(T=256, seed=0):
+    w = S.WORKLOADS["tiny"]
+    return S.io_to_f64(S.to_io(S.keys(w, T_total=T, t1=T), "f32"), "f32")
+
+
+@pytest.mark.parametrize("g", [8, 4])
+def test_encode_nsn_invariants(codebooks, g):
+    """Methodology §1: after the shift the channel mean is 0, after the second
+    normalize every token has norm sqrt(d), and the byproducts (s1, o, s2)
+    rebuild the token exactly from the transformed vector."""
+    x = _tiny_keys()
+    enc = O.encode(x, codebooks[g], want_w=True)
+    H = scipy.linalg.hadamard(D) / np.sqrt(D)
+    w = enc["w"][0, 0]
+    u = w @ H  # H symmetric, H^2 = I
+    s1, s2, o = enc["s1"][0, 0], enc["s2"][0, 0], enc["o"][0, 0]
+    assert np.abs(np.linalg.norm(w, axis=1) - np.sqrt(D)).max() < 1e-12
+    assert np.abs(np.linalg.norm(u, axis=1) - np.sqrt(D)).max() < 1e-12
+    z = s2[:, None] * u
+    assert np.abs(z.mean(0)).max() < 1e-12 * np.abs(o).max()
+    rebuilt = s1[:, None] * (z + o[None, :])
+    assert np.abs(rebuilt - x[0, 0]).max() < 1e-12 * np.abs(x).max()
+    # the mean is taken over normalised tokens: o = mean of x / s1
+    assert np.abs(o - (x[0, 0] / s1[:, None]).mean(0)).max() < 1e-12
+
+
+@pytest.mark.parametrize("g", [8, 4])
+def test_encode_codes_are_nearest_codewords(codebooks, g):
+    """Methodology §3: every sub-vector maps to its nearest codeword (SciPy's
+    cdist + first-index argmin as the independent brute force)."""
+    x = _tiny_keys(T=32)
+    C = codebooks[g]
+    enc = O.encode(x, C, want_w=True)
+    sub = enc["w"][0, 0].reshape(-1, g)
+    dist = scipy.spatial.distance.cdist(sub, C.astype(np.float64), "sqeuclidean")
+    assert np.array_equal(enc["codes"][0, 0].reshape(-1), dist.argmin(1).astype(np.uint8))
+
+
+def test_encode_given_shift_uses_it(codebooks):
+    x = _tiny_keys(T=16)
+    o = np.random.default_rng(3).standard_normal((1, 1, D)) * 0.1
+    enc = O.encode(x, codebooks[4], shift=o, want_w=True)
+    assert np.array_equal(enc["o"], o)
+    H = scipy.linalg.hadamard(D) / np.sqrt(D)
+    u = enc["w"][0, 0] @ H
+    rebuilt = enc["s1"][0, 0][:, None] * (enc["s2"][0, 0][:, None] * u + o[0, 0][None, :])
+    assert np.abs(rebuilt - x[0, 0]).max() < 1e-12 * np.abs(x).max()
+
+
+def test_encode_degenerate_tokens():
+    """Zero token -> s1 = 0; a single token in compute mode -> z = 0, s2 = 0,
+    w = 0, so every code is the codeword of least norm (lowest index on ties)."""
+    C = np.full((256, 4), 3.0, dtype=np.float32)
+    C[5] = [1, 0, 0, 0]
+    C[9] = [0, 1, 0, 0]  # same norm as C[5]: the tie goes to index 5
+    x = np.zeros((1, 1, 1, D))
+    enc = O.encode(x, C)
+    assert enc["s1"][0, 0, 0] == 0 and enc["s2"][0, 0, 0] == 0
+    assert (enc["codes"] == 5).all()
+    x = np.random.default_rng(0).standard_normal((1, 1, 1, D))
+    enc = O.encode(x, C)
+    assert enc["s1"][0, 0, 0] > 0 and enc["s2"][0, 0, 0] == 0
+    assert (enc["codes"] == 5).all()
+    enc0 = O.encode(np.zeros((1, 1, 0, D)), C)
+    assert enc0["codes"].shape == (1, 1, 0, D // 4) and (enc0["o"] == 0).all()
+
+
+@pytest.mark.parametrize("g,T", [(8, 16), (4, 8)])
+def test_roundtrip_with_planted_codebook(g, T):
+    """Plant the transformed sub-vectors themselves as codewords (in shuffled
+    order): encode must pick exactly those indices, and dequant must give
+    back the input up to fp32 storage rounding of codebook, s1, s2, o."""
+    x = _tiny_keys(T=T)
+    rng = np.random.default_rng(7)
+    probe = rng.standard_normal((256, g)).astype(np.float32)
+    w = O.encode(x, probe, want_w=True)["w"][0, 0]
+    sub = w.reshape(-1, g)
+    assert sub.shape[0] == 256
+    perm = rng.permutation(256)
+    C = np.empty((256, g), dtype=np.float32)
+    C[perm] = sub.astype(np.float32)  # sub-vector i becomes codeword perm[i]
+    enc = O.encode(x, C)
+    assert np.array_equal(enc["codes"][0, 0].reshape(-1), perm.astype(np.uint8))
+    s1, s2, o = O.stored(enc)
+    xh = O.dequant(enc["codes"], s1, s2, o, C)
+    assert np.abs(xh - x).max() < 2e-6 * np.abs(x).max()
+
+
+def test_dequant_closed_form():
+    """All codes 0 with C_0 = e_0 (g = 4): w_hat has ones at coordinates 4j, and
+    by Walsh-function orthogonality H w_hat = (32/sqrt(128)) on coordinates
+    0..3 and 0 elsewhere."""
+    C = np.zeros((256, 4), dtype=np.float32)
+    C[0, 0] = 1.0
+    T = 3
+    codes = np.zeros((1, 1, T, 32), dtype=np.uint8)
+    s1 = np.array([[[1.0, 2.0, 0.5]]], dtype=np.float32)
+    s2 = np.array([[[1.0, 0.25, 3.0]]], dtype=np.float32)
+    o = np.linspace(-1, 1, D, dtype=np.float32).reshape(1, 1, D)
+    xh = O.dequant(codes, s1, s2, o, C)[0, 0]
+    hw = np.zeros(D)
+    hw[:4] = 32 / np.sqrt(D)
+    for t in range(T):
+        ref = float(s1[0, 0, t]) * (float(s2[0, 0, t]) * hw + o[0, 0].astype(np.float64))
+        assert np.abs(xh[t] - ref).max() < 1e-12
+
+
+def test_transformed_channels_are_near_standard_normal(codebooks):
+    """Methodology §1-§2 (Lemma 1 and the CLT argument): after NSN and the
+    Hadamard transform every channel has mean ~0 and variance ~1."""
+    w = S.WORKLOADS["encode-8x4096"]
+    x = S.io_to_f64(S.to_io(S.keys(w, b0=0, b1=1)[:, :2], "bf16"), "bf16")
+    enc = O.encode(x, codebooks[4], want_w=True)
+    for h in range(2):
+        wt = enc["w"][0, h]
+        T = wt.shape[0]
+        assert np.abs(wt.mean(0)).max() < 6 / np.sqrt(T)
+        assert np.abs(wt.var(0) - 1).max() < 0.1
+
+
+# --------------------------------------------------------------- attention --
+def _sdpa(q, K, V, scale):
+    return torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None], torch.from_numpy(K)[None], torch.from_numpy(V)[None],
+        scale=scale)[0].numpy()
+
+
+def test_attention_matches_torch_sdpa_with_gqa_and_lengths():
+    rng = np.random.default_rng(1)
+    B, Hq, Hkv, T = 3, 8, 2, 37
+    q = rng.standard_normal((B, Hq, D))
+    K = rng.standard_normal((B, Hkv, T, D)) * 1.5
+    V = rng.standard_normal((B, Hkv, T, D))
+    lens = np.array([37, 1, 20])
+    out = O.attention(q, K, V, lens)
+    G = Hq // Hkv
+    for b in range(B):
+        for h in range(Hq):
+            L = lens[b]
+            ref = _sdpa(q[b, h][None], K[b, h // G, :L], V[b, h // G, :L], 1 / np.sqrt(D))[0]
+            assert np.abs(out[b, h] - ref).max() < 1e-12
+
+
+def test_attention_special_cases():
+    rng = np.random.default_rng(2)
+    K = rng.standard_normal((1, 1, 50, D))
+    V = rng.standard_normal((1, 1, 50, D))
+    out = O.attention(np.zeros((1, 1, D)), K, V)       # q = 0 -> mean of v
+    assert np.abs(out[0, 0] - V[0, 0].mean(0)).max() < 1e-12
+    out = O.attention(rng.standard_normal((1, 1, D)), K, V, [1])  # one token -> v_0
+    assert np.abs(out[0, 0] - V[0, 0, 0]).max() < 1e-15
+    out = O.attention(rng.standard_normal((1, 1, D)), K, V, [0])  # empty -> 0
+    assert (out == 0).all()
+
+
+# ------------------------------------------------------------ input recipe --
+def test_synthetic_normals_are_standard_normal():
+    import scipy.stats
+    n = S.normal(123, 0, 0, 200000)
+    assert abs(n.mean()) < 0.01 and abs(n.var() - 1) < 0.01
+    assert scipy.stats.kstest(n, "norm").pvalue > 1e-3
+    # counter-based: any slice equals the same slice of the whole stream
+    assert np.array_equal(S.normal(123, 0, 1001, 77), n[1001:1078])
+
+
+def test_synthetic_keys_have_outlier_channels():
+    w = S.WORKLOADS["tiny"]
+    K = S.keys(w)
+    chans, signs = w.kdist.channels(D)
+    assert chans == [0, 32, 64, 96]
+    m = np.abs(K[0, 0]).mean(0)
+    assert all(m[c] > 5 for c in chans) and np.median(m) < 2
+    sub = S.keys(w, t0=100, t1=120, T_total=256)
+    assert np.array_equal(sub[0, 0], K[0, 0, 100:120])
