@@ -23,7 +23,8 @@
  *     from the quantized cache and the NSN byproducts.
  * Readings where the text is silent (stated once, used everywhere):
  *   s = ||v|| / sqrt(d) so that v / s has norm sqrt(d); a zero-norm token maps
- *   to the zero vector and keeps s = 0; H is the orthonormal Sylvester
+ *   to the zero vector and keeps s = 0, and a shift residual at or below
+ *   2^-20 of the token/shift magnitude counts as zero; H is the orthonormal Sylvester
  *   Hadamard matrix in natural order, H[i][j] = (-1)^popcount(i & j) / sqrt(d);
  *   sub-vector j covers coordinates [j*g, (j+1)*g); argmin ties go to the
  *   lowest index; k-means starts from the first k samples, runs a fixed
@@ -192,13 +193,18 @@ int oracle_encode_head(const double* x, int64_t T, int d, int g, const float* C,
     }
     for (int64_t t = 0; t < T; ++t) {
         double* yt = y + (size_t)t * d;
-        /* z = y - o; Normalize again: s2 = ||z|| / sqrt(d), u = z / s2. */
-        double ss = 0.0;
+        /* z = y - o; Normalize again: s2 = ||z|| / sqrt(d), u = z / s2.
+         * A residual at or below 2^-20 of sqrt(||y||^2 + ||o||^2) counts as
+         * zero (s2 = 0, u = 0): fp32-stored byproducts cannot resolve it, and
+         * it is exactly what a one-token prompt (o = y) produces. */
+        double ss = 0.0, yy = 0.0, oo = 0.0;
         for (int c = 0; c < d; ++c) {
+            yy += yt[c] * yt[c];
+            oo += o_out[c] * o_out[c];
             yt[c] -= o_out[c];
             ss += yt[c] * yt[c];
         }
-        double s = sqrt(ss) / sqrt_d;
+        double s = ss <= 0x1p-40 * (yy + oo) ? 0.0 : sqrt(ss) / sqrt_d;
         s2[t] = s;
         for (int c = 0; c < d; ++c) u[c] = s > 0.0 ? yt[c] / s : 0.0;
         /* Hadamard (Methodology §2), then nearest codeword per sub-vector. */

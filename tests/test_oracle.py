@@ -158,6 +158,11 @@ def test_encode_degenerate_tokens():
     enc = O.encode(x, C)
     assert enc["s1"][0, 0, 0] > 0 and enc["s2"][0, 0, 0] == 0
     assert (enc["codes"] == 5).all()
+    # identical tokens: o equals every y, the residual vanishes (rounding-level
+    # leftovers of the mean count as zero), so s2 = 0 for each of them
+    x = np.repeat(np.random.default_rng(1).standard_normal((1, 1, 1, D)), 3, axis=2)
+    enc = O.encode(x, C)
+    assert (enc["s2"] == 0).all() and (enc["codes"] == 5).all()
     enc0 = O.encode(np.zeros((1, 1, 0, D)), C)
     assert enc0["codes"].shape == (1, 1, 0, D // 4) and (enc0["o"] == 0).all()
 
