@@ -1,0 +1,214 @@
+"""B200-native NSNQuant KV-cache quantization and quantized decode attention.
+
+Thin Python binding over the C ABI in include/nsnq.h (libnsnq.so): argument
+marshalling only. Every step of the path runs in the library's sm_100a CUDA
+kernels; PyTorch supplies device memory and the current stream. There is no
+CPU fallback: if the library is missing, loading raises.
+
+    cb    = Codebook(centroids_fp32_256xg.cuda())
+    cache = Cache.empty(B, H, cap, sub_dim=cb.sub_dim, device="cuda")
+    nsnq_encode(x, cb, cache)                      # prompt: shift computed
+    nsnq_encode(x_new, cb, cache, t_offset=T, shift_mode=SHIFT_GIVEN)
+    out = nsnq_attn_decode(q, k_cache, v_cache, k_cb, v_cb, seq_lens, max_len)
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_build", "libnsnq.so")
+
+NSNQ_OK, NSNQ_ERR_INVALID_ARG, NSNQ_ERR_UNSUPPORTED, NSNQ_ERR_WORKSPACE, NSNQ_ERR_CUDA = range(5)
+NSNQ_F32, NSNQ_BF16 = 0, 1
+SHIFT_COMPUTE, SHIFT_GIVEN = 0, 1
+HEAD_DIM = 128
+N_CENTROIDS = 256
+
+EXPORTED = ("nsnq_status_string", "nsnq_last_error", "nsnq_encode_workspace", "nsnq_encode",
+            "nsnq_dequant", "nsnq_attn_workspace", "nsnq_attn_decode")
+
+
+class NSNQError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        super().__init__(f"{_status_name(status)}: {detail}")
+        self.status = status
+
+
+class _Codebook(ctypes.Structure):
+    _fields_ = [("centroids", ctypes.c_void_p), ("n_centroids", ctypes.c_int),
+                ("sub_dim", ctypes.c_int)]
+
+
+class _Cache(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("shift", ctypes.c_void_p), ("cap", ctypes.c_int64)]
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load libnsnq.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m attention_decode_b200.build`"
+                           " (the library has no CPU fallback)")
+    L = ctypes.CDLL(path)
+    vp, i64, ci, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    L.nsnq_status_string.argtypes = [ci]
+    L.nsnq_status_string.restype = ctypes.c_char_p
+    L.nsnq_last_error.argtypes = []
+    L.nsnq_last_error.restype = ctypes.c_char_p
+    L.nsnq_encode_workspace.argtypes = [ci, ci, i64, ci]
+    L.nsnq_encode_workspace.restype = sz
+    L.nsnq_encode.argtypes = [vp, ci, ci, ci, i64, ci, i64, i64, i64, i64, ci, _Codebook, _Cache,
+                              vp, sz, vp]
+    L.nsnq_encode.restype = ci
+    L.nsnq_dequant.argtypes = [_Cache, _Codebook, ci, ci, i64, i64, ci, vp, vp]
+    L.nsnq_dequant.restype = ci
+    L.nsnq_attn_workspace.argtypes = [ci, ci, ci, ci, i64]
+    L.nsnq_attn_workspace.restype = sz
+    L.nsnq_attn_decode.argtypes = [vp, ci, _Cache, _Cache, _Codebook, _Codebook, vp, i64, ci, ci,
+                                   ci, ci, ctypes.c_float, vp, ci, vp, sz, vp]
+    L.nsnq_attn_decode.restype = ci
+    _lib = L
+    return L
+
+
+def _status_name(s: int) -> str:
+    try:
+        return load().nsnq_status_string(s).decode()
+    except Exception:
+        return f"status {s}"
+
+
+def _check(status: int):
+    if status != NSNQ_OK:
+        raise NSNQError(status, load().nsnq_last_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return NSNQ_F32
+    if t.dtype == torch.bfloat16:
+        return NSNQ_BF16
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+@dataclasses.dataclass
+class Codebook:
+    """Global codebook: [256][sub_dim] fp32 on the device."""
+    centroids: torch.Tensor
+
+    @property
+    def sub_dim(self) -> int:
+        return int(self.centroids.shape[1])
+
+    def _c(self) -> _Codebook:
+        return _Codebook(_ptr(self.centroids), int(self.centroids.shape[0]), self.sub_dim)
+
+
+@dataclasses.dataclass
+class Cache:
+    """One quantized tensor (K or V): codes [B][H][cap][D/g] uint8,
+    scales [B][H][cap][2] fp32 (s1, s2), shift [B][H][D] fp32 (o)."""
+    codes: torch.Tensor
+    scales: torch.Tensor
+    shift: torch.Tensor
+
+    @property
+    def cap(self) -> int:
+        return int(self.codes.shape[2])
+
+    @classmethod
+    def empty(cls, B: int, H: int, cap: int, sub_dim: int, device="cuda", D: int = HEAD_DIM):
+        return cls(torch.zeros(B, H, cap, D // sub_dim, dtype=torch.uint8, device=device),
+                   torch.zeros(B, H, cap, 2, dtype=torch.float32, device=device),
+                   torch.zeros(B, H, D, dtype=torch.float32, device=device))
+
+    def _c(self) -> _Cache:
+        return _Cache(_ptr(self.codes), _ptr(self.scales), _ptr(self.shift), self.cap)
+
+
+def nsnq_encode_workspace(B: int, H: int, T: int, D: int = HEAD_DIM) -> int:
+    return int(load().nsnq_encode_workspace(B, H, T, D))
+
+
+def nsnq_attn_workspace(B: int, Hq: int, Hkv: int, max_len: int, D: int = HEAD_DIM) -> int:
+    return int(load().nsnq_attn_workspace(B, Hq, Hkv, D, max_len))
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def nsnq_encode(x: torch.Tensor, cb: Codebook, cache: Cache, t_offset: int = 0,
+                shift_mode: int = SHIFT_COMPUTE, workspace: Optional[torch.Tensor] = None,
+                stream=None) -> torch.Tensor:
+    """Encode x [B][H][T][D] (fp32 or bf16; channels contiguous) into cache
+    positions [t_offset, t_offset + T). Returns the workspace (its first two
+    uint64 hold the near-tie counters)."""
+    B, H, T, D = x.shape
+    if x.stride(3) != 1:
+        raise ValueError("x must have contiguous channels")
+    need = nsnq_encode_workspace(B, H, T, D)
+    if workspace is None:
+        workspace = _workspace(need, x.device)
+    _check(load().nsnq_encode(_ptr(x), _dtype_code(x), B, H, T, D, x.stride(0), x.stride(1),
+                              x.stride(2), t_offset, shift_mode, cb._c(), cache._c(),
+                              _ptr(workspace), workspace.numel() * workspace.element_size(),
+                              _stream(stream)))
+    return workspace
+
+
+def encode_stats(workspace: torch.Tensor):
+    """(token-heads, sub-vectors) decided on the fp64 near-tie path by the last encode."""
+    v = workspace[:16].cpu().view(torch.int64)
+    return int(v[0]), int(v[1])
+
+
+def nsnq_dequant(cache: Cache, cb: Codebook, B: int, H: int, t0: int, T: int,
+                 out: Optional[torch.Tensor] = None, D: int = HEAD_DIM, stream=None) -> torch.Tensor:
+    """Reconstruct tokens [t0, t0+T): returns fp32 [B][H][T][D]."""
+    if out is None:
+        out = torch.empty(B, H, T, D, dtype=torch.float32, device=cache.codes.device)
+    _check(load().nsnq_dequant(cache._c(), cb._c(), B, H, t0, T, D, _ptr(out), _stream(stream)))
+    return out
+
+
+def nsnq_attn_decode(q: torch.Tensor, k_cache: Cache, v_cache: Cache, k_cb: Codebook,
+                     v_cb: Codebook, seq_lens: torch.Tensor, max_len: int, Hkv: int,
+                     softmax_scale: float = 0.0, out_dtype: torch.dtype = torch.bfloat16,
+                     out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """One decode step: q [B][Hq][D] -> out [B][Hq][D] over the quantized caches."""
+    B, Hq, D = q.shape
+    if out is None:
+        out = torch.empty(B, Hq, D, dtype=out_dtype, device=q.device)
+    if workspace is None:
+        workspace = _workspace(nsnq_attn_workspace(B, Hq, Hkv, max_len, D), q.device)
+    if seq_lens.dtype != torch.int32:
+        raise TypeError("seq_lens must be int32")
+    _check(load().nsnq_attn_decode(_ptr(q), _dtype_code(q), k_cache._c(), v_cache._c(), k_cb._c(),
+                                   v_cb._c(), _ptr(seq_lens), max_len, B, Hq, Hkv, D,
+                                   float(softmax_scale), _ptr(out), _dtype_code(out),
+                                   _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                   _stream(stream)))
+    return out

@@ -1,0 +1,215 @@
+// C ABI of the NSNQuant library: argument validation, workspace planning and
+// kernel launches. Every check runs on the host before anything is launched.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+
+#include "../../include/nsnq.h"
+#include "internal.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+nsnq_status fail(nsnq_status s, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+nsnq_status ok() {
+    g_err[0] = '\0';
+    return NSNQ_OK;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+nsnq_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(NSNQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+nsnq_status check_codebook(const nsnq_codebook& cb, const char* name) {
+    if (!cb.centroids) return fail(NSNQ_ERR_INVALID_ARG, "%s.centroids is NULL", name);
+    if (!aligned(cb.centroids, 16))
+        return fail(NSNQ_ERR_INVALID_ARG, "%s.centroids must be 16-byte aligned", name);
+    if (cb.n_centroids != nsnq::kNCentroids)
+        return fail(NSNQ_ERR_UNSUPPORTED, "%s.n_centroids = %d (only 256 is supported)", name,
+                    cb.n_centroids);
+    if (cb.sub_dim != 4 && cb.sub_dim != 8)
+        return fail(NSNQ_ERR_UNSUPPORTED, "%s.sub_dim = %d (4 or 8 supported)", name, cb.sub_dim);
+    return NSNQ_OK;
+}
+
+nsnq_status check_cache(const nsnq_cache& c, const char* name, bool need_shift) {
+    if (!c.codes || !c.scales || (need_shift && !c.shift))
+        return fail(NSNQ_ERR_INVALID_ARG, "%s has a NULL buffer", name);
+    if (!aligned(c.codes, 16) || !aligned(c.scales, 16) || (c.shift && !aligned(c.shift, 16)))
+        return fail(NSNQ_ERR_INVALID_ARG, "%s buffers must be 16-byte aligned", name);
+    if (c.cap < 0) return fail(NSNQ_ERR_INVALID_ARG, "%s.cap = %lld < 0", name, (long long)c.cap);
+    return NSNQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* nsnq_status_string(nsnq_status s) {
+    switch (s) {
+        case NSNQ_OK: return "NSNQ_OK";
+        case NSNQ_ERR_INVALID_ARG: return "NSNQ_ERR_INVALID_ARG";
+        case NSNQ_ERR_UNSUPPORTED: return "NSNQ_ERR_UNSUPPORTED";
+        case NSNQ_ERR_WORKSPACE: return "NSNQ_ERR_WORKSPACE";
+        case NSNQ_ERR_CUDA: return "NSNQ_ERR_CUDA";
+    }
+    return "NSNQ_ERR_UNKNOWN";
+}
+
+const char* nsnq_last_error(void) { return g_err; }
+
+size_t nsnq_encode_workspace(int B, int H, int64_t T, int D) {
+    if (B < 0 || H < 0 || T < 0 || D != nsnq::kHeadDim) return 0;
+    return nsnq::plan_encode(B, H, T).total;
+}
+
+nsnq_status nsnq_encode(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t T, int D,
+                        int64_t stride_b, int64_t stride_h, int64_t stride_t, int64_t t_offset,
+                        nsnq_shift_mode mode, nsnq_codebook cb, nsnq_cache cache,
+                        void* workspace, size_t workspace_bytes, nsnq_stream stream) {
+    if (D != nsnq::kHeadDim) return fail(NSNQ_ERR_UNSUPPORTED, "D = %d (only 128 is supported)", D);
+    if (x_dtype != NSNQ_F32 && x_dtype != NSNQ_BF16)
+        return fail(NSNQ_ERR_UNSUPPORTED, "x_dtype = %d", (int)x_dtype);
+    if (mode != NSNQ_SHIFT_COMPUTE && mode != NSNQ_SHIFT_GIVEN)
+        return fail(NSNQ_ERR_INVALID_ARG, "shift mode = %d", (int)mode);
+    if (B < 0 || H < 0 || T < 0)
+        return fail(NSNQ_ERR_INVALID_ARG, "negative size B=%d H=%d T=%lld", B, H, (long long)T);
+    if (B > 65535 || H > 65535) return fail(NSNQ_ERR_UNSUPPORTED, "B or H above 65535");
+    nsnq_status s = check_codebook(cb, "cb");
+    if (s != NSNQ_OK) return s;
+    s = check_cache(cache, "cache", true);
+    if (s != NSNQ_OK) return s;
+    if (t_offset < 0 || t_offset > cache.cap || T > cache.cap - t_offset)
+        return fail(NSNQ_ERR_INVALID_ARG, "positions [%lld, %lld) exceed cache capacity %lld",
+                    (long long)t_offset, (long long)(t_offset + T), (long long)cache.cap);
+    if (B == 0 || H == 0 || T == 0) return ok();
+    if (!x) return fail(NSNQ_ERR_INVALID_ARG, "x is NULL");
+    const int64_t esz = x_dtype == NSNQ_BF16 ? 2 : 4;
+    if (!aligned(x, 16) || (stride_b * esz) % 16 || (stride_h * esz) % 16 || (stride_t * esz) % 16)
+        return fail(NSNQ_ERR_INVALID_ARG, "x and its strides must be 16-byte aligned");
+    if (stride_b < 0 || stride_h < 0 || stride_t < D)
+        return fail(NSNQ_ERR_INVALID_ARG, "strides must be non-negative with stride_t >= D");
+    const nsnq::EncodePlan plan = nsnq::plan_encode(B, H, T);
+    if (!workspace || workspace_bytes < plan.total)
+        return fail(NSNQ_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", plan.total,
+                    workspace ? workspace_bytes : (size_t)0);
+    if (!aligned(workspace, nsnq::kWsAlign))
+        return fail(NSNQ_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+
+    nsnq::EncodeArgs a{};
+    a.x = x;
+    a.x_bf16 = x_dtype == NSNQ_BF16;
+    a.B = B; a.H = H; a.T = T;
+    a.sb = stride_b; a.sh = stride_h; a.st = stride_t;
+    a.t_offset = t_offset;
+    a.given_shift = mode == NSNQ_SHIFT_GIVEN;
+    a.C = cb.centroids;
+    a.sub = cb.sub_dim;
+    a.codes = cache.codes; a.scales = cache.scales; a.shift = cache.shift; a.cap = cache.cap;
+    char* ws = static_cast<char*>(workspace);
+    a.stats = reinterpret_cast<unsigned long long*>(ws);
+    a.partial = reinterpret_cast<double*>(ws + plan.partial_off);
+    a.o64 = reinterpret_cast<double*>(ws + plan.o64_off);
+    a.nchunk1 = plan.nchunk1;
+    a.chunk1 = plan.chunk1;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(ws, 0, nsnq::kEncodeStatsBytes, st);
+    if (e != cudaSuccess) return cuda_fail(e, "workspace reset");
+    e = nsnq::launch_encode(a, st);
+    if (e != cudaSuccess) return cuda_fail(e, "encode launch");
+    return ok();
+}
+
+nsnq_status nsnq_dequant(nsnq_cache cache, nsnq_codebook cb, int B, int H, int64_t t0, int64_t T,
+                         int D, float* out, nsnq_stream stream) {
+    if (D != nsnq::kHeadDim) return fail(NSNQ_ERR_UNSUPPORTED, "D = %d (only 128 is supported)", D);
+    if (B < 0 || H < 0 || T < 0 || t0 < 0)
+        return fail(NSNQ_ERR_INVALID_ARG, "negative size or offset");
+    nsnq_status s = check_codebook(cb, "cb");
+    if (s != NSNQ_OK) return s;
+    s = check_cache(cache, "cache", true);
+    if (s != NSNQ_OK) return s;
+    if (t0 > cache.cap || T > cache.cap - t0)
+        return fail(NSNQ_ERR_INVALID_ARG, "positions [%lld, %lld) exceed cache capacity %lld",
+                    (long long)t0, (long long)(t0 + T), (long long)cache.cap);
+    if (B == 0 || H == 0 || T == 0) return ok();
+    if (!out || !aligned(out, 16)) return fail(NSNQ_ERR_INVALID_ARG, "out NULL or not 16-byte aligned");
+    nsnq::DequantArgs a{};
+    a.codes = cache.codes; a.scales = cache.scales; a.shift = cache.shift; a.cap = cache.cap;
+    a.C = cb.centroids; a.sub = cb.sub_dim;
+    a.B = B; a.H = H; a.t0 = t0; a.T = T;
+    a.out = out;
+    cudaError_t e = nsnq::launch_dequant(a, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "dequant launch");
+    return ok();
+}
+
+size_t nsnq_attn_workspace(int B, int Hq, int Hkv, int D, int64_t max_len) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || D != nsnq::kHeadDim || max_len < 0) return 0;
+    return nsnq::plan_attention(B, Hq, Hkv, max_len).total;
+}
+
+nsnq_status nsnq_attn_decode(const void* q, nsnq_dtype q_dtype, nsnq_cache k_cache,
+                             nsnq_cache v_cache, nsnq_codebook k_cb, nsnq_codebook v_cb,
+                             const int32_t* seq_lens, int64_t max_len, int B, int Hq, int Hkv,
+                             int D, float softmax_scale, void* out, nsnq_dtype out_dtype,
+                             void* workspace, size_t workspace_bytes, nsnq_stream stream) {
+    if (D != nsnq::kHeadDim) return fail(NSNQ_ERR_UNSUPPORTED, "D = %d (only 128 is supported)", D);
+    if ((q_dtype != NSNQ_F32 && q_dtype != NSNQ_BF16) ||
+        (out_dtype != NSNQ_F32 && out_dtype != NSNQ_BF16))
+        return fail(NSNQ_ERR_UNSUPPORTED, "q/out dtype must be NSNQ_F32 or NSNQ_BF16");
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv)
+        return fail(NSNQ_ERR_INVALID_ARG, "need B >= 0 and Hq a positive multiple of Hkv (B=%d Hq=%d Hkv=%d)",
+                    B, Hq, Hkv);
+    if (B > 65535 || Hq > 65535) return fail(NSNQ_ERR_UNSUPPORTED, "B or Hq above 65535");
+    if (!isfinite(softmax_scale)) return fail(NSNQ_ERR_INVALID_ARG, "softmax_scale is not finite");
+    nsnq_status s = check_codebook(k_cb, "k_cb");
+    if (s != NSNQ_OK) return s;
+    s = check_codebook(v_cb, "v_cb");
+    if (s != NSNQ_OK) return s;
+    s = check_cache(k_cache, "k_cache", true);
+    if (s != NSNQ_OK) return s;
+    s = check_cache(v_cache, "v_cache", true);
+    if (s != NSNQ_OK) return s;
+    if (max_len < 0 || max_len > k_cache.cap || max_len > v_cache.cap)
+        return fail(NSNQ_ERR_INVALID_ARG, "max_len = %lld must be in [0, min(cap)]",
+                    (long long)max_len);
+    if (B == 0) return ok();
+    if (!q || !out || !seq_lens) return fail(NSNQ_ERR_INVALID_ARG, "q, out or seq_lens is NULL");
+    if (!aligned(q, 16) || !aligned(out, 16) || !aligned(seq_lens, 4))
+        return fail(NSNQ_ERR_INVALID_ARG, "q and out must be 16-byte aligned");
+    const nsnq::AttnPlan plan = nsnq::plan_attention(B, Hq, Hkv, max_len);
+    if (!workspace || workspace_bytes < plan.total)
+        return fail(NSNQ_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", plan.total,
+                    workspace ? workspace_bytes : (size_t)0);
+    if (!aligned(workspace, nsnq::kWsAlign))
+        return fail(NSNQ_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    nsnq::AttnArgs a{};
+    a.q = q; a.q_bf16 = q_dtype == NSNQ_BF16;
+    a.kcodes = k_cache.codes; a.kscales = k_cache.scales; a.kshift = k_cache.shift;
+    a.kcap = k_cache.cap; a.kC = k_cb.centroids; a.ksub = k_cb.sub_dim;
+    a.vcodes = v_cache.codes; a.vscales = v_cache.scales; a.vshift = v_cache.shift;
+    a.vcap = v_cache.cap; a.vC = v_cb.centroids; a.vsub = v_cb.sub_dim;
+    a.seq_lens = seq_lens; a.max_len = max_len;
+    a.B = B; a.Hq = Hq; a.Hkv = Hkv;
+    const float scale = softmax_scale == 0.f ? 1.0f / sqrtf((float)D) : softmax_scale;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.out = out; a.out_bf16 = out_dtype == NSNQ_BF16;
+    a.part = static_cast<float*>(workspace);
+    a.plan = plan;
+    cudaError_t e = nsnq::launch_attention(a, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+    return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,362 @@
+// Decode attention over the NSNQuant-quantized KV cache on sm_100a
+// (gist.science "NSNQuant ...", Technical Summary, Methodology §4: the score
+// folds the NSN byproducts s1, s2, o into a kernel that reads the codes).
+//
+// With k_hat = s1 (s2 H w_hat + o) and H symmetric orthonormal:
+//   q . k_hat = s1 * (s2 * (H q) . w_hat + q . o)
+//             = s1 * (s2 * sum_j L[j][code_j] + gamma),  L[j][c] = (Hq)_j . C_c
+//   sum_t p_t v_hat_t = H (sum_t p_t s1_t s2_t w_hat_t) + (sum_t p_t s1_t) o_V
+// so a CTA rotates q once, builds L in shared memory, streams codes and
+// accumulates values in the Hadamard domain; a combine kernel merges the
+// context splits (online-softmax rescaling) and applies H once per head.
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace nsnq {
+
+constexpr int kAttnWarps = 8;
+constexpr int kAttnThreads = kAttnWarps * 32;
+
+template <int GC, int KSUB, int VSUB>
+struct AttnSmem {
+    static constexpr int KJ = kD / KSUB, VJ = kD / VSUB;
+    static constexpr size_t lut = (size_t)KJ * kNC * GC;  // floats
+    static constexpr size_t cv = (size_t)kNC * VSUB;
+    static constexpr size_t ck = (size_t)kNC * KSUB;
+    static constexpr size_t qrot = (size_t)GC * kD;
+    static constexpr size_t gam = 8;
+    static constexpr size_t wst = (size_t)kAttnWarps * 32 * GC;
+    static constexpr size_t floats = lut + cv + ck + qrot + gam + wst;
+    static constexpr size_t bytes = floats * 4 + (size_t)kAttnWarps * 32 * VJ;
+    static constexpr size_t merge_floats = (size_t)kAttnWarps * GC * (3 + kD);
+    static_assert(merge_floats <= lut, "merge area must fit in the LUT region");
+};
+
+template <typename QT>
+__device__ __forceinline__ void load_q4(const void* q, int64_t off, float (&v)[4]) {
+    load4(reinterpret_cast<const QT*>(q) + off, v);
+}
+
+template <int GC, int KSUB, int VSUB, typename QT>
+__global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a) {
+    using S = AttnSmem<GC, KSUB, VSUB>;
+    constexpr int KJ = S::KJ, VJ = S::VJ;
+    extern __shared__ __align__(16) float sm[];
+    float* lut = sm;
+    float* Cv = lut + S::lut;
+    float* Ck = Cv + S::cv;
+    float* qrot = Ck + S::ck;
+    float* gam = qrot + S::qrot;
+    float* wst = gam + S::gam;
+    uint8_t* cst = reinterpret_cast<uint8_t*>(wst + S::wst);
+
+    const int split = blockIdx.x, grp = blockIdx.y, b = blockIdx.z;
+    const int G = a.Hq / a.Hkv;
+    const int kvh = grp / a.plan.ngroups, hg = grp % a.plan.ngroups;
+    const int qh0 = kvh * G + hg * GC;
+    const int64_t bkv = (int64_t)b * a.Hkv + kvh;
+    const int nsplit = a.plan.nsplit;
+    int64_t len = a.seq_lens[b];
+    len = len < 0 ? 0 : (len > a.max_len ? a.max_len : len);
+    const int64_t ts = (int64_t)split * a.plan.split_len;
+    const int64_t te = min(ts + a.plan.split_len, len);
+    const int tid = threadIdx.x, lane = lane_id(), warp = tid >> 5;
+
+    if (ts >= te) {  // empty split: neutral partial
+        for (int idx = tid; idx < GC * kPartStride; idx += kAttnThreads) {
+            const int h = idx / kPartStride, c = idx % kPartStride;
+            float* P = a.part + (((int64_t)b * a.Hq + qh0 + h) * nsplit + split) * kPartStride;
+            P[c] = (c == kD) ? -INFINITY : 0.f;
+        }
+        return;
+    }
+
+    for (int i = tid; i < kNC * KSUB; i += kAttnThreads) Ck[i] = a.kC[i];
+    for (int i = tid; i < kNC * VSUB; i += kAttnThreads) Cv[i] = a.vC[i];
+    if (warp < GC) {
+        float qv[4];
+        load_q4<QT>(a.q, ((int64_t)b * a.Hq + qh0 + warp) * kD + 4 * lane, qv);
+        const float4 o = reinterpret_cast<const float4*>(a.kshift + bkv * kD)[lane];
+        const float g = warp_sum(fmaf(qv[3], o.w, fmaf(qv[2], o.z, fmaf(qv[1], o.y, qv[0] * o.x))));
+        fwht128_lane4(qv);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) qrot[warp * kD + 4 * lane + r] = qv[r] * kRsqrtD;
+        if (lane == 0) gam[warp] = g;
+    }
+    __syncthreads();
+    // L[j][c][h] = (Hq_h)[j*KSUB : (j+1)*KSUB] . C_c
+    for (int e = tid; e < KJ * kNC; e += kAttnThreads) {
+        const int j = e >> 8, c = e & (kNC - 1);
+        float ck[KSUB];
+#pragma unroll
+        for (int r = 0; r < KSUB; ++r) ck[r] = Ck[c * KSUB + r];
+#pragma unroll
+        for (int h = 0; h < GC; ++h) {
+            float s = 0.f;
+#pragma unroll
+            for (int r = 0; r < KSUB; ++r) s = fmaf(qrot[h * kD + j * KSUB + r], ck[r], s);
+            lut[(size_t)e * GC + h] = s;
+        }
+    }
+    __syncthreads();
+
+    float gm[GC];
+#pragma unroll
+    for (int h = 0; h < GC; ++h) gm[h] = gam[h];
+    float m[GC], l[GC], be[GC], A[GC][VSUB];
+#pragma unroll
+    for (int h = 0; h < GC; ++h) {
+        m[h] = -INFINITY; l[h] = 0.f; be[h] = 0.f;
+#pragma unroll
+        for (int r = 0; r < VSUB; ++r) A[h][r] = 0.f;
+    }
+    const uint8_t* kc = a.kcodes + bkv * a.kcap * KJ;
+    const uint8_t* vc = a.vcodes + bkv * a.vcap * VJ;
+    const float2* ks = reinterpret_cast<const float2*>(a.kscales) + bkv * a.kcap;
+    const float2* vs = reinterpret_cast<const float2*>(a.vscales) + bkv * a.vcap;
+    uint8_t* my_codes = cst + (size_t)warp * 32 * VJ;
+    float* my_w = wst + (size_t)warp * 32 * GC;
+    constexpr int TPI = 32 / VJ;  // tokens per V iteration (1 at VSUB=4, 2 at VSUB=8)
+    const int jj = lane % VJ, sub_t = lane / VJ;
+
+    for (int64_t base = ts + warp * 32; base < te; base += kAttnWarps * 32) {
+        const int64_t t = base + lane;
+        const bool valid = t < te;
+        float sc[GC];
+#pragma unroll
+        for (int h = 0; h < GC; ++h) sc[h] = 0.f;
+        float2 k2 = make_float2(0.f, 0.f), v2 = make_float2(0.f, 0.f);
+        if (valid) {
+            const uint4* kr = reinterpret_cast<const uint4*>(kc + t * KJ);
+#pragma unroll
+            for (int q4 = 0; q4 < KJ / 16; ++q4) {
+                const uint4 w4 = kr[q4];
+                const uint32_t wd[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                for (int wi = 0; wi < 4; ++wi) {
+#pragma unroll
+                    for (int by = 0; by < 4; ++by) {
+                        const int j = q4 * 16 + wi * 4 + by;
+                        const int code = (wd[wi] >> (8 * by)) & 0xff;
+                        const float* e = lut + ((size_t)(j << 8) + code) * GC;
+                        if constexpr (GC == 4) {
+                            const float4 ev = *reinterpret_cast<const float4*>(e);
+                            sc[0] += ev.x; sc[1] += ev.y; sc[2] += ev.z; sc[3] += ev.w;
+                        } else {
+#pragma unroll
+                            for (int h = 0; h < GC; ++h) sc[h] += e[h];
+                        }
+                    }
+                }
+            }
+            k2 = ks[t];
+            v2 = vs[t];
+            const uint4* vr = reinterpret_cast<const uint4*>(vc + t * VJ);
+            uint4* dst = reinterpret_cast<uint4*>(my_codes + lane * VJ);
+#pragma unroll
+            for (int q4 = 0; q4 < VJ / 16; ++q4) dst[q4] = vr[q4];
+        }
+#pragma unroll
+        for (int h = 0; h < GC; ++h) {
+            const float logit = valid ? k2.x * fmaf(k2.y, sc[h], gm[h]) * a.scale_log2 : -INFINITY;
+            const float mx = warp_max(logit);
+            const float mn = fmaxf(m[h], mx);
+            const float alpha = (mn == -INFINITY) ? 1.f : exp2f(m[h] - mn);
+            const float p = valid ? exp2f(logit - mn) : 0.f;
+            l[h] = fmaf(l[h], alpha, p);
+            be[h] = fmaf(be[h], alpha, p * v2.x);
+#pragma unroll
+            for (int r = 0; r < VSUB; ++r) A[h][r] *= alpha;
+            my_w[lane * GC + h] = p * v2.x * v2.y;
+            m[h] = mn;
+        }
+        __syncwarp();
+        const int nt = (int)min((int64_t)32, te - base);
+        for (int i = 0; i < nt; i += TPI) {
+            const int tt = i + sub_t;
+            if (tt < nt) {
+                const int code = my_codes[tt * VJ + jj];
+                float wv[GC];
+#pragma unroll
+                for (int h = 0; h < GC; ++h) wv[h] = my_w[tt * GC + h];
+                const float* cp = Cv + code * VSUB;
+#pragma unroll
+                for (int r = 0; r < VSUB; ++r) {
+                    const float c = cp[r];
+#pragma unroll
+                    for (int h = 0; h < GC; ++h) A[h][r] = fmaf(wv[h], c, A[h][r]);
+                }
+            }
+        }
+        __syncwarp();
+    }
+
+#pragma unroll
+    for (int h = 0; h < GC; ++h) {
+        l[h] = warp_sum(l[h]);
+        be[h] = warp_sum(be[h]);
+        if constexpr (TPI == 2) {
+#pragma unroll
+            for (int r = 0; r < VSUB; ++r) A[h][r] += __shfl_xor_sync(kFull, A[h][r], 16);
+        }
+    }
+    __syncthreads();  // LUT no longer needed: reuse it for the CTA merge
+    float* mw = sm;
+    float* lw = mw + kAttnWarps * GC;
+    float* bw = lw + kAttnWarps * GC;
+    float* Aw = bw + kAttnWarps * GC;  // [warp][h][128]
+    if (lane == 0) {
+#pragma unroll
+        for (int h = 0; h < GC; ++h) {
+            mw[warp * GC + h] = m[h]; lw[warp * GC + h] = l[h]; bw[warp * GC + h] = be[h];
+        }
+    }
+    if (lane < VJ) {
+#pragma unroll
+        for (int h = 0; h < GC; ++h)
+#pragma unroll
+            for (int r = 0; r < VSUB; ++r) Aw[(warp * GC + h) * kD + jj * VSUB + r] = A[h][r];
+    }
+    __syncthreads();
+    for (int idx = tid; idx < GC * (kD + 2); idx += kAttnThreads) {
+        const int h = idx / (kD + 2), c = idx % (kD + 2);
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, mw[w * GC + h]);
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < kAttnWarps; ++w) {
+            const float mv = mw[w * GC + h];
+            const float f = (mv == -INFINITY) ? 0.f : exp2f(mv - M);
+            float v;
+            if (c < kD) v = Aw[(w * GC + h) * kD + c];
+            else if (c == kD) v = lw[w * GC + h];
+            else v = bw[w * GC + h];
+            acc = fmaf(f, v, acc);
+        }
+        float* P = a.part + (((int64_t)b * a.Hq + qh0 + h) * nsplit + split) * kPartStride;
+        if (c < kD) P[c] = acc;
+        else if (c == kD) { P[kD] = M; P[kD + 1] = acc; }
+        else P[kD + 2] = acc;  // c == kD + 1: beta
+    }
+}
+
+// Merge the splits of one (batch, query head): rescale by exp2(m_s - M),
+// apply H to the rotated-domain sum, add beta * o_V, divide by l.
+__global__ void __launch_bounds__(kD) attn_combine_kernel(AttnArgs a) {
+    __shared__ float As[kD];
+    __shared__ float LB[2];
+    const int bq = blockIdx.x;
+    const int b = bq / a.Hq, qh = bq % a.Hq;
+    const int kvh = qh / (a.Hq / a.Hkv);
+    const int nsplit = a.plan.nsplit;
+    const float* P = a.part + (int64_t)bq * nsplit * kPartStride;
+    const int c = threadIdx.x;
+    float M = -INFINITY;
+    for (int s = 0; s < nsplit; ++s) M = fmaxf(M, P[(int64_t)s * kPartStride + kD]);
+    float acc = 0.f, L = 0.f, Be = 0.f;
+    if (M != -INFINITY) {
+        for (int s = 0; s < nsplit; ++s) {
+            const float* Ps = P + (int64_t)s * kPartStride;
+            const float ms = Ps[kD];
+            const float f = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
+            acc = fmaf(f, Ps[c], acc);
+            L = fmaf(f, Ps[kD + 1], L);
+            Be = fmaf(f, Ps[kD + 2], Be);
+        }
+    }
+    As[c] = acc;
+    if (c == 0) { LB[0] = L; LB[1] = Be; }
+    __syncthreads();
+    if (threadIdx.x >= 32) return;
+    const int lane = lane_id();
+    float v[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) v[r] = As[4 * lane + r];
+    fwht128_lane4(v);
+    const float Lt = LB[0], Bt = LB[1];
+    const float inv = Lt > 0.f ? 1.0f / Lt : 0.f;
+    const float4 o = reinterpret_cast<const float4*>(a.vshift + ((int64_t)b * a.Hkv + kvh) * kD)[lane];
+    float r4[4];
+    r4[0] = fmaf(Bt, o.x, v[0] * kRsqrtD) * inv;
+    r4[1] = fmaf(Bt, o.y, v[1] * kRsqrtD) * inv;
+    r4[2] = fmaf(Bt, o.z, v[2] * kRsqrtD) * inv;
+    r4[3] = fmaf(Bt, o.w, v[3] * kRsqrtD) * inv;
+    if (a.out_bf16) {
+        uint2 pk;
+        pk.x = (uint32_t)f32_to_bf16_rn(r4[0]) | ((uint32_t)f32_to_bf16_rn(r4[1]) << 16);
+        pk.y = (uint32_t)f32_to_bf16_rn(r4[2]) | ((uint32_t)f32_to_bf16_rn(r4[3]) << 16);
+        reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(a.out) + (int64_t)bq * kD)[lane] = pk;
+    } else {
+        reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + (int64_t)bq * kD)[lane] =
+            make_float4(r4[0], r4[1], r4[2], r4[3]);
+    }
+}
+
+// ---------------------------------------------------------------- host --
+static int device_sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        return 148;
+    }
+    return n;
+}
+
+AttnPlan plan_attention(int B, int Hq, int Hkv, int64_t max_len) {
+    AttnPlan p{};
+    const int G = Hq / Hkv;
+    p.gc = (G % 4 == 0) ? 4 : (G % 2 == 0 ? 2 : 1);
+    p.ngroups = G / p.gc;
+    const int64_t units = (int64_t)B * Hkv * p.ngroups;
+    const int64_t target = 4LL * device_sms();
+    int64_t want = (target + units - 1) / units;
+    if (want < 1) want = 1;
+    const int64_t L = max_len > 0 ? max_len : 1;
+    int64_t sl = (L + want - 1) / want;
+    sl = (sl + 255) / 256 * 256;
+    if (sl < 256) sl = 256;
+    p.split_len = sl;
+    p.nsplit = (int)((L + sl - 1) / sl);
+    p.total = align_up((size_t)B * Hq * p.nsplit * kPartStride * sizeof(float), kWsAlign);
+    return p;
+}
+
+template <int GC, int KSUB, int VSUB, typename QT>
+static cudaError_t launch_split(const AttnArgs& a, cudaStream_t s) {
+    using S = AttnSmem<GC, KSUB, VSUB>;
+    auto kern = attn_split_kernel<GC, KSUB, VSUB, QT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)S::bytes);
+    if (e != cudaSuccess) return e;
+    const dim3 grid(a.plan.nsplit, a.Hkv * a.plan.ngroups, a.B);
+    kern<<<grid, kAttnThreads, S::bytes, s>>>(a);
+    return cudaGetLastError();
+}
+
+template <int GC, typename QT>
+static cudaError_t launch_split_sub(const AttnArgs& a, cudaStream_t s) {
+    if (a.ksub == 4 && a.vsub == 4) return launch_split<GC, 4, 4, QT>(a, s);
+    if (a.ksub == 4 && a.vsub == 8) return launch_split<GC, 4, 8, QT>(a, s);
+    if (a.ksub == 8 && a.vsub == 4) return launch_split<GC, 8, 4, QT>(a, s);
+    return launch_split<GC, 8, 8, QT>(a, s);
+}
+
+template <typename QT>
+static cudaError_t launch_split_gc(const AttnArgs& a, cudaStream_t s) {
+    if (a.plan.gc == 4) return launch_split_sub<4, QT>(a, s);
+    if (a.plan.gc == 2) return launch_split_sub<2, QT>(a, s);
+    return launch_split_sub<1, QT>(a, s);
+}
+
+cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s) {
+    cudaError_t e = a.q_bf16 ? launch_split_gc<__nv_bfloat16>(a, s) : launch_split_gc<float>(a, s);
+    if (e != cudaSuccess) return e;
+    attn_combine_kernel<<<a.B * a.Hq, kD, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace nsnq

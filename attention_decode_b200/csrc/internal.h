@@ -1,0 +1,102 @@
+// Host-side interfaces between the C ABI layer and the kernel launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace nsnq {
+
+constexpr int kHeadDim = 128;      // the only head_dim the kernels support
+constexpr int kNCentroids = 256;   // one byte per code
+constexpr size_t kWsAlign = 256;
+constexpr size_t kEncodeStatsBytes = 64;
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// ------------------------------------------------------------------ encode --
+struct EncodeArgs {
+    const void* x;
+    int x_bf16;
+    int B, H;
+    int64_t T;
+    int64_t sb, sh, st;
+    int64_t t_offset;
+    int given_shift;
+    const float* C;
+    int sub;
+    uint8_t* codes;
+    float* scales;
+    float* shift;
+    int64_t cap;
+    // workspace views
+    unsigned long long* stats;  // [8]
+    double* partial;            // [B][H][nchunk1][128]
+    double* o64;                // [B][H][128]
+    int nchunk1;
+    int64_t chunk1;
+};
+
+struct EncodePlan {
+    int nchunk1;
+    int64_t chunk1;
+    size_t partial_off, o64_off, total;
+};
+
+EncodePlan plan_encode(int B, int H, int64_t T);
+cudaError_t launch_encode(const EncodeArgs& a, cudaStream_t s);
+
+// ----------------------------------------------------------------- dequant --
+struct DequantArgs {
+    const uint8_t* codes;
+    const float* scales;
+    const float* shift;
+    int64_t cap;
+    const float* C;
+    int sub;
+    int B, H;
+    int64_t t0, T;
+    float* out;
+};
+cudaError_t launch_dequant(const DequantArgs& a, cudaStream_t s);
+
+// --------------------------------------------------------------- attention --
+constexpr int kPartStride = 132;  // 128 rotated-domain values + (m, l, beta, pad)
+
+struct AttnPlan {
+    int gc;          // query heads per CTA
+    int ngroups;     // head groups per kv-head
+    int64_t split_len;
+    int nsplit;
+    size_t total;
+};
+
+AttnPlan plan_attention(int B, int Hq, int Hkv, int64_t max_len);
+
+struct AttnArgs {
+    const void* q;
+    int q_bf16;
+    const uint8_t* kcodes;
+    const float* kscales;
+    const float* kshift;
+    int64_t kcap;
+    const float* kC;
+    int ksub;
+    const uint8_t* vcodes;
+    const float* vscales;
+    const float* vshift;
+    int64_t vcap;
+    const float* vC;
+    int vsub;
+    const int32_t* seq_lens;
+    int64_t max_len;
+    int B, Hq, Hkv;
+    float scale_log2;
+    void* out;
+    int out_bf16;
+    float* part;
+    AttnPlan plan;
+};
+cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s);
+
+}  // namespace nsnq

@@ -1,0 +1,419 @@
+#!/usr/bin/env python3
+"""Benchmark: NSNQuant KV-cache encode + quantized decode attention on B200.
+
+One step = the hot path over one batch of the Llama-3-8B layer workload
+(8 sequences x 8 kv-heads x 4096 prompt tokens, head_dim 128, bf16, 2 bits
+per coordinate): encode K, encode V (normalize-shift-normalize, Hadamard,
+nearest-codeword VQ), then one decode-attention query per sequence over the
+fresh quantized cache (32 query heads, GQA 4:1). `value` is KV tokens encoded
+per second over the whole step, all ranks together (weak scaling: every rank
+runs its own batch; no collective on the data path).
+
+The same run also times decode attention alone at the 32k-context workload
+(16 x 32 query heads / 8 kv-heads x 32768 tokens, 2 bit) and reports its HBM
+GB/s under "attention".
+
+  python bench.py [--gpus N --steps K --warmup W]          # CUDA path
+  python bench.py --impl reference ...                     # the CPU oracle
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import nsnq_synth as S  # noqa: E402
+
+GOLDEN = os.path.join(ROOT, "tests", "golden")
+METRIC = "KV tokens/s encoded and quantized decode-attn HBM GB/s (fraction of peak), 1 B200"
+STEP_WORKLOAD = "encode-8x4096"
+ATTN_WORKLOAD = "decode-16x32k-2b"
+STEP_HQ = 32
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_codebook(g: int) -> np.ndarray:
+    return np.fromfile(os.path.join(GOLDEN, f"codebook_g{g}.f32"), dtype="<f4").reshape(256, g)
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def encode_bytes_per_token_head(sub: int, in_bytes: int = 2) -> int:
+    """Algorithmic bytes of encode per token-head: input row, codes, (s1, s2)."""
+    return 128 * in_bytes + 128 // sub + 8
+
+
+def attn_bytes_per_token(ksub: int, vsub: int) -> int:
+    """Algorithmic bytes of attention per (batch, kv-head, token): K and V codes plus scales."""
+    return 128 // ksub + 128 // vsub + 16
+
+
+# ------------------------------------------------------------------ clocks --
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100", "-f", self.path],
+                stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------- CUDA arm --
+def run_cuda(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    torch.cuda.set_device(local)
+    from attention_decode_b200 import build as nbuild
+    nbuild.build()
+    import attention_decode_b200 as nsnq
+
+    dev = torch.device("cuda", local)
+    w = S.WORKLOADS[STEP_WORKLOAD]
+    B, H, T, Hq = w.B, w.Hkv, w.T, STEP_HQ
+    cb = nsnq.Codebook(torch.from_numpy(load_codebook(w.sub_dim)).to(dev))
+    # Inputs: seeded synthetic K/V of the workload (ranks draw disjoint sequences).
+    kx = S.to_io(S.keys(w), "bf16")
+    vx = S.to_io(S.values(w), "bf16")
+    qx = S.to_io(S.queries(S.Workload(**{**w.__dict__, "Hq": Hq}), step=rank), "bf16")
+    host = {n: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
+            for n, a in (("k", kx), ("v", vx), ("q", qx))}
+    k = host["k"].to(dev)
+    v = host["v"].to(dev)
+    q = host["q"].to(dev)
+    kc = nsnq.Cache.empty(B, H, T, w.sub_dim, device=dev)
+    vc = nsnq.Cache.empty(B, H, T, w.sub_dim, device=dev)
+    ws_e = torch.empty(nsnq.nsnq_encode_workspace(B, H, T), dtype=torch.uint8, device=dev)
+    ws_a = torch.empty(max(256, nsnq.nsnq_attn_workspace(B, Hq, H, T)), dtype=torch.uint8, device=dev)
+    seq = torch.full((B,), T, dtype=torch.int32, device=dev)
+    out = torch.empty(B, Hq, 128, dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(kin, vin, qin):
+        nsnq.nsnq_encode(kin, cb, kc, workspace=ws_e)
+        nsnq.nsnq_encode(vin, cb, vc, workspace=ws_e)
+        nsnq.nsnq_attn_decode(qin, kc, vc, cb, cb, seq, T, Hkv=H, out=out, workspace=ws_a)
+
+    LAUNCHES_PER_STEP = 3 + 3 + 2  # (stats, shift, encode) x 2 + (split, combine)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step(k, v, q)
+    torch.cuda.synchronize()
+
+    # ---- timed device-resident steps (L2 flushed before each step) ----
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            e = ev[i]
+            e[0].record(stream)
+            nsnq.nsnq_encode(k, cb, kc, workspace=ws_e)
+            e[1].record(stream)
+            nsnq.nsnq_encode(v, cb, vc, workspace=ws_e)
+            e[2].record(stream)
+            nsnq.nsnq_attn_decode(q, kc, vc, cb, cb, seq, T, Hkv=H, out=out, workspace=ws_a)
+            e[3].record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    step_ms = [e[0].elapsed_time(e[3]) for e in ev]
+    enc_ms = [e[0].elapsed_time(e[1]) for e in ev] + [e[1].elapsed_time(e[2]) for e in ev]
+    att_small_ms = [e[2].elapsed_time(e[3]) for e in ev]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    tokens_per_step = B * T * world
+    value = tokens_per_step / (ms_per_step / 1e3)
+
+    # ---- end to end: pinned host K/V in, result out, through the public API ----
+    res_host = torch.empty(B, Hq, 128, dtype=torch.bfloat16).pin_memory()
+    codes_host = torch.empty(2, *kc.codes.shape, dtype=torch.uint8).pin_memory()
+    scales_host = torch.empty(2, *kc.scales.shape, dtype=torch.float32).pin_memory()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e2e_ms = 0.0
+    for i in range(args.steps):
+        flush.zero_()
+        e0.record(stream)
+        k.copy_(host["k"], non_blocking=True)
+        v.copy_(host["v"], non_blocking=True)
+        q.copy_(host["q"], non_blocking=True)
+        step(k, v, q)
+        res_host.copy_(out, non_blocking=True)
+        codes_host[0].copy_(kc.codes, non_blocking=True)
+        codes_host[1].copy_(vc.codes, non_blocking=True)
+        scales_host[0].copy_(kc.scales, non_blocking=True)
+        scales_host[1].copy_(vc.scales, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        e2e_ms += e0.elapsed_time(e1)
+    barrier()
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = sum(host[n].numel() * host[n].element_size() for n in ("k", "v", "q"))
+    d2h = (res_host.numel() * 2 + codes_host.numel() + scales_host.numel() * 4)
+    e2e = {"value": tokens_per_step / (e2e_ms / args.steps / 1e3), "unit": "KV tokens/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    # ---- roofline of the dominant call (encode), algorithmic bytes ----
+    hbm, peak_kind = peaks()
+    enc_bytes = B * H * T * encode_bytes_per_token_head(w.sub_dim)
+    enc_avg_ms = sum(enc_ms) / len(enc_ms)
+    enc_gbs = enc_bytes / (enc_avg_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(enc_gbs, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(enc_gbs / hbm, 4), "peak_kind": peak_kind,
+                "kernel": "nsnq_encode (nsn_stats + nsn_shift + nsn_encode, one tensor)",
+                "algorithmic_bytes_per_launch": enc_bytes,
+                "traffic": args.traffic}
+
+    # ---- decode attention alone at the 32k workload ----
+    attention = run_attention_bench(args, nsnq, dev, world, barrier, hbm, peak_kind)
+
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": "KV tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded K with outlier channels x LogNormal token scale, V ~ N(0,1))",
+        "config": {"workload": "encode-8x4096 + decode (Llama-3-8B layer: B 8, Hkv 8, Hq 32, "
+                               "T 4096, d 128, 2 bit/coord)",
+                   "global_batch": B * world, "seq_len": T, "parallelism": f"replicas x{world}",
+                   "l2": "flushed (256 MB write) before every timed step"},
+        "stages_ms": {"encode_per_tensor": round(enc_avg_ms, 4),
+                      "attention_4k": round(sum(att_small_ms) / len(att_small_ms), 4)},
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "roofline": roofline, "attention": attention, "e2e": e2e, "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(args)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_attention_bench(args, nsnq, dev, world, barrier, hbm, peak_kind):
+    """Decode attention over a 32k-token 2-bit cache built by encoding seeded
+    K/V of the workload's distribution (generated on the device)."""
+    import torch
+    import torch.distributed as dist
+    w = S.WORKLOADS[ATTN_WORKLOAD]
+    B, H, Hq, T = w.B, w.Hkv, w.Hq, w.T
+    cb = nsnq.Codebook(torch.from_numpy(load_codebook(w.sub_dim)).to(dev))
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1234)
+    kc = nsnq.Cache.empty(B, H, T, w.sub_dim, device=dev)
+    vc = nsnq.Cache.empty(B, H, T, w.sub_dim, device=dev)
+    chans, signs = w.kdist.channels(128)
+    bias = torch.zeros(128, device=dev)
+    bias[chans] = torch.tensor(signs, device=dev) * w.kdist.bias
+    for b in range(B):  # one sequence at a time keeps the bf16 staging at 8 MB x 8
+        z = torch.randn(1, H, T, 128, generator=gen, device=dev)
+        s = torch.exp(w.kdist.sigma * torch.randn(1, H, T, 1, generator=gen, device=dev))
+        x = ((z + bias) * s).to(torch.bfloat16)
+        sub = nsnq.Cache(kc.codes[b:b + 1], kc.scales[b:b + 1], kc.shift[b:b + 1])
+        nsnq.nsnq_encode(x, cb, sub)
+        x = torch.randn(1, H, T, 128, generator=gen, device=dev).to(torch.bfloat16)
+        sub = nsnq.Cache(vc.codes[b:b + 1], vc.scales[b:b + 1], vc.shift[b:b + 1])
+        nsnq.nsnq_encode(x, cb, sub)
+    q = torch.randn(B, Hq, 128, generator=gen, device=dev).to(torch.bfloat16)
+    seq = torch.full((B,), T, dtype=torch.int32, device=dev)
+    out = torch.empty(B, Hq, 128, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(nsnq.nsnq_attn_workspace(B, Hq, H, T), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        nsnq.nsnq_attn_decode(q, kc, vc, cb, cb, seq, T, Hkv=H, out=out, workspace=ws)
+    stream = torch.cuda.current_stream()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for e0, e1 in evs:
+        flush.zero_()
+        e0.record(stream)
+        nsnq.nsnq_attn_decode(q, kc, vc, cb, cb, seq, T, Hkv=H, out=out, workspace=ws)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = [a.elapsed_time(b) for a, b in evs]
+    avg = sum(ms) / len(ms)
+    if world > 1:
+        t = torch.tensor([avg], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        avg = float(t.item())
+    nbytes = B * H * T * attn_bytes_per_token(w.sub_dim, w.sub_dim)
+    gbs = nbytes / (avg / 1e3) / 1e9
+    return {"metric": "decode-attn HBM GB/s (algorithmic bytes)", "value": round(gbs * world, 1),
+            "unit": "GB/s", "ms_per_call": round(avg, 4),
+            "workload": "decode-16x32k-2b (B 16, Hq 32, Hkv 8, T 32768, d 128, 2 bit K and V)",
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(gbs / hbm, 4), "peak_kind": peak_kind,
+                         "kernel": "nsnq_attn_decode (attn_split + attn_combine)",
+                         "algorithmic_bytes_per_launch": nbytes, "traffic": None},
+            "l2": "flushed before every call (cache 335 MB > L2 anyway)"}
+
+
+# ------------------------------------------------------------ oracle arm --
+def oracle_step_sample(n_seq: int = 1, n_heads: int = 8):
+    """The oracle on a bounded sample of the step: n_seq sequences x n_heads
+    kv-heads (K and V encode, dequant, attention for their query heads).
+    Returns (seconds, tokens-equivalent processed)."""
+    from oracle import oracle as O
+    w = S.WORKLOADS[STEP_WORKLOAD]
+    C = load_codebook(w.sub_dim)
+    k = S.io_to_f64(S.to_io(S.keys(w, b0=0, b1=n_seq)[:, :n_heads], "bf16"), "bf16")
+    v = S.io_to_f64(S.to_io(S.values(w, b0=0, b1=n_seq)[:, :n_heads], "bf16"), "bf16")
+    G = STEP_HQ // w.Hkv
+    q = S.io_to_f64(S.to_io(S.queries(S.Workload(**{**w.__dict__, "Hq": STEP_HQ}), B=n_seq)
+                            [:, :n_heads * G], "bf16"), "bf16")
+    t0 = time.perf_counter()
+    ok, ov = O.encode(k, C), O.encode(v, C)
+    Kh = O.dequant(ok["codes"], *O.stored(ok), C)
+    Vh = O.dequant(ov["codes"], *O.stored(ov), C)
+    O.attention(q, Kh, Vh)
+    dt = time.perf_counter() - t0
+    # tokens are counted over all kv-heads of the layer: scale by the sampled fraction
+    tokens = n_seq * w.T * (n_heads / w.Hkv)
+    return dt, tokens
+
+
+def cpu_baseline(args):
+    dt, tokens = oracle_step_sample(1, 8)
+    return {"value": round(tokens / dt, 2), "unit": "KV tokens/s", "cores": 1, "kind": "oracle",
+            "sample": "1 sequence x 8 kv-heads x 4096 tokens (K+V encode, dequant, attention of 32 "
+                      f"query heads), single-threaded fp64 C, {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from oracle import build as obuild
+    obuild.build()
+    for _ in range(args.warmup):
+        oracle_step_sample(1, 1)
+    times, toks = [], 0.0
+    for _ in range(args.steps):
+        dt, tokens = oracle_step_sample(1, 2)
+        times.append(dt)
+        toks = tokens
+    avg = sum(times) / len(times)
+    value = toks / avg
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "KV tokens/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(avg * 1e3, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "encode-8x4096 + decode (Llama-3-8B layer: B 8, Hkv 8, Hq 32, "
+                               "T 4096, d 128, 2 bit/coord)", "global_batch": 8, "seq_len": 4096,
+                   "parallelism": "none (CPU oracle)"},
+        "cpu_baseline": {"value": round(value, 2), "unit": "KV tokens/s", "cores": 1,
+                         "kind": "oracle",
+                         "sample": "per step: 1 sequence x 2 kv-heads x 4096 tokens (K+V encode, "
+                                   "dequant, attention of 8 query heads), scaled to all 8 kv-heads"},
+        "e2e": {"value": round(value, 2), "unit": "KV tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["nsnq", "reference"], default="nsnq")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="dram bytes per launch of the roofline kernel from an ncu capture")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_cuda(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,157 @@
+/*
+ * nsnq.h -- C ABI of the B200 (sm_100a) NSNQuant KV-cache library.
+ *
+ * NSNQuant ("NSNQuant: A Double Normalization Approach for Calibration-Free
+ * Low-Bit Vector Quantization of KV Cache", as summarised on gist.science,
+ * Technical Summary) quantizes each key/value token in four steps:
+ *   (Methodology §1) Normalize-Shift-Normalize: s1 = ||x||/sqrt(D), y = x/s1;
+ *       o = channel-wise mean of y over the prompt; z = y - o;
+ *       s2 = ||z||/sqrt(D), u = z/s2 (so ||u|| = sqrt(D));
+ *   (Methodology §2) w = H u with the naive orthonormal Hadamard matrix H
+ *       (Sylvester order, entries +-1/sqrt(D));
+ *   (Methodology §3) each sub-vector w[j*g:(j+1)*g] is replaced by the index
+ *       of its nearest codeword in one global 256-entry codebook built by
+ *       k-means on standard-normal samples (g = 8: 1 bit/coordinate,
+ *       g = 4: 2 bits/coordinate);
+ *   (Methodology §4) attention scores and outputs are computed from the codes
+ *       and the byproducts (s1, s2, o) directly.
+ * Reconstruction: x_hat = s1 * (s2 * H w_hat + o).
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers unless stated otherwise. The
+ *    caller owns every buffer, the workspace and the stream; the library
+ *    allocates no memory and keeps no state besides a thread-local error
+ *    message. Calls are asynchronous on `stream` (NULL = legacy default
+ *    stream) and never synchronise.
+ *  - Arguments are validated on the host before anything is launched; on
+ *    error the call returns a non-zero status, writes nothing, launches
+ *    nothing, and nsnq_last_error() describes the problem. A failed launch
+ *    returns NSNQ_ERR_CUDA. Faults that happen later on the device surface on
+ *    the stream like any CUDA error.
+ *  - Supported: D = 128, 256 centroids, sub_dim in {4, 8}, Hq % Hkv == 0.
+ *    Query head h reads kv-head h / (Hq / Hkv).
+ *  - Cache layout (one nsnq_cache per tensor, K and V separately):
+ *      codes  uint8 [B][H][cap][D/sub_dim], sub-vector j ascending
+ *      scales fp32  [B][H][cap][2] = (s1, s2)
+ *      shift  fp32  [B][H][D]      = o
+ */
+#ifndef NSNQ_H_
+#define NSNQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t (the runtime's stream handle); NULL is the legacy default stream. */
+typedef struct CUstream_st* nsnq_stream;
+
+typedef enum {
+    NSNQ_OK = 0,
+    NSNQ_ERR_INVALID_ARG = 1,  /* null pointer, bad size, stride or range */
+    NSNQ_ERR_UNSUPPORTED = 2,  /* valid but not implemented (D != 128, sub_dim, ...) */
+    NSNQ_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required */
+    NSNQ_ERR_CUDA = 4          /* a CUDA call or kernel launch failed */
+} nsnq_status;
+
+typedef enum { NSNQ_F32 = 0, NSNQ_BF16 = 1 } nsnq_dtype;
+
+typedef enum {
+    NSNQ_SHIFT_COMPUTE = 0,  /* o = mean of the normalized tokens of this call (a prompt) */
+    NSNQ_SHIFT_GIVEN = 1     /* o read from cache.shift (tokens appended after the prompt) */
+} nsnq_shift_mode;
+
+typedef struct {
+    const float* centroids;  /* device, [n_centroids][sub_dim] fp32, 16-byte aligned */
+    int n_centroids;         /* must be 256 (one byte per code) */
+    int sub_dim;             /* 4 (2 bits/coordinate) or 8 (1 bit/coordinate) */
+} nsnq_codebook;
+
+typedef struct {
+    uint8_t* codes;   /* device, [B][H][cap][D/sub_dim] */
+    float* scales;    /* device, [B][H][cap][2] = (s1, s2) */
+    float* shift;     /* device, [B][H][D] = o */
+    int64_t cap;      /* token capacity per (batch, head) */
+} nsnq_cache;
+
+/* Human-readable name of a status code (static string). */
+const char* nsnq_status_string(nsnq_status status);
+
+/* Detail of the last error returned on the calling thread ("" if none). */
+const char* nsnq_last_error(void);
+
+/*
+ * Workspace bytes nsnq_encode needs for this shape (any shift mode). The
+ * first 64 bytes hold counters the call resets and fills:
+ *   uint64 [0] token-heads re-encoded on the fp64 near-tie path,
+ *   uint64 [1] sub-vectors whose code was decided on that path.
+ */
+size_t nsnq_encode_workspace(int B, int H, int64_t T, int D);
+
+/*
+ * nsnq_encode -- NSN normalize/shift/normalize, Hadamard transform and
+ * nearest-codeword quantization of T tokens per (batch, head)
+ * (Methodology §1-§3), written to cache positions [t_offset, t_offset+T).
+ *
+ *   x         device, element (b, h, t, c) at x[b*stride_b + h*stride_h +
+ *             t*stride_t + c] (strides in elements, channels contiguous),
+ *             dtype x_dtype (fp32 or bf16); 16-byte aligned rows.
+ *   mode      NSNQ_SHIFT_COMPUTE: o = mean over the T tokens of x/s1, stored
+ *             to cache.shift (fp32); NSNQ_SHIFT_GIVEN: o = cache.shift.
+ *   cb        codebook; cache: codes/scales written, shift read or written.
+ *   workspace device scratch of at least nsnq_encode_workspace(B, H, T, D)
+ *             bytes, 256-byte aligned.
+ * Codes equal the nearest codeword of the exact (fp64) transformed token;
+ * sub-vectors whose two best fp32 distances are within a relative 1e-4 are
+ * re-decided in fp64. Stored s1, s2, o are fp32 roundings. A zero-norm
+ * token (or a zero residual after the shift) maps to the zero vector with
+ * s = 0. T = 0 is a no-op.
+ */
+nsnq_status nsnq_encode(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t T, int D,
+                        int64_t stride_b, int64_t stride_h, int64_t stride_t, int64_t t_offset,
+                        nsnq_shift_mode mode, nsnq_codebook cb, nsnq_cache cache,
+                        void* workspace, size_t workspace_bytes, nsnq_stream stream);
+
+/*
+ * nsnq_dequant -- reconstruct tokens [t0, t0+T) of every (batch, head):
+ * out = s1 * (s2 * H w_hat + o), w_hat the concatenated codewords
+ * (Methodology §1: the byproducts reconstruct the tensor).
+ *   out  device fp32 [B][H][T][D], 16-byte aligned.
+ * No workspace. T = 0 is a no-op.
+ */
+nsnq_status nsnq_dequant(nsnq_cache cache, nsnq_codebook cb, int B, int H, int64_t t0, int64_t T,
+                         int D, float* out, nsnq_stream stream);
+
+/* Workspace bytes nsnq_attn_decode needs (split-context partials). */
+size_t nsnq_attn_workspace(int B, int Hq, int Hkv, int D, int64_t max_len);
+
+/*
+ * nsnq_attn_decode -- one decode step of attention for one query token per
+ * sequence, reading the quantized K/V caches directly (Methodology §4):
+ *   score_t = scale * q . k_hat_t
+ *           = scale * s1_t * (s2_t * sum_j L[j][code_t,j] + q . o_K),
+ *     L[j][c] = (H q)[j*g:(j+1)*g] . C_c   (H symmetric, so q . H w = (Hq) . w),
+ *   out = sum_t softmax(score)_t v_hat_t
+ *       = (H sum_t p_t s1_t s2_t w_hat_t + (sum_t p_t s1_t) o_V) / sum_t p_t.
+ *   q        device [B][Hq][D], q_dtype (fp32 or bf16).
+ *   k_cache, v_cache, k_cb, v_cb: caches and their codebooks (sub_dims may differ).
+ *   seq_lens device int32 [B]; sequence b attends to its first
+ *            min(seq_lens[b], max_len) tokens (0 gives a zero output).
+ *   max_len  host upper bound on seq_lens, <= both caps; sizes the split plan.
+ *   softmax_scale  0 means 1/sqrt(D).
+ *   out      device [B][Hq][D], out_dtype (fp32 or bf16, rounded to nearest even).
+ *   workspace  >= nsnq_attn_workspace(B, Hq, Hkv, D, max_len) bytes, 256-byte aligned.
+ */
+nsnq_status nsnq_attn_decode(const void* q, nsnq_dtype q_dtype, nsnq_cache k_cache,
+                             nsnq_cache v_cache, nsnq_codebook k_cb, nsnq_codebook v_cb,
+                             const int32_t* seq_lens, int64_t max_len, int B, int Hq, int Hkv,
+                             int D, float softmax_scale, void* out, nsnq_dtype out_dtype,
+                             void* workspace, size_t workspace_bytes, nsnq_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NSNQ_H_ */

@@ -1,0 +1,139 @@
+"""C ABI checks that need no GPU: the library builds and loads, exports every
+entry point include/nsnq.h declares, and rejects bad arguments on the host
+before anything is launched."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import attention_decode_b200 as nsnq
+from attention_decode_b200 import build as nbuild
+from tests.conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "nsnq.h")
+FAKE = 0x10000  # a 16-byte aligned non-null address: validation never dereferences it
+
+
+@pytest.fixture(scope="module")
+def lib():
+    nbuild.build()
+    return nsnq.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(nsnq_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_exported_set(lib):
+    decl = declared_functions()
+    assert set(decl) == set(nsnq.EXPORTED), decl
+    for name in decl:
+        assert hasattr(lib, name), name
+
+
+def test_symbols_in_dynamic_table(lib):
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", nsnq.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    for name in declared_functions():
+        assert re.search(rf"\bT {name}\b", out), name
+
+
+def test_status_strings(lib):
+    assert lib.nsnq_status_string(0) == b"NSNQ_OK"
+    assert lib.nsnq_status_string(3) == b"NSNQ_ERR_WORKSPACE"
+
+
+def _cb(sub=4, n=256, ptr=FAKE):
+    return nsnq._Codebook(ptr, n, sub)
+
+
+def _cache(cap=100):
+    return nsnq._Cache(FAKE, FAKE, FAKE, cap)
+
+
+def _encode(lib, **kw):
+    a = dict(x=FAKE, dt=nsnq.NSNQ_BF16, B=1, H=1, T=10, D=128, sb=128 * 10, sh=128 * 10, st=128,
+             off=0, mode=0, cb=_cb(), cache=_cache(), ws=FAKE, wsb=1 << 20, stream=None)
+    a.update(kw)
+    return lib.nsnq_encode(a["x"], a["dt"], a["B"], a["H"], a["T"], a["D"], a["sb"], a["sh"],
+                           a["st"], a["off"], a["mode"], a["cb"], a["cache"], a["ws"], a["wsb"],
+                           a["stream"])
+
+
+def test_encode_validation(lib):
+    assert _encode(lib, D=64) == nsnq.NSNQ_ERR_UNSUPPORTED
+    assert _encode(lib, cb=_cb(sub=5)) == nsnq.NSNQ_ERR_UNSUPPORTED
+    assert _encode(lib, cb=_cb(n=128)) == nsnq.NSNQ_ERR_UNSUPPORTED
+    assert _encode(lib, cb=_cb(ptr=None)) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert _encode(lib, x=None) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert _encode(lib, x=FAKE + 2) == nsnq.NSNQ_ERR_INVALID_ARG        # misaligned
+    assert _encode(lib, st=100) == nsnq.NSNQ_ERR_INVALID_ARG            # stride_t < D
+    assert _encode(lib, off=95) == nsnq.NSNQ_ERR_INVALID_ARG            # past capacity
+    assert _encode(lib, T=-1) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert _encode(lib, mode=7) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert _encode(lib, ws=None) == nsnq.NSNQ_ERR_WORKSPACE
+    need = lib.nsnq_encode_workspace(1, 1, 10, 128)
+    assert need > 0
+    assert _encode(lib, wsb=need - 1) == nsnq.NSNQ_ERR_WORKSPACE
+    assert b"workspace" in lib.nsnq_last_error()
+    assert _encode(lib, T=0) == nsnq.NSNQ_OK                            # no-op, no launch
+    assert lib.nsnq_last_error() == b""
+
+
+def test_encode_workspace_grows_with_tokens(lib):
+    a = lib.nsnq_encode_workspace(8, 8, 4096, 128)
+    b = lib.nsnq_encode_workspace(8, 8, 8192, 128)
+    assert 0 < a < b and a % 256 == 0
+    assert lib.nsnq_encode_workspace(8, 8, 4096, 64) == 0
+
+
+def test_dequant_validation(lib):
+    f = lambda **kw: lib.nsnq_dequant(kw.get("cache", _cache()), kw.get("cb", _cb()), 1, 1,
+                                      kw.get("t0", 0), kw.get("T", 10), kw.get("D", 128),
+                                      kw.get("out", FAKE), None)
+    assert f(D=256) == nsnq.NSNQ_ERR_UNSUPPORTED
+    assert f(t0=95) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert f(out=None) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert f(out=FAKE + 4) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert f(cache=nsnq._Cache(None, FAKE, FAKE, 100)) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert f(T=0) == nsnq.NSNQ_OK
+
+
+def _attn(lib, **kw):
+    a = dict(q=FAKE, qdt=nsnq.NSNQ_BF16, kc=_cache(), vc=_cache(), kcb=_cb(4), vcb=_cb(8),
+             lens=FAKE, max_len=100, B=2, Hq=8, Hkv=2, D=128, scale=0.0, out=FAKE,
+             odt=nsnq.NSNQ_BF16, ws=FAKE, wsb=1 << 24)
+    a.update(kw)
+    return lib.nsnq_attn_decode(a["q"], a["qdt"], a["kc"], a["vc"], a["kcb"], a["vcb"], a["lens"],
+                                a["max_len"], a["B"], a["Hq"], a["Hkv"], a["D"], a["scale"],
+                                a["out"], a["odt"], a["ws"], a["wsb"], None)
+
+
+def test_attention_validation(lib):
+    assert _attn(lib, Hq=6, Hkv=4) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert _attn(lib, max_len=101) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert _attn(lib, vc=_cache(cap=50)) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert _attn(lib, lens=None) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert _attn(lib, qdt=9) == nsnq.NSNQ_ERR_UNSUPPORTED
+    assert _attn(lib, vcb=_cb(3)) == nsnq.NSNQ_ERR_UNSUPPORTED
+    assert _attn(lib, scale=float("nan")) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert _attn(lib, wsb=16) == nsnq.NSNQ_ERR_WORKSPACE
+    assert _attn(lib, B=0) == nsnq.NSNQ_OK
+    need = lib.nsnq_attn_workspace(2, 8, 2, 128, 100)
+    assert need > 0 and need % 256 == 0
+    assert lib.nsnq_attn_workspace(2, 8, 3, 128, 100) == 0
+
+
+def test_binding_has_no_fallback(tmp_path):
+    """The binding raises when the library file is absent; it never computes on the CPU."""
+    import importlib
+    mod = importlib.reload(nsnq)
+    mod._lib = None
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        mod.load(str(tmp_path / "missing.so"))
+    mod._lib = None
+    mod.load()
