@@ -30,7 +30,7 @@ HEAD_DIM = 128
 N_CENTROIDS = 256
 
 EXPORTED = ("nsnq_status_string", "nsnq_last_error", "nsnq_encode_workspace", "nsnq_encode",
-            "nsnq_dequant", "nsnq_attn_workspace", "nsnq_attn_decode")
+            "nsnq_dequant", "nsnq_attn_workspace", "nsnq_attn_decode", "nsnq_attn_decode_noalloc")
 
 
 class NSNQError(RuntimeError):
@@ -78,6 +78,9 @@ def load(path: str = LIB_PATH):
     L.nsnq_attn_decode.argtypes = [vp, ci, _Cache, _Cache, _Codebook, _Codebook, vp, i64, ci, ci,
                                    ci, ci, ctypes.c_float, vp, ci, vp, sz, vp]
     L.nsnq_attn_decode.restype = ci
+    L.nsnq_attn_decode_noalloc.argtypes = [vp, ci, _Cache, _Cache, _Codebook, _Codebook, vp, i64,
+                                           ci, ci, ci, ci, ctypes.c_float, vp, ci, vp]
+    L.nsnq_attn_decode_noalloc.restype = ci
     _lib = L
     return L
 
@@ -211,4 +214,23 @@ def nsnq_attn_decode(q: torch.Tensor, k_cache: Cache, v_cache: Cache, k_cb: Code
                                    float(softmax_scale), _ptr(out), _dtype_code(out),
                                    _ptr(workspace), workspace.numel() * workspace.element_size(),
                                    _stream(stream)))
+    return out
+
+
+def nsnq_attn_decode_noalloc(q: torch.Tensor, k_cache: Cache, v_cache: Cache, k_cb: Codebook,
+                             v_cb: Codebook, seq_lens: torch.Tensor, max_len: int, Hkv: int,
+                             softmax_scale: float = 0.0, out_dtype: torch.dtype = torch.bfloat16,
+                             out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """nsnq_attn_decode without a workspace: the split partials live in the
+    library's fixed 4 MiB device array (for callers that cannot allocate).
+    Calls on one device must not overlap on the GPU."""
+    B, Hq, D = q.shape
+    if out is None:
+        out = torch.empty(B, Hq, D, dtype=out_dtype, device=q.device)
+    if seq_lens.dtype != torch.int32:
+        raise TypeError("seq_lens must be int32")
+    _check(load().nsnq_attn_decode_noalloc(_ptr(q), _dtype_code(q), k_cache._c(), v_cache._c(),
+                                           k_cb._c(), v_cb._c(), _ptr(seq_lens), max_len, B, Hq,
+                                           Hkv, D, float(softmax_scale), _ptr(out),
+                                           _dtype_code(out), _stream(stream)))
     return out

@@ -53,6 +53,16 @@ nsnq_status check_cache(const nsnq_cache& c, const char* name, bool need_shift) 
 
 }  // namespace
 
+namespace nsnq {
+nsnq_status set_error(nsnq_status s, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return s;
+}
+}  // namespace nsnq
+
 extern "C" {
 
 const char* nsnq_status_string(nsnq_status s) {

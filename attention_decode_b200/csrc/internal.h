@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "../../include/nsnq.h"
+
 namespace nsnq {
 
 constexpr int kHeadDim = 128;      // the only head_dim the kernels support
@@ -13,6 +15,9 @@ constexpr size_t kWsAlign = 256;
 constexpr size_t kEncodeStatsBytes = 64;
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Record a printf-style message as the calling thread's nsnq_last_error().
+nsnq_status set_error(nsnq_status s, const char* fmt, ...);
 
 // ------------------------------------------------------------------ encode --
 struct EncodeArgs {

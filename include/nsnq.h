@@ -21,7 +21,7 @@
  *  - All tensor pointers are DEVICE pointers unless stated otherwise. The
  *    caller owns every buffer, the workspace and the stream; the library
  *    allocates no memory and keeps no state besides a thread-local error
- *    message. Calls are asynchronous on `stream` (NULL = legacy default
+ *    message (and the fixed device array of nsnq_attn_decode_noalloc). Calls are asynchronous on `stream` (NULL = legacy default
  *    stream) and never synchronise.
  *  - Arguments are validated on the host before anything is launched; on
  *    error the call returns a non-zero status, writes nothing, launches
@@ -149,6 +149,36 @@ nsnq_status nsnq_attn_decode(const void* q, nsnq_dtype q_dtype, nsnq_cache k_cac
                              const int32_t* seq_lens, int64_t max_len, int B, int Hq, int Hkv,
                              int D, float softmax_scale, void* out, nsnq_dtype out_dtype,
                              void* workspace, size_t workspace_bytes, nsnq_stream stream);
+
+/*
+ * nsnq_attn_decode_noalloc -- nsnq_attn_decode for callers that cannot
+ * allocate device memory (no workspace argument). The method has no
+ * counterpart for this: it is a packaging of the same kernels.
+ *
+ * Who needs it: code that cannot call cudaMalloc or reach an allocator --
+ * a plugin inside an engine that owns all device memory, a real-time loop
+ * where an allocation (which may synchronise the device) is not allowed, or
+ * a C caller without an allocator. The caller still passes q, the caches,
+ * seq_lens and out; only the split-context partials move into a fixed
+ * 4 MiB array in device global memory that the library defines. Every GPU
+ * that loads the library reserves those 4 MiB until the process exits.
+ *
+ * Limit: shapes whose partials need more than 4 MiB
+ * (nsnq_attn_workspace(B, Hq, Hkv, D, max_len) > 4194304) are rejected with
+ * NSNQ_ERR_WORKSPACE before anything is launched.
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture. The array is shared by all calls and keeps the
+ * last call's contents; nothing in it needs to start at zero. Calls that
+ * overlap on the GPU (different streams, or different host threads on the
+ * same device) race on the array: serialise them. Arguments, errors and
+ * results are otherwise exactly those of nsnq_attn_decode.
+ */
+nsnq_status nsnq_attn_decode_noalloc(const void* q, nsnq_dtype q_dtype, nsnq_cache k_cache,
+                                     nsnq_cache v_cache, nsnq_codebook k_cb, nsnq_codebook v_cb,
+                                     const int32_t* seq_lens, int64_t max_len, int B, int Hq,
+                                     int Hkv, int D, float softmax_scale, void* out,
+                                     nsnq_dtype out_dtype, nsnq_stream stream);
 
 #ifdef __cplusplus
 }
