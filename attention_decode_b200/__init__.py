@@ -29,8 +29,9 @@ SHIFT_COMPUTE, SHIFT_GIVEN = 0, 1
 HEAD_DIM = 128
 N_CENTROIDS = 256
 
-EXPORTED = ("nsnq_status_string", "nsnq_last_error", "nsnq_encode_workspace", "nsnq_encode",
-            "nsnq_dequant", "nsnq_attn_workspace", "nsnq_attn_decode", "nsnq_attn_decode_noalloc")
+EXPORTED = ("nsnq_status_string", "nsnq_last_error", "nsnq_codebook_index_bytes",
+            "nsnq_codebook_index_build", "nsnq_encode_workspace", "nsnq_encode", "nsnq_dequant",
+            "nsnq_attn_workspace", "nsnq_attn_decode", "nsnq_attn_decode_noalloc")
 
 
 class NSNQError(RuntimeError):
@@ -41,7 +42,7 @@ class NSNQError(RuntimeError):
 
 class _Codebook(ctypes.Structure):
     _fields_ = [("centroids", ctypes.c_void_p), ("n_centroids", ctypes.c_int),
-                ("sub_dim", ctypes.c_int)]
+                ("sub_dim", ctypes.c_int), ("index", ctypes.c_void_p)]
 
 
 class _Cache(ctypes.Structure):
@@ -66,6 +67,10 @@ def load(path: str = LIB_PATH):
     L.nsnq_status_string.restype = ctypes.c_char_p
     L.nsnq_last_error.argtypes = []
     L.nsnq_last_error.restype = ctypes.c_char_p
+    L.nsnq_codebook_index_bytes.argtypes = [ci]
+    L.nsnq_codebook_index_bytes.restype = sz
+    L.nsnq_codebook_index_build.argtypes = [_Codebook, vp, sz, vp]
+    L.nsnq_codebook_index_build.restype = ci
     L.nsnq_encode_workspace.argtypes = [ci, ci, i64, ci]
     L.nsnq_encode_workspace.restype = sz
     L.nsnq_encode.argtypes = [vp, ci, ci, ci, i64, ci, i64, i64, i64, i64, ci, _Codebook, _Cache,
@@ -117,15 +122,30 @@ def _dtype_code(t: torch.Tensor) -> int:
 
 @dataclasses.dataclass
 class Codebook:
-    """Global codebook: [256][sub_dim] fp32 on the device."""
+    """Global codebook: [256][sub_dim] fp32 on the device. A 2-bit
+    (sub_dim 4) codebook also carries its search index, built on first use
+    by nsnq_codebook_index_build."""
     centroids: torch.Tensor
+    index: Optional[torch.Tensor] = None
 
     @property
     def sub_dim(self) -> int:
         return int(self.centroids.shape[1])
 
+    def prepare(self, stream=None) -> "Codebook":
+        if self.sub_dim == 4 and self.index is None:
+            n = int(load().nsnq_codebook_index_bytes(4))
+            idx = torch.empty(n, dtype=torch.uint8, device=self.centroids.device)
+            raw = _Codebook(_ptr(self.centroids), int(self.centroids.shape[0]), 4, None)
+            _check(load().nsnq_codebook_index_build(raw, _ptr(idx), n, _stream(stream)))
+            self.index = idx
+        return self
+
     def _c(self) -> _Codebook:
-        return _Codebook(_ptr(self.centroids), int(self.centroids.shape[0]), self.sub_dim)
+        if self.sub_dim == 4 and self.index is None and self.centroids.is_cuda:
+            self.prepare()
+        return _Codebook(_ptr(self.centroids), int(self.centroids.shape[0]), self.sub_dim,
+                         _ptr(self.index))
 
 
 @dataclasses.dataclass
@@ -182,9 +202,10 @@ def nsnq_encode(x: torch.Tensor, cb: Codebook, cache: Cache, t_offset: int = 0,
 
 
 def encode_stats(workspace: torch.Tensor):
-    """(token-heads, sub-vectors) decided on the fp64 near-tie path by the last encode."""
-    v = workspace[:16].cpu().view(torch.int64)
-    return int(v[0]), int(v[1])
+    """(token-heads, sub-vectors) decided on the fp64 near-tie path by the last
+    encode, and whether the codebook index did not match the centroids."""
+    v = workspace[:24].cpu().view(torch.int64)
+    return int(v[0]), int(v[1]), int(v[2])
 
 
 def nsnq_dequant(cache: Cache, cb: Codebook, B: int, H: int, t0: int, T: int,

@@ -78,6 +78,32 @@ const char* nsnq_status_string(nsnq_status s) {
 
 const char* nsnq_last_error(void) { return g_err; }
 
+size_t nsnq_codebook_index_bytes(int sub_dim) {
+    return sub_dim == 4 ? nsnq::index_bytes() : 0;
+}
+
+nsnq_status nsnq_codebook_index_build(nsnq_codebook cb, void* index, size_t index_bytes,
+                                      nsnq_stream stream) {
+    nsnq_status s = check_codebook(cb, "cb");
+    if (s != NSNQ_OK) return s;
+    if (cb.sub_dim != 4) return fail(NSNQ_ERR_UNSUPPORTED, "only sub_dim 4 codebooks take an index");
+    if (!index || !aligned(index, 16))
+        return fail(NSNQ_ERR_INVALID_ARG, "index NULL or not 16-byte aligned");
+    if (index_bytes < nsnq::index_bytes())
+        return fail(NSNQ_ERR_WORKSPACE, "index of %zu bytes needed, %zu given", nsnq::index_bytes(),
+                    index_bytes);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = nsnq::launch_index_build(cb.centroids, index, st);
+    if (e != cudaSuccess) return cuda_fail(e, "index build launch");
+    uint32_t hdr[4] = {0, 0, 0, 0};
+    e = cudaMemcpyAsync(hdr, index, sizeof(hdr), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "index build");
+    if (hdr[2] != 0)
+        return fail(NSNQ_ERR_UNSUPPORTED, "codebook index needs %u list entries (limit 65535)", hdr[1]);
+    return ok();
+}
+
 size_t nsnq_encode_workspace(int B, int H, int64_t T, int D) {
     if (B < 0 || H < 0 || T < 0 || D != nsnq::kHeadDim) return 0;
     return nsnq::plan_encode(B, H, T).total;
@@ -115,6 +141,9 @@ nsnq_status nsnq_encode(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t
                     workspace ? workspace_bytes : (size_t)0);
     if (!aligned(workspace, nsnq::kWsAlign))
         return fail(NSNQ_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    if (cb.sub_dim == 4 && (!cb.index || !aligned(cb.index, 16)))
+        return fail(NSNQ_ERR_INVALID_ARG,
+                    "cb.index is NULL or misaligned: build it with nsnq_codebook_index_build");
 
     nsnq::EncodeArgs a{};
     a.x = x;
@@ -125,6 +154,7 @@ nsnq_status nsnq_encode(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t
     a.given_shift = mode == NSNQ_SHIFT_GIVEN;
     a.C = cb.centroids;
     a.sub = cb.sub_dim;
+    a.index = cb.index;
     a.codes = cache.codes; a.scales = cache.scales; a.shift = cache.shift; a.cap = cache.cap;
     char* ws = static_cast<char*>(workspace);
     a.stats = reinterpret_cast<unsigned long long*>(ws);

@@ -16,22 +16,34 @@
 
 namespace nsnq {
 
-constexpr int kAttnWarps = 8;
+constexpr int kAttnWarps = 12;
 constexpr int kAttnThreads = kAttnWarps * 32;
 
+// Shared-memory map of the split kernel (bytes):
+//   lut   fp32 [256][KJ][GC]        L[c][j][h] = (H q_h)_j . C^K_c
+//   vrep  fp32 [256][VSUB/4][8] x4  V codewords, 8 interleaved copies of each
+//                                   16-byte piece, so the 8 lanes of a
+//                                   quarter-warp read 8 different bank groups
+//   qrot  fp32 [GC][128], gam fp32 [8]
+//   per warp: V codes [32][VJ] bytes, weights [32][GC] (w, w) pairs
+// The K codebook is staged in the per-warp area while the LUT is built.
 template <int GC, int KSUB, int VSUB>
 struct AttnSmem {
     static constexpr int KJ = kD / KSUB, VJ = kD / VSUB;
-    static constexpr size_t lut = (size_t)KJ * kNC * GC;  // floats
-    static constexpr size_t cv = (size_t)kNC * VSUB;
-    static constexpr size_t ck = (size_t)kNC * KSUB;
-    static constexpr size_t qrot = (size_t)GC * kD;
-    static constexpr size_t gam = 8;
-    static constexpr size_t wst = (size_t)kAttnWarps * 32 * GC;
-    static constexpr size_t floats = lut + cv + ck + qrot + gam + wst;
-    static constexpr size_t bytes = floats * 4 + (size_t)kAttnWarps * 32 * VJ;
-    static constexpr size_t merge_floats = (size_t)kAttnWarps * GC * (3 + kD);
-    static_assert(merge_floats <= lut, "merge area must fit in the LUT region");
+    static constexpr size_t lut = (size_t)kNC * KJ * GC * 4;
+    static constexpr size_t vrep = (size_t)kNC * (VSUB / 4) * 8 * 16;
+    static constexpr size_t qrot = (size_t)GC * kD * 4 + 32;
+    static constexpr size_t wcodes = (size_t)32 * VJ;
+    static constexpr size_t wweights = (size_t)32 * GC * 8;
+    static constexpr size_t per_warp = wcodes + wweights;
+    static constexpr size_t o_vrep = lut;
+    static constexpr size_t o_qrot = o_vrep + vrep;
+    static constexpr size_t o_warp = o_qrot + qrot;
+    static constexpr size_t bytes = o_warp + per_warp * kAttnWarps;
+    static constexpr size_t merge = (size_t)kAttnWarps * GC * (3 + kD) * 4;
+    static_assert(merge <= lut, "merge area must fit in the LUT region");
+    static_assert((size_t)kNC * KSUB * 4 <= per_warp * kAttnWarps, "K codebook staging");
+    static_assert(bytes <= 232448, "shared memory per block");
 };
 
 template <typename QT>
@@ -39,18 +51,43 @@ __device__ __forceinline__ void load_q4(const void* q, int64_t off, float (&v)[4
     load4(reinterpret_cast<const QT*>(q) + off, v);
 }
 
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ float2 upk2(uint64_t u) {
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(u));
+    return r;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
 template <int GC, int KSUB, int VSUB, typename QT>
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a) {
     using S = AttnSmem<GC, KSUB, VSUB>;
     constexpr int KJ = S::KJ, VJ = S::VJ;
-    extern __shared__ __align__(16) float sm[];
-    float* lut = sm;
-    float* Cv = lut + S::lut;
-    float* Ck = Cv + S::cv;
-    float* qrot = Ck + S::ck;
-    float* gam = qrot + S::qrot;
-    float* wst = gam + S::gam;
-    uint8_t* cst = reinterpret_cast<uint8_t*>(wst + S::wst);
+    constexpr int KW = KJ / 4;  // 32-bit words per K code row
+    extern __shared__ __align__(16) uint8_t smb[];
+    float* lut = reinterpret_cast<float*>(smb);
+    float4* vrep = reinterpret_cast<float4*>(smb + S::o_vrep);
+    float* qrot = reinterpret_cast<float*>(smb + S::o_qrot);
+    float* gam = qrot + GC * kD;
+    uint8_t* warp_area = smb + S::o_warp;
+    float* Ck = reinterpret_cast<float*>(warp_area);  // staged K codebook (prologue only)
 
     const int split = blockIdx.x, grp = blockIdx.y, b = blockIdx.z;
     const int G = a.Hq / a.Hkv;
@@ -73,8 +110,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a)
         return;
     }
 
+    // ---- prologue: K codebook, fp16 V table, rotated queries, LUT ----
     for (int i = tid; i < kNC * KSUB; i += kAttnThreads) Ck[i] = a.kC[i];
-    for (int i = tid; i < kNC * VSUB; i += kAttnThreads) Cv[i] = a.vC[i];
+    for (int i = tid; i < kNC * (VSUB / 4) * 8; i += kAttnThreads)  // [piece][copy]
+        vrep[i] = reinterpret_cast<const float4*>(a.vC)[i >> 3];
     if (warp < GC) {
         float qv[4];
         load_q4<QT>(a.q, ((int64_t)b * a.Hq + qh0 + warp) * kD + 4 * lane, qv);
@@ -86,18 +125,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a)
         if (lane == 0) gam[warp] = g;
     }
     __syncthreads();
-    // L[j][c][h] = (Hq_h)[j*KSUB : (j+1)*KSUB] . C_c
-    for (int e = tid; e < KJ * kNC; e += kAttnThreads) {
-        const int j = e >> 8, c = e & (kNC - 1);
+    for (int e = tid; e < kNC * KJ; e += kAttnThreads) {
+        const int c = e / KJ, j = e % KJ;
         float ck[KSUB];
 #pragma unroll
         for (int r = 0; r < KSUB; ++r) ck[r] = Ck[c * KSUB + r];
 #pragma unroll
         for (int h = 0; h < GC; ++h) {
-            float s = 0.f;
+            float sum = 0.f;
 #pragma unroll
-            for (int r = 0; r < KSUB; ++r) s = fmaf(qrot[h * kD + j * KSUB + r], ck[r], s);
-            lut[(size_t)e * GC + h] = s;
+            for (int r = 0; r < KSUB; ++r) sum = fmaf(qrot[h * kD + j * KSUB + r], ck[r], sum);
+            lut[(size_t)e * GC + h] = sum;
         }
     }
     __syncthreads();
@@ -105,59 +143,77 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a)
     float gm[GC];
 #pragma unroll
     for (int h = 0; h < GC; ++h) gm[h] = gam[h];
-    float m[GC], l[GC], be[GC], A[GC][VSUB];
+    float m[GC], l[GC], be[GC];
+    uint64_t acc[GC][VSUB / 2];
 #pragma unroll
     for (int h = 0; h < GC; ++h) {
         m[h] = -INFINITY; l[h] = 0.f; be[h] = 0.f;
 #pragma unroll
-        for (int r = 0; r < VSUB; ++r) A[h][r] = 0.f;
+        for (int r = 0; r < VSUB / 2; ++r) acc[h][r] = 0ull;
     }
     const uint8_t* kc = a.kcodes + bkv * a.kcap * KJ;
     const uint8_t* vc = a.vcodes + bkv * a.vcap * VJ;
     const float2* ks = reinterpret_cast<const float2*>(a.kscales) + bkv * a.kcap;
     const float2* vs = reinterpret_cast<const float2*>(a.vscales) + bkv * a.vcap;
-    uint8_t* my_codes = cst + (size_t)warp * 32 * VJ;
-    float* my_w = wst + (size_t)warp * 32 * GC;
-    constexpr int TPI = 32 / VJ;  // tokens per V iteration (1 at VSUB=4, 2 at VSUB=8)
+    uint8_t* my_codes = warp_area + (size_t)warp * S::per_warp;
+    uint64_t* my_w = reinterpret_cast<uint64_t*>(my_codes + S::wcodes);  // [32][GC] (w, w)
+    constexpr int TPI = 32 / VJ;  // tokens per V step (1 at VSUB=4, 2 at VSUB=8)
     const int jj = lane % VJ, sub_t = lane / VJ;
+    const int t7 = lane & 7;
 
     for (int64_t base = ts + warp * 32; base < te; base += kAttnWarps * 32) {
         const int64_t t = base + lane;
         const bool valid = t < te;
-        float sc[GC];
-#pragma unroll
-        for (int h = 0; h < GC; ++h) sc[h] = 0.f;
+        // ---- scores: lane = token; sub-vector order s ^ (lane & 7) keeps the
+        //      eight lanes of a quarter-warp on eight different bank groups
+        uint32_t kw[KW];
         float2 k2 = make_float2(0.f, 0.f), v2 = make_float2(0.f, 0.f);
         if (valid) {
             const uint4* kr = reinterpret_cast<const uint4*>(kc + t * KJ);
 #pragma unroll
-            for (int q4 = 0; q4 < KJ / 16; ++q4) {
-                const uint4 w4 = kr[q4];
-                const uint32_t wd[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-                for (int wi = 0; wi < 4; ++wi) {
-#pragma unroll
-                    for (int by = 0; by < 4; ++by) {
-                        const int j = q4 * 16 + wi * 4 + by;
-                        const int code = (wd[wi] >> (8 * by)) & 0xff;
-                        const float* e = lut + ((size_t)(j << 8) + code) * GC;
-                        if constexpr (GC == 4) {
-                            const float4 ev = *reinterpret_cast<const float4*>(e);
-                            sc[0] += ev.x; sc[1] += ev.y; sc[2] += ev.z; sc[3] += ev.w;
-                        } else {
-#pragma unroll
-                            for (int h = 0; h < GC; ++h) sc[h] += e[h];
-                        }
-                    }
-                }
+            for (int q4 = 0; q4 < KW / 4; ++q4) {
+                const uint4 w4 = __ldg(kr + q4);
+                kw[4 * q4] = w4.x; kw[4 * q4 + 1] = w4.y; kw[4 * q4 + 2] = w4.z; kw[4 * q4 + 3] = w4.w;
             }
-            k2 = ks[t];
-            v2 = vs[t];
+            k2 = __ldg(ks + t);
+            v2 = __ldg(vs + t);
             const uint4* vr = reinterpret_cast<const uint4*>(vc + t * VJ);
             uint4* dst = reinterpret_cast<uint4*>(my_codes + lane * VJ);
 #pragma unroll
-            for (int q4 = 0; q4 < VJ / 16; ++q4) dst[q4] = vr[q4];
+            for (int q4 = 0; q4 < VJ / 16; ++q4) dst[q4] = __ldg(vr + q4);
+        } else {
+#pragma unroll
+            for (int i = 0; i < KW; ++i) kw[i] = 0u;
         }
+        float sc[GC];
+        if constexpr (GC == 4) {
+            uint64_t s01 = 0ull, s23 = 0ull;
+            const float4* lut4 = reinterpret_cast<const float4*>(lut);
+#pragma unroll
+            for (int s = 0; s < KJ; ++s) {
+                const int j = s ^ t7;
+                const uint32_t word = (t7 & 4) ? kw[(s >> 2) ^ 1] : kw[s >> 2];
+                const uint32_t code = __byte_perm(word, 0u, 0x4440u | (uint32_t)((s ^ t7) & 3));
+                const float4 e = lut4[code * KJ + j];
+                s01 = fadd2(s01, pk2(e.x, e.y));
+                s23 = fadd2(s23, pk2(e.z, e.w));
+            }
+            const float2 a01 = upk2(s01), a23 = upk2(s23);
+            sc[0] = a01.x; sc[1] = a01.y; sc[2] = a23.x; sc[3] = a23.y;
+        } else {
+#pragma unroll
+            for (int h = 0; h < GC; ++h) sc[h] = 0.f;
+#pragma unroll
+            for (int s = 0; s < KJ; ++s) {
+                const int j = s ^ t7;
+                const uint32_t word = (t7 & 4) ? kw[(s >> 2) ^ 1] : kw[s >> 2];
+                const uint32_t code = __byte_perm(word, 0u, 0x4440u | (uint32_t)((s ^ t7) & 3));
+                const float* e = lut + ((size_t)code * KJ + j) * GC;
+#pragma unroll
+                for (int h = 0; h < GC; ++h) sc[h] += e[h];
+            }
+        }
+        // ---- online softmax (log2 domain) ----
 #pragma unroll
         for (int h = 0; h < GC; ++h) {
             const float logit = valid ? k2.x * fmaf(k2.y, sc[h], gm[h]) * a.scale_log2 : -INFINITY;
@@ -167,26 +223,34 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a)
             const float p = valid ? exp2f(logit - mn) : 0.f;
             l[h] = fmaf(l[h], alpha, p);
             be[h] = fmaf(be[h], alpha, p * v2.x);
+            const uint64_t al = pk2(alpha, alpha);
 #pragma unroll
-            for (int r = 0; r < VSUB; ++r) A[h][r] *= alpha;
-            my_w[lane * GC + h] = p * v2.x * v2.y;
+            for (int r = 0; r < VSUB / 2; ++r) acc[h][r] = fmul2(acc[h][r], al);
+            const float wv = p * v2.x * v2.y;
+            my_w[lane * GC + h] = pk2(wv, wv);
             m[h] = mn;
         }
         __syncwarp();
+        // ---- values: lane = sub-vector, fp32 codewords and accumulation ----
         const int nt = (int)min((int64_t)32, te - base);
+        const float4* myrep = vrep + (lane & 7);
         for (int i = 0; i < nt; i += TPI) {
             const int tt = i + sub_t;
             if (tt < nt) {
                 const int code = my_codes[tt * VJ + jj];
-                float wv[GC];
+                float c[VSUB];
 #pragma unroll
-                for (int h = 0; h < GC; ++h) wv[h] = my_w[tt * GC + h];
-                const float* cp = Cv + code * VSUB;
+                for (int k = 0; k < VSUB / 4; ++k) {
+                    const float4 cv = myrep[(code * (VSUB / 4) + k) * 8];
+                    c[4 * k] = cv.x; c[4 * k + 1] = cv.y; c[4 * k + 2] = cv.z; c[4 * k + 3] = cv.w;
+                }
+                const uint64_t* wv = my_w + tt * GC;
 #pragma unroll
-                for (int r = 0; r < VSUB; ++r) {
-                    const float c = cp[r];
+                for (int h = 0; h < GC; ++h) {
+                    const uint64_t wp = wv[h];
 #pragma unroll
-                    for (int h = 0; h < GC; ++h) A[h][r] = fmaf(wv[h], c, A[h][r]);
+                    for (int r = 0; r < VSUB / 2; ++r)
+                        acc[h][r] = ffma2(pk2(c[2 * r], c[2 * r + 1]), wp, acc[h][r]);
                 }
             }
         }
@@ -199,11 +263,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a)
         be[h] = warp_sum(be[h]);
         if constexpr (TPI == 2) {
 #pragma unroll
-            for (int r = 0; r < VSUB; ++r) A[h][r] += __shfl_xor_sync(kFull, A[h][r], 16);
+            for (int r = 0; r < VSUB / 2; ++r) {
+                const float2 v = upk2(acc[h][r]);
+                acc[h][r] = pk2(v.x + __shfl_xor_sync(kFull, v.x, 16), v.y + __shfl_xor_sync(kFull, v.y, 16));
+            }
         }
     }
     __syncthreads();  // LUT no longer needed: reuse it for the CTA merge
-    float* mw = sm;
+    float* mw = lut;
     float* lw = mw + kAttnWarps * GC;
     float* bw = lw + kAttnWarps * GC;
     float* Aw = bw + kAttnWarps * GC;  // [warp][h][128]
@@ -217,7 +284,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a)
 #pragma unroll
         for (int h = 0; h < GC; ++h)
 #pragma unroll
-            for (int r = 0; r < VSUB; ++r) Aw[(warp * GC + h) * kD + jj * VSUB + r] = A[h][r];
+            for (int r = 0; r < VSUB / 2; ++r) {
+                const float2 v = upk2(acc[h][r]);
+                Aw[(warp * GC + h) * kD + jj * VSUB + 2 * r] = v.x;
+                Aw[(warp * GC + h) * kD + jj * VSUB + 2 * r + 1] = v.y;
+            }
     }
     __syncthreads();
     for (int idx = tid; idx < GC * (kD + 2); idx += kAttnThreads) {
@@ -225,7 +296,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a)
         float M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, mw[w * GC + h]);
-        float acc = 0.f;
+        float accm = 0.f;
 #pragma unroll
         for (int w = 0; w < kAttnWarps; ++w) {
             const float mv = mw[w * GC + h];
@@ -234,12 +305,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a)
             if (c < kD) v = Aw[(w * GC + h) * kD + c];
             else if (c == kD) v = lw[w * GC + h];
             else v = bw[w * GC + h];
-            acc = fmaf(f, v, acc);
+            accm = fmaf(f, v, accm);
         }
         float* P = a.part + (((int64_t)b * a.Hq + qh0 + h) * nsplit + split) * kPartStride;
-        if (c < kD) P[c] = acc;
-        else if (c == kD) { P[kD] = M; P[kD + 1] = acc; }
-        else P[kD + 2] = acc;  // c == kD + 1: beta
+        if (c < kD) P[c] = accm;
+        else if (c == kD) { P[kD] = M; P[kD + 1] = accm; }
+        else P[kD + 2] = accm;  // c == kD + 1: beta
     }
 }
 

@@ -338,11 +338,13 @@ static cudaError_t launch_encode_t(const EncodeArgs& a, cudaStream_t s) {
         nsn_stats_kernel<XT><<<dim3(a.nchunk1, a.H, a.B), kStatsThreads, 0, s>>>(a);
         nsn_shift_kernel<<<a.B * a.H, kD, 0, s>>>(a);
     }
+    if (a.sub == 4) {
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        return launch_encode_pruned(a, s);
+    }
     const dim3 grid((unsigned)((a.T + kEncodeChunk - 1) / kEncodeChunk), a.H, a.B);
-    if (a.sub == 4)
-        nsn_encode_kernel<XT, 4><<<grid, kEncodeThreads, 0, s>>>(a);
-    else
-        nsn_encode_kernel<XT, 8><<<grid, kEncodeThreads, 0, s>>>(a);
+    nsn_encode_kernel<XT, 8><<<grid, kEncodeThreads, 0, s>>>(a);
     return cudaGetLastError();
 }
 

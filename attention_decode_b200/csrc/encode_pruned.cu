@@ -1,0 +1,428 @@
+// NSNQuant encode for 4-dimensional sub-vectors (2 bits/coordinate) on
+// sm_100a: normalize-shift-normalize, Hadamard transform and the exact
+// nearest codeword found through the grid-cell index of vq_index.cuh
+// (gist.science "NSNQuant ...", Technical Summary, Methodology §1-§3).
+//
+// Persistent CTAs of 512 threads keep the index (cell offsets + candidate
+// lists) and an 8-way replicated copy of the codebook in shared memory.
+// Two threads share a token-head: each holds 64 of its 128 coordinates, runs
+// six FWHT stages in registers (packed f32x2 adds) and one across the pair,
+// then searches its 16 sub-vectors: cell -> candidate list (sorted by a
+// lower bound of the distance) -> distances until the next lower bound
+// exceeds the best distance plus the near-tie band. Near ties and heavily
+// cancelled residuals are re-decided from an fp64 recomputation.
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "vq_index.cuh"
+
+namespace nsnq {
+
+constexpr int kPrunedThreads = 512;
+constexpr int kWarps = kPrunedThreads / 32;
+constexpr int kWarpTile = 16;              // token-heads per warp tile (2 threads each)
+constexpr float kCancel = 1e-3f;           // s2 below this: residual decided in fp64
+
+// shared-memory map (bytes)
+constexpr size_t kSmReps = 0;                                  // float4 [256][8]
+constexpr size_t kSmShift = kSmReps + size_t(kNC) * 8 * 16;   // float [warps][136]
+constexpr size_t kSmHash = kSmShift + size_t(kPrunedThreads / 32) * 136 * 4;
+constexpr size_t kSmOffsets = kSmHash + 16;                    // uint16 [kCells + 1]
+constexpr size_t kSmEntries = kSmOffsets + kIdxSmemOffsetsBytes;
+constexpr size_t kSmBytes = kSmEntries + size_t(kMaxEntries + 1) * 2;
+
+__device__ __forceinline__ uint64_t pk(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ float2 upk(uint64_t u) {
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(u));
+    return r;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t cb_hash_term(uint32_t bits, uint32_t i) {
+    uint32_t h = bits * 0x9E3779B1u ^ (i * 0x85EBCA77u + 0x165667B1u);
+    h ^= h >> 15;
+    h *= 0x2C1B3C6Du;
+    h ^= h >> 13;
+    return h;
+}
+
+template <typename XT>
+__device__ __forceinline__ void load64(const XT* p, float (&v)[64]);
+template <>
+__device__ __forceinline__ void load64<__nv_bfloat16>(const __nv_bfloat16* p, float (&v)[64]) {
+    const uint4* q = reinterpret_cast<const uint4*>(p);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint4 a = __ldg(q + i);
+        const uint32_t u[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            v[8 * i + 2 * k] = __uint_as_float(u[k] << 16);
+            v[8 * i + 2 * k + 1] = __uint_as_float(u[k] & 0xffff0000u);
+        }
+    }
+}
+template <>
+__device__ __forceinline__ void load64<float>(const float* p, float (&v)[64]) {
+    const float4* q = reinterpret_cast<const float4*>(p);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float4 a = __ldg(q + i);
+        v[4 * i] = a.x; v[4 * i + 1] = a.y; v[4 * i + 2] = a.z; v[4 * i + 3] = a.w;
+    }
+}
+
+// Exact decision for the flagged sub-vectors of one token-head, shared by
+// the two threads of a pair (pair_mask): fp64 NSN of the whole token, then
+// w_j = H_j u for each flagged sub-vector and a full fp64 scan of the
+// codebook (lowest index on ties). Returns the fp64 (s1, s2).
+template <typename XT>
+__device__ __noinline__ void exact_path(const XT* xrow, const double* o64, const float* o32,
+                                       const float4* reps, const uint16_t* offs,
+                                       const uint16_t* ents, int half, unsigned pair_mask,
+                                       uint32_t my_mask, uint32_t both_mask, uint32_t (&codes)[4],
+                                       double& s1_out, double& s2_out) {
+    float v[64];
+    load64<XT>(xrow + 64 * half, v);
+    const double sqrt_d = sqrt((double)kD);
+    double ss = 0.0;
+    for (int k = 0; k < 64; ++k) ss = __dadd_rn(ss, __dmul_rn((double)v[k], (double)v[k]));
+    ss = __dadd_rn(ss, __shfl_xor_sync(pair_mask, ss, 1));
+    const double s1 = sqrt(ss) / sqrt_d;
+    double u[64];
+    double ss2 = 0.0, yy = 0.0, oo = 0.0;
+    for (int k = 0; k < 64; ++k) {
+        const double o = o64 ? o64[64 * half + k] : (double)o32[64 * half + k];
+        const double y = s1 > 0.0 ? (double)v[k] / s1 : 0.0;
+        const double z = __dadd_rn(y, -o);
+        u[k] = z;
+        ss2 = __dadd_rn(ss2, __dmul_rn(z, z));
+        yy = __dadd_rn(yy, __dmul_rn(y, y));
+        oo = __dadd_rn(oo, __dmul_rn(o, o));
+    }
+    ss2 = __dadd_rn(ss2, __shfl_xor_sync(pair_mask, ss2, 1));
+    yy = __dadd_rn(yy, __shfl_xor_sync(pair_mask, yy, 1));
+    oo = __dadd_rn(oo, __shfl_xor_sync(pair_mask, oo, 1));
+    // a residual at or below 2^-20 of the token/shift magnitude counts as zero
+    const double s2 = ss2 <= 0x1p-40 * (yy + oo) ? 0.0 : sqrt(ss2) / sqrt_d;
+    for (int k = 0; k < 64; ++k) u[k] = s2 > 0.0 ? u[k] / s2 : 0.0;
+    const double hs = 1.0 / sqrt_d;
+    uint32_t todo = both_mask;
+    while (todo) {
+        const int j = __ffs(todo) - 1;  // global sub-vector index 0..31
+        todo &= todo - 1;
+        double w[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int row = 4 * j + r;
+            double acc = 0.0;
+            for (int k = 0; k < 64; ++k) {
+                const int col = 64 * half + k;
+                const double h = (__popc(row & col) & 1) ? -hs : hs;
+                acc = __dadd_rn(acc, __dmul_rn(h, u[k]));
+            }
+            w[r] = __dadd_rn(acc, __shfl_xor_sync(pair_mask, acc, 1));
+        }
+        if ((my_mask >> j) & 1u) {
+            // The cell list holds every codeword that can be nearest anywhere in
+            // the (expanded) cell, so the exact argmin over it is the global one.
+            int cell = 0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                int bi = __float2int_rd(fmaf((float)w[i], kInvW, kBinBias));
+                bi = min(max(bi, 0), kNb - 1);
+                cell = cell * kNb + bi;
+            }
+            double bd = INFINITY;
+            int bi = 0;
+            for (uint32_t q = offs[cell]; q < offs[cell + 1]; ++q) {
+                const int c = ents[q] & 0xff;
+                const float4 cv = reps[c * 8];
+                double d = 0.0, e;
+                e = w[0] - (double)cv.x; d = __dadd_rn(d, __dmul_rn(e, e));
+                e = w[1] - (double)cv.y; d = __dadd_rn(d, __dmul_rn(e, e));
+                e = w[2] - (double)cv.z; d = __dadd_rn(d, __dmul_rn(e, e));
+                e = w[3] - (double)cv.w; d = __dadd_rn(d, __dmul_rn(e, e));
+                if (d < bd || (d == bd && c < bi)) { bd = d; bi = c; }
+            }
+            const int jj = j - 16 * half;
+            const int sh = 8 * (jj & 3);
+            codes[jj >> 2] = (codes[jj >> 2] & ~(0xffu << sh)) | ((uint32_t)bi << sh);
+        }
+    }
+    s1_out = s1;
+    s2_out = s2;
+}
+
+// Candidate walk of one sub-vector w through its cell's list.
+struct Walk {
+    uint64_t w01, w23;
+    uint32_t p, e;
+    float d1, d2;
+    int i1;
+
+    __device__ __forceinline__ void init(float w0, float w1, float w2, float w3,
+                                         const uint16_t* offs) {
+        int cell = 0;
+        const float wv[4] = {w0, w1, w2, w3};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            int bi = __float2int_rd(fmaf(wv[i], kInvW, kBinBias));
+            bi = min(max(bi, 0), kNb - 1);
+            cell = cell * kNb + bi;
+        }
+        p = offs[cell];
+        e = offs[cell + 1];
+        w01 = pk(w0, w1);
+        w23 = pk(w2, w3);
+        d1 = INFINITY; d2 = INFINITY; i1 = 0;
+    }
+
+    // Evaluate up to two more entries (the second against the band of the
+    // best distance before the first, which costs at most one extra
+    // evaluation and never skips a contender); marks the walk finished
+    // (p = e) once the next lower bound leaves the band or the list ends.
+    __device__ __forceinline__ void step(const uint16_t* ents, const float4* myrep) {
+        if (p >= e) return;
+        const uint32_t ent0 = ents[p];
+        const bool has1 = p + 1 < e;
+        const uint32_t ent1 = has1 ? ents[p + 1] : 0u;
+        // lower bounds are floor(lb * 64) in the high byte: compare in integers
+        const uint32_t lim = (uint32_t)fminf(fmaf(d1, (1.0f + kTieRel) * kLbScale, kTieAbs * kLbScale), 1.0e6f);
+        if ((ent0 >> 8) > lim) { p = e; return; }
+        const bool take1 = has1 && (ent1 >> 8) <= lim;
+        const float4 cv0 = myrep[(ent0 & 0xff) * 8];
+        const float4 cv1 = myrep[(ent1 & 0xff) * 8];
+        const uint64_t a01 = sub2(w01, pk(cv0.x, cv0.y)), a23 = sub2(w23, pk(cv0.z, cv0.w));
+        const uint64_t b01 = sub2(w01, pk(cv1.x, cv1.y)), b23 = sub2(w23, pk(cv1.z, cv1.w));
+        const float2 da = upk(fma2(a23, a23, mul2(a01, a01)));
+        const float2 db = upk(fma2(b23, b23, mul2(b01, b01)));
+        const float dA = da.x + da.y;
+        const float dB = take1 ? db.x + db.y : INFINITY;
+        d2 = fminf(d2, fmaxf(d1, dA));
+        i1 = dA < d1 ? (int)(ent0 & 0xff) : i1;
+        d1 = fminf(d1, dA);
+        d2 = fminf(d2, fmaxf(d1, dB));
+        i1 = dB < d1 ? (int)(ent1 & 0xff) : i1;
+        d1 = fminf(d1, dB);
+        p = take1 ? p + 2 : e;
+    }
+
+    __device__ __forceinline__ bool tie() const { return (d2 - d1) <= fmaf(kTieRel, d1, kTieAbs); }
+};
+
+template <typename XT>
+__global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(EncodeArgs a) {
+    extern __shared__ __align__(16) uint8_t sm[];
+    float4* reps = reinterpret_cast<float4*>(sm + kSmReps);
+    float* shift_s = reinterpret_cast<float*>(sm + kSmShift);
+    const uint16_t* offs = reinterpret_cast<const uint16_t*>(sm + kSmOffsets);
+    const uint16_t* ents = reinterpret_cast<const uint16_t*>(sm + kSmEntries);
+    const int tid = threadIdx.x, lane = lane_id();
+    const int half = lane & 1;
+    const unsigned pair_mask = 3u << (lane & 30);
+
+    // ---- stage the index and the replicated codebook ----
+    const IndexHeader* hdr = reinterpret_cast<const IndexHeader*>(a.index);
+    const uint32_t n_ent = min(hdr->n_entries, (uint32_t)kMaxEntries);
+    unsigned* hash_s = reinterpret_cast<unsigned*>(sm + kSmHash);
+    if (tid == 0) *hash_s = 0u;
+    __syncthreads();
+    {
+        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.index) + kIdxOffsets);
+        uint4* dst = reinterpret_cast<uint4*>(sm + kSmOffsets);
+        const size_t nbytes = kIdxSmemOffsetsBytes + ((size_t)n_ent * 2 + 15) / 16 * 16;
+        for (size_t i = tid; i < nbytes / 16; i += kPrunedThreads) dst[i] = src[i];
+        for (int i = tid; i < kNC * 8; i += kPrunedThreads)
+            reps[i] = reinterpret_cast<const float4*>(a.C)[i >> 3];
+        uint32_t h = 0;
+        for (int i = tid; i < kNC * 4; i += kPrunedThreads) h ^= cb_hash_term(__float_as_uint(a.C[i]), i);
+#pragma unroll
+        for (int m = 16; m; m >>= 1) h ^= __shfl_xor_sync(kFull, h, m);
+        if (lane == 0) atomicXor(hash_s, h);
+    }
+    __syncthreads();
+    if (tid == 0 && blockIdx.x == 0 && a.stats &&
+        (*hash_s != hdr->pad[0] || hdr->magic != kIndexMagic || hdr->overflow))
+        atomicOr(&a.stats[2], 1ull);
+
+    // Each warp owns tiles of 16 consecutive token-heads of one (batch, head)
+    // and keeps its own copy of that head's shift: no CTA barrier in the loop.
+    const int warp = tid >> 5;
+    float* wshift = shift_s + warp * 136;  // [128 + 4 pad + 4]
+    const int64_t tiles_per_bh = (a.T + kWarpTile - 1) / kWarpTile;
+    const int64_t ntiles = (int64_t)a.B * a.H * tiles_per_bh;
+    const float4* shift4 = reinterpret_cast<const float4*>(wshift);
+    int64_t cur_bh = -1;
+    // Warp tiles are handed out by a counter in the workspace (reset by the
+    // host before the launch), so warps that hit slow tiles do not hold back
+    // a static share of the work.
+    for (;;) {
+        unsigned long long tl = 0;
+        if (lane == 0) tl = atomicAdd(&a.stats[3], 1ull);
+        const int64_t tile = (int64_t)__shfl_sync(kFull, tl, 0);
+        if (tile >= ntiles) break;
+        const int64_t bh = tile / tiles_per_bh;
+        const int64_t t = (tile - bh * tiles_per_bh) * kWarpTile + (lane >> 1);
+        const int b = (int)(bh / a.H), h = (int)(bh - (int64_t)b * a.H);
+        if (bh != cur_bh) {  // warp-uniform
+            __syncwarp();
+            const float4 o = reinterpret_cast<const float4*>(a.shift + bh * kD)[lane];
+            reinterpret_cast<float4*>(wshift)[lane + (lane >= 16 ? 1 : 0)] = o;
+            __syncwarp();
+            cur_bh = bh;
+        }
+        const bool valid = t < a.T;
+        const XT* xrow = reinterpret_cast<const XT*>(a.x) + b * a.sb + h * a.sh +
+                         (valid ? t : 0) * a.st;
+        float v[64];
+        if (valid) {
+            load64<XT>(xrow + 64 * half, v);
+        } else {
+#pragma unroll
+            for (int k = 0; k < 64; ++k) v[k] = 0.f;
+        }
+        // ---- normalize, shift, normalize ----
+        uint64_t acc0 = 0, acc1 = 0;
+#pragma unroll
+        for (int k = 0; k < 64; k += 4) {
+            const uint64_t p0 = pk(v[k], v[k + 1]), p1 = pk(v[k + 2], v[k + 3]);
+            acc0 = fma2(p0, p0, acc0);
+            acc1 = fma2(p1, p1, acc1);
+        }
+        float2 s01 = upk(add2(acc0, acc1));
+        float ss = s01.x + s01.y;
+        ss += __shfl_xor_sync(kFull, ss, 1);
+        const float s1 = sqrtf(ss * (1.0f / kD));
+        const float inv1 = s1 > 0.f ? 1.0f / s1 : 0.f;
+        const float4* o4 = shift4 + 17 * half;  // upper half stored 4 floats further
+        acc0 = 0; acc1 = 0;
+        const uint64_t inv2 = pk(inv1, inv1);
+#pragma unroll
+        for (int k = 0; k < 64; k += 4) {
+            const float4 o = o4[k >> 2];
+            const uint64_t z0 = fma2(pk(v[k], v[k + 1]), inv2, pk(-o.x, -o.y));
+            const uint64_t z1 = fma2(pk(v[k + 2], v[k + 3]), inv2, pk(-o.z, -o.w));
+            acc0 = fma2(z0, z0, acc0);
+            acc1 = fma2(z1, z1, acc1);
+            const float2 a0 = upk(z0), a1 = upk(z1);
+            v[k] = a0.x; v[k + 1] = a0.y; v[k + 2] = a1.x; v[k + 3] = a1.y;
+        }
+        s01 = upk(add2(acc0, acc1));
+        float ss2 = s01.x + s01.y;
+        ss2 += __shfl_xor_sync(kFull, ss2, 1);
+        const float s2 = sqrtf(ss2 * (1.0f / kD));
+        const bool cancel = s2 < kCancel;
+        const float sc = s2 > 0.f ? kRsqrtD / s2 : 0.f;
+        // ---- FWHT: bits 0..4 on packed pairs (v[i], v[i+32]), bit 5 in-thread, bit 6 across the pair
+        uint64_t P[32];
+        const uint64_t sc2 = pk(sc, sc);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) P[i] = mul2(pk(v[i], v[i + 32]), sc2);
+#pragma unroll
+        for (int bit = 1; bit < 32; bit <<= 1) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                if (i & bit) continue;
+                const uint64_t x0 = P[i], x1 = P[i | bit];
+                P[i] = add2(x0, x1);
+                P[i | bit] = sub2(x0, x1);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const float2 q = upk(P[i]);
+            v[i] = q.x + q.y;
+            v[i + 32] = q.x - q.y;
+        }
+#pragma unroll
+        for (int k = 0; k < 64; ++k) {
+            const float p = __shfl_xor_sync(kFull, v[k], 1);
+            v[k] = half ? (p - v[k]) : (v[k] + p);
+        }
+        // ---- nearest codeword of the 16 sub-vectors this thread holds ----
+        uint32_t codes[4] = {0u, 0u, 0u, 0u};
+        uint32_t tie = 0;
+        const float4* myrep = reps + (lane & 7);
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) {
+            Walk A;
+            A.init(v[4 * jj], v[4 * jj + 1], v[4 * jj + 2], v[4 * jj + 3], offs);
+            while (A.p < A.e) A.step(ents, myrep);
+            codes[jj >> 2] |= (uint32_t)A.i1 << (8 * (jj & 3));
+            if (cancel || A.tie()) tie |= 1u << jj;
+        }
+        if (!valid) tie = 0;
+        // ---- exact fp64 decision where the fp32 search is not conclusive ----
+        const uint32_t my_mask = tie << (16 * half);
+        const uint32_t both = my_mask | __shfl_xor_sync(kFull, my_mask, 1);
+        float s1o = s1, s2o = s2;
+        if (both) {
+            const double* o64 = a.given_shift ? nullptr : a.o64 + bh * kD;
+            double s1d, s2d;
+            exact_path<XT>(xrow, o64, a.shift + bh * kD, reps, offs, ents, half, pair_mask,
+                           my_mask, both, codes, s1d, s2d);
+            s1o = (float)s1d;
+            s2o = (float)s2d;
+            if (half == 0 && a.stats) {
+                atomicAdd(&a.stats[0], 1ull);
+                atomicAdd(&a.stats[1], (unsigned long long)__popc(both));
+            }
+        }
+        if (valid) {
+            const int64_t row = bh * a.cap + a.t_offset + t;
+            reinterpret_cast<uint4*>(a.codes + row * 32)[half] =
+                make_uint4(codes[0], codes[1], codes[2], codes[3]);
+            if (half == 0) reinterpret_cast<float2*>(a.scales)[row] = make_float2(s1o, s2o);
+        }
+    }
+}
+
+size_t pruned_smem_bytes() { return kSmBytes; }
+
+template <typename XT>
+static cudaError_t launch_pruned_t(const EncodeArgs& a, cudaStream_t s) {
+    auto kern = nsn_encode_pruned_kernel<XT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmBytes);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t ntiles = (int64_t)a.B * a.H * ((a.T + kWarpTile - 1) / kWarpTile);
+    const int64_t ctas = (ntiles + kWarps - 1) / kWarps;
+    const int grid = (int)(ctas < sms ? ctas : sms);
+    kern<<<grid, kPrunedThreads, kSmBytes, s>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_encode_pruned(const EncodeArgs& a, cudaStream_t s) {
+    return a.x_bf16 ? launch_pruned_t<__nv_bfloat16>(a, s) : launch_pruned_t<float>(a, s);
+}
+
+}  // namespace nsnq

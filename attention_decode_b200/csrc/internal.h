@@ -30,6 +30,7 @@ struct EncodeArgs {
     int given_shift;
     const float* C;
     int sub;
+    const void* index;  // search index (sub == 4)
     uint8_t* codes;
     float* scales;
     float* shift;
@@ -50,6 +51,9 @@ struct EncodePlan {
 
 EncodePlan plan_encode(int B, int H, int64_t T);
 cudaError_t launch_encode(const EncodeArgs& a, cudaStream_t s);
+cudaError_t launch_encode_pruned(const EncodeArgs& a, cudaStream_t s);
+size_t index_bytes();
+cudaError_t launch_index_build(const float* C, void* index, cudaStream_t s);
 
 // ----------------------------------------------------------------- dequant --
 struct DequantArgs {

@@ -43,9 +43,16 @@ def encode_case(B, H, T, reps, dev):
     x = _keys(gen, B, H, T, dev)
     cache = nsnq.Cache.empty(B, H, T, 4, device=dev)
     ws = torch.empty(nsnq.nsnq_encode_workspace(B, H, T), dtype=torch.uint8, device=dev)
+    cb.prepare()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     for _ in range(reps):
+        e0.record()
         nsnq.nsnq_encode(x, cb, cache, workspace=ws)
+        e1.record()
     torch.cuda.synchronize()
+    th, sv, mism = nsnq.encode_stats(ws)
+    print(f"last call {e0.elapsed_time(e1):.3f} ms; fp64 path: {th} of {B * H * T} token-heads, "
+          f"{sv} sub-vectors; index mismatch {mism}")
 
 
 def attn_case(B, Hq, Hkv, T, sub, reps, dev):

@@ -67,57 +67,59 @@ def attn_bytes_per_token(ksub: int, vsub: int) -> int:
 
 # ------------------------------------------------------------------ clocks --
 class ClockSampler:
-    """nvidia-smi clock/throttle samples during the timed region."""
+    """Polls nvidia-smi (one query every ~100 ms) for SM clock and throttle
+    reasons while the timed regions run."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, gpu_index: int):
+        import threading
         self.gpu = gpu_index
-        self.proc = None
-        self.path = None
+        self.rows = []
+        self.stop = threading.Event()
+        self.thread = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self.stop.is_set():
+            try:
+                out = subprocess.run(
+                    ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                     "--format=csv,noheader,nounits"], capture_output=True, text=True,
+                    timeout=5).stdout.strip()
+                if out:
+                    self.rows.append([p.strip() for p in out.split(",")])
+            except Exception:
+                return
+            self.stop.wait(0.1)
 
     def __enter__(self):
-        try:
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
-            os.close(fd)
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100", "-f", self.path],
-                stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+        self.thread.start()
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
+        self.stop.set()
+        self.thread.join(timeout=10)
 
     def summary(self):
-        if not self.path or not os.path.exists(self.path):
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
         sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
+        for r in self.rows:
+            if len(r) < 7:
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
+                sm.append(float(r[0]))
+                mx = float(r[1])
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
+            for n, v in zip(self.NAMES, r[3:7]):
                 if v.lower() == "active":
                     reasons.add(n)
-        os.unlink(self.path)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
 
 
 # --------------------------------------------------------------- CUDA arm --
@@ -170,6 +172,8 @@ def run_cuda(args):
         if world > 1:
             dist.barrier()
 
+    clk = ClockSampler(local).__enter__()
+    time.sleep(0.3)
     for _ in range(args.warmup):
         step(k, v, q)
     torch.cuda.synchronize()
@@ -178,7 +182,7 @@ def run_cuda(args):
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    if True:
         for i in range(args.steps):
             flush.zero_()
             e = ev[i]
@@ -249,6 +253,7 @@ def run_cuda(args):
 
     # ---- decode attention alone at the 32k workload ----
     attention = run_attention_bench(args, nsnq, dev, world, barrier, hbm, peak_kind)
+    clk.__exit__(None, None, None)
 
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "KV tokens/s", "n_gpus": world,

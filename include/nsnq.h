@@ -67,6 +67,9 @@ typedef struct {
     const float* centroids;  /* device, [n_centroids][sub_dim] fp32, 16-byte aligned */
     int n_centroids;         /* must be 256 (one byte per code) */
     int sub_dim;             /* 4 (2 bits/coordinate) or 8 (1 bit/coordinate) */
+    const void* index;       /* device search index built from these centroids by
+                                nsnq_codebook_index_build; required by nsnq_encode when
+                                sub_dim == 4, ignored otherwise (may be NULL) */
 } nsnq_codebook;
 
 typedef struct {
@@ -83,10 +86,34 @@ const char* nsnq_status_string(nsnq_status status);
 const char* nsnq_last_error(void);
 
 /*
+ * Bytes of the nearest-codeword search index of a sub_dim = 4 codebook
+ * (0 for sub_dim = 8, which needs none).
+ */
+size_t nsnq_codebook_index_bytes(int sub_dim);
+
+/*
+ * nsnq_codebook_index_build -- one-time preparation of a 2-bit codebook for
+ * nsnq_encode (no counterpart on the pages: it accelerates the exact
+ * nearest-codeword search of Methodology §3). Each coordinate of the
+ * transformed sub-vector is binned on a fixed grid; for every grid cell the
+ * index lists, sorted by a lower bound of their distance over the cell, the
+ * codewords that can be nearest (or within the near-tie band of the
+ * nearest) somewhere in the cell. cb.index is ignored; on success set
+ * cb.index = index for later calls. `index` must hold
+ * nsnq_codebook_index_bytes(4) bytes (16-byte aligned). This call waits for
+ * `stream` to finish (it checks that the lists fit) and returns
+ * NSNQ_ERR_UNSUPPORTED if they do not.
+ */
+nsnq_status nsnq_codebook_index_build(nsnq_codebook cb, void* index, size_t index_bytes,
+                                      nsnq_stream stream);
+
+/*
  * Workspace bytes nsnq_encode needs for this shape (any shift mode). The
  * first 64 bytes hold counters the call resets and fills:
  *   uint64 [0] token-heads re-encoded on the fp64 near-tie path,
- *   uint64 [1] sub-vectors whose code was decided on that path.
+ *   uint64 [1] sub-vectors whose code was decided on that path,
+ *   uint64 [2] nonzero if cb.index was not built from cb.centroids,
+ *   uint64 [3] used internally (work counter).
  */
 size_t nsnq_encode_workspace(int B, int H, int64_t T, int D);
 

@@ -47,8 +47,8 @@ def test_status_strings(lib):
     assert lib.nsnq_status_string(3) == b"NSNQ_ERR_WORKSPACE"
 
 
-def _cb(sub=4, n=256, ptr=FAKE):
-    return nsnq._Codebook(ptr, n, sub)
+def _cb(sub=4, n=256, ptr=FAKE, index=FAKE):
+    return nsnq._Codebook(ptr, n, sub, index)
 
 
 def _cache(cap=100):
@@ -76,12 +76,23 @@ def test_encode_validation(lib):
     assert _encode(lib, T=-1) == nsnq.NSNQ_ERR_INVALID_ARG
     assert _encode(lib, mode=7) == nsnq.NSNQ_ERR_INVALID_ARG
     assert _encode(lib, ws=None) == nsnq.NSNQ_ERR_WORKSPACE
+    assert _encode(lib, cb=_cb(index=None)) == nsnq.NSNQ_ERR_INVALID_ARG     # 2-bit needs its index
+    assert b"nsnq_codebook_index_build" in lib.nsnq_last_error()
+    assert _encode(lib, cb=_cb(sub=8, index=None), T=0) == nsnq.NSNQ_OK
     need = lib.nsnq_encode_workspace(1, 1, 10, 128)
     assert need > 0
     assert _encode(lib, wsb=need - 1) == nsnq.NSNQ_ERR_WORKSPACE
     assert b"workspace" in lib.nsnq_last_error()
     assert _encode(lib, T=0) == nsnq.NSNQ_OK                            # no-op, no launch
     assert lib.nsnq_last_error() == b""
+
+
+def test_index_build_validation(lib):
+    assert lib.nsnq_codebook_index_bytes(4) > 0 and lib.nsnq_codebook_index_bytes(8) == 0
+    need = lib.nsnq_codebook_index_bytes(4)
+    assert lib.nsnq_codebook_index_build(_cb(sub=8), FAKE, need, None) == nsnq.NSNQ_ERR_UNSUPPORTED
+    assert lib.nsnq_codebook_index_build(_cb(), None, need, None) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert lib.nsnq_codebook_index_build(_cb(), FAKE, need - 1, None) == nsnq.NSNQ_ERR_WORKSPACE
 
 
 def test_encode_workspace_grows_with_tokens(lib):

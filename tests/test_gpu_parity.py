@@ -53,7 +53,8 @@ def test_encode_matches_oracle(codebooks, case):
     assert n_bad == 0, (n_mis, n_bad, worst)
     P.check_scales(cache.scales.cpu().numpy(), ora)
     P.check_shift(cache.shift.cpu().numpy(), ora["o"])
-    th, sv = nsnq.encode_stats(ws)
+    th, sv, mismatch = nsnq.encode_stats(ws)
+    assert mismatch == 0
     assert th <= max(4, B * H * T // 50)
 
 
@@ -217,3 +218,54 @@ def test_pipeline_tiny_config(codebooks):
     assert np.array_equal(vc.codes.cpu().numpy(), ov["codes"])
     e, _ = P.attn_errors(P.out_to_np(out), ref, False)
     assert (e <= 1.0).all(), e.max()
+
+
+def _parse_index(idx: np.ndarray):
+    hdr = idx[:64].view(np.uint32)
+    n_cells = int(hdr[3])
+    offs = idx[64:64 + 2 * (n_cells + 1)].view(np.uint16).astype(np.int64)
+    start = 64 + ((2 * (n_cells + 1) + 15) // 16) * 16
+    ents = idx[start:start + 2 * int(hdr[1])].view(np.uint16)
+    return hdr, offs, ents
+
+
+def test_codebook_index_lists_contain_the_nearest(codebooks):
+    """Grid-cell candidate lists of the 2-bit search index: for sampled points
+    (standard normal, and heavy-tailed) the true nearest codeword (brute
+    force) is in the point's cell list, and each list is sorted by a valid
+    lower bound of the distance over the cell."""
+    C = codebooks[4]
+    cb = P.codebook(C).prepare()
+    idx = cb.index.cpu().numpy()
+    hdr, offs, ents = _parse_index(idx)
+    assert hdr[0] == 0x4E534E51 and hdr[2] == 0 and hdr[1] < 65536
+    nb, R, W = 10, 2.4, 0.6
+    assert hdr[3] == nb ** 4
+    rng = np.random.default_rng(5)
+    pts = np.concatenate([rng.standard_normal((20000, 4)), 3 * rng.standard_t(3, (5000, 4))])
+    pts = np.clip(pts, -11.3, 11.3)
+    b = np.clip(np.floor(pts.astype(np.float32) * np.float32(1 / 0.6) + np.float32(R / W + 1)),
+                0, nb - 1).astype(np.int64)
+    cell = ((b[:, 0] * nb + b[:, 1]) * nb + b[:, 2]) * nb + b[:, 3]
+    d2 = ((pts[:, None, :] - C[None].astype(np.float64)) ** 2).sum(-1)
+    nearest = d2.argmin(1)
+    for i in range(len(pts)):
+        lst = ents[offs[cell[i]]:offs[cell[i] + 1]]
+        codes, lbq = lst & 0xFF, lst >> 8
+        assert nearest[i] in codes, i
+        assert (np.diff(lbq.astype(np.int64)) >= 0).all()
+        assert (lbq / 64.0 <= d2[i, codes] + 1e-9).all()
+
+
+def test_encode_detects_index_of_another_codebook(codebooks):
+    C = codebooks[4]
+    other = P.codebook((C * np.float32(1.01)).astype(np.float32)).prepare()
+    good = P.codebook(C)
+    w = _workload(1, 2, 100, "bf16", 4)
+    io, _ = _inputs(w, "K")
+    x = P.to_dev(io, "bf16")
+    cache = nsnq.Cache.empty(1, 2, 100, 4)
+    ws = nsnq.nsnq_encode(x, nsnq.Codebook(good.centroids, other.index), cache)
+    assert nsnq.encode_stats(ws)[2] != 0
+    ws = nsnq.nsnq_encode(x, good, cache)
+    assert nsnq.encode_stats(ws)[2] == 0
