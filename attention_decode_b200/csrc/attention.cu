@@ -25,7 +25,7 @@ constexpr int kAttnThreads = kAttnWarps * 32;
 //                                   16-byte piece, so the 8 lanes of a
 //                                   quarter-warp read 8 different bank groups
 //   qrot  fp32 [GC][128], gam fp32 [8]
-//   per warp: V codes [32][VJ] bytes, weights [32][GC] (w, w) pairs
+//   per warp: V codes [32][VJ] bytes, weights [32][GC padded to 4] fp32
 // The K codebook is staged in the per-warp area while the LUT is built.
 template <int GC, int KSUB, int VSUB>
 struct AttnSmem {
@@ -34,7 +34,7 @@ struct AttnSmem {
     static constexpr size_t vrep = (size_t)kNC * (VSUB / 4) * 8 * 16;
     static constexpr size_t qrot = (size_t)GC * kD * 4 + 32;
     static constexpr size_t wcodes = (size_t)32 * VJ;
-    static constexpr size_t wweights = (size_t)32 * GC * 8;
+    static constexpr size_t wweights = (size_t)32 * ((GC + 3) / 4) * 16;
     static constexpr size_t per_warp = wcodes + wweights;
     static constexpr size_t o_vrep = lut;
     static constexpr size_t o_qrot = o_vrep + vrep;
@@ -156,7 +156,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a)
     const float2* ks = reinterpret_cast<const float2*>(a.kscales) + bkv * a.kcap;
     const float2* vs = reinterpret_cast<const float2*>(a.vscales) + bkv * a.vcap;
     uint8_t* my_codes = warp_area + (size_t)warp * S::per_warp;
-    uint64_t* my_w = reinterpret_cast<uint64_t*>(my_codes + S::wcodes);  // [32][GC] (w, w)
+    constexpr int GP = (GC + 3) / 4 * 4;  // weights per token, padded to a float4
+    float* my_w = reinterpret_cast<float*>(my_codes + S::wcodes);  // [32][GP]
     constexpr int TPI = 32 / VJ;  // tokens per V step (1 at VSUB=4, 2 at VSUB=8)
     const int jj = lane % VJ, sub_t = lane / VJ;
     const int t7 = lane & 7;
@@ -226,8 +227,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a)
             const uint64_t al = pk2(alpha, alpha);
 #pragma unroll
             for (int r = 0; r < VSUB / 2; ++r) acc[h][r] = fmul2(acc[h][r], al);
-            const float wv = p * v2.x * v2.y;
-            my_w[lane * GC + h] = pk2(wv, wv);
+            my_w[lane * GP + h] = p * v2.x * v2.y;
             m[h] = mn;
         }
         __syncwarp();
@@ -244,10 +244,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a)
                     const float4 cv = myrep[(code * (VSUB / 4) + k) * 8];
                     c[4 * k] = cv.x; c[4 * k + 1] = cv.y; c[4 * k + 2] = cv.z; c[4 * k + 3] = cv.w;
                 }
-                const uint64_t* wv = my_w + tt * GC;
+                float wv[GP];
+#pragma unroll
+                for (int q4 = 0; q4 < GP / 4; ++q4) {
+                    const float4 w4 = reinterpret_cast<const float4*>(my_w + tt * GP)[q4];
+                    wv[4 * q4] = w4.x; wv[4 * q4 + 1] = w4.y; wv[4 * q4 + 2] = w4.z; wv[4 * q4 + 3] = w4.w;
+                }
 #pragma unroll
                 for (int h = 0; h < GC; ++h) {
-                    const uint64_t wp = wv[h];
+                    const uint64_t wp = pk2(wv[h], wv[h]);
 #pragma unroll
                     for (int r = 0; r < VSUB / 2; ++r)
                         acc[h][r] = ffma2(pk2(c[2 * r], c[2 * r + 1]), wp, acc[h][r]);

@@ -99,8 +99,10 @@ __device__ __forceinline__ void load64<float>(const float* p, float (&v)[64]) {
 
 // Exact decision for the flagged sub-vectors of one token-head, shared by
 // the two threads of a pair (pair_mask): fp64 NSN of the whole token, then
-// w_j = H_j u for each flagged sub-vector and a full fp64 scan of the
-// codebook (lowest index on ties). Returns the fp64 (s1, s2).
+// w_j = H_j u for each flagged sub-vector and an fp64 scan of its cell list
+// (which holds every codeword that can be nearest there; lowest index on
+// exact ties). Returns the fp64 (s1, s2). Kept in registers (no local
+// arrays) and division-free, since one slow warp holds its SM.
 template <typename XT>
 __device__ __noinline__ void exact_path(const XT* xrow, const double* o64, const float* o32,
                                        const float4* reps, const uint16_t* offs,
@@ -109,28 +111,31 @@ __device__ __noinline__ void exact_path(const XT* xrow, const double* o64, const
                                        double& s1_out, double& s2_out) {
     float v[64];
     load64<XT>(xrow + 64 * half, v);
+    const double* o64h = o64 ? o64 + 64 * half : nullptr;
+    const float* o32h = o32 + 64 * half;
     const double sqrt_d = sqrt((double)kD);
     double ss = 0.0;
-    for (int k = 0; k < 64; ++k) ss = __dadd_rn(ss, __dmul_rn((double)v[k], (double)v[k]));
-    ss = __dadd_rn(ss, __shfl_xor_sync(pair_mask, ss, 1));
+#pragma unroll
+    for (int k = 0; k < 64; ++k) ss = fma((double)v[k], (double)v[k], ss);
+    ss += __shfl_xor_sync(pair_mask, ss, 1);
     const double s1 = sqrt(ss) / sqrt_d;
-    double u[64];
+    const double inv1 = s1 > 0.0 ? 1.0 / s1 : 0.0;
     double ss2 = 0.0, yy = 0.0, oo = 0.0;
+#pragma unroll 8
     for (int k = 0; k < 64; ++k) {
-        const double o = o64 ? o64[64 * half + k] : (double)o32[64 * half + k];
-        const double y = s1 > 0.0 ? (double)v[k] / s1 : 0.0;
-        const double z = __dadd_rn(y, -o);
-        u[k] = z;
-        ss2 = __dadd_rn(ss2, __dmul_rn(z, z));
-        yy = __dadd_rn(yy, __dmul_rn(y, y));
-        oo = __dadd_rn(oo, __dmul_rn(o, o));
+        const double o = o64h ? o64h[k] : (double)o32h[k];
+        const double y = (double)v[k] * inv1;
+        const double z = y - o;
+        ss2 = fma(z, z, ss2);
+        yy = fma(y, y, yy);
+        oo = fma(o, o, oo);
     }
-    ss2 = __dadd_rn(ss2, __shfl_xor_sync(pair_mask, ss2, 1));
-    yy = __dadd_rn(yy, __shfl_xor_sync(pair_mask, yy, 1));
-    oo = __dadd_rn(oo, __shfl_xor_sync(pair_mask, oo, 1));
+    ss2 += __shfl_xor_sync(pair_mask, ss2, 1);
+    yy += __shfl_xor_sync(pair_mask, yy, 1);
+    oo += __shfl_xor_sync(pair_mask, oo, 1);
     // a residual at or below 2^-20 of the token/shift magnitude counts as zero
     const double s2 = ss2 <= 0x1p-40 * (yy + oo) ? 0.0 : sqrt(ss2) / sqrt_d;
-    for (int k = 0; k < 64; ++k) u[k] = s2 > 0.0 ? u[k] / s2 : 0.0;
+    const double inv2 = s2 > 0.0 ? 1.0 / s2 : 0.0;
     const double hs = 1.0 / sqrt_d;
     uint32_t todo = both_mask;
     while (todo) {
@@ -141,16 +146,15 @@ __device__ __noinline__ void exact_path(const XT* xrow, const double* o64, const
         for (int r = 0; r < 4; ++r) {
             const int row = 4 * j + r;
             double acc = 0.0;
+#pragma unroll 8
             for (int k = 0; k < 64; ++k) {
-                const int col = 64 * half + k;
-                const double h = (__popc(row & col) & 1) ? -hs : hs;
-                acc = __dadd_rn(acc, __dmul_rn(h, u[k]));
+                const double o = o64h ? o64h[k] : (double)o32h[k];
+                const double u = ((double)v[k] * inv1 - o) * inv2;
+                acc += (__popc(row & (64 * half + k)) & 1) ? -u : u;
             }
-            w[r] = __dadd_rn(acc, __shfl_xor_sync(pair_mask, acc, 1));
+            w[r] = (acc + __shfl_xor_sync(pair_mask, acc, 1)) * hs;
         }
         if ((my_mask >> j) & 1u) {
-            // The cell list holds every codeword that can be nearest anywhere in
-            // the (expanded) cell, so the exact argmin over it is the global one.
             int cell = 0;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -163,11 +167,9 @@ __device__ __noinline__ void exact_path(const XT* xrow, const double* o64, const
             for (uint32_t q = offs[cell]; q < offs[cell + 1]; ++q) {
                 const int c = ents[q] & 0xff;
                 const float4 cv = reps[c * 8];
-                double d = 0.0, e;
-                e = w[0] - (double)cv.x; d = __dadd_rn(d, __dmul_rn(e, e));
-                e = w[1] - (double)cv.y; d = __dadd_rn(d, __dmul_rn(e, e));
-                e = w[2] - (double)cv.z; d = __dadd_rn(d, __dmul_rn(e, e));
-                e = w[3] - (double)cv.w; d = __dadd_rn(d, __dmul_rn(e, e));
+                const double e0 = w[0] - (double)cv.x, e1 = w[1] - (double)cv.y;
+                const double e2 = w[2] - (double)cv.z, e3 = w[3] - (double)cv.w;
+                const double d = e0 * e0 + e1 * e1 + e2 * e2 + e3 * e3;
                 if (d < bd || (d == bd && c < bi)) { bd = d; bi = c; }
             }
             const int jj = j - 16 * half;
