@@ -26,7 +26,6 @@ constexpr int kAttnThreads = kAttnWarps * 32;
 //                                   quarter-warp read 8 different bank groups
 //   qrot  fp32 [GC][128], gam fp32 [8]
 //   per warp: V codes [32][VJ] bytes, weights [32][GC padded to 4] fp32
-// The K codebook is staged in the per-warp area while the LUT is built.
 template <int GC, int KSUB, int VSUB>
 struct AttnSmem {
     static constexpr int KJ = kD / KSUB, VJ = kD / VSUB;
@@ -42,7 +41,6 @@ struct AttnSmem {
     static constexpr size_t bytes = o_warp + per_warp * kAttnWarps;
     static constexpr size_t merge = (size_t)kAttnWarps * GC * (3 + kD) * 4;
     static_assert(merge <= lut, "merge area must fit in the LUT region");
-    static_assert((size_t)kNC * KSUB * 4 <= per_warp * kAttnWarps, "K codebook staging");
     static_assert(bytes <= 232448, "shared memory per block");
 };
 
@@ -76,6 +74,22 @@ __device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
     asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
     return d;
 }
+// Balanced split of the flattened (unit, token) space over the CTAs: CTA c
+// covers virtual tokens [cta_begin(c), cta_begin(c + 1)).
+__host__ __device__ inline int64_t cta_begin(int c, const AttnPlan& p) {
+    const int64_t W = p.units * p.L;
+    return (W / p.ctas) * c + ((W % p.ctas) * c) / p.ctas;
+}
+// The CTA whose range holds virtual token v.
+__host__ __device__ inline int first_cta(int64_t v, const AttnPlan& p) {
+    const int64_t W = p.units * p.L;
+    int c = (int)((double)v * (double)p.ctas / (double)(W > 0 ? W : 1));
+    c = c < 0 ? 0 : (c >= p.ctas ? p.ctas - 1 : c);
+    while (c + 1 < p.ctas && cta_begin(c + 1, p) <= v) ++c;
+    while (c > 0 && cta_begin(c, p) > v) --c;
+    return c;
+}
+
 template <int GC, int KSUB, int VSUB, typename QT>
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a) {
     using S = AttnSmem<GC, KSUB, VSUB>;
@@ -87,33 +101,42 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a)
     float* qrot = reinterpret_cast<float*>(smb + S::o_qrot);
     float* gam = qrot + GC * kD;
     uint8_t* warp_area = smb + S::o_warp;
-    float* Ck = reinterpret_cast<float*>(warp_area);  // staged K codebook (prologue only)
 
-    const int split = blockIdx.x, grp = blockIdx.y, b = blockIdx.z;
-    const int G = a.Hq / a.Hkv;
-    const int kvh = grp / a.plan.ngroups, hg = grp % a.plan.ngroups;
-    const int qh0 = kvh * G + hg * GC;
-    const int64_t bkv = (int64_t)b * a.Hkv + kvh;
-    const int nsplit = a.plan.nsplit;
-    int64_t len = a.seq_lens[b];
-    len = len < 0 ? 0 : (len > a.max_len ? a.max_len : len);
-    const int64_t ts = (int64_t)split * a.plan.split_len;
-    const int64_t te = min(ts + a.plan.split_len, len);
     const int tid = threadIdx.x, lane = lane_id(), warp = tid >> 5;
+    const int G = a.Hq / a.Hkv;
+    const int cta = blockIdx.x;
+    const int64_t L = a.plan.L;
+    const int nslot = a.plan.nslot;
+    // This CTA's share of the flattened (unit, token) space; a unit is one
+    // (batch, kv-head, head group) and spans L virtual tokens.
+    const int64_t vbeg = cta_begin(cta, a.plan), vend = cta_begin(cta + 1, a.plan);
 
-    if (ts >= te) {  // empty split: neutral partial
-        for (int idx = tid; idx < GC * kPartStride; idx += kAttnThreads) {
-            const int h = idx / kPartStride, c = idx % kPartStride;
-            float* P = a.part + (((int64_t)b * a.Hq + qh0 + h) * nsplit + split) * kPartStride;
-            P[c] = (c == kD) ? -INFINITY : 0.f;
-        }
-        return;
-    }
-
-    // ---- prologue: K codebook, fp16 V table, rotated queries, LUT ----
-    for (int i = tid; i < kNC * KSUB; i += kAttnThreads) Ck[i] = a.kC[i];
     for (int i = tid; i < kNC * (VSUB / 4) * 8; i += kAttnThreads)  // [piece][copy]
         vrep[i] = reinterpret_cast<const float4*>(a.vC)[i >> 3];
+
+  for (int64_t u = vbeg / L; u < a.plan.units && u * L < vend; ++u) {
+    const int64_t per_b = (int64_t)a.Hkv * a.plan.ngroups;
+    const int b = (int)(u / per_b);
+    const int kvh = (int)((u % per_b) / a.plan.ngroups), hg = (int)(u % a.plan.ngroups);
+    const int qh0 = kvh * G + hg * GC;
+    const int64_t bkv = (int64_t)b * a.Hkv + kvh;
+    const int slot = cta - first_cta(u * L, a.plan);
+    int64_t len = a.seq_lens[b];
+    len = len < 0 ? 0 : (len > a.max_len ? a.max_len : len);
+    const int64_t ts = max(vbeg, u * L) - u * L;
+    const int64_t te = min(min(vend, (u + 1) * L) - u * L, len);
+    __syncthreads();  // the previous segment is done with the LUT, qrot and merge area
+
+    if (ts >= te) {  // nothing to attend in this segment: neutral partial
+        for (int idx = tid; idx < GC * kPartStride; idx += kAttnThreads) {
+            const int h = idx / kPartStride, c = idx % kPartStride;
+            float* P = a.part + (((int64_t)b * a.Hq + qh0 + h) * nslot + slot) * kPartStride;
+            P[c] = (c == kD) ? -INFINITY : 0.f;
+        }
+        continue;
+    }
+
+    // ---- segment prologue: rotated queries, q . o_K, LUT ----
     if (warp < GC) {
         float qv[4];
         load_q4<QT>(a.q, ((int64_t)b * a.Hq + qh0 + warp) * kD + 4 * lane, qv);
@@ -129,7 +152,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a)
         const int c = e / KJ, j = e % KJ;
         float ck[KSUB];
 #pragma unroll
-        for (int r = 0; r < KSUB; ++r) ck[r] = Ck[c * KSUB + r];
+        for (int r = 0; r < KSUB; ++r) ck[r] = __ldg(a.kC + c * KSUB + r);
 #pragma unroll
         for (int h = 0; h < GC; ++h) {
             float sum = 0.f;
@@ -312,11 +335,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a)
             else v = bw[w * GC + h];
             accm = fmaf(f, v, accm);
         }
-        float* P = a.part + (((int64_t)b * a.Hq + qh0 + h) * nsplit + split) * kPartStride;
+        float* P = a.part + (((int64_t)b * a.Hq + qh0 + h) * nslot + slot) * kPartStride;
         if (c < kD) P[c] = accm;
         else if (c == kD) { P[kD] = M; P[kD + 1] = accm; }
         else P[kD + 2] = accm;  // c == kD + 1: beta
     }
+  }
 }
 
 // Merge the splits of one (batch, query head): rescale by exp2(m_s - M),
@@ -326,15 +350,20 @@ __global__ void __launch_bounds__(kD) attn_combine_kernel(AttnArgs a) {
     __shared__ float LB[2];
     const int bq = blockIdx.x;
     const int b = bq / a.Hq, qh = bq % a.Hq;
-    const int kvh = qh / (a.Hq / a.Hkv);
-    const int nsplit = a.plan.nsplit;
-    const float* P = a.part + (int64_t)bq * nsplit * kPartStride;
+    const int G = a.Hq / a.Hkv;
+    const int kvh = qh / G, hg = (qh % G) / a.plan.gc;
+    const int64_t u = ((int64_t)b * a.Hkv + kvh) * a.plan.ngroups + hg;
+    const int nslot = a.plan.nslot;
+    const int used = a.plan.L > 0
+                         ? first_cta(u * a.plan.L + a.plan.L - 1, a.plan) - first_cta(u * a.plan.L, a.plan) + 1
+                         : 0;
+    const float* P = a.part + (int64_t)bq * nslot * kPartStride;
     const int c = threadIdx.x;
     float M = -INFINITY;
-    for (int s = 0; s < nsplit; ++s) M = fmaxf(M, P[(int64_t)s * kPartStride + kD]);
+    for (int s = 0; s < used; ++s) M = fmaxf(M, P[(int64_t)s * kPartStride + kD]);
     float acc = 0.f, L = 0.f, Be = 0.f;
     if (M != -INFINITY) {
-        for (int s = 0; s < nsplit; ++s) {
+        for (int s = 0; s < used; ++s) {
             const float* Ps = P + (int64_t)s * kPartStride;
             const float ms = Ps[kD];
             const float f = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
@@ -387,17 +416,11 @@ AttnPlan plan_attention(int B, int Hq, int Hkv, int64_t max_len) {
     const int G = Hq / Hkv;
     p.gc = (G % 4 == 0) ? 4 : (G % 2 == 0 ? 2 : 1);
     p.ngroups = G / p.gc;
-    const int64_t units = (int64_t)B * Hkv * p.ngroups;
-    const int64_t target = 4LL * device_sms();
-    int64_t want = (target + units - 1) / units;
-    if (want < 1) want = 1;
-    const int64_t L = max_len > 0 ? max_len : 1;
-    int64_t sl = (L + want - 1) / want;
-    sl = (sl + 255) / 256 * 256;
-    if (sl < 256) sl = 256;
-    p.split_len = sl;
-    p.nsplit = (int)((L + sl - 1) / sl);
-    p.total = align_up((size_t)B * Hq * p.nsplit * kPartStride * sizeof(float), kWsAlign);
+    p.units = (int64_t)B * Hkv * p.ngroups;
+    p.L = max_len;
+    p.ctas = device_sms();  // one CTA per SM (the tables fill shared memory)
+    p.nslot = (int)((p.ctas + p.units - 1) / (p.units > 0 ? p.units : 1)) + 1;
+    p.total = align_up((size_t)B * Hq * p.nslot * kPartStride * sizeof(float), kWsAlign);
     return p;
 }
 
@@ -408,8 +431,7 @@ static cudaError_t launch_split(const AttnArgs& a, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)S::bytes);
     if (e != cudaSuccess) return e;
-    const dim3 grid(a.plan.nsplit, a.Hkv * a.plan.ngroups, a.B);
-    kern<<<grid, kAttnThreads, S::bytes, s>>>(a);
+    kern<<<a.plan.ctas, kAttnThreads, S::bytes, s>>>(a);
     return cudaGetLastError();
 }
 

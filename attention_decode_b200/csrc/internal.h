@@ -75,8 +75,10 @@ constexpr int kPartStride = 132;  // 128 rotated-domain values + (m, l, beta, pa
 struct AttnPlan {
     int gc;          // query heads per CTA
     int ngroups;     // head groups per kv-head
-    int64_t split_len;
-    int nsplit;
+    int64_t units;   // (batch, kv-head, head group) triples
+    int64_t L;       // virtual tokens per unit (max_len)
+    int ctas;        // CTAs of the split kernel (one per SM)
+    int nslot;       // partial rows per (batch, query head)
     size_t total;
 };
 
