@@ -153,12 +153,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a)
         float ck[KSUB];
 #pragma unroll
         for (int r = 0; r < KSUB; ++r) ck[r] = __ldg(a.kC + c * KSUB + r);
+        float sum[GC];
 #pragma unroll
         for (int h = 0; h < GC; ++h) {
-            float sum = 0.f;
+            sum[h] = 0.f;
 #pragma unroll
-            for (int r = 0; r < KSUB; ++r) sum = fmaf(qrot[h * kD + j * KSUB + r], ck[r], sum);
-            lut[(size_t)e * GC + h] = sum;
+            for (int r = 0; r < KSUB; ++r) sum[h] = fmaf(qrot[h * kD + j * KSUB + r], ck[r], sum[h]);
+        }
+        if constexpr (GC == 4) {
+            reinterpret_cast<float4*>(lut)[e] = make_float4(sum[0], sum[1], sum[2], sum[3]);
+        } else {
+#pragma unroll
+            for (int h = 0; h < GC; ++h) lut[(size_t)e * GC + h] = sum[h];
         }
     }
     __syncthreads();

@@ -29,27 +29,54 @@ constexpr int kEncodeThreads = 128;
 constexpr int64_t kEncodeChunk = 64;  // tokens per pass-2 CTA
 
 // --------------------------------------------------------------- pass 1 --
-__device__ __forceinline__ void load16(const float* p, float (&v)[16]) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        float4 a = reinterpret_cast<const float4*>(p)[i];
-        v[4 * i] = a.x; v[4 * i + 1] = a.y; v[4 * i + 2] = a.z; v[4 * i + 3] = a.w;
+// Lane layout: 8 lanes per token (16 channels each), 4 tokens per warp step.
+// Each warp keeps kStatsDepth steps of loads in flight (the kernel streams
+// x once from HBM and needs the bytes in flight to cover the latency).
+constexpr int kStatsDepth = 4;
+
+template <typename XT>
+struct Raw16;
+template <>
+struct Raw16<__nv_bfloat16> {
+    uint4 u[2];
+    __device__ __forceinline__ void load(const __nv_bfloat16* p) {
+        const uint4* q = reinterpret_cast<const uint4*>(p);
+        u[0] = __ldg(q);
+        u[1] = __ldg(q + 1);
     }
-}
-__device__ __forceinline__ void load16(const __nv_bfloat16* p, float (&v)[16]) {
+    __device__ __forceinline__ void zero() { u[0] = u[1] = make_uint4(0, 0, 0, 0); }
+    __device__ __forceinline__ void unpack(float (&v)[16]) const {
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        uint4 a = reinterpret_cast<const uint4*>(p)[i];
-        uint32_t u[4] = {a.x, a.y, a.z, a.w};
+        for (int i = 0; i < 2; ++i) {
+            const uint32_t w[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            v[8 * i + 2 * k] = __uint_as_float(u[k] << 16);
-            v[8 * i + 2 * k + 1] = __uint_as_float(u[k] & 0xffff0000u);
+            for (int k = 0; k < 4; ++k) {
+                v[8 * i + 2 * k] = __uint_as_float(w[k] << 16);
+                v[8 * i + 2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+            }
         }
     }
-}
+};
+template <>
+struct Raw16<float> {
+    float4 f[4];
+    __device__ __forceinline__ void load(const float* p) {
+        const float4* q = reinterpret_cast<const float4*>(p);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) f[i] = __ldg(q + i);
+    }
+    __device__ __forceinline__ void zero() {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) f[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    __device__ __forceinline__ void unpack(float (&v)[16]) const {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            v[4 * i] = f[i].x; v[4 * i + 1] = f[i].y; v[4 * i + 2] = f[i].z; v[4 * i + 3] = f[i].w;
+        }
+    }
+};
 
-// Lane layout: 8 lanes per token (16 channels each), 4 tokens per warp step.
 template <typename XT>
 __global__ void __launch_bounds__(kStatsThreads) nsn_stats_kernel(EncodeArgs a) {
     const int chunk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -59,28 +86,35 @@ __global__ void __launch_bounds__(kStatsThreads) nsn_stats_kernel(EncodeArgs a) 
     const int64_t t1 = min(t0 + a.chunk1, a.T);
     const XT* xb = reinterpret_cast<const XT*>(a.x) + b * a.sb + h * a.sh + 16 * cg;
     const double sqrt_d = sqrt((double)kD);
+    constexpr int64_t kStride = 4 * (kStatsThreads / 32);  // tokens per CTA step
     double acc[16];
 #pragma unroll
     for (int c = 0; c < 16; ++c) acc[c] = 0.0;
-    for (int64_t base = t0 + warp * 4; base < t1; base += 4 * (kStatsThreads / 32)) {
-        const int64_t t = base + tk;
-        float v[16];
-        if (t < t1) {
-            load16(xb + t * a.st, v);
-        } else {
+    Raw16<XT> buf[kStatsDepth];
 #pragma unroll
-            for (int c = 0; c < 16; ++c) v[c] = 0.f;
-        }
-        double ss = 0.0;
+    for (int d = 0; d < kStatsDepth; ++d) {
+        const int64_t t = t0 + warp * 4 + d * kStride + tk;
+        if (t < t1) buf[d].load(xb + t * a.st); else buf[d].zero();
+    }
+    for (int64_t base = t0 + warp * 4; base < t1; base += kStatsDepth * kStride) {
 #pragma unroll
-        for (int c = 0; c < 16; ++c) ss = fma((double)v[c], (double)v[c], ss);
-        ss += __shfl_xor_sync(kFull, ss, 1);
-        ss += __shfl_xor_sync(kFull, ss, 2);
-        ss += __shfl_xor_sync(kFull, ss, 4);
-        if (ss > 0.0) {
-            const double inv = 1.0 / (sqrt(ss) / sqrt_d);
+        for (int d = 0; d < kStatsDepth; ++d) {
+            float v[16];
+            buf[d].unpack(v);
+            // refill this slot kStatsDepth steps ahead
+            const int64_t tn = base + (d + kStatsDepth) * kStride + tk;
+            if (tn < t1) buf[d].load(xb + tn * a.st); else buf[d].zero();
+            double ss = 0.0;
 #pragma unroll
-            for (int c = 0; c < 16; ++c) acc[c] = fma((double)v[c], inv, acc[c]);
+            for (int c = 0; c < 16; ++c) ss = fma((double)v[c], (double)v[c], ss);
+            ss += __shfl_xor_sync(kFull, ss, 1);
+            ss += __shfl_xor_sync(kFull, ss, 2);
+            ss += __shfl_xor_sync(kFull, ss, 4);
+            if (ss > 0.0) {
+                const double inv = rsqrt(ss) * sqrt_d;  // 1 / s1
+#pragma unroll
+                for (int c = 0; c < 16; ++c) acc[c] = fma((double)v[c], inv, acc[c]);
+            }
         }
     }
     // Sum the four token slots of each channel group, then the warps.

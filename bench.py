@@ -24,7 +24,6 @@ import os
 import statistics
 import subprocess
 import sys
-import tempfile
 import time
 
 import numpy as np
@@ -67,30 +66,47 @@ def attn_bytes_per_token(ksub: int, vsub: int) -> int:
 
 # ------------------------------------------------------------------ clocks --
 class ClockSampler:
-    """Polls nvidia-smi (one query every ~100 ms) for SM clock and throttle
-    reasons while the timed regions run."""
+    """Samples SM clock and throttle reasons through NVML every ~2 ms (nvidia-smi
+    polling as a fallback) while the timed regions run."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
     NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, gpu_index: int):
         import threading
         self.gpu = gpu_index
-        self.rows = []
+        self.rows = []  # (sm_mhz, max_mhz, set(reasons))
         self.stop = threading.Event()
         self.thread = threading.Thread(target=self._run, daemon=True)
 
     def _run(self):
+        try:
+            import pynvml as N
+            N.nvmlInit()
+            hdl = N.nvmlDeviceGetHandleByIndex(self.gpu)
+            bits = {"hw_slowdown": N.nvmlClocksThrottleReasonHwSlowdown,
+                    "hw_thermal_slowdown": N.nvmlClocksThrottleReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": N.nvmlClocksThrottleReasonSwThermalSlowdown,
+                    "sw_power_cap": N.nvmlClocksThrottleReasonSwPowerCap}
+            mx = N.nvmlDeviceGetMaxClockInfo(hdl, N.NVML_CLOCK_SM)
+            while not self.stop.is_set():
+                sm = N.nvmlDeviceGetClockInfo(hdl, N.NVML_CLOCK_SM)
+                r = N.nvmlDeviceGetCurrentClocksThrottleReasons(hdl)
+                self.rows.append((float(sm), float(mx), {k for k, v in bits.items() if r & v}))
+                self.stop.wait(0.002)
+            return
+        except Exception:
+            pass
+        fields = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+                  "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_power_cap")
         while not self.stop.is_set():
             try:
-                out = subprocess.run(
-                    ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                     "--format=csv,noheader,nounits"], capture_output=True, text=True,
-                    timeout=5).stdout.strip()
-                if out:
-                    self.rows.append([p.strip() for p in out.split(",")])
+                out = subprocess.run(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={fields}",
+                                      "--format=csv,noheader,nounits"], capture_output=True,
+                                     text=True, timeout=5).stdout.strip()
+                p = [x.strip() for x in out.split(",")]
+                self.rows.append((float(p[0]), float(p[1]),
+                                  {n for n, v in zip(self.NAMES, p[2:6]) if v.lower() == "active"}))
             except Exception:
                 return
             self.stop.wait(0.1)
@@ -104,22 +120,13 @@ class ClockSampler:
         self.thread.join(timeout=10)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        for r in self.rows:
-            if len(r) < 7:
-                continue
-            try:
-                sm.append(float(r[0]))
-                mx = float(r[1])
-            except ValueError:
-                continue
-            for n, v in zip(self.NAMES, r[3:7]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
+        if not self.rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        reasons = set()
+        for r in self.rows:
+            reasons |= r[2]
+        return {"sm_mhz": statistics.median(r[0] for r in self.rows), "sm_max_mhz": self.rows[-1][1],
+                "reasons": sorted(reasons), "samples": len(self.rows)}
 
 
 # --------------------------------------------------------------- CUDA arm --
@@ -364,9 +371,9 @@ def oracle_step_sample(n_seq: int = 1, n_heads: int = 8):
 
 
 def cpu_baseline(args):
-    dt, tokens = oracle_step_sample(1, 8)
+    dt, tokens = oracle_step_sample(4, 8)
     return {"value": round(tokens / dt, 2), "unit": "KV tokens/s", "cores": 1, "kind": "oracle",
-            "sample": "1 sequence x 8 kv-heads x 4096 tokens (K+V encode, dequant, attention of 32 "
+            "sample": "4 sequences x 8 kv-heads x 4096 tokens (K+V encode, dequant, attention of 32 "
                       f"query heads), single-threaded fp64 C, {dt:.1f} s"}
 
 
