@@ -129,6 +129,19 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(self.rows)}
 
 
+# ------------------------------------------------------------- reduction --
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The largest value over all ranks (timings are reported as the max)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64,
+                     device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # --------------------------------------------------------------- CUDA arm --
 def run_cuda(args):
     import torch
@@ -205,11 +218,7 @@ def run_cuda(args):
     step_ms = [e[0].elapsed_time(e[3]) for e in ev]
     enc_ms = [e[0].elapsed_time(e[1]) for e in ev] + [e[1].elapsed_time(e[2]) for e in ev]
     att_small_ms = [e[2].elapsed_time(e[3]) for e in ev]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
     ms_per_step = total_ms / args.steps
     tokens_per_step = B * T * world
     value = tokens_per_step / (ms_per_step / 1e3)
@@ -238,10 +247,7 @@ def run_cuda(args):
         e1.synchronize()
         e2e_ms += e0.elapsed_time(e1)
     barrier()
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
     h2d = sum(host[n].numel() * host[n].element_size() for n in ("k", "v", "q"))
     d2h = (res_host.numel() * 2 + codes_host.numel() + scales_host.numel() * 4)
     e2e = {"value": tokens_per_step / (e2e_ms / args.steps / 1e3), "unit": "KV tokens/s",
@@ -329,11 +335,7 @@ def run_attention_bench(args, nsnq, dev, world, barrier, hbm, peak_kind):
     torch.cuda.synchronize()
     barrier()
     ms = [a.elapsed_time(b) for a, b in evs]
-    avg = sum(ms) / len(ms)
-    if world > 1:
-        t = torch.tensor([avg], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        avg = float(t.item())
+    avg = max_over_ranks(sum(ms) / len(ms), world, dev)
     nbytes = B * H * T * attn_bytes_per_token(w.sub_dim, w.sub_dim)
     gbs = nbytes / (avg / 1e3) / 1e9
     return {"metric": "decode-attn HBM GB/s (algorithmic bytes)", "value": round(gbs * world, 1),
