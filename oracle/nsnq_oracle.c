@@ -151,12 +151,14 @@ static int nearest_codeword(const double* w, const float* C, int K, int g) {
  *   shift_given = 0: o is the channel mean of the normalized tokens;
  *               = 1: o is taken from o_in (tokens appended to a cache whose
  *                    shift was computed over the prompt)
+ *   adaptive_scale = 1: s2 is multiplied by ||w||^2 / (w . w_hat), the
+ *               scale adjustment of Methodology §3 (see below).
  * Outputs: codes [T][d/g], s1 [T], s2 [T], o_out [d], and optionally
  * w_out [T][d] (the transformed tokens that were quantized).
  */
 int oracle_encode_head(const double* x, int64_t T, int d, int g, const float* C, int K,
-                       int shift_given, const double* o_in, uint8_t* codes, double* s1,
-                       double* s2, double* o_out, double* w_out) {
+                       int shift_given, const double* o_in, int adaptive_scale, uint8_t* codes,
+                       double* s1, double* s2, double* o_out, double* w_out) {
     if (d <= 0 || (d & (d - 1)) != 0 || g <= 0 || d % g != 0 || g > 64 || K <= 0 || K > 256 ||
         T < 0 || (shift_given && !o_in) || !C || !o_out)
         return ORACLE_ERR_ARG;
@@ -212,6 +214,22 @@ int oracle_encode_head(const double* x, int64_t T, int d, int g, const float* C,
         if (w_out) memcpy(w_out + (size_t)t * d, w, (size_t)d * sizeof(double));
         for (int j = 0; j < J; ++j)
             codes[(size_t)t * J + j] = (uint8_t)nearest_codeword(w + (size_t)j * g, C, K, g);
+        /* Scale adjustment (Methodology §3): the quantized vector w_hat is
+         * scaled by a = ||w||^2 / (w . w_hat) so that its component along w
+         * equals w (the remaining error is orthogonal to w); a is folded into
+         * the stored s2. a = 1 when w . w_hat <= 0 (nothing to align). */
+        if (adaptive_scale) {
+            double ww = 0.0, wq = 0.0;
+            for (int j = 0; j < J; ++j) {
+                const int c = codes[(size_t)t * J + j];
+                for (int r = 0; r < g; ++r) {
+                    const double wi = w[j * g + r];
+                    ww += wi * wi;
+                    wq += wi * (double)C[(size_t)c * g + r];
+                }
+            }
+            if (wq > 0.0) s2[t] *= ww / wq;
+        }
     }
     free(H); free(y); free(u); free(w);
     return ORACLE_OK;

@@ -31,7 +31,8 @@ def lib():
         L.oracle_kmeans.argtypes = [dp, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                     dp, i64p]
         L.oracle_encode_head.argtypes = [dp, ctypes.c_int64, ctypes.c_int, ctypes.c_int, fp,
-                                         ctypes.c_int, ctypes.c_int, dp, u8p, dp, dp, dp, dp]
+                                         ctypes.c_int, ctypes.c_int, dp, ctypes.c_int, u8p, dp, dp,
+                                         dp, dp]
         L.oracle_dequant_head.argtypes = [u8p, fp, fp, fp, ctypes.c_int64, ctypes.c_int,
                                           ctypes.c_int, fp, ctypes.c_int, dp]
         L.oracle_attention_head.argtypes = [dp, ctypes.c_int, dp, dp, ctypes.c_int64,
@@ -73,11 +74,12 @@ def kmeans(X: np.ndarray, k: int, iters: int):
 
 
 def encode(x: np.ndarray, codebook: np.ndarray, shift: Optional[np.ndarray] = None,
-           want_w: bool = False):
+           want_w: bool = False, adaptive_scale: bool = False):
     """Encode x [B][H][T][d] (exact fp64 values of the I/O type).
 
     shift None -> the shift is computed per (b, h) over the T tokens;
-    else shift [B][H][d] is used as given.
+    else shift [B][H][d] is used as given. adaptive_scale -> s2 carries the
+    scale adjustment ||w||^2 / (w . w_hat).
     Returns dict with codes uint8 [B][H][T][d/g], s1, s2 fp64 [B][H][T],
     o fp64 [B][H][d] and (optionally) w fp64 [B][H][T][d].
     """
@@ -104,7 +106,8 @@ def encode(x: np.ndarray, codebook: np.ndarray, shift: Optional[np.ndarray] = No
             _check(lib().oracle_encode_head(
                 _p(np.ascontiguousarray(x[b, h]), ctypes.c_double), T, d, g,
                 _p(C, ctypes.c_float), K, 1 if shift is not None else 0,
-                _p(oin, ctypes.c_double), _p(cb, ctypes.c_uint8), _p(s1b, ctypes.c_double),
+                _p(oin, ctypes.c_double), 1 if adaptive_scale else 0,
+                _p(cb, ctypes.c_uint8), _p(s1b, ctypes.c_double),
                 _p(s2b, ctypes.c_double), _p(ob, ctypes.c_double), _p(wb, ctypes.c_double)),
                 "encode")
             codes[b, h] = cb

@@ -274,3 +274,33 @@ def test_synthetic_keys_have_outlier_channels():
     assert all(m[c] > 5 for c in chans) and np.median(m) < 2
     sub = S.keys(w, t0=100, t1=120, T_total=256)
     assert np.array_equal(sub[0, 0], K[0, 0, 100:120])
+
+
+@pytest.mark.parametrize("g", [8, 4])
+def test_adaptive_scale_leaves_error_orthogonal_to_the_token(codebooks, g):
+    """Methodology §3, scale adjustment: the scaled quantized vector keeps the
+    component along the original, so after removing the shift the
+    reconstruction error is orthogonal to the original token, and the codes
+    are those of the plain encoding."""
+    x = _tiny_keys(T=64)
+    C = codebooks[g]
+    plain = O.encode(x, C)
+    adj = O.encode(x, C, adaptive_scale=True)
+    assert np.array_equal(plain["codes"], adj["codes"])
+    assert np.array_equal(plain["s1"], adj["s1"]) and np.array_equal(plain["o"], adj["o"])
+    # no float32 storage here: rebuild with the exact byproducts
+    H = scipy.linalg.hadamard(D) / np.sqrt(D)
+    wh = C[adj["codes"][0, 0]].reshape(64, D).astype(np.float64)
+    s1, s2, o = adj["s1"][0, 0], adj["s2"][0, 0], adj["o"][0, 0]
+    xr = s1[:, None] * (s2[:, None] * (wh @ H) + o[None, :])
+    xc = x[0, 0] - s1[:, None] * o[None, :]          # original minus shift part
+    err = xr - x[0, 0]
+    cos = (err * xc).sum(1) / (np.linalg.norm(err, axis=1) * np.linalg.norm(xc, axis=1))
+    assert np.abs(cos).max() < 1e-10
+    # the plain encoding's error is not orthogonal
+    whp = wh
+    xp = plain["s1"][0, 0][:, None] * (plain["s2"][0, 0][:, None] * (whp @ H) + o[None, :])
+    ep = xp - x[0, 0]
+    assert np.abs((ep * xc).sum(1)).max() > 1e-3
+    ratio = adj["s2"][0, 0] / plain["s2"][0, 0]
+    assert (ratio > 0.5).all() and (ratio < 2.0).all()
