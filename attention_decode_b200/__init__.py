@@ -26,6 +26,7 @@ LIB_PATH = os.path.join(_HERE, "_build", "libnsnq.so")
 NSNQ_OK, NSNQ_ERR_INVALID_ARG, NSNQ_ERR_UNSUPPORTED, NSNQ_ERR_WORKSPACE, NSNQ_ERR_CUDA = range(5)
 NSNQ_F32, NSNQ_BF16 = 0, 1
 SHIFT_COMPUTE, SHIFT_GIVEN = 0, 1
+ENCODE_DEFAULT, ENCODE_ADAPTIVE_SCALE = 0, 1
 HEAD_DIM = 128
 N_CENTROIDS = 256
 
@@ -73,8 +74,8 @@ def load(path: str = LIB_PATH):
     L.nsnq_codebook_index_build.restype = ci
     L.nsnq_encode_workspace.argtypes = [ci, ci, i64, ci]
     L.nsnq_encode_workspace.restype = sz
-    L.nsnq_encode.argtypes = [vp, ci, ci, ci, i64, ci, i64, i64, i64, i64, ci, _Codebook, _Cache,
-                              vp, sz, vp]
+    L.nsnq_encode.argtypes = [vp, ci, ci, ci, i64, ci, i64, i64, i64, i64, ci, ctypes.c_uint,
+                              _Codebook, _Cache, vp, sz, vp]
     L.nsnq_encode.restype = ci
     L.nsnq_dequant.argtypes = [_Cache, _Codebook, ci, ci, i64, i64, ci, vp, vp]
     L.nsnq_dequant.restype = ci
@@ -184,7 +185,7 @@ def _workspace(nbytes: int, device) -> torch.Tensor:
 
 def nsnq_encode(x: torch.Tensor, cb: Codebook, cache: Cache, t_offset: int = 0,
                 shift_mode: int = SHIFT_COMPUTE, workspace: Optional[torch.Tensor] = None,
-                stream=None) -> torch.Tensor:
+                stream=None, flags: int = ENCODE_DEFAULT) -> torch.Tensor:
     """Encode x [B][H][T][D] (fp32 or bf16; channels contiguous) into cache
     positions [t_offset, t_offset + T). Returns the workspace (its first two
     uint64 hold the near-tie counters)."""
@@ -195,7 +196,7 @@ def nsnq_encode(x: torch.Tensor, cb: Codebook, cache: Cache, t_offset: int = 0,
     if workspace is None:
         workspace = _workspace(need, x.device)
     _check(load().nsnq_encode(_ptr(x), _dtype_code(x), B, H, T, D, x.stride(0), x.stride(1),
-                              x.stride(2), t_offset, shift_mode, cb._c(), cache._c(),
+                              x.stride(2), t_offset, shift_mode, flags, cb._c(), cache._c(),
                               _ptr(workspace), workspace.numel() * workspace.element_size(),
                               _stream(stream)))
     return workspace

@@ -111,13 +111,15 @@ size_t nsnq_encode_workspace(int B, int H, int64_t T, int D) {
 
 nsnq_status nsnq_encode(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t T, int D,
                         int64_t stride_b, int64_t stride_h, int64_t stride_t, int64_t t_offset,
-                        nsnq_shift_mode mode, nsnq_codebook cb, nsnq_cache cache,
+                        nsnq_shift_mode mode, unsigned flags, nsnq_codebook cb, nsnq_cache cache,
                         void* workspace, size_t workspace_bytes, nsnq_stream stream) {
     if (D != nsnq::kHeadDim) return fail(NSNQ_ERR_UNSUPPORTED, "D = %d (only 128 is supported)", D);
     if (x_dtype != NSNQ_F32 && x_dtype != NSNQ_BF16)
         return fail(NSNQ_ERR_UNSUPPORTED, "x_dtype = %d", (int)x_dtype);
     if (mode != NSNQ_SHIFT_COMPUTE && mode != NSNQ_SHIFT_GIVEN)
         return fail(NSNQ_ERR_INVALID_ARG, "shift mode = %d", (int)mode);
+    if (flags & ~(unsigned)NSNQ_ENCODE_ADAPTIVE_SCALE)
+        return fail(NSNQ_ERR_INVALID_ARG, "unknown encode flags 0x%x", flags);
     if (B < 0 || H < 0 || T < 0)
         return fail(NSNQ_ERR_INVALID_ARG, "negative size B=%d H=%d T=%lld", B, H, (long long)T);
     if (B > 65535 || H > 65535) return fail(NSNQ_ERR_UNSUPPORTED, "B or H above 65535");
@@ -152,6 +154,7 @@ nsnq_status nsnq_encode(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t
     a.sb = stride_b; a.sh = stride_h; a.st = stride_t;
     a.t_offset = t_offset;
     a.given_shift = mode == NSNQ_SHIFT_GIVEN;
+    a.adaptive = (flags & NSNQ_ENCODE_ADAPTIVE_SCALE) ? 1 : 0;
     a.C = cb.centroids;
     a.sub = cb.sub_dim;
     a.index = cb.index;

@@ -301,6 +301,7 @@ __global__ void __launch_bounds__(kEncodeThreads) nsn_encode_kernel(EncodeArgs a
 
         const Best best = search_fp32<SUB>(w, Cs);
         int code = best.i1;
+        double wsub[4] = {w[0], w[1], w[2], w[3]};  // the transformed coordinates (fp64 if re-decided)
         const bool tie = cancel || (best.d2 - best.d1) <= kTieRel * best.d1 + kTieAbs;
         const unsigned tie_mask = __ballot_sync(kFull, tie);
         if (tie_mask) {
@@ -338,10 +339,26 @@ __global__ void __launch_bounds__(kEncodeThreads) nsn_encode_kernel(EncodeArgs a
             if (tie) code = c64;
             s1 = (float)s1d;
             s2 = (float)s2d;
+#pragma unroll
+            for (int r = 0; r < 4; ++r) wsub[r] = zd[r];
             if (lane == 0 && a.stats) {
                 atomicAdd(&a.stats[0], 1ull);
                 atomicAdd(&a.stats[1], (unsigned long long)(__popc(tie_mask) / (SUB / 4)));
             }
+        }
+        if (a.adaptive) {
+            // Scale adjustment: s2 *= ||w||^2 / (w . w_hat); lane holds coordinates
+            // 4l..4l+3, i.e. the (lane & 1) half of sub-vector lane / 2 when SUB = 8.
+            const float* cw = Cs + code * SUB + (SUB == 8 ? 4 * (lane & 1) : 0);
+            double ww = 0.0, wq = 0.0;
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                ww += wsub[r] * wsub[r];
+                wq += wsub[r] * (double)cw[r];
+            }
+            ww = warp_sum_d(ww);
+            wq = warp_sum_d(wq);
+            s2 = (float)((double)s2 * (wq > 0.0 ? ww / wq : 1.0));
         }
         const int64_t row = bh * a.cap + a.t_offset + t;
         if constexpr (SUB == 4) {

@@ -101,14 +101,17 @@ __device__ __forceinline__ void load64<float>(const float* p, float (&v)[64]) {
 // the two threads of a pair (pair_mask): fp64 NSN of the whole token, then
 // w_j = H_j u for each flagged sub-vector and an fp64 scan of its cell list
 // (which holds every codeword that can be nearest there; lowest index on
-// exact ties). Returns the fp64 (s1, s2). Kept in registers (no local
-// arrays) and division-free, since one slow warp holds its SM.
+// exact ties). Returns the fp64 (s1, s2) and, summed over the pair's
+// re-decided sub-vectors, w . C[new code] and w . C[previous code] (for the
+// scale adjustment). Kept in registers (no local arrays) and division-free,
+// since one slow warp holds its SM.
 template <typename XT>
 __device__ __noinline__ void exact_path(const XT* xrow, const double* o64, const float* o32,
                                        const float4* reps, const uint16_t* offs,
                                        const uint16_t* ents, int half, unsigned pair_mask,
                                        uint32_t my_mask, uint32_t both_mask, uint32_t (&codes)[4],
-                                       double& s1_out, double& s2_out) {
+                                       double& s1_out, double& s2_out, double& wq_new_out,
+                                       double& wq_old_out) {
     float v[64];
     load64<XT>(xrow + 64 * half, v);
     const double* o64h = o64 ? o64 + 64 * half : nullptr;
@@ -137,6 +140,7 @@ __device__ __noinline__ void exact_path(const XT* xrow, const double* o64, const
     const double s2 = ss2 <= 0x1p-40 * (yy + oo) ? 0.0 : sqrt(ss2) / sqrt_d;
     const double inv2 = s2 > 0.0 ? 1.0 / s2 : 0.0;
     const double hs = 1.0 / sqrt_d;
+    double wq_new = 0.0, wq_old = 0.0;
     uint32_t todo = both_mask;
     while (todo) {
         const int j = __ffs(todo) - 1;  // global sub-vector index 0..31
@@ -174,11 +178,17 @@ __device__ __noinline__ void exact_path(const XT* xrow, const double* o64, const
             }
             const int jj = j - 16 * half;
             const int sh = 8 * (jj & 3);
+            const float4 cn = reps[bi * 8];
+            const float4 co = reps[((codes[jj >> 2] >> sh) & 0xffu) * 8];
             codes[jj >> 2] = (codes[jj >> 2] & ~(0xffu << sh)) | ((uint32_t)bi << sh);
+            wq_new += w[0] * (double)cn.x + w[1] * (double)cn.y + w[2] * (double)cn.z + w[3] * (double)cn.w;
+            wq_old += w[0] * (double)co.x + w[1] * (double)co.y + w[2] * (double)co.z + w[3] * (double)co.w;
         }
     }
     s1_out = s1;
     s2_out = s2;
+    wq_new_out = wq_new + __shfl_xor_sync(pair_mask, wq_new, 1);
+    wq_old_out = wq_old + __shfl_xor_sync(pair_mask, wq_old, 1);
 }
 
 // Candidate walk of one sub-vector w through its cell's list.
@@ -238,7 +248,10 @@ struct Walk {
     __device__ __forceinline__ bool tie() const { return (d2 - d1) <= fmaf(kTieRel, d1, kTieAbs); }
 };
 
-template <typename XT>
+// ADAPT: also apply the scale adjustment s2 *= ||w||^2 / (w . w_hat). Since
+// u = z / s2 has ||u||^2 = d and H is orthonormal, ||w||^2 = d; only w . w_hat
+// is accumulated, in the search loop.
+template <typename XT, bool ADAPT>
 __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(EncodeArgs a) {
     extern __shared__ __align__(16) uint8_t sm[];
     float4* reps = reinterpret_cast<float4*>(sm + kSmReps);
@@ -370,6 +383,7 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
         // ---- nearest codeword of the 16 sub-vectors this thread holds ----
         uint32_t codes[4] = {0u, 0u, 0u, 0u};
         uint32_t tie = 0;
+        float wq = 0.f;
         const float4* myrep = reps + (lane & 7);
 #pragma unroll
         for (int jj = 0; jj < 16; ++jj) {
@@ -378,23 +392,35 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
             while (A.p < A.e) A.step(ents, myrep);
             codes[jj >> 2] |= (uint32_t)A.i1 << (8 * (jj & 3));
             if (cancel || A.tie()) tie |= 1u << jj;
+            if constexpr (ADAPT) {
+                const float4 c = myrep[A.i1 * 8];
+                wq = fmaf(v[4 * jj + 3], c.w, fmaf(v[4 * jj + 2], c.z,
+                     fmaf(v[4 * jj + 1], c.y, fmaf(v[4 * jj], c.x, wq))));
+            }
         }
         if (!valid) tie = 0;
         // ---- exact fp64 decision where the fp32 search is not conclusive ----
         const uint32_t my_mask = tie << (16 * half);
         const uint32_t both = my_mask | __shfl_xor_sync(kFull, my_mask, 1);
         float s1o = s1, s2o = s2;
+        double wqd = 0.0;
+        if constexpr (ADAPT) wqd = (double)(wq + __shfl_xor_sync(kFull, wq, 1));
         if (both) {
             const double* o64 = a.given_shift ? nullptr : a.o64 + bh * kD;
-            double s1d, s2d;
+            double s1d, s2d, wq_new, wq_old;
             exact_path<XT>(xrow, o64, a.shift + bh * kD, reps, offs, ents, half, pair_mask,
-                           my_mask, both, codes, s1d, s2d);
+                           my_mask, both, codes, s1d, s2d, wq_new, wq_old);
             s1o = (float)s1d;
             s2o = (float)s2d;
+            // on cancellation every sub-vector was re-decided from the fp64 w
+            wqd = cancel ? wq_new : wqd + (wq_new - wq_old);
             if (half == 0 && a.stats) {
                 atomicAdd(&a.stats[0], 1ull);
                 atomicAdd(&a.stats[1], (unsigned long long)__popc(both));
             }
+        }
+        if constexpr (ADAPT) {
+            if (wqd > 0.0) s2o = (float)((double)s2o * ((double)kD / wqd));
         }
         if (valid) {
             const int64_t row = bh * a.cap + a.t_offset + t;
@@ -407,9 +433,9 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
 
 size_t pruned_smem_bytes() { return kSmBytes; }
 
-template <typename XT>
+template <typename XT, bool ADAPT>
 static cudaError_t launch_pruned_t(const EncodeArgs& a, cudaStream_t s) {
-    auto kern = nsn_encode_pruned_kernel<XT>;
+    auto kern = nsn_encode_pruned_kernel<XT, ADAPT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmBytes);
     if (e != cudaSuccess) return e;
@@ -424,7 +450,9 @@ static cudaError_t launch_pruned_t(const EncodeArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_encode_pruned(const EncodeArgs& a, cudaStream_t s) {
-    return a.x_bf16 ? launch_pruned_t<__nv_bfloat16>(a, s) : launch_pruned_t<float>(a, s);
+    if (a.adaptive)
+        return a.x_bf16 ? launch_pruned_t<__nv_bfloat16, true>(a, s) : launch_pruned_t<float, true>(a, s);
+    return a.x_bf16 ? launch_pruned_t<__nv_bfloat16, false>(a, s) : launch_pruned_t<float, false>(a, s);
 }
 
 }  // namespace nsnq

@@ -28,6 +28,7 @@ struct EncodeArgs {
     int64_t sb, sh, st;
     int64_t t_offset;
     int given_shift;
+    int adaptive;  // scale adjustment folded into s2
     const float* C;
     int sub;
     const void* index;  // search index (sub == 4)

@@ -63,6 +63,15 @@ typedef enum {
     NSNQ_SHIFT_GIVEN = 1     /* o read from cache.shift (tokens appended after the prompt) */
 } nsnq_shift_mode;
 
+typedef enum {
+    NSNQ_ENCODE_DEFAULT = 0,
+    /* Scale adjustment (Methodology §3): the quantized token w_hat is scaled by
+     * ||w||^2 / (w . w_hat) so that its component along the transformed token w
+     * equals w (the error left is orthogonal to w); the factor multiplies the
+     * stored s2, so dequant and attention need no change. */
+    NSNQ_ENCODE_ADAPTIVE_SCALE = 1
+} nsnq_encode_flags;
+
 typedef struct {
     const float* centroids;  /* device, [n_centroids][sub_dim] fp32, 16-byte aligned */
     int n_centroids;         /* must be 256 (one byte per code) */
@@ -127,6 +136,7 @@ size_t nsnq_encode_workspace(int B, int H, int64_t T, int D);
  *             dtype x_dtype (fp32 or bf16); 16-byte aligned rows.
  *   mode      NSNQ_SHIFT_COMPUTE: o = mean over the T tokens of x/s1, stored
  *             to cache.shift (fp32); NSNQ_SHIFT_GIVEN: o = cache.shift.
+ *   flags     NSNQ_ENCODE_DEFAULT or NSNQ_ENCODE_ADAPTIVE_SCALE.
  *   cb        codebook; cache: codes/scales written, shift read or written.
  *   workspace device scratch of at least nsnq_encode_workspace(B, H, T, D)
  *             bytes, 256-byte aligned.
@@ -138,7 +148,7 @@ size_t nsnq_encode_workspace(int B, int H, int64_t T, int D);
  */
 nsnq_status nsnq_encode(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t T, int D,
                         int64_t stride_b, int64_t stride_h, int64_t stride_t, int64_t t_offset,
-                        nsnq_shift_mode mode, nsnq_codebook cb, nsnq_cache cache,
+                        nsnq_shift_mode mode, unsigned flags, nsnq_codebook cb, nsnq_cache cache,
                         void* workspace, size_t workspace_bytes, nsnq_stream stream);
 
 /*

@@ -57,11 +57,11 @@ def _cache(cap=100):
 
 def _encode(lib, **kw):
     a = dict(x=FAKE, dt=nsnq.NSNQ_BF16, B=1, H=1, T=10, D=128, sb=128 * 10, sh=128 * 10, st=128,
-             off=0, mode=0, cb=_cb(), cache=_cache(), ws=FAKE, wsb=1 << 20, stream=None)
+             off=0, mode=0, flags=0, cb=_cb(), cache=_cache(), ws=FAKE, wsb=1 << 20, stream=None)
     a.update(kw)
     return lib.nsnq_encode(a["x"], a["dt"], a["B"], a["H"], a["T"], a["D"], a["sb"], a["sh"],
-                           a["st"], a["off"], a["mode"], a["cb"], a["cache"], a["ws"], a["wsb"],
-                           a["stream"])
+                           a["st"], a["off"], a["mode"], a["flags"], a["cb"], a["cache"], a["ws"],
+                           a["wsb"], a["stream"])
 
 
 def test_encode_validation(lib):
@@ -75,6 +75,7 @@ def test_encode_validation(lib):
     assert _encode(lib, off=95) == nsnq.NSNQ_ERR_INVALID_ARG            # past capacity
     assert _encode(lib, T=-1) == nsnq.NSNQ_ERR_INVALID_ARG
     assert _encode(lib, mode=7) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert _encode(lib, flags=2) == nsnq.NSNQ_ERR_INVALID_ARG
     assert _encode(lib, ws=None) == nsnq.NSNQ_ERR_WORKSPACE
     assert _encode(lib, cb=_cb(index=None)) == nsnq.NSNQ_ERR_INVALID_ARG     # 2-bit needs its index
     assert b"nsnq_codebook_index_build" in lib.nsnq_last_error()

@@ -269,3 +269,40 @@ def test_encode_detects_index_of_another_codebook(codebooks):
     assert nsnq.encode_stats(ws)[2] != 0
     ws = nsnq.nsnq_encode(x, good, cache)
     assert nsnq.encode_stats(ws)[2] == 0
+
+
+@pytest.mark.parametrize("sub,T,dtype,kdist", [(4, 700, "bf16", S.K_MODERATE), (8, 300, "f32", S.K_MODERATE),
+                                                (4, 400, "bf16", S.K_STRONG)])
+def test_encode_adaptive_scale_matches_oracle(codebooks, sub, T, dtype, kdist):
+    """Scale adjustment (Methodology §3): same codes, s2 multiplied by
+    ||w||^2 / (w . w_hat), against the oracle's fp64 value."""
+    w = _workload(2, 2, T, dtype, sub, kdist)
+    io, x64 = _inputs(w, "K")
+    C = codebooks[sub]
+    ora = O.encode(x64, C, want_w=True, adaptive_scale=True)
+    cache = nsnq.Cache.empty(2, 2, T, sub)
+    nsnq.nsnq_encode(P.to_dev(io, dtype), P.codebook(C), cache, flags=nsnq.ENCODE_ADAPTIVE_SCALE)
+    torch.cuda.synchronize()
+    _, n_bad, worst = P.code_report(cache.codes.cpu().numpy(), ora["codes"], ora["w"], C)
+    assert n_bad == 0, worst
+    P.check_scales(cache.scales.cpu().numpy(), ora)
+    P.check_shift(cache.shift.cpu().numpy(), ora["o"])
+
+
+@pytest.mark.parametrize("sub", [4, 8])
+def test_encode_adaptive_scale_given_shift(codebooks, sub):
+    """Scale adjustment with a given shift (the append path), a far-off shift
+    included so that some tokens take the fp64 path."""
+    w = _workload(1, 2, 260, "bf16", sub)
+    io, x64 = _inputs(w, "K")
+    C = codebooks[sub]
+    o_given = (np.random.default_rng(3).standard_normal((1, 2, D)) * 0.3).astype(np.float32)
+    ora = O.encode(x64, C, shift=o_given.astype(np.float64), want_w=True, adaptive_scale=True)
+    cache = nsnq.Cache.empty(1, 2, 260, sub)
+    cache.shift.copy_(torch.from_numpy(o_given))
+    nsnq.nsnq_encode(P.to_dev(io, "bf16"), P.codebook(C), cache, shift_mode=nsnq.SHIFT_GIVEN,
+                     flags=nsnq.ENCODE_ADAPTIVE_SCALE)
+    torch.cuda.synchronize()
+    _, n_bad, worst = P.code_report(cache.codes.cpu().numpy(), ora["codes"], ora["w"], C)
+    assert n_bad == 0, worst
+    P.check_scales(cache.scales.cpu().numpy(), ora)
