@@ -173,3 +173,81 @@ def stored(enc: dict):
     """The fp32 values an encoder stores for (s1, s2, o)."""
     return (enc["s1"].astype(np.float32), enc["s2"].astype(np.float32),
             enc["o"].astype(np.float32))
+
+
+def attention_with_residual(q: np.ndarray, Khat: np.ndarray, Vhat: np.ndarray, seq_lens,
+                            Kres: np.ndarray, Vres: np.ndarray, res_lens,
+                            scale: Optional[float] = None) -> np.ndarray:
+    """Decode attention over [quantized part || full-precision residual]
+    (Methodology §4, Implementation Details, Residuals: the cache is a
+    quantized part plus a full-precision residual of recent tokens).
+
+    Khat/Vhat [B][Hkv][T][d] dense dequantized, sequence b uses its first
+    seq_lens[b] rows; Kres/Vres [B][Hkv][R][d] the residual tokens as stored,
+    sequence b uses its first res_lens[b] rows, which come after its quantized
+    tokens. One softmax over both parts. Returns fp64 [B][Hq][d]."""
+    B, Hq, d = q.shape
+    out = np.zeros((B, Hq, d))
+    for b in range(B):
+        L, r = int(seq_lens[b]), int(res_lens[b])
+        Kb = np.concatenate([np.asarray(Khat[b:b + 1, :, :L], dtype=np.float64),
+                             np.asarray(Kres[b:b + 1, :, :r], dtype=np.float64)], axis=2)
+        Vb = np.concatenate([np.asarray(Vhat[b:b + 1, :, :L], dtype=np.float64),
+                             np.asarray(Vres[b:b + 1, :, :r], dtype=np.float64)], axis=2)
+        out[b:b + 1] = attention(q[b:b + 1], Kb, Vb, scale=scale)
+    return out
+
+
+def decode_with_residual(k_prompt: np.ndarray, v_prompt: np.ndarray, k_new: np.ndarray,
+                         v_new: np.ndarray, queries: np.ndarray, Ck: np.ndarray, Cv: np.ndarray,
+                         R: int, scale: Optional[float] = None):
+    """The serving loop with a residual window of R tokens (Methodology §4,
+    Implementation Details, Residuals), every sequence in lock-step.
+
+    Readings: the prompt [B][Hkv][T][d] is quantized whole, its shift o
+    computed over its T tokens; decode step s appends token s of
+    k_new/v_new [B][Hkv][S][d] to the residual; when the residual then holds
+    R tokens it is flushed: encoded with the stored o (not refreshed) and
+    appended to the quantized cache, and the residual is emptied; the step's
+    query queries[s] [B][Hq][d] then attends over [quantized || residual].
+    Inputs are the exact values of the I/O type. Returns (outputs fp64
+    [S][B][Hq][d], final state dict: codes/s1/s2 per tensor over the
+    quantized tokens, o, number of quantized and residual tokens)."""
+    B, Hkv, T, d = k_prompt.shape
+    S = k_new.shape[2]
+    enc = {"K": encode(k_prompt, Ck), "V": encode(v_prompt, Cv)}
+    o = {n: enc[n]["o"] for n in enc}
+    codes = {n: [enc[n]["codes"]] for n in enc}
+    s1 = {n: [enc[n]["s1"]] for n in enc}
+    s2 = {n: [enc[n]["s2"]] for n in enc}
+    C = {"K": Ck, "V": Cv}
+    res = {"K": k_new[:, :, :0], "V": v_new[:, :, :0]}
+    new = {"K": k_new, "V": v_new}
+    outs = np.zeros((S,) + queries.shape[1:])
+    for s in range(S):
+        for n in res:
+            res[n] = np.concatenate([res[n], new[n][:, :, s:s + 1]], axis=2)
+        if res["K"].shape[2] == R:
+            for n in res:
+                e = encode(res[n], C[n], shift=o[n])
+                codes[n].append(e["codes"])
+                s1[n].append(e["s1"])
+                s2[n].append(e["s2"])
+                res[n] = res[n][:, :, :0]
+        hat = {}
+        for n in res:
+            cs = np.concatenate(codes[n], axis=2)
+            a1 = np.concatenate(s1[n], axis=2)
+            a2 = np.concatenate(s2[n], axis=2)
+            hat[n] = dequant(cs, a1.astype(np.float32), a2.astype(np.float32),
+                             o[n].astype(np.float32), C[n])
+        nq = hat["K"].shape[2]
+        nr = res["K"].shape[2]
+        outs[s] = attention_with_residual(queries[s], hat["K"], hat["V"], [nq] * B,
+                                          res["K"], res["V"], [nr] * B, scale=scale)
+    state = {"n_quant": T + (S // R) * R if R > 0 else T, "n_res": S % R}
+    for n in res:
+        state[n] = {"codes": np.concatenate(codes[n], axis=2),
+                    "s1": np.concatenate(s1[n], axis=2), "s2": np.concatenate(s2[n], axis=2),
+                    "o": o[n]}
+    return outs, state

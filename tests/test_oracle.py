@@ -304,3 +304,94 @@ def test_adaptive_scale_leaves_error_orthogonal_to_the_token(codebooks, g):
     assert np.abs((ep * xc).sum(1)).max() > 1e-3
     ratio = adj["s2"][0, 0] / plain["s2"][0, 0]
     assert (ratio > 0.5).all() and (ratio < 2.0).all()
+
+
+# --------------------------------------------------------- residual window --
+def test_residual_attention_matches_sdpa_over_concatenation():
+    """Methodology §4 (Residuals): one softmax over the quantized tokens and
+    the full-precision residual, each sequence with its own two lengths
+    (empty parts included), checked against torch SDPA over the
+    concatenated rows."""
+    rng = np.random.default_rng(4)
+    B, Hq, Hkv, T, R = 4, 4, 2, 23, 9
+    q = rng.standard_normal((B, Hq, D))
+    K = rng.standard_normal((B, Hkv, T, D)) * 1.3
+    V = rng.standard_normal((B, Hkv, T, D))
+    Kr = rng.standard_normal((B, Hkv, R, D)) * 1.3 + 0.5
+    Vr = rng.standard_normal((B, Hkv, R, D)) - 0.7
+    lens, rlens = [23, 0, 5, 0], [0, 9, 4, 0]
+    out = O.attention_with_residual(q, K, V, lens, Kr, Vr, rlens)
+    G = Hq // Hkv
+    for b in range(B):
+        for h in range(Hq):
+            Kc = np.concatenate([K[b, h // G, :lens[b]], Kr[b, h // G, :rlens[b]]])
+            Vc = np.concatenate([V[b, h // G, :lens[b]], Vr[b, h // G, :rlens[b]]])
+            if Kc.shape[0] == 0:
+                assert (out[b, h] == 0).all()
+                continue
+            ref = _sdpa(q[b, h][None], Kc, Vc, 1 / np.sqrt(D))[0]
+            assert np.abs(out[b, h] - ref).max() < 1e-12
+
+
+def _loop_inputs(B=2, Hkv=2, Hq=4, T=40, S_=11, seed=3):
+    rng = np.random.default_rng(seed)
+    mk = lambda *s: rng.standard_normal(s).astype(np.float32).astype(np.float64)
+    kp = mk(B, Hkv, T, D) + np.where(np.arange(D) % 32 == 0, 4.0, 0.0)
+    return kp, mk(B, Hkv, T, D), mk(B, Hkv, S_, D) * 1.2, mk(B, Hkv, S_, D), mk(S_, B, Hq, D)
+
+
+def test_decode_loop_flushes_equal_a_one_shot_encode_with_the_stored_shift(codebooks):
+    """Residual window R = 4 over 11 decode steps: two flushes. Every flushed
+    token is encoded with the prompt's shift, so the cache equals a one-shot
+    encoding of the first 8 new tokens with that shift; 3 tokens stay."""
+    kp, vp, kn, vn, qs = _loop_inputs()
+    C = codebooks[4]
+    outs, st = O.decode_with_residual(kp, vp, kn, vn, qs, C, C, R=4)
+    assert st["n_quant"] == 40 + 8 and st["n_res"] == 3
+    for n, x in (("K", kn), ("V", vn)):
+        prompt = O.encode(kp if n == "K" else vp, C)
+        one = O.encode(x[:, :, :8], C, shift=prompt["o"])
+        assert np.array_equal(st[n]["codes"][:, :, :40], prompt["codes"])
+        assert np.array_equal(st[n]["codes"][:, :, 40:], one["codes"])
+        assert np.array_equal(st[n]["s2"][:, :, 40:], one["s2"])
+        assert np.array_equal(st[n]["o"], prompt["o"])
+
+
+def test_decode_loop_without_a_flush_attends_to_the_raw_new_tokens(codebooks):
+    """R above the number of steps: the new tokens stay at full precision, so
+    step s is SDPA over [dequantized prompt || the first s + 1 raw tokens]."""
+    kp, vp, kn, vn, qs = _loop_inputs(S_=5)
+    C = codebooks[8]
+    outs, st = O.decode_with_residual(kp, vp, kn, vn, qs, C, C, R=64)
+    assert st["n_res"] == 5
+    eK, eV = O.encode(kp, C), O.encode(vp, C)
+    Kh = O.dequant(eK["codes"], *O.stored(eK), C)
+    Vh = O.dequant(eV["codes"], *O.stored(eV), C)
+    G = qs.shape[2] // kp.shape[1]
+    for s in range(5):
+        for b in range(2):
+            for h in range(4):
+                Kc = np.concatenate([Kh[b, h // G], kn[b, h // G, :s + 1]])
+                Vc = np.concatenate([Vh[b, h // G], vn[b, h // G, :s + 1]])
+                ref = _sdpa(qs[s, b, h][None], Kc, Vc, 1 / np.sqrt(D))[0]
+                assert np.abs(outs[s, b, h] - ref).max() < 1e-12
+
+
+def test_decode_loop_with_a_one_token_window_quantizes_every_token(codebooks):
+    """R = 1: each new token is flushed at once, so every step attends over a
+    fully quantized cache with no residual."""
+    kp, vp, kn, vn, qs = _loop_inputs(S_=3)
+    C = codebooks[4]
+    outs, st = O.decode_with_residual(kp, vp, kn, vn, qs, C, C, R=1)
+    assert st["n_res"] == 0 and st["n_quant"] == 43
+    eK, eV = O.encode(kp, C), O.encode(vp, C)
+    for s in range(3):
+        fK = O.encode(kn[:, :, :s + 1], C, shift=eK["o"])
+        fV = O.encode(vn[:, :, :s + 1], C, shift=eV["o"])
+        cat = lambda a, b, k: np.concatenate([a[k], b[k]], axis=2)
+        Kh = O.dequant(cat(eK, fK, "codes"), cat(eK, fK, "s1").astype(np.float32),
+                       cat(eK, fK, "s2").astype(np.float32), eK["o"].astype(np.float32), C)
+        Vh = O.dequant(cat(eV, fV, "codes"), cat(eV, fV, "s1").astype(np.float32),
+                       cat(eV, fV, "s2").astype(np.float32), eV["o"].astype(np.float32), C)
+        ref = O.attention(qs[s], Kh, Vh)
+        assert np.abs(outs[s] - ref).max() < 1e-12
