@@ -10,6 +10,14 @@ CPU fallback: if the library is missing, loading raises.
     nsnq_encode(x, cb, cache)                      # prompt: shift computed
     nsnq_encode(x_new, cb, cache, t_offset=T, shift_mode=SHIFT_GIVEN)
     out = nsnq_attn_decode(q, k_cache, v_cache, k_cb, v_cb, seq_lens, max_len)
+
+With a full-precision residual window of R recent tokens (DecodeCache does
+the bookkeeping for sequences decoded in lock-step):
+
+    dc = DecodeCache(B, Hkv, cap, k_cb, v_cb, window=R)
+    dc.prefill(k_prompt, v_prompt)
+    dc.append(k_new, v_new)          # flushes (quantizes) a full window
+    out = dc.attend(q)
 """
 from __future__ import annotations
 
@@ -32,7 +40,8 @@ N_CENTROIDS = 256
 
 EXPORTED = ("nsnq_status_string", "nsnq_last_error", "nsnq_codebook_index_bytes",
             "nsnq_codebook_index_build", "nsnq_encode_workspace", "nsnq_encode", "nsnq_dequant",
-            "nsnq_attn_workspace", "nsnq_attn_decode", "nsnq_attn_decode_noalloc")
+            "nsnq_attn_workspace", "nsnq_attn_decode", "nsnq_attn_decode_res",
+            "nsnq_residual_write", "nsnq_attn_decode_noalloc")
 
 
 class NSNQError(RuntimeError):
@@ -49,6 +58,11 @@ class _Codebook(ctypes.Structure):
 class _Cache(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
                 ("shift", ctypes.c_void_p), ("cap", ctypes.c_int64)]
+
+
+class _Residual(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("dtype", ctypes.c_int),
+                ("lens", ctypes.c_void_p), ("cap", ctypes.c_int64)]
 
 
 _lib = None
@@ -84,6 +98,12 @@ def load(path: str = LIB_PATH):
     L.nsnq_attn_decode.argtypes = [vp, ci, _Cache, _Cache, _Codebook, _Codebook, vp, i64, ci, ci,
                                    ci, ci, ctypes.c_float, vp, ci, vp, sz, vp]
     L.nsnq_attn_decode.restype = ci
+    L.nsnq_attn_decode_res.argtypes = [vp, ci, _Cache, _Cache, _Codebook, _Codebook, vp, i64,
+                                       _Residual, ci, ci, ci, ci, ctypes.c_float, vp, ci, vp, sz,
+                                       vp]
+    L.nsnq_attn_decode_res.restype = ci
+    L.nsnq_residual_write.argtypes = [vp, ci, ci, ci, i64, ci, i64, i64, i64, i64, vp, ci, i64, vp]
+    L.nsnq_residual_write.restype = ci
     L.nsnq_attn_decode_noalloc.argtypes = [vp, ci, _Cache, _Cache, _Codebook, _Codebook, vp, i64,
                                            ci, ci, ci, ci, ctypes.c_float, vp, ci, vp]
     L.nsnq_attn_decode_noalloc.restype = ci
@@ -256,3 +276,134 @@ def nsnq_attn_decode_noalloc(q: torch.Tensor, k_cache: Cache, v_cache: Cache, k_
                                            Hkv, D, float(softmax_scale), _ptr(out),
                                            _dtype_code(out), _stream(stream)))
     return out
+
+
+@dataclasses.dataclass
+class Residual:
+    """Full-precision residual window: k, v [B][Hkv][cap][D] (fp32 or bf16)
+    and lens int32 [B] (tokens held per sequence)."""
+    k: torch.Tensor
+    v: torch.Tensor
+    lens: torch.Tensor
+
+    @property
+    def cap(self) -> int:
+        return int(self.k.shape[2])
+
+    @classmethod
+    def empty(cls, B: int, H: int, cap: int, dtype=torch.bfloat16, device="cuda",
+              D: int = HEAD_DIM):
+        return cls(torch.zeros(B, H, cap, D, dtype=dtype, device=device),
+                   torch.zeros(B, H, cap, D, dtype=dtype, device=device),
+                   torch.zeros(B, dtype=torch.int32, device=device))
+
+    def _c(self) -> _Residual:
+        return _Residual(_ptr(self.k), _ptr(self.v), _dtype_code(self.k), _ptr(self.lens),
+                         self.cap)
+
+
+def nsnq_residual_write(x: torch.Tensor, buf: torch.Tensor, t_offset: int, stream=None):
+    """Copy x [B][H][T][D] into rows [t_offset, t_offset + T) of buf [B][H][cap][D]."""
+    B, H, T, D = x.shape
+    if x.stride(3) != 1 or not buf.is_contiguous():
+        raise ValueError("x must have contiguous channels and buf must be contiguous")
+    if tuple(buf.shape[:2]) != (B, H) or buf.shape[3] != D:
+        raise ValueError(f"buf shape {tuple(buf.shape)} does not match x {tuple(x.shape)}")
+    _check(load().nsnq_residual_write(_ptr(x), _dtype_code(x), B, H, T, D, x.stride(0),
+                                      x.stride(1), x.stride(2), t_offset, _ptr(buf),
+                                      _dtype_code(buf), int(buf.shape[2]), _stream(stream)))
+
+
+def nsnq_attn_decode_res(q: torch.Tensor, k_cache: Cache, v_cache: Cache, k_cb: Codebook,
+                         v_cb: Codebook, seq_lens: torch.Tensor, max_len: int, Hkv: int,
+                         res: Optional[Residual], softmax_scale: float = 0.0,
+                         out_dtype: torch.dtype = torch.bfloat16,
+                         out: Optional[torch.Tensor] = None,
+                         workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Decode step over [quantized tokens || residual window tokens]."""
+    B, Hq, D = q.shape
+    if out is None:
+        out = torch.empty(B, Hq, D, dtype=out_dtype, device=q.device)
+    if workspace is None:
+        workspace = _workspace(nsnq_attn_workspace(B, Hq, Hkv, max_len, D), q.device)
+    if seq_lens.dtype != torch.int32 or (res is not None and res.lens.dtype != torch.int32):
+        raise TypeError("seq_lens and res.lens must be int32")
+    rc = res._c() if res is not None else _Residual(None, None, NSNQ_BF16, None, 0)
+    _check(load().nsnq_attn_decode_res(_ptr(q), _dtype_code(q), k_cache._c(), v_cache._c(),
+                                       k_cb._c(), v_cb._c(), _ptr(seq_lens), max_len, rc, B, Hq,
+                                       Hkv, D, float(softmax_scale), _ptr(out), _dtype_code(out),
+                                       _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(),
+                                       _stream(stream)))
+    return out
+
+
+class DecodeCache:
+    """Quantized K/V caches plus a full-precision residual window of `window`
+    tokens, for sequences decoded in lock-step (one length for the batch).
+
+    prefill() quantizes the whole prompt (shift computed over it); append()
+    puts the new token in the window and, once the window holds `window`
+    tokens, flushes it: the window is quantized with the stored shift and
+    appended to the caches, and the window empties. attend() runs one
+    decode step over [quantized || window]. Bookkeeping only: every step
+    runs in the library's kernels."""
+
+    def __init__(self, B: int, Hkv: int, cap: int, k_cb: Codebook, v_cb: Codebook, window: int,
+                 res_dtype=torch.bfloat16, device="cuda", flags: int = ENCODE_DEFAULT):
+        if window <= 0:
+            raise ValueError("window must be positive")
+        self.B, self.Hkv, self.window, self.flags = B, Hkv, window, flags
+        self.k_cb, self.v_cb = k_cb, v_cb
+        self.k = Cache.empty(B, Hkv, cap, k_cb.sub_dim, device)
+        self.v = Cache.empty(B, Hkv, cap, v_cb.sub_dim, device)
+        self.res = Residual.empty(B, Hkv, window, res_dtype, device)
+        self.seq_lens = torch.zeros(B, dtype=torch.int32, device=device)
+        self.n_quant = 0
+        self.n_res = 0
+        self._prefilled = False
+
+    def prefill(self, k: torch.Tensor, v: torch.Tensor, stream=None):
+        if self._prefilled:
+            raise RuntimeError("prefill() was already called")
+        T = int(k.shape[2])
+        nsnq_encode(k, self.k_cb, self.k, stream=stream, flags=self.flags)
+        nsnq_encode(v, self.v_cb, self.v, stream=stream, flags=self.flags)
+        self.n_quant = T
+        self.seq_lens.fill_(T)
+        self._prefilled = True
+
+    def append(self, k_new: torch.Tensor, v_new: torch.Tensor, stream=None):
+        """k_new, v_new [B][Hkv][D] or [B][Hkv][1][D]: one token per sequence."""
+        if not self._prefilled:
+            raise RuntimeError("prefill() first: the window is quantized with the prompt's shift")
+        if k_new.dim() == 3:
+            k_new, v_new = k_new.unsqueeze(2), v_new.unsqueeze(2)
+        nsnq_residual_write(k_new, self.res.k, self.n_res, stream)
+        nsnq_residual_write(v_new, self.res.v, self.n_res, stream)
+        self.n_res += 1
+        if self.n_res == self.window:
+            self.flush(stream)
+        else:
+            self.res.lens.fill_(self.n_res)
+
+    def flush(self, stream=None):
+        if self.n_res == 0:
+            return
+        if self.n_quant + self.n_res > self.k.cap:
+            raise RuntimeError("quantized cache is full")
+        n = self.n_res
+        nsnq_encode(self.res.k[:, :, :n], self.k_cb, self.k, t_offset=self.n_quant,
+                    shift_mode=SHIFT_GIVEN, stream=stream, flags=self.flags)
+        nsnq_encode(self.res.v[:, :, :n], self.v_cb, self.v, t_offset=self.n_quant,
+                    shift_mode=SHIFT_GIVEN, stream=stream, flags=self.flags)
+        self.n_quant += n
+        self.n_res = 0
+        self.seq_lens.fill_(self.n_quant)
+        self.res.lens.fill_(0)
+
+    def attend(self, q: torch.Tensor, softmax_scale: float = 0.0,
+               out_dtype: torch.dtype = torch.bfloat16, stream=None) -> torch.Tensor:
+        return nsnq_attn_decode_res(q, self.k, self.v, self.k_cb, self.v_cb, self.seq_lens,
+                                    self.n_quant, self.Hkv, self.res, softmax_scale, out_dtype,
+                                    stream=stream)

@@ -202,11 +202,12 @@ size_t nsnq_attn_workspace(int B, int Hq, int Hkv, int D, int64_t max_len) {
     return nsnq::plan_attention(B, Hq, Hkv, max_len).total;
 }
 
-nsnq_status nsnq_attn_decode(const void* q, nsnq_dtype q_dtype, nsnq_cache k_cache,
-                             nsnq_cache v_cache, nsnq_codebook k_cb, nsnq_codebook v_cb,
-                             const int32_t* seq_lens, int64_t max_len, int B, int Hq, int Hkv,
-                             int D, float softmax_scale, void* out, nsnq_dtype out_dtype,
-                             void* workspace, size_t workspace_bytes, nsnq_stream stream) {
+nsnq_status nsnq_attn_decode_res(const void* q, nsnq_dtype q_dtype, nsnq_cache k_cache,
+                                 nsnq_cache v_cache, nsnq_codebook k_cb, nsnq_codebook v_cb,
+                                 const int32_t* seq_lens, int64_t max_len, nsnq_residual res,
+                                 int B, int Hq, int Hkv, int D, float softmax_scale, void* out,
+                                 nsnq_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                                 nsnq_stream stream) {
     if (D != nsnq::kHeadDim) return fail(NSNQ_ERR_UNSUPPORTED, "D = %d (only 128 is supported)", D);
     if ((q_dtype != NSNQ_F32 && q_dtype != NSNQ_BF16) ||
         (out_dtype != NSNQ_F32 && out_dtype != NSNQ_BF16))
@@ -227,6 +228,15 @@ nsnq_status nsnq_attn_decode(const void* q, nsnq_dtype q_dtype, nsnq_cache k_cac
     if (max_len < 0 || max_len > k_cache.cap || max_len > v_cache.cap)
         return fail(NSNQ_ERR_INVALID_ARG, "max_len = %lld must be in [0, min(cap)]",
                     (long long)max_len);
+    if (res.cap < 0) return fail(NSNQ_ERR_INVALID_ARG, "res.cap = %lld < 0", (long long)res.cap);
+    if (res.cap > 0) {
+        if (res.dtype != NSNQ_F32 && res.dtype != NSNQ_BF16)
+            return fail(NSNQ_ERR_UNSUPPORTED, "res.dtype must be NSNQ_F32 or NSNQ_BF16");
+        if (B > 0 && (!res.k || !res.v || !res.lens))
+            return fail(NSNQ_ERR_INVALID_ARG, "res.k, res.v or res.lens is NULL");
+        if (!aligned(res.k, 16) || !aligned(res.v, 16) || !aligned(res.lens, 4))
+            return fail(NSNQ_ERR_INVALID_ARG, "res.k and res.v must be 16-byte aligned");
+    }
     if (B == 0) return ok();
     if (!q || !out || !seq_lens) return fail(NSNQ_ERR_INVALID_ARG, "q, out or seq_lens is NULL");
     if (!aligned(q, 16) || !aligned(out, 16) || !aligned(seq_lens, 4))
@@ -250,8 +260,56 @@ nsnq_status nsnq_attn_decode(const void* q, nsnq_dtype q_dtype, nsnq_cache k_cac
     a.out = out; a.out_bf16 = out_dtype == NSNQ_BF16;
     a.part = static_cast<float*>(workspace);
     a.plan = plan;
+    if (res.cap > 0) {
+        a.rk = res.k; a.rv = res.v; a.r_bf16 = res.dtype == NSNQ_BF16;
+        a.res_lens = res.lens; a.rcap = res.cap;
+    }
     cudaError_t e = nsnq::launch_attention(a, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+    return ok();
+}
+
+nsnq_status nsnq_attn_decode(const void* q, nsnq_dtype q_dtype, nsnq_cache k_cache,
+                             nsnq_cache v_cache, nsnq_codebook k_cb, nsnq_codebook v_cb,
+                             const int32_t* seq_lens, int64_t max_len, int B, int Hq, int Hkv,
+                             int D, float softmax_scale, void* out, nsnq_dtype out_dtype,
+                             void* workspace, size_t workspace_bytes, nsnq_stream stream) {
+    nsnq_residual none{};
+    return nsnq_attn_decode_res(q, q_dtype, k_cache, v_cache, k_cb, v_cb, seq_lens, max_len, none,
+                                B, Hq, Hkv, D, softmax_scale, out, out_dtype, workspace,
+                                workspace_bytes, stream);
+}
+
+nsnq_status nsnq_residual_write(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t T, int D,
+                                int64_t stride_b, int64_t stride_h, int64_t stride_t,
+                                int64_t t_offset, void* buf, nsnq_dtype buf_dtype, int64_t cap,
+                                nsnq_stream stream) {
+    if (D != nsnq::kHeadDim) return fail(NSNQ_ERR_UNSUPPORTED, "D = %d (only 128 is supported)", D);
+    if ((x_dtype != NSNQ_F32 && x_dtype != NSNQ_BF16) ||
+        (buf_dtype != NSNQ_F32 && buf_dtype != NSNQ_BF16))
+        return fail(NSNQ_ERR_UNSUPPORTED, "x/buf dtype must be NSNQ_F32 or NSNQ_BF16");
+    if (B < 0 || H < 0 || T < 0 || cap < 0)
+        return fail(NSNQ_ERR_INVALID_ARG, "negative size B=%d H=%d T=%lld cap=%lld", B, H,
+                    (long long)T, (long long)cap);
+    if (t_offset < 0 || t_offset > cap || T > cap - t_offset)
+        return fail(NSNQ_ERR_INVALID_ARG, "rows [%lld, %lld) exceed capacity %lld",
+                    (long long)t_offset, (long long)(t_offset + T), (long long)cap);
+    if (B == 0 || H == 0 || T == 0) return ok();
+    if (!x || !buf) return fail(NSNQ_ERR_INVALID_ARG, "x or buf is NULL");
+    const int64_t esz = x_dtype == NSNQ_BF16 ? 2 : 4;
+    if (!aligned(x, 16) || (stride_b * esz) % 16 || (stride_h * esz) % 16 || (stride_t * esz) % 16)
+        return fail(NSNQ_ERR_INVALID_ARG, "x and its strides must be 16-byte aligned");
+    if (stride_b < 0 || stride_h < 0 || stride_t < D)
+        return fail(NSNQ_ERR_INVALID_ARG, "strides must be non-negative with stride_t >= D");
+    if (!aligned(buf, 16)) return fail(NSNQ_ERR_INVALID_ARG, "buf must be 16-byte aligned");
+    nsnq::ResWriteArgs a{};
+    a.x = x; a.x_bf16 = x_dtype == NSNQ_BF16;
+    a.B = B; a.H = H; a.T = T;
+    a.sb = stride_b; a.sh = stride_h; a.st = stride_t;
+    a.t_offset = t_offset;
+    a.buf = buf; a.buf_bf16 = buf_dtype == NSNQ_BF16; a.cap = cap;
+    cudaError_t e = nsnq::launch_residual_write(a, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "residual write launch");
     return ok();
 }
 

@@ -349,10 +349,63 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a)
   }
 }
 
+// Residual tokens scored per combine pass (one score per token in shared memory).
+constexpr int kResChunk = 256;
+
 // Merge the splits of one (batch, query head): rescale by exp2(m_s - M),
-// apply H to the rotated-domain sum, add beta * o_V, divide by l.
+// apply H to the rotated-domain sum, add beta * o_V, divide by l. Tokens of
+// the full-precision residual window join the same softmax here: their
+// scores q . k * scale are taken in fp32 chunk by chunk (an online max over
+// the chunks), their values accumulate in the original domain.
+template <typename RT>
+__device__ __forceinline__ void combine_residual(const AttnArgs& a, int b, int qh, int kvh,
+                                                 int64_t rlen, float& M, float& acc, float& L,
+                                                 float& Be, float& racc, float* qs, float* ps) {
+    const int c = threadIdx.x, lane = lane_id(), warp = c >> 5;
+    const int64_t qoff = ((int64_t)b * a.Hq + qh) * kD + c;
+    qs[c] = a.q_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(a.q)[qoff])
+                     : reinterpret_cast<const float*>(a.q)[qoff];
+    __syncthreads();
+    float q4[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) q4[r] = qs[4 * lane + r];
+    const int64_t base = ((int64_t)b * a.Hkv + kvh) * a.rcap;
+    const RT* K = reinterpret_cast<const RT*>(a.rk) + base * kD;
+    const RT* V = reinterpret_cast<const RT*>(a.rv) + base * kD;
+    for (int64_t t0 = 0; t0 < rlen; t0 += kResChunk) {
+        const int n = (int)(rlen - t0 < kResChunk ? rlen - t0 : kResChunk);
+        for (int i = warp; i < n; i += kD / 32) {
+            float k4[4];
+            load4(K + (t0 + i) * kD + 4 * lane, k4);
+            float d = fmaf(q4[3], k4[3], fmaf(q4[2], k4[2], fmaf(q4[1], k4[1], q4[0] * k4[0])));
+            d = warp_sum(d);
+            if (lane == 0) ps[i] = d * a.scale_log2;
+        }
+        __syncthreads();
+        float mc = -INFINITY;
+        for (int i = 0; i < n; ++i) mc = fmaxf(mc, ps[i]);
+        const float Mn = fmaxf(M, mc);
+        const float f = M == -INFINITY ? 0.f : exp2f(M - Mn);
+        acc *= f; L *= f; Be *= f; racc *= f;
+        M = Mn;
+        __syncthreads();  // every thread has read the scores
+        for (int i = c; i < n; i += kD) ps[i] = exp2f(ps[i] - M);
+        __syncthreads();
+        for (int i = 0; i < n; ++i) {
+            const float p = ps[i];
+            L += p;
+            const RT vv = V[(t0 + i) * kD + c];
+            racc = fmaf(p, (float)vv, racc);
+        }
+        __syncthreads();  // before the next chunk overwrites ps
+    }
+}
+
 __global__ void __launch_bounds__(kD) attn_combine_kernel(AttnArgs a) {
     __shared__ float As[kD];
+    __shared__ float Rs[kD];
+    __shared__ float qs[kD];
+    __shared__ float ps[kResChunk];
     __shared__ float LB[2];
     const int bq = blockIdx.x;
     const int b = bq / a.Hq, qh = bq % a.Hq;
@@ -367,7 +420,7 @@ __global__ void __launch_bounds__(kD) attn_combine_kernel(AttnArgs a) {
     const int c = threadIdx.x;
     float M = -INFINITY;
     for (int s = 0; s < used; ++s) M = fmaxf(M, P[(int64_t)s * kPartStride + kD]);
-    float acc = 0.f, L = 0.f, Be = 0.f;
+    float acc = 0.f, L = 0.f, Be = 0.f, racc = 0.f;
     if (M != -INFINITY) {
         for (int s = 0; s < used; ++s) {
             const float* Ps = P + (int64_t)s * kPartStride;
@@ -378,7 +431,16 @@ __global__ void __launch_bounds__(kD) attn_combine_kernel(AttnArgs a) {
             Be = fmaf(f, Ps[kD + 2], Be);
         }
     }
+    int64_t rlen = a.rcap > 0 ? (int64_t)a.res_lens[b] : 0;
+    rlen = rlen < 0 ? 0 : (rlen > a.rcap ? a.rcap : rlen);
+    if (rlen > 0) {  // block-uniform
+        if (a.r_bf16)
+            combine_residual<__nv_bfloat16>(a, b, qh, kvh, rlen, M, acc, L, Be, racc, qs, ps);
+        else
+            combine_residual<float>(a, b, qh, kvh, rlen, M, acc, L, Be, racc, qs, ps);
+    }
     As[c] = acc;
+    Rs[c] = racc;
     if (c == 0) { LB[0] = L; LB[1] = Be; }
     __syncthreads();
     if (threadIdx.x >= 32) return;
@@ -390,11 +452,12 @@ __global__ void __launch_bounds__(kD) attn_combine_kernel(AttnArgs a) {
     const float Lt = LB[0], Bt = LB[1];
     const float inv = Lt > 0.f ? 1.0f / Lt : 0.f;
     const float4 o = reinterpret_cast<const float4*>(a.vshift + ((int64_t)b * a.Hkv + kvh) * kD)[lane];
+    const float4 rr = reinterpret_cast<const float4*>(Rs)[lane];
     float r4[4];
-    r4[0] = fmaf(Bt, o.x, v[0] * kRsqrtD) * inv;
-    r4[1] = fmaf(Bt, o.y, v[1] * kRsqrtD) * inv;
-    r4[2] = fmaf(Bt, o.z, v[2] * kRsqrtD) * inv;
-    r4[3] = fmaf(Bt, o.w, v[3] * kRsqrtD) * inv;
+    r4[0] = (fmaf(Bt, o.x, v[0] * kRsqrtD) + rr.x) * inv;
+    r4[1] = (fmaf(Bt, o.y, v[1] * kRsqrtD) + rr.y) * inv;
+    r4[2] = (fmaf(Bt, o.z, v[2] * kRsqrtD) + rr.z) * inv;
+    r4[3] = (fmaf(Bt, o.w, v[3] * kRsqrtD) + rr.w) * inv;
     if (a.out_bf16) {
         uint2 pk;
         pk.x = (uint32_t)f32_to_bf16_rn(r4[0]) | ((uint32_t)f32_to_bf16_rn(r4[1]) << 16);

@@ -108,7 +108,26 @@ struct AttnArgs {
     int out_bf16;
     float* part;
     AttnPlan plan;
+    // full-precision residual window ([B][Hkv][rcap][D]; rcap = 0: none)
+    const void* rk;
+    const void* rv;
+    int r_bf16;
+    const int32_t* res_lens;
+    int64_t rcap;
 };
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s);
+
+struct ResWriteArgs {
+    const void* x;
+    int x_bf16;
+    int B, H;
+    int64_t T;
+    int64_t sb, sh, st;
+    int64_t t_offset;
+    void* buf;
+    int buf_bf16;
+    int64_t cap;
+};
+cudaError_t launch_residual_write(const ResWriteArgs& a, cudaStream_t s);
 
 }  // namespace nsnq

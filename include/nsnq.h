@@ -141,8 +141,8 @@ size_t nsnq_encode_workspace(int B, int H, int64_t T, int D);
  *   workspace device scratch of at least nsnq_encode_workspace(B, H, T, D)
  *             bytes, 256-byte aligned.
  * Codes equal the nearest codeword of the exact (fp64) transformed token;
- * sub-vectors whose two best fp32 distances are within a relative 1e-4 are
- * re-decided in fp64. Stored s1, s2, o are fp32 roundings. A zero-norm
+ * sub-vectors whose two best fp32 distances are within a relative 2e-5
+ * (sub_dim 4) or 1e-4 (sub_dim 8) are re-decided in fp64. Stored s1, s2, o are fp32 roundings. A zero-norm
  * token (or a zero residual after the shift) maps to the zero vector with
  * s = 0. T = 0 is a no-op.
  */
@@ -186,6 +186,50 @@ nsnq_status nsnq_attn_decode(const void* q, nsnq_dtype q_dtype, nsnq_cache k_cac
                              const int32_t* seq_lens, int64_t max_len, int B, int Hq, int Hkv,
                              int D, float softmax_scale, void* out, nsnq_dtype out_dtype,
                              void* workspace, size_t workspace_bytes, nsnq_stream stream);
+
+/*
+ * Full-precision residual window (Methodology §4, Implementation Details,
+ * Residuals): the most recent tokens of each sequence, kept unquantized
+ * until the window fills; then they are quantized (nsnq_encode with
+ * NSNQ_SHIFT_GIVEN on the window, t_offset = the sequence's quantized
+ * length) and the window is emptied.
+ */
+typedef struct {
+    const void* k;        /* device [B][Hkv][cap][D] of dtype, 16-byte aligned */
+    const void* v;        /* device [B][Hkv][cap][D] of dtype, 16-byte aligned */
+    nsnq_dtype dtype;     /* NSNQ_F32 or NSNQ_BF16 */
+    const int32_t* lens;  /* device int32 [B]: residual tokens of sequence b */
+    int64_t cap;          /* rows per (batch, kv-head) */
+} nsnq_residual;
+
+/*
+ * nsnq_attn_decode_res -- nsnq_attn_decode over the first seq_lens[b]
+ * quantized tokens followed by the first min(max(res.lens[b], 0), res.cap)
+ * residual tokens of each sequence, one softmax over both:
+ *   out = (H A + beta o_V + sum_r p_r v_r) / (sum_t p_t + sum_r p_r),
+ * residual scores scale * q . k_r in fp32 from the stored K rows.
+ * res.cap = 0 (pointers may then be NULL) is exactly nsnq_attn_decode.
+ * A sequence with no token at all gets a zero output. Other arguments,
+ * the workspace and the errors are those of nsnq_attn_decode.
+ */
+nsnq_status nsnq_attn_decode_res(const void* q, nsnq_dtype q_dtype, nsnq_cache k_cache,
+                                 nsnq_cache v_cache, nsnq_codebook k_cb, nsnq_codebook v_cb,
+                                 const int32_t* seq_lens, int64_t max_len, nsnq_residual res,
+                                 int B, int Hq, int Hkv, int D, float softmax_scale, void* out,
+                                 nsnq_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                                 nsnq_stream stream);
+
+/*
+ * nsnq_residual_write -- copy T tokens of every (batch, head) into rows
+ * [t_offset, t_offset + T) of a residual buffer buf [B][H][cap][D] of
+ * buf_dtype, converting (fp32 to bf16 rounds to nearest even; the other
+ * directions are exact). x is laid out as for nsnq_encode. The rows must
+ * fit: 0 <= t_offset and t_offset + T <= cap. T = 0 is a no-op.
+ */
+nsnq_status nsnq_residual_write(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t T, int D,
+                                int64_t stride_b, int64_t stride_h, int64_t stride_t,
+                                int64_t t_offset, void* buf, nsnq_dtype buf_dtype, int64_t cap,
+                                nsnq_stream stream);
 
 /*
  * nsnq_attn_decode_noalloc -- nsnq_attn_decode for callers that cannot

@@ -200,7 +200,7 @@ def attention_with_residual(q: np.ndarray, Khat: np.ndarray, Vhat: np.ndarray, s
 
 def decode_with_residual(k_prompt: np.ndarray, v_prompt: np.ndarray, k_new: np.ndarray,
                          v_new: np.ndarray, queries: np.ndarray, Ck: np.ndarray, Cv: np.ndarray,
-                         R: int, scale: Optional[float] = None):
+                         R: int, scale: Optional[float] = None, adaptive_scale: bool = False):
     """The serving loop with a residual window of R tokens (Methodology §4,
     Implementation Details, Residuals), every sequence in lock-step.
 
@@ -212,10 +212,12 @@ def decode_with_residual(k_prompt: np.ndarray, v_prompt: np.ndarray, k_new: np.n
     query queries[s] [B][Hq][d] then attends over [quantized || residual].
     Inputs are the exact values of the I/O type. Returns (outputs fp64
     [S][B][Hq][d], final state dict: codes/s1/s2 per tensor over the
-    quantized tokens, o, number of quantized and residual tokens)."""
+    quantized tokens, o, number of quantized and residual tokens).
+    adaptive_scale applies the scale adjustment at every encode."""
     B, Hkv, T, d = k_prompt.shape
     S = k_new.shape[2]
-    enc = {"K": encode(k_prompt, Ck), "V": encode(v_prompt, Cv)}
+    enc = {"K": encode(k_prompt, Ck, adaptive_scale=adaptive_scale),
+           "V": encode(v_prompt, Cv, adaptive_scale=adaptive_scale)}
     o = {n: enc[n]["o"] for n in enc}
     codes = {n: [enc[n]["codes"]] for n in enc}
     s1 = {n: [enc[n]["s1"]] for n in enc}
@@ -229,7 +231,7 @@ def decode_with_residual(k_prompt: np.ndarray, v_prompt: np.ndarray, k_new: np.n
             res[n] = np.concatenate([res[n], new[n][:, :, s:s + 1]], axis=2)
         if res["K"].shape[2] == R:
             for n in res:
-                e = encode(res[n], C[n], shift=o[n])
+                e = encode(res[n], C[n], shift=o[n], adaptive_scale=adaptive_scale)
                 codes[n].append(e["codes"])
                 s1[n].append(e["s1"])
                 s2[n].append(e["s2"])

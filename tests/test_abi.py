@@ -140,6 +140,51 @@ def test_attention_validation(lib):
     assert lib.nsnq_attn_workspace(2, 8, 3, 128, 100) == 0
 
 
+def _attn_res(lib, res, **kw):
+    a = dict(q=FAKE, qdt=nsnq.NSNQ_BF16, kc=_cache(), vc=_cache(), kcb=_cb(4), vcb=_cb(8),
+             lens=FAKE, max_len=100, B=2, Hq=8, Hkv=2, D=128, scale=0.0, out=FAKE,
+             odt=nsnq.NSNQ_BF16, ws=FAKE, wsb=1 << 24)
+    a.update(kw)
+    return lib.nsnq_attn_decode_res(a["q"], a["qdt"], a["kc"], a["vc"], a["kcb"], a["vcb"],
+                                    a["lens"], a["max_len"], res, a["B"], a["Hq"], a["Hkv"],
+                                    a["D"], a["scale"], a["out"], a["odt"], a["ws"], a["wsb"],
+                                    None)
+
+
+def test_residual_attention_validation(lib):
+    R = lambda k=FAKE, v=FAKE, dt=nsnq.NSNQ_BF16, lens=FAKE, cap=16: nsnq._Residual(k, v, dt, lens, cap)
+    assert _attn_res(lib, R(cap=-1)) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert _attn_res(lib, R(k=None)) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert _attn_res(lib, R(lens=None)) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert _attn_res(lib, R(v=FAKE + 8)) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert _attn_res(lib, R(dt=7)) == nsnq.NSNQ_ERR_UNSUPPORTED
+    assert _attn_res(lib, R(), Hq=6, Hkv=4) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert _attn_res(lib, R(), wsb=16) == nsnq.NSNQ_ERR_WORKSPACE
+    assert _attn_res(lib, R(), B=0) == nsnq.NSNQ_OK
+    # no window: NULL pointers are accepted (the call is nsnq_attn_decode)
+    assert _attn_res(lib, R(k=None, v=None, lens=None, cap=0), B=0) == nsnq.NSNQ_OK
+
+
+def test_residual_write_validation(lib):
+    def f(**kw):
+        a = dict(x=FAKE, dt=nsnq.NSNQ_BF16, B=2, H=2, T=1, D=128, sb=512, sh=256, st=128, off=3,
+                 buf=FAKE, bdt=nsnq.NSNQ_BF16, cap=4)
+        a.update(kw)
+        return lib.nsnq_residual_write(a["x"], a["dt"], a["B"], a["H"], a["T"], a["D"], a["sb"],
+                                       a["sh"], a["st"], a["off"], a["buf"], a["bdt"], a["cap"],
+                                       None)
+    assert f(off=4) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert f(T=2) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert f(off=-1) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert f(D=64) == nsnq.NSNQ_ERR_UNSUPPORTED
+    assert f(bdt=5) == nsnq.NSNQ_ERR_UNSUPPORTED
+    assert f(x=None) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert f(buf=FAKE + 2) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert f(st=100) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert f(sh=12) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert f(T=0) == nsnq.NSNQ_OK
+
+
 def test_binding_has_no_fallback(tmp_path):
     """The binding raises when the library file is absent; it never computes on the CPU."""
     import importlib
