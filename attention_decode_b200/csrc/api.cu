@@ -6,6 +6,7 @@
 
 #include "../../include/nsnq.h"
 #include "internal.h"
+#include "vq_index.cuh"
 
 namespace {
 
@@ -100,7 +101,8 @@ nsnq_status nsnq_codebook_index_build(nsnq_codebook cb, void* index, size_t inde
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return cuda_fail(e, "index build");
     if (hdr[2] != 0)
-        return fail(NSNQ_ERR_UNSUPPORTED, "codebook index needs %u list entries (limit 65535)", hdr[1]);
+        return fail(NSNQ_ERR_UNSUPPORTED, "codebook index needs %u list entry pairs (limit %d)", hdr[1],
+                    nsnq::kMaxPairs);
     return ok();
 }
 

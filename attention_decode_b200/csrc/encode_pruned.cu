@@ -30,7 +30,7 @@ constexpr size_t kSmShift = kSmReps + size_t(kNC) * 8 * 16;   // float [warps][1
 constexpr size_t kSmHash = kSmShift + size_t(kPrunedThreads / 32) * 136 * 4;
 constexpr size_t kSmOffsets = kSmHash + 16;                    // uint16 [kCells + 1]
 constexpr size_t kSmEntries = kSmOffsets + kIdxSmemOffsetsBytes;
-constexpr size_t kSmBytes = kSmEntries + size_t(kMaxEntries + 1) * 2;
+constexpr size_t kSmBytes = kSmEntries + size_t(kMaxPairs) * 4;
 
 __device__ __forceinline__ uint64_t pk(float a, float b) {
     uint64_t r;
@@ -161,14 +161,11 @@ __device__ __noinline__ void exact_path(const XT* xrow, const double* o64, const
         if ((my_mask >> j) & 1u) {
             int cell = 0;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                int bi = __float2int_rd(fmaf((float)w[i], kInvW, kBinBias));
-                bi = min(max(bi, 0), kNb - 1);
-                cell = cell * kNb + bi;
-            }
+            for (int i = 0; i < 4; ++i) cell = cell * kNb + bin_of((float)w[i]);
             double bd = INFINITY;
             int bi = 0;
-            for (uint32_t q = offs[cell]; q < offs[cell + 1]; ++q) {
+            // every entry of the list, the padding codeword included (it never wins)
+            for (uint32_t q = 2u * offs[cell]; q < 2u * offs[cell + 1]; ++q) {
                 const int c = ents[q] & 0xff;
                 const float4 cv = reps[c * 8];
                 const double e0 = w[0] - (double)cv.x, e1 = w[1] - (double)cv.y;
@@ -200,14 +197,7 @@ struct Walk {
 
     __device__ __forceinline__ void init(float w0, float w1, float w2, float w3,
                                          const uint16_t* offs) {
-        int cell = 0;
-        const float wv[4] = {w0, w1, w2, w3};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            int bi = __float2int_rd(fmaf(wv[i], kInvW, kBinBias));
-            bi = min(max(bi, 0), kNb - 1);
-            cell = cell * kNb + bi;
-        }
+        const int cell = ((bin_of(w0) * kNb + bin_of(w1)) * kNb + bin_of(w2)) * kNb + bin_of(w3);
         p = offs[cell];
         e = offs[cell + 1];
         w01 = pk(w0, w1);
@@ -215,19 +205,18 @@ struct Walk {
         d1 = INFINITY; d2 = INFINITY; i1 = 0;
     }
 
-    // Evaluate up to two more entries (the second against the band of the
+    // Evaluate the next pair of entries (the second against the band of the
     // best distance before the first, which costs at most one extra
     // evaluation and never skips a contender); marks the walk finished
     // (p = e) once the next lower bound leaves the band or the list ends.
-    __device__ __forceinline__ void step(const uint16_t* ents, const float4* myrep) {
+    __device__ __forceinline__ void step(const uint32_t* pairs, const float4* myrep) {
         if (p >= e) return;
-        const uint32_t ent0 = ents[p];
-        const bool has1 = p + 1 < e;
-        const uint32_t ent1 = has1 ? ents[p + 1] : 0u;
+        const uint32_t pr = pairs[p];
+        const uint32_t ent0 = pr & 0xffffu, ent1 = pr >> 16;
         // lower bounds are floor(lb * 64) in the high byte: compare in integers
         const uint32_t lim = (uint32_t)fminf(fmaf(d1, (1.0f + kTieRel) * kLbScale, kTieAbs * kLbScale), 1.0e6f);
         if ((ent0 >> 8) > lim) { p = e; return; }
-        const bool take1 = has1 && (ent1 >> 8) <= lim;
+        const bool take1 = (ent1 >> 8) <= lim;
         const float4 cv0 = myrep[(ent0 & 0xff) * 8];
         const float4 cv1 = myrep[(ent1 & 0xff) * 8];
         const uint64_t a01 = sub2(w01, pk(cv0.x, cv0.y)), a23 = sub2(w23, pk(cv0.z, cv0.w));
@@ -242,7 +231,7 @@ struct Walk {
         d2 = fminf(d2, fmaxf(d1, dB));
         i1 = dB < d1 ? (int)(ent1 & 0xff) : i1;
         d1 = fminf(d1, dB);
-        p = take1 ? p + 2 : e;
+        p = take1 ? p + 1 : e;
     }
 
     __device__ __forceinline__ bool tie() const { return (d2 - d1) <= fmaf(kTieRel, d1, kTieAbs); }
@@ -258,20 +247,21 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
     float* shift_s = reinterpret_cast<float*>(sm + kSmShift);
     const uint16_t* offs = reinterpret_cast<const uint16_t*>(sm + kSmOffsets);
     const uint16_t* ents = reinterpret_cast<const uint16_t*>(sm + kSmEntries);
+    const uint32_t* pairs = reinterpret_cast<const uint32_t*>(sm + kSmEntries);
     const int tid = threadIdx.x, lane = lane_id();
     const int half = lane & 1;
     const unsigned pair_mask = 3u << (lane & 30);
 
     // ---- stage the index and the replicated codebook ----
     const IndexHeader* hdr = reinterpret_cast<const IndexHeader*>(a.index);
-    const uint32_t n_ent = min(hdr->n_entries, (uint32_t)kMaxEntries);
+    const uint32_t n_pairs = min(hdr->n_pairs, (uint32_t)kMaxPairs);
     unsigned* hash_s = reinterpret_cast<unsigned*>(sm + kSmHash);
     if (tid == 0) *hash_s = 0u;
     __syncthreads();
     {
         const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.index) + kIdxOffsets);
         uint4* dst = reinterpret_cast<uint4*>(sm + kSmOffsets);
-        const size_t nbytes = kIdxSmemOffsetsBytes + ((size_t)n_ent * 2 + 15) / 16 * 16;
+        const size_t nbytes = kIdxSmemOffsetsBytes + ((size_t)n_pairs * 4 + 15) / 16 * 16;
         for (size_t i = tid; i < nbytes / 16; i += kPrunedThreads) dst[i] = src[i];
         for (int i = tid; i < kNC * 8; i += kPrunedThreads)
             reps[i] = reinterpret_cast<const float4*>(a.C)[i >> 3];
@@ -389,7 +379,7 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
         for (int jj = 0; jj < 16; ++jj) {
             Walk A;
             A.init(v[4 * jj], v[4 * jj + 1], v[4 * jj + 2], v[4 * jj + 3], offs);
-            while (A.p < A.e) A.step(ents, myrep);
+            while (A.p < A.e) A.step(pairs, myrep);
             codes[jj >> 2] |= (uint32_t)A.i1 << (8 * (jj & 3));
             if (cancel || A.tie()) tie |= 1u << jj;
             if constexpr (ADAPT) {

@@ -1,8 +1,9 @@
 // Builder of the nearest-codeword search index for 4-dimensional
 // sub-vectors (see vq_index.cuh). Runs once per codebook on the device:
 //   vq_index_cells_kernel(count)  per grid cell: which codewords survive
-//   vq_index_scan_kernel          counts -> uint16 offsets, header
-//   vq_index_cells_kernel(fill)   per grid cell: survivors sorted by lower bound
+//   vq_index_scan_kernel          pair counts -> uint16 pair offsets, header
+//   vq_index_cells_kernel(fill)   per grid cell: survivors sorted by lower bound,
+//                                 an odd list padded with a dominated codeword
 // Dominance tests run in fp64 over cells expanded by kBoxEps.
 #include <math.h>
 
@@ -22,16 +23,8 @@ __device__ __forceinline__ void cell_box(int cell, double (&lo)[4], double (&hi)
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        if (b[i] == 0) {
-            lo[i] = -kOuter; hi[i] = -(double)kR;
-        } else if (b[i] == kNb - 1) {
-            lo[i] = (double)kR; hi[i] = kOuter;
-        } else {
-            lo[i] = -(double)kR + (double)(b[i] - 1) * (double)kW;
-            hi[i] = lo[i] + (double)kW;
-        }
-        lo[i] -= kBoxEps;
-        hi[i] += kBoxEps;
+        lo[i] = bin_edge(b[i]) - kBoxEps;
+        hi[i] = bin_edge(b[i] + 1) + kBoxEps;
     }
 }
 
@@ -91,7 +84,7 @@ __global__ void __launch_bounds__(kNC) vq_index_cells_kernel(const float* __rest
     const int count = __syncthreads_count(alive);
     uint16_t* offsets = reinterpret_cast<uint16_t*>(index + kIdxOffsets);
     if (!kFill) {
-        if (c == 0) offsets[cell] = (uint16_t)count;
+        if (c == 0) offsets[cell] = (uint16_t)((count + 1) / 2);
         if (cell == 0) {
             // codebook hash (xor is order-free; the term mixes in the position)
             uint32_t h = 0;
@@ -112,18 +105,23 @@ __global__ void __launch_bounds__(kNC) vq_index_cells_kernel(const float* __rest
     }
     const IndexHeader* hdr = reinterpret_cast<const IndexHeader*>(index);
     if (hdr->overflow) return;
+    __shared__ int pad_code;
+    if (c == 0) pad_code = kNC;
     surv[c] = alive;
     lbqs[c] = lbq;
     __syncthreads();
+    if (!alive) atomicMin(&pad_code, c);  // a dominated codeword exists whenever count < 256
+    __syncthreads();
+    uint16_t* entries = reinterpret_cast<uint16_t*>(index + kIdxEntries) + 2 * (size_t)offsets[cell];
+    if ((count & 1) && c == 0) entries[count] = (uint16_t)(pad_code | (255 << 8));
     if (!alive) return;
     int rank = 0;
     for (int c2 = 0; c2 < kNC; ++c2)
         rank += surv[c2] && (lbqs[c2] < lbq || (lbqs[c2] == lbq && c2 < c));
-    uint16_t* entries = reinterpret_cast<uint16_t*>(index + kIdxEntries);
-    entries[offsets[cell] + rank] = (uint16_t)(c | (lbq << 8));
+    entries[rank] = (uint16_t)(c | (lbq << 8));
 }
 
-// counts (in the offsets array) -> exclusive offsets; one CTA.
+// pair counts (in the offsets array) -> exclusive pair offsets; one CTA.
 __global__ void __launch_bounds__(1024) vq_index_scan_kernel(uint8_t* __restrict__ index) {
     __shared__ uint32_t part[1024];
     uint16_t* offsets = reinterpret_cast<uint16_t*>(index + kIdxOffsets);
@@ -147,7 +145,7 @@ __global__ void __launch_bounds__(1024) vq_index_scan_kernel(uint8_t* __restrict
     }
     const uint32_t total = part[1023];
     uint32_t run = part[t] - s;
-    const bool overflow = total > (uint32_t)kMaxEntries;
+    const bool overflow = total > (uint32_t)kMaxPairs;
 #pragma unroll
     for (int k = 0; k < per; ++k) {
         const int i = t * per + k;
@@ -157,7 +155,7 @@ __global__ void __launch_bounds__(1024) vq_index_scan_kernel(uint8_t* __restrict
     if (t == 0) {
         IndexHeader* hdr = reinterpret_cast<IndexHeader*>(index);
         if (!overflow) offsets[kCells] = (uint16_t)total;
-        hdr->n_entries = total;
+        hdr->n_pairs = total;
         hdr->overflow = overflow ? 1u : 0u;
         hdr->cells = kCells;
         hdr->magic = kIndexMagic;

@@ -2,32 +2,51 @@
 // (2 bits/coordinate), shared by the builder and the encode kernel.
 //
 // The transformed coordinates are near N(0, 1) (NSN + Hadamard, gist.science
-// "NSNQuant ...", Methodology §1-§2), so each coordinate is binned on a
-// uniform grid: kNb bins per coordinate, the inner kNb-2 bins of width kW
-// covering [-kR, kR) and two outer bins reaching to +-kOuter (every
-// coordinate of w satisfies |w_i| <= ||w|| = sqrt(128) < kOuter). For every
-// grid cell the index lists the codewords that can be nearest (or within the
-// near-tie margin of the nearest) for some point of the cell, sorted by a
-// lower bound of their squared distance over the cell. A codeword is left
-// out only if another codeword is closer by a margin everywhere in the cell
-// (expanded by kBoxEps), so the list's best codeword is the exact nearest.
+// "NSNQuant ...", Methodology §1-§2), so each coordinate is binned on a grid
+// that is fine where the data is dense: kNb = 10 bins per coordinate with
+// edges at 0, +-kE1, +-kE2, +-kE3, +-kE4 (about 1.3x the deciles of N(0, 1))
+// and two outer bins reaching to +-kOuter (every coordinate of w satisfies
+// |w_i| <= ||w|| = sqrt(128) < kOuter). For every grid cell the index lists
+// the codewords that can be nearest (or within the near-tie margin of the
+// nearest) for some point of the cell, sorted by a lower bound of their
+// squared distance over the cell. A codeword is left out only if another
+// codeword is closer by a margin everywhere in the cell (expanded by
+// kBoxEps), so the list's best codeword is the exact nearest.
+//
+// Lists are stored as pairs of 16-bit entries (code | lbq << 8, lbq =
+// floor(64 * lower bound) clamped to 255) so that one 32-bit load fetches
+// two; an odd list is padded with a codeword that is dominated in the cell
+// (never nearest and never within the near-tie margin) and lbq 255.
+// Offsets count pairs.
 #pragma once
 
+#include <math.h>
 #include <stdint.h>
 
 namespace nsnq {
 
 constexpr int kNb = 10;                           // bins per coordinate
-constexpr float kR = 2.4f;                        // inner grid covers [-kR, kR)
-constexpr float kW = 0.6f;                        // inner bin width
-constexpr float kInvW = 1.0f / 0.6f;
-constexpr float kBinBias = 2.4f / 0.6f + 1.0f;    // bin = floor(w / kW + kBinBias), clamped
+constexpr float kE1 = 0.32f, kE2 = 0.68f, kE3 = 1.09f, kE4 = 1.66f;  // positive inner edges
 constexpr double kOuter = 12.0;                   // outer bins end here (> sqrt(128))
 constexpr double kBoxEps = 1e-3;                  // cell expansion covering fp32 error in w
 constexpr int kCells = kNb * kNb * kNb * kNb;
-constexpr int kMaxEntries = 65535;                // offsets are uint16
+constexpr int kMaxPairs = 42496;                  // list capacity in entry pairs (shared memory)
 constexpr float kLbScale = 64.0f;                 // lower bounds stored as floor(lb * 64), <= 255
-constexpr uint32_t kIndexMagic = 0x4e534e51u;     // "NSNQ"
+constexpr uint32_t kIndexMagic = 0x4e534e52u;
+
+// Bin of one coordinate: bins 0..4 below zero, 5..9 at or above it.
+__host__ __device__ __forceinline__ int bin_of(float x) {
+    const float a = fabsf(x);
+    const int c = (a >= kE1) + (a >= kE2) + (a >= kE3) + (a >= kE4);
+    return x >= 0.f ? 5 + c : 4 - c;
+}
+
+// Edge k of the bins (k = 0..kNb): bin b covers [bin_edge(b), bin_edge(b + 1)].
+__host__ __device__ __forceinline__ double bin_edge(int k) {
+    const double e[kNb + 1] = {-kOuter, -(double)kE4, -(double)kE3, -(double)kE2, -(double)kE1, 0.0,
+                               (double)kE1, (double)kE2, (double)kE3, (double)kE4, kOuter};
+    return e[k];
+}
 
 // Near-tie rule of the fp32 search: a sub-vector whose two best distances
 // are within kTieRel * d1 + kTieAbs is re-decided in fp64 (the fp32 error of
@@ -39,18 +58,18 @@ constexpr float kTieAbs = 1e-6f;
 
 struct IndexHeader {
     uint32_t magic;
-    uint32_t n_entries;  // total list entries
-    uint32_t overflow;   // nonzero if the lists did not fit kMaxEntries
+    uint32_t n_pairs;    // total list entry pairs
+    uint32_t overflow;   // nonzero if the lists did not fit kMaxPairs
     uint32_t cells;
-    uint32_t pad[12];
+    uint32_t pad[12];    // pad[0]: hash of the codebook the index was built for
 };
 static_assert(sizeof(IndexHeader) == 64, "index header is 64 bytes");
 
 // byte offsets inside the index buffer
 constexpr size_t kIdxOffsets = 64;                                   // uint16[kCells + 1]
-constexpr size_t kIdxEntries = 64 + ((size_t(kCells + 1) * 2 + 15) / 16) * 16;  // uint16[]
-constexpr size_t kIdxBytes = kIdxEntries + size_t(kMaxEntries + 1) * 2;
-// smem image: offsets + entries (without the header)
+constexpr size_t kIdxEntries = 64 + ((size_t(kCells + 1) * 2 + 15) / 16) * 16;  // uint32[] pairs
+constexpr size_t kIdxBytes = kIdxEntries + size_t(kMaxPairs) * 4;
+// shared-memory image: offsets + entries (without the header)
 constexpr size_t kIdxSmemOffsetsBytes = kIdxEntries - kIdxOffsets;
 
 }  // namespace nsnq

@@ -225,36 +225,49 @@ def _parse_index(idx: np.ndarray):
     n_cells = int(hdr[3])
     offs = idx[64:64 + 2 * (n_cells + 1)].view(np.uint16).astype(np.int64)
     start = 64 + ((2 * (n_cells + 1) + 15) // 16) * 16
-    ents = idx[start:start + 2 * int(hdr[1])].view(np.uint16)
-    return hdr, offs, ents
+    ents = idx[start:start + 4 * int(hdr[1])].view(np.uint16)   # pairs of entries
+    return hdr, 2 * offs, ents
+
+
+def _bins(x: np.ndarray) -> np.ndarray:
+    """The index's binning of one coordinate: edges 0, +-0.32, +-0.68, +-1.09, +-1.66."""
+    x = x.astype(np.float32)
+    a = np.abs(x)
+    c = sum((a >= np.float32(e)).astype(np.int64) for e in (0.32, 0.68, 1.09, 1.66))
+    return np.where(x >= 0, 5 + c, 4 - c)
 
 
 def test_codebook_index_lists_contain_the_nearest(codebooks):
     """Grid-cell candidate lists of the 2-bit search index: for sampled points
     (standard normal, and heavy-tailed) the true nearest codeword (brute
-    force) is in the point's cell list, and each list is sorted by a valid
-    lower bound of the distance over the cell."""
+    force) is in the point's cell list, each list is sorted by a valid lower
+    bound of the distance over the cell, and the entry padding an odd list
+    is farther than the nearest codeword."""
     C = codebooks[4]
     cb = P.codebook(C).prepare()
     idx = cb.index.cpu().numpy()
     hdr, offs, ents = _parse_index(idx)
-    assert hdr[0] == 0x4E534E51 and hdr[2] == 0 and hdr[1] < 65536
-    nb, R, W = 10, 2.4, 0.6
+    assert hdr[0] == 0x4E534E52 and hdr[2] == 0
+    nb = 10
     assert hdr[3] == nb ** 4
     rng = np.random.default_rng(5)
     pts = np.concatenate([rng.standard_normal((20000, 4)), 3 * rng.standard_t(3, (5000, 4))])
     pts = np.clip(pts, -11.3, 11.3)
-    b = np.clip(np.floor(pts.astype(np.float32) * np.float32(1 / 0.6) + np.float32(R / W + 1)),
-                0, nb - 1).astype(np.int64)
+    b = _bins(pts)
     cell = ((b[:, 0] * nb + b[:, 1]) * nb + b[:, 2]) * nb + b[:, 3]
     d2 = ((pts[:, None, :] - C[None].astype(np.float64)) ** 2).sum(-1)
     nearest = d2.argmin(1)
     for i in range(len(pts)):
         lst = ents[offs[cell[i]]:offs[cell[i] + 1]]
+        assert len(lst) % 2 == 0 and len(lst) > 0
         codes, lbq = lst & 0xFF, lst >> 8
         assert nearest[i] in codes, i
         assert (np.diff(lbq.astype(np.int64)) >= 0).all()
-        assert (lbq / 64.0 <= d2[i, codes] + 1e-9).all()
+        assert (lbq[:-1] / 64.0 <= d2[i, codes[:-1]] + 1e-9).all()
+        # the last entry is a listed codeword (valid bound) or the padding
+        # (lbq 255, a codeword farther than the nearest everywhere in the cell)
+        last = d2[i, codes[-1]]
+        assert lbq[-1] / 64.0 <= last + 1e-9 or (lbq[-1] == 255 and last > d2[i, nearest[i]])
 
 
 def test_encode_detects_index_of_another_codebook(codebooks):
