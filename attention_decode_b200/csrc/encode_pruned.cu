@@ -28,7 +28,8 @@ constexpr float kCancel = 1e-3f;           // s2 below this: residual decided in
 constexpr size_t kSmReps = 0;                                  // float4 [256][8]
 constexpr size_t kSmShift = kSmReps + size_t(kNC) * 8 * 16;   // float [warps][136]
 constexpr size_t kSmHash = kSmShift + size_t(kPrunedThreads / 32) * 136 * 4;
-constexpr size_t kSmOffsets = kSmHash + 16;                    // uint16 [kCells + 1]
+constexpr size_t kSmBinTab = kSmHash + 16;                     // uint8 [kBinTabSize]
+constexpr size_t kSmOffsets = kSmBinTab + kBinTabSize;         // uint16 [kCells + 1]
 constexpr size_t kSmEntries = kSmOffsets + kIdxSmemOffsetsBytes;
 constexpr size_t kSmBytes = kSmEntries + size_t(kMaxPairs) * 4;
 
@@ -188,6 +189,12 @@ __device__ __noinline__ void exact_path(const XT* xrow, const double* o64, const
     wq_old_out = wq_old + __shfl_xor_sync(pair_mask, wq_old, 1);
 }
 
+// Bin of one coordinate through the shared-memory bin table.
+__device__ __forceinline__ int bin_fast(float x, const uint8_t* tab) {
+    const unsigned t = (unsigned)__float2int_rd(fmaf(x, kBinGrid, (float)kBinTabZero));
+    return tab[min(t, (unsigned)kBinTabSize - 1u)];
+}
+
 // Candidate walk of one sub-vector w through its cell's list.
 struct Walk {
     uint64_t w01, w23;
@@ -196,8 +203,9 @@ struct Walk {
     int i1;
 
     __device__ __forceinline__ void init(float w0, float w1, float w2, float w3,
-                                         const uint16_t* offs) {
-        const int cell = ((bin_of(w0) * kNb + bin_of(w1)) * kNb + bin_of(w2)) * kNb + bin_of(w3);
+                                         const uint16_t* offs, const uint8_t* tab) {
+        const int cell = ((bin_fast(w0, tab) * kNb + bin_fast(w1, tab)) * kNb + bin_fast(w2, tab)) * kNb +
+                         bin_fast(w3, tab);
         p = offs[cell];
         e = offs[cell + 1];
         w01 = pk(w0, w1);
@@ -205,25 +213,29 @@ struct Walk {
         d1 = INFINITY; d2 = INFINITY; i1 = 0;
     }
 
-    // Evaluate the next pair of entries (the second against the band of the
-    // best distance before the first, which costs at most one extra
-    // evaluation and never skips a contender); marks the walk finished
-    // (p = e) once the next lower bound leaves the band or the list ends.
+    // Evaluate the next pair of entries (p < e) against the band of the best
+    // distance before the pair, which costs at most one extra evaluation and
+    // never skips a contender; marks the walk finished (p = e) once a lower
+    // bound leaves the band or the list ends. Branch-free.
     __device__ __forceinline__ void step(const uint32_t* pairs, const float4* myrep) {
-        if (p >= e) return;
         const uint32_t pr = pairs[p];
         const uint32_t ent0 = pr & 0xffffu, ent1 = pr >> 16;
-        // lower bounds are floor(lb * 64) in the high byte: compare in integers
-        const uint32_t lim = (uint32_t)fminf(fmaf(d1, (1.0f + kTieRel) * kLbScale, kTieAbs * kLbScale), 1.0e6f);
-        if ((ent0 >> 8) > lim) { p = e; return; }
-        const bool take1 = (ent1 >> 8) <= lim;
+        // Lower bounds are floor(lb * 64) in the high byte of each entry. The
+        // band's limit, 64 d1 (1 + rel) rounded to the nearest integer (never
+        // below floor(64 (d1 (1 + rel) + abs)), abs < 1/128), is the low
+        // mantissa of y = 2^23 + 64 d1 (1 + rel); a larger y (d1 >= 2^17 or
+        // infinite) has larger bits and admits every entry.
+        const float y = fmaf(d1, (1.0f + kTieRel) * kLbScale, 8388608.0f);
+        const uint32_t lim = __float_as_uint(y);
+        const bool take0 = (0x4b000000u | (ent0 >> 8)) <= lim;
+        const bool take1 = (0x4b000000u | (ent1 >> 8)) <= lim;
         const float4 cv0 = myrep[(ent0 & 0xff) * 8];
         const float4 cv1 = myrep[(ent1 & 0xff) * 8];
         const uint64_t a01 = sub2(w01, pk(cv0.x, cv0.y)), a23 = sub2(w23, pk(cv0.z, cv0.w));
         const uint64_t b01 = sub2(w01, pk(cv1.x, cv1.y)), b23 = sub2(w23, pk(cv1.z, cv1.w));
         const float2 da = upk(fma2(a23, a23, mul2(a01, a01)));
         const float2 db = upk(fma2(b23, b23, mul2(b01, b01)));
-        const float dA = da.x + da.y;
+        const float dA = take0 ? da.x + da.y : INFINITY;
         const float dB = take1 ? db.x + db.y : INFINITY;
         d2 = fminf(d2, fmaxf(d1, dA));
         i1 = dA < d1 ? (int)(ent0 & 0xff) : i1;
@@ -248,8 +260,10 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
     const uint16_t* offs = reinterpret_cast<const uint16_t*>(sm + kSmOffsets);
     const uint16_t* ents = reinterpret_cast<const uint16_t*>(sm + kSmEntries);
     const uint32_t* pairs = reinterpret_cast<const uint32_t*>(sm + kSmEntries);
+    uint8_t* bintab = sm + kSmBinTab;
     const int tid = threadIdx.x, lane = lane_id();
     const int half = lane & 1;
+    const float sgn = half ? -1.0f : 1.0f;
     const unsigned pair_mask = 3u << (lane & 30);
 
     // ---- stage the index and the replicated codebook ----
@@ -265,6 +279,8 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
         for (size_t i = tid; i < nbytes / 16; i += kPrunedThreads) dst[i] = src[i];
         for (int i = tid; i < kNC * 8; i += kPrunedThreads)
             reps[i] = reinterpret_cast<const float4*>(a.C)[i >> 3];
+        for (int t = tid; t < kBinTabSize; t += kPrunedThreads)
+            bintab[t] = (uint8_t)bin_of((float)(t - kBinTabZero) * (1.0f / kBinGrid));
         uint32_t h = 0;
         for (int i = tid; i < kNC * 4; i += kPrunedThreads) h ^= cb_hash_term(__float_as_uint(a.C[i]), i);
 #pragma unroll
@@ -298,7 +314,8 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
         if (bh != cur_bh) {  // warp-uniform
             __syncwarp();
             const float4 o = reinterpret_cast<const float4*>(a.shift + bh * kD)[lane];
-            reinterpret_cast<float4*>(wshift)[lane + (lane >= 16 ? 1 : 0)] = o;
+            reinterpret_cast<float4*>(wshift)[lane + (lane >= 16 ? 1 : 0)] =
+                make_float4(-o.x, -o.y, -o.z, -o.w);  // -o: the shift is subtracted
             __syncwarp();
             cur_bh = bh;
         }
@@ -331,8 +348,8 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
 #pragma unroll
         for (int k = 0; k < 64; k += 4) {
             const float4 o = o4[k >> 2];
-            const uint64_t z0 = fma2(pk(v[k], v[k + 1]), inv2, pk(-o.x, -o.y));
-            const uint64_t z1 = fma2(pk(v[k + 2], v[k + 3]), inv2, pk(-o.z, -o.w));
+            const uint64_t z0 = fma2(pk(v[k], v[k + 1]), inv2, pk(o.x, o.y));
+            const uint64_t z1 = fma2(pk(v[k + 2], v[k + 3]), inv2, pk(o.z, o.w));
             acc0 = fma2(z0, z0, acc0);
             acc1 = fma2(z1, z1, acc1);
             const float2 a0 = upk(z0), a1 = upk(z1);
@@ -368,7 +385,7 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
 #pragma unroll
         for (int k = 0; k < 64; ++k) {
             const float p = __shfl_xor_sync(kFull, v[k], 1);
-            v[k] = half ? (p - v[k]) : (v[k] + p);
+            v[k] = fmaf(v[k], sgn, p);  // lower half v + p, upper half p - v
         }
         // ---- nearest codeword of the 16 sub-vectors this thread holds ----
         uint32_t codes[4] = {0u, 0u, 0u, 0u};
@@ -378,7 +395,7 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
 #pragma unroll
         for (int jj = 0; jj < 16; ++jj) {
             Walk A;
-            A.init(v[4 * jj], v[4 * jj + 1], v[4 * jj + 2], v[4 * jj + 3], offs);
+            A.init(v[4 * jj], v[4 * jj + 1], v[4 * jj + 2], v[4 * jj + 3], offs, bintab);
             while (A.p < A.e) A.step(pairs, myrep);
             codes[jj >> 2] |= (uint32_t)A.i1 << (8 * (jj & 3));
             if (cancel || A.tie()) tie |= 1u << jj;

@@ -4,8 +4,9 @@
 // The transformed coordinates are near N(0, 1) (NSN + Hadamard, gist.science
 // "NSNQuant ...", Methodology §1-§2), so each coordinate is binned on a grid
 // that is fine where the data is dense: kNb = 10 bins per coordinate with
-// edges at 0, +-kE1, +-kE2, +-kE3, +-kE4 (about 1.3x the deciles of N(0, 1))
-// and two outer bins reaching to +-kOuter (every coordinate of w satisfies
+// edges at 0, +-kE1, +-kE2, +-kE3, +-kE4 (about 1.3x the deciles of N(0, 1),
+// rounded to multiples of 1/32 so that a table over a 1/32 grid gives the
+// bin exactly) and two outer bins reaching to +-kOuter (every coordinate of w satisfies
 // |w_i| <= ||w|| = sqrt(128) < kOuter). For every grid cell the index lists
 // the codewords that can be nearest (or within the near-tie margin of the
 // nearest) for some point of the cell, sorted by a lower bound of their
@@ -26,19 +27,24 @@
 namespace nsnq {
 
 constexpr int kNb = 10;                           // bins per coordinate
-constexpr float kE1 = 0.32f, kE2 = 0.68f, kE3 = 1.09f, kE4 = 1.66f;  // positive inner edges
+constexpr float kE1 = 0.3125f, kE2 = 0.6875f, kE3 = 1.09375f, kE4 = 1.65625f;  // positive inner edges
 constexpr double kOuter = 12.0;                   // outer bins end here (> sqrt(128))
 constexpr double kBoxEps = 1e-3;                  // cell expansion covering fp32 error in w
 constexpr int kCells = kNb * kNb * kNb * kNb;
-constexpr int kMaxPairs = 42496;                  // list capacity in entry pairs (shared memory)
+constexpr int kMaxPairs = 41984;                  // list capacity in entry pairs (shared memory)
+// Bin table: entry t is the bin of (t - kBinTabZero) / kBinGrid, so a
+// coordinate x has bin table[floor(x * kBinGrid) + kBinTabZero] (|x| < 12).
+constexpr float kBinGrid = 32.0f;
+constexpr int kBinTabZero = 384;
+constexpr int kBinTabSize = 768;
 constexpr float kLbScale = 64.0f;                 // lower bounds stored as floor(lb * 64), <= 255
 constexpr uint32_t kIndexMagic = 0x4e534e52u;
 
-// Bin of one coordinate: bins 0..4 below zero, 5..9 at or above it.
+// Bin of one coordinate: the number of inner edges at or below x (bins are
+// closed below, open above, like floor() on the 1/32 grid of the table).
 __host__ __device__ __forceinline__ int bin_of(float x) {
-    const float a = fabsf(x);
-    const int c = (a >= kE1) + (a >= kE2) + (a >= kE3) + (a >= kE4);
-    return x >= 0.f ? 5 + c : 4 - c;
+    return (x >= -kE4) + (x >= -kE3) + (x >= -kE2) + (x >= -kE1) + (x >= 0.f) + (x >= kE1) +
+           (x >= kE2) + (x >= kE3) + (x >= kE4);
 }
 
 // Edge k of the bins (k = 0..kNb): bin b covers [bin_edge(b), bin_edge(b + 1)].

@@ -230,11 +230,11 @@ def _parse_index(idx: np.ndarray):
 
 
 def _bins(x: np.ndarray) -> np.ndarray:
-    """The index's binning of one coordinate: edges 0, +-0.32, +-0.68, +-1.09, +-1.66."""
+    """The index's binning of one coordinate: the number of edges (0, +-10/32, +-22/32,
+    +-35/32, +-53/32) at or below it."""
     x = x.astype(np.float32)
-    a = np.abs(x)
-    c = sum((a >= np.float32(e)).astype(np.int64) for e in (0.32, 0.68, 1.09, 1.66))
-    return np.where(x >= 0, 5 + c, 4 - c)
+    edges = (0.3125, 0.6875, 1.09375, 1.65625)
+    return sum((x >= np.float32(e)).astype(np.int64) for e in sorted([-e for e in edges] + [0.0] + list(edges)))
 
 
 def test_codebook_index_lists_contain_the_nearest(codebooks):
