@@ -98,95 +98,81 @@ __device__ __forceinline__ void load64<float>(const float* p, float (&v)[64]) {
     }
 }
 
-// Exact decision for the flagged sub-vectors of one token-head, shared by
-// the two threads of a pair (pair_mask): fp64 NSN of the whole token, then
-// w_j = H_j u for each flagged sub-vector and an fp64 scan of its cell list
-// (which holds every codeword that can be nearest there; lowest index on
-// exact ties). Returns the fp64 (s1, s2) and, summed over the pair's
-// re-decided sub-vectors, w . C[new code] and w . C[previous code] (for the
-// scale adjustment). Kept in registers (no local arrays) and division-free,
-// since one slow warp holds its SM.
+// Exact decision for one token-head, by the whole warp: fp64 NSN of the
+// token (lane l holds channels 4l..4l+3), fp64 Hadamard transform across the
+// warp, after which lane l holds sub-vector l of w; each flagged lane scans
+// its cell list in fp64 (the list holds every codeword that can be nearest
+// there; lowest index on exact ties). Returns this lane's code (old_code when
+// not flagged), the fp64 (s1, s2) and, summed over the warp, w . C[code] over
+// all sub-vectors and w . (C[new] - C[old]) over the flagged ones (for the
+// scale adjustment). Kept short and warp-wide: a slow warp holds its SM.
 template <typename XT>
-__device__ __noinline__ void exact_path(const XT* xrow, const double* o64, const float* o32,
+__device__ __noinline__ int exact_warp(const XT* xtok, const double* o64, const float* o32,
                                        const float4* reps, const uint16_t* offs,
-                                       const uint16_t* ents, int half, unsigned pair_mask,
-                                       uint32_t my_mask, uint32_t both_mask, uint32_t (&codes)[4],
-                                       double& s1_out, double& s2_out, double& wq_new_out,
-                                       double& wq_old_out) {
-    float v[64];
-    load64<XT>(xrow + 64 * half, v);
-    const double* o64h = o64 ? o64 + 64 * half : nullptr;
-    const float* o32h = o32 + 64 * half;
-    const double sqrt_d = sqrt((double)kD);
-    double ss = 0.0;
+                                       const uint16_t* ents, uint32_t flags, int old_code,
+                                       double& s1_out, double& s2_out, double& wq_all,
+                                       double& wq_delta) {
+    const int lane = lane_id();
+    float xf[4];
+    load4(xtok + 4 * lane, xf);
+    double x[4], o[4];
 #pragma unroll
-    for (int k = 0; k < 64; ++k) ss = fma((double)v[k], (double)v[k], ss);
-    ss += __shfl_xor_sync(pair_mask, ss, 1);
+    for (int r = 0; r < 4; ++r) {
+        x[r] = (double)xf[r];
+        o[r] = o64 ? o64[4 * lane + r] : (double)o32[4 * lane + r];
+    }
+    const double sqrt_d = sqrt((double)kD);
+    const double ss = warp_sum_d(x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3]);
     const double s1 = sqrt(ss) / sqrt_d;
     const double inv1 = s1 > 0.0 ? 1.0 / s1 : 0.0;
-    double ss2 = 0.0, yy = 0.0, oo = 0.0;
-#pragma unroll 8
-    for (int k = 0; k < 64; ++k) {
-        const double o = o64h ? o64h[k] : (double)o32h[k];
-        const double y = (double)v[k] * inv1;
-        const double z = y - o;
-        ss2 = fma(z, z, ss2);
+    double z[4], ss2 = 0.0, yy = 0.0, oo = 0.0;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const double y = x[r] * inv1;
+        z[r] = y - o[r];
+        ss2 = fma(z[r], z[r], ss2);
         yy = fma(y, y, yy);
-        oo = fma(o, o, oo);
+        oo = fma(o[r], o[r], oo);
     }
-    ss2 += __shfl_xor_sync(pair_mask, ss2, 1);
-    yy += __shfl_xor_sync(pair_mask, yy, 1);
-    oo += __shfl_xor_sync(pair_mask, oo, 1);
+    ss2 = warp_sum_d(ss2);
+    yy = warp_sum_d(yy);
+    oo = warp_sum_d(oo);
     // a residual at or below 2^-20 of the token/shift magnitude counts as zero
     const double s2 = ss2 <= 0x1p-40 * (yy + oo) ? 0.0 : sqrt(ss2) / sqrt_d;
     const double inv2 = s2 > 0.0 ? 1.0 / s2 : 0.0;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) z[r] *= inv2;
+    fwht128_lane4(z);  // unnormalised: w = z / sqrt(d)
     const double hs = 1.0 / sqrt_d;
-    double wq_new = 0.0, wq_old = 0.0;
-    uint32_t todo = both_mask;
-    while (todo) {
-        const int j = __ffs(todo) - 1;  // global sub-vector index 0..31
-        todo &= todo - 1;
-        double w[4];
+    double w[4];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const int row = 4 * j + r;
-            double acc = 0.0;
-#pragma unroll 8
-            for (int k = 0; k < 64; ++k) {
-                const double o = o64h ? o64h[k] : (double)o32h[k];
-                const double u = ((double)v[k] * inv1 - o) * inv2;
-                acc += (__popc(row & (64 * half + k)) & 1) ? -u : u;
-            }
-            w[r] = (acc + __shfl_xor_sync(pair_mask, acc, 1)) * hs;
-        }
-        if ((my_mask >> j) & 1u) {
-            int cell = 0;
+    for (int r = 0; r < 4; ++r) w[r] = z[r] * hs;
+    int code = old_code;
+    if ((flags >> lane) & 1u) {
+        int cell = 0;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) cell = cell * kNb + bin_of((float)w[i]);
-            double bd = INFINITY;
-            int bi = 0;
-            // every entry of the list, the padding codeword included (it never wins)
-            for (uint32_t q = 2u * offs[cell]; q < 2u * offs[cell + 1]; ++q) {
-                const int c = ents[q] & 0xff;
-                const float4 cv = reps[c * 8];
-                const double e0 = w[0] - (double)cv.x, e1 = w[1] - (double)cv.y;
-                const double e2 = w[2] - (double)cv.z, e3 = w[3] - (double)cv.w;
-                const double d = e0 * e0 + e1 * e1 + e2 * e2 + e3 * e3;
-                if (d < bd || (d == bd && c < bi)) { bd = d; bi = c; }
-            }
-            const int jj = j - 16 * half;
-            const int sh = 8 * (jj & 3);
-            const float4 cn = reps[bi * 8];
-            const float4 co = reps[((codes[jj >> 2] >> sh) & 0xffu) * 8];
-            codes[jj >> 2] = (codes[jj >> 2] & ~(0xffu << sh)) | ((uint32_t)bi << sh);
-            wq_new += w[0] * (double)cn.x + w[1] * (double)cn.y + w[2] * (double)cn.z + w[3] * (double)cn.w;
-            wq_old += w[0] * (double)co.x + w[1] * (double)co.y + w[2] * (double)co.z + w[3] * (double)co.w;
+        for (int i = 0; i < 4; ++i) cell = cell * kNb + bin_of((float)w[i]);
+        double bd = INFINITY;
+        int bi = 0;
+        // every entry of the list, the padding codeword included (it never wins)
+        for (uint32_t q = 2u * offs[cell]; q < 2u * offs[cell + 1]; ++q) {
+            const int c = ents[q] & 0xff;
+            const float4 cv = reps[c * 8];
+            const double e0 = w[0] - (double)cv.x, e1 = w[1] - (double)cv.y;
+            const double e2 = w[2] - (double)cv.z, e3 = w[3] - (double)cv.w;
+            const double d = e0 * e0 + e1 * e1 + e2 * e2 + e3 * e3;
+            if (d < bd || (d == bd && c < bi)) { bd = d; bi = c; }
         }
+        code = bi;
     }
+    const float4 cn = reps[code * 8], co = reps[old_code * 8];
+    const double qn = w[0] * (double)cn.x + w[1] * (double)cn.y + w[2] * (double)cn.z + w[3] * (double)cn.w;
+    const double qo = w[0] * (double)co.x + w[1] * (double)co.y + w[2] * (double)co.z + w[3] * (double)co.w;
+    wq_all = warp_sum_d(qn);
+    wq_delta = warp_sum_d(((flags >> lane) & 1u) ? qn - qo : 0.0);
     s1_out = s1;
     s2_out = s2;
-    wq_new_out = wq_new + __shfl_xor_sync(pair_mask, wq_new, 1);
-    wq_old_out = wq_old + __shfl_xor_sync(pair_mask, wq_old, 1);
+    return code;
 }
 
 // Bin of one coordinate through the shared-memory bin table.
@@ -213,10 +199,10 @@ struct Walk {
         d1 = INFINITY; d2 = INFINITY; i1 = 0;
     }
 
-    // Evaluate the next pair of entries (p < e) against the band of the best
-    // distance before the pair, which costs at most one extra evaluation and
-    // never skips a contender; marks the walk finished (p = e) once a lower
-    // bound leaves the band or the list ends. Branch-free.
+    // Evaluate the next pair of entries (p < e); the walk ends (p = e) after
+    // a pair whose second lower bound leaves the band of the best distance
+    // before the pair, or at the end of the list (entries are sorted by lower
+    // bound, so no contender is skipped). Branch-free.
     __device__ __forceinline__ void step(const uint32_t* pairs, const float4* myrep) {
         const uint32_t pr = pairs[p];
         const uint32_t ent0 = pr & 0xffffu, ent1 = pr >> 16;
@@ -227,7 +213,6 @@ struct Walk {
         // infinite) has larger bits and admits every entry.
         const float y = fmaf(d1, (1.0f + kTieRel) * kLbScale, 8388608.0f);
         const uint32_t lim = __float_as_uint(y);
-        const bool take0 = (0x4b000000u | (ent0 >> 8)) <= lim;
         const bool take1 = (0x4b000000u | (ent1 >> 8)) <= lim;
         const float4 cv0 = myrep[(ent0 & 0xff) * 8];
         const float4 cv1 = myrep[(ent1 & 0xff) * 8];
@@ -235,8 +220,11 @@ struct Walk {
         const uint64_t b01 = sub2(w01, pk(cv1.x, cv1.y)), b23 = sub2(w23, pk(cv1.z, cv1.w));
         const float2 da = upk(fma2(a23, a23, mul2(a01, a01)));
         const float2 db = upk(fma2(b23, b23, mul2(b01, b01)));
-        const float dA = take0 ? da.x + da.y : INFINITY;
-        const float dB = take1 ? db.x + db.y : INFINITY;
+        // Both entries count even past the band: they are listed codewords
+        // (or the padding, farther than the nearest by the margin), so they
+        // can only tighten d1 or reveal a true near-tie.
+        const float dA = da.x + da.y;
+        const float dB = db.x + db.y;
         d2 = fminf(d2, fmaxf(d1, dA));
         i1 = dA < d1 ? (int)(ent0 & 0xff) : i1;
         d1 = fminf(d1, dA);
@@ -264,7 +252,6 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
     const int tid = threadIdx.x, lane = lane_id();
     const int half = lane & 1;
     const float sgn = half ? -1.0f : 1.0f;
-    const unsigned pair_mask = 3u << (lane & 30);
 
     // ---- stage the index and the replicated codebook ----
     const IndexHeader* hdr = reinterpret_cast<const IndexHeader*>(a.index);
@@ -407,23 +394,51 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
         }
         if (!valid) tie = 0;
         // ---- exact fp64 decision where the fp32 search is not conclusive ----
+        // Token-heads with a flagged sub-vector are re-done one at a time by
+        // the whole warp; results go back to the owning pair of lanes.
         const uint32_t my_mask = tie << (16 * half);
         const uint32_t both = my_mask | __shfl_xor_sync(kFull, my_mask, 1);
         float s1o = s1, s2o = s2;
         double wqd = 0.0;
         if constexpr (ADAPT) wqd = (double)(wq + __shfl_xor_sync(kFull, wq, 1));
-        if (both) {
+        uint32_t pending = __ballot_sync(kFull, both != 0u && half == 0);
+        if (pending) {
             const double* o64 = a.given_shift ? nullptr : a.o64 + bh * kD;
-            double s1d, s2d, wq_new, wq_old;
-            exact_path<XT>(xrow, o64, a.shift + bh * kD, reps, offs, ents, half, pair_mask,
-                           my_mask, both, codes, s1d, s2d, wq_new, wq_old);
-            s1o = (float)s1d;
-            s2o = (float)s2d;
-            // on cancellation every sub-vector was re-decided from the fp64 w
-            wqd = cancel ? wq_new : wqd + (wq_new - wq_old);
-            if (half == 0 && a.stats) {
-                atomicAdd(&a.stats[0], 1ull);
-                atomicAdd(&a.stats[1], (unsigned long long)__popc(both));
+            const XT* xhead = reinterpret_cast<const XT*>(a.x) + b * a.sb + h * a.sh;
+            const int64_t t0 = t - (lane >> 1);  // first token of the tile
+            while (pending) {
+                const int src = __ffs(pending) - 1;  // even lane of the token-head's pair
+                pending &= pending - 1;
+                const uint32_t flags = __shfl_sync(kFull, both, src);
+                // current code of sub-vector `lane` (held by lane src + lane / 16)
+                uint32_t word = 0u;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint32_t wk = __shfl_sync(kFull, codes[k], src + (lane >> 4));
+                    if (k == ((lane & 15) >> 2)) word = wk;
+                }
+                const int old_code = (int)((word >> (8 * (lane & 3))) & 0xffu);
+                double s1d, s2d, wq_all, wq_delta;
+                const int code = exact_warp<XT>(xhead + (t0 + (src >> 1)) * a.st, o64,
+                                                a.shift + bh * kD, reps, offs, ents, flags,
+                                                old_code, s1d, s2d, wq_all, wq_delta);
+                const bool mine = (lane >> 1) == (src >> 1);
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) {
+                    const uint32_t c = (uint32_t)__shfl_sync(kFull, code, 16 * half + jj);
+                    const int sh = 8 * (jj & 3);
+                    if (mine) codes[jj >> 2] = (codes[jj >> 2] & ~(0xffu << sh)) | (c << sh);
+                }
+                if (mine) {
+                    s1o = (float)s1d;
+                    s2o = (float)s2d;
+                    // all re-decided (always so on cancellation): the fp64 sum
+                    wqd = flags == kFull ? wq_all : wqd + wq_delta;
+                }
+                if (lane == 0 && a.stats) {
+                    atomicAdd(&a.stats[0], 1ull);
+                    atomicAdd(&a.stats[1], (unsigned long long)__popc(flags));
+                }
             }
         }
         if constexpr (ADAPT) {
