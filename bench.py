@@ -54,6 +54,25 @@ def peaks():
         return 6650.0, "fallback"
 
 
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "roofline_traffic.json")
+
+
+def measured_traffic(call: str):
+    """DRAM bytes per launch of `call` from the committed ncu record, or None
+    when the kernel sources changed since the capture (hash mismatch)."""
+    import hashlib
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)[call]
+        h = hashlib.sha256()
+        for name in rec["sources"]:
+            with open(os.path.join(ROOT, "attention_decode_b200", "csrc", name), "rb") as f:
+                h.update(f.read())
+        return int(rec["bytes_per_launch"]) if h.hexdigest() == rec["source_sha256"] else None
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def encode_bytes_per_token_head(sub: int, in_bytes: int = 2) -> int:
     """Algorithmic bytes of encode per token-head: input row, codes, (s1, s2)."""
     return 128 * in_bytes + 128 // sub + 8
@@ -262,7 +281,7 @@ def run_cuda(args):
                 "frac": round(enc_gbs / hbm, 4), "peak_kind": peak_kind,
                 "kernel": "nsnq_encode (nsn_stats + nsn_shift + nsn_encode, one tensor)",
                 "algorithmic_bytes_per_launch": enc_bytes,
-                "traffic": args.traffic}
+                "traffic": args.traffic if args.traffic is not None else measured_traffic("nsnq_encode")}
 
     # ---- decode attention alone at the 32k workload ----
     attention = run_attention_bench(args, nsnq, dev, world, barrier, hbm, peak_kind)
@@ -344,7 +363,8 @@ def run_attention_bench(args, nsnq, dev, world, barrier, hbm, peak_kind):
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
                          "frac": round(gbs / hbm, 4), "peak_kind": peak_kind,
                          "kernel": "nsnq_attn_decode (attn_split + attn_combine)",
-                         "algorithmic_bytes_per_launch": nbytes, "traffic": None},
+                         "algorithmic_bytes_per_launch": nbytes,
+                         "traffic": measured_traffic("nsnq_attn_decode")},
             "l2": "flushed before every call (cache 335 MB > L2 anyway)"}
 
 

@@ -68,3 +68,21 @@ def test_reference_arm_prints_one_json_line():
     assert d["impl"] == "reference" and d["unit"] == "KV tokens/s" and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
     assert d["higher_is_better"] is True and d["warmup"] >= 3
+
+
+def test_traffic_record_is_dropped_when_the_kernel_changes(tmp_path, monkeypatch):
+    """The roofline's measured DRAM traffic is reported only while the kernel
+    sources still hash to the value recorded with the ncu capture."""
+    import hashlib
+    import json
+    import bench
+    src = ["common.cuh"]
+    path = os.path.join(bench.ROOT, "attention_decode_b200", "csrc", "common.cuh")
+    good = hashlib.sha256(open(path, "rb").read()).hexdigest()
+    rec = tmp_path / "traffic.json"
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(rec))
+    rec.write_text(json.dumps({"k": {"sources": src, "source_sha256": good, "bytes_per_launch": 123}}))
+    assert bench.measured_traffic("k") == 123
+    rec.write_text(json.dumps({"k": {"sources": src, "source_sha256": "0" * 64, "bytes_per_launch": 123}}))
+    assert bench.measured_traffic("k") is None
+    assert bench.measured_traffic("missing") is None
