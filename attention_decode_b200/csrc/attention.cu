@@ -16,7 +16,7 @@
 
 namespace nsnq {
 
-constexpr int kAttnWarps = 12;
+constexpr int kAttnWarps = 16;
 constexpr int kAttnThreads = kAttnWarps * 32;
 
 // Shared-memory map of the split kernel (bytes):
@@ -263,30 +263,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a)
         // ---- values: lane = sub-vector, fp32 codewords and accumulation ----
         const int nt = (int)min((int64_t)32, te - base);
         const float4* myrep = vrep + (lane & 7);
-        for (int i = 0; i < nt; i += TPI) {
-            const int tt = i + sub_t;
-            if (tt < nt) {
-                const int code = my_codes[tt * VJ + jj];
-                float c[VSUB];
+        // one token's value codewords into the head accumulators (lane = sub-vector)
+        auto vstep = [&](int tt) {
+            const int code = my_codes[tt * VJ + jj];
+            float c[VSUB];
 #pragma unroll
-                for (int k = 0; k < VSUB / 4; ++k) {
-                    const float4 cv = myrep[(code * (VSUB / 4) + k) * 8];
-                    c[4 * k] = cv.x; c[4 * k + 1] = cv.y; c[4 * k + 2] = cv.z; c[4 * k + 3] = cv.w;
-                }
-                float wv[GP];
-#pragma unroll
-                for (int q4 = 0; q4 < GP / 4; ++q4) {
-                    const float4 w4 = reinterpret_cast<const float4*>(my_w + tt * GP)[q4];
-                    wv[4 * q4] = w4.x; wv[4 * q4 + 1] = w4.y; wv[4 * q4 + 2] = w4.z; wv[4 * q4 + 3] = w4.w;
-                }
-#pragma unroll
-                for (int h = 0; h < GC; ++h) {
-                    const uint64_t wp = pk2(wv[h], wv[h]);
-#pragma unroll
-                    for (int r = 0; r < VSUB / 2; ++r)
-                        acc[h][r] = ffma2(pk2(c[2 * r], c[2 * r + 1]), wp, acc[h][r]);
-                }
+            for (int k = 0; k < VSUB / 4; ++k) {
+                const float4 cv = myrep[(code * (VSUB / 4) + k) * 8];
+                c[4 * k] = cv.x; c[4 * k + 1] = cv.y; c[4 * k + 2] = cv.z; c[4 * k + 3] = cv.w;
             }
+            float wv[GP];
+#pragma unroll
+            for (int q4 = 0; q4 < GP / 4; ++q4) {
+                const float4 w4 = reinterpret_cast<const float4*>(my_w + tt * GP)[q4];
+                wv[4 * q4] = w4.x; wv[4 * q4 + 1] = w4.y; wv[4 * q4 + 2] = w4.z; wv[4 * q4 + 3] = w4.w;
+            }
+#pragma unroll
+            for (int h = 0; h < GC; ++h) {
+                const uint64_t wp = pk2(wv[h], wv[h]);
+#pragma unroll
+                for (int r = 0; r < VSUB / 2; ++r)
+                    acc[h][r] = ffma2(pk2(c[2 * r], c[2 * r + 1]), wp, acc[h][r]);
+            }
+        };
+        if (nt == 32) {  // full batch: unrolled so that several gathers are in flight
+#pragma unroll 8
+            for (int i = 0; i < 32; i += TPI) vstep(i + sub_t);
+        } else {
+            for (int i = 0; i < nt; i += TPI)
+                if (i + sub_t < nt) vstep(i + sub_t);
         }
         __syncwarp();
     }
