@@ -7,7 +7,8 @@
 //   nsn_shift_kernel   per (b, h): o = sum / T (fp64, kept in the workspace
 //                      for the near-tie path) and its fp32 copy in the cache
 //   pass 2             NSN + FWHT + nearest codeword: encode_pruned.cu
-//                      (2 bit, search index) or encode1.cu (1 bit, all codewords)
+//                      (2 bit, search index) or encode1_tc.cu (1 bit, all
+//                      codewords scored on the tensor cores)
 #include <math.h>
 
 #include "common.cuh"
@@ -157,7 +158,7 @@ static cudaError_t launch_encode_t(const EncodeArgs& a, cudaStream_t s) {
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    return a.sub == 4 ? launch_encode_pruned(a, s) : launch_encode1(a, s);
+    return a.sub == 4 ? launch_encode_pruned(a, s) : launch_encode1_tc(a, s);
 }
 
 cudaError_t launch_encode(const EncodeArgs& a, cudaStream_t s) {

@@ -53,7 +53,7 @@ struct EncodePlan {
 EncodePlan plan_encode(int B, int H, int64_t T);
 cudaError_t launch_encode(const EncodeArgs& a, cudaStream_t s);
 cudaError_t launch_encode_pruned(const EncodeArgs& a, cudaStream_t s);
-cudaError_t launch_encode1(const EncodeArgs& a, cudaStream_t s);
+cudaError_t launch_encode1_tc(const EncodeArgs& a, cudaStream_t s);
 size_t index_bytes();
 cudaError_t launch_index_build(const float* C, void* index, cudaStream_t s);
 
