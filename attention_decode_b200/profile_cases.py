@@ -6,6 +6,8 @@ Cases (seeded synthetic inputs generated on the device):
   encode-16x8x4096     encode one bf16 tensor, 16 x 8 kv-heads x 4096 tokens, 2 bit
                        (134 MB of input: larger than L2)
   encode-8x8x4096      the benchmark's per-tensor encode (67 MB)
+  encode1-16x8x4096    1-bit encode (tensor-core scoring), 16 x 8 kv-heads x 4096 tokens
+  encode1-8x8x4096     1-bit encode, 8 x 8 kv-heads x 4096 tokens
   attn-16x32k-2b       decode attention, B 16, Hq 32, Hkv 8, 32768 tokens, 2 bit
   attn-16x32k-1b       the same with 1-bit K and V
   attn-64x8k-gqa8      decode attention, B 64, Hq 64, Hkv 8, 8192 tokens, 2 bit
@@ -36,12 +38,12 @@ def _keys(gen, B, H, T, dev):
     return ((z + bias) * s).to(torch.bfloat16)
 
 
-def encode_case(B, H, T, reps, dev):
+def encode_case(B, H, T, reps, dev, sub=4):
     gen = torch.Generator(device=dev)
     gen.manual_seed(0)
-    cb = _codebook(4, dev)
+    cb = _codebook(sub, dev)
     x = _keys(gen, B, H, T, dev)
-    cache = nsnq.Cache.empty(B, H, T, 4, device=dev)
+    cache = nsnq.Cache.empty(B, H, T, sub, device=dev)
     ws = torch.empty(nsnq.nsnq_encode_workspace(B, H, T), dtype=torch.uint8, device=dev)
     cb.prepare()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -78,6 +80,8 @@ def attn_case(B, Hq, Hkv, T, sub, reps, dev):
 CASES = {
     "encode-16x8x4096": lambda r, d: encode_case(16, 8, 4096, r, d),
     "encode-8x8x4096": lambda r, d: encode_case(8, 8, 4096, r, d),
+    "encode1-16x8x4096": lambda r, d: encode_case(16, 8, 4096, r, d, sub=8),
+    "encode1-8x8x4096": lambda r, d: encode_case(8, 8, 4096, r, d, sub=8),
     "attn-16x32k-2b": lambda r, d: attn_case(16, 32, 8, 32768, 4, r, d),
     "attn-16x32k-1b": lambda r, d: attn_case(16, 32, 8, 32768, 8, r, d),
     "attn-64x8k-gqa8": lambda r, d: attn_case(64, 64, 8, 8192, 4, r, d),
