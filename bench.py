@@ -285,6 +285,7 @@ def run_cuda(args):
 
     # ---- decode attention alone at the 32k workload ----
     attention = run_attention_bench(args, nsnq, dev, world, barrier, hbm, peak_kind)
+    encode_1bit = run_encode1_bench(args, nsnq, dev, world, barrier, hbm, peak_kind, k)
     clk.__exit__(None, None, None)
 
     result = {
@@ -299,7 +300,8 @@ def run_cuda(args):
         "stages_ms": {"encode_per_tensor": round(enc_avg_ms, 4),
                       "attention_4k": round(sum(att_small_ms) / len(att_small_ms), 4)},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
-        "roofline": roofline, "attention": attention, "e2e": e2e, "clocks": clk.summary(),
+        "roofline": roofline, "attention": attention, "encode_1bit": encode_1bit, "e2e": e2e,
+        "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(args)
@@ -366,6 +368,42 @@ def run_attention_bench(args, nsnq, dev, world, barrier, hbm, peak_kind):
                          "algorithmic_bytes_per_launch": nbytes,
                          "traffic": measured_traffic("nsnq_attn_decode")},
             "l2": "flushed before every call (cache 335 MB > L2 anyway)"}
+
+
+def run_encode1_bench(args, nsnq, dev, world, barrier, hbm, peak_kind, x):
+    """The 1-bit encode (tensor-core scoring) of the step's K tensor."""
+    import torch
+    B, H, T = x.shape[0], x.shape[1], x.shape[2]
+    cb = nsnq.Codebook(torch.from_numpy(load_codebook(8)).to(dev))
+    cache = nsnq.Cache.empty(B, H, T, 8, device=dev)
+    ws = torch.empty(nsnq.nsnq_encode_workspace(B, H, T), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        nsnq.nsnq_encode(x, cb, cache, workspace=ws)
+    stream = torch.cuda.current_stream()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for e0, e1 in evs:
+        flush.zero_()
+        e0.record(stream)
+        nsnq.nsnq_encode(x, cb, cache, workspace=ws)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    avg = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / len(evs), world, dev)
+    nbytes = B * H * T * encode_bytes_per_token_head(8)
+    gbs = nbytes / (avg / 1e3) / 1e9
+    return {"metric": "KV tokens/s encoded at 1 bit", "value": round(B * T * world / (avg / 1e3), 1),
+            "unit": "KV tokens/s (one tensor)", "ms_per_call": round(avg, 4),
+            "workload": "encode-8x4096 keys at 1 bit/coord (g = 8), codewords scored on the tensor cores",
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(gbs / hbm, 4), "peak_kind": peak_kind,
+                         "kernel": "nsnq_encode at 1 bit (nsn_stats + nsn_shift + nsn_encode1_tc)",
+                         "algorithmic_bytes_per_launch": nbytes,
+                         "traffic": measured_traffic("nsnq_encode_1bit")},
+            "l2": "flushed before every call"}
 
 
 # ------------------------------------------------------------ oracle arm --
