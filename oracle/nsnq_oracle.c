@@ -305,3 +305,30 @@ int oracle_attention_head(const double* q, int G, const double* Kh, const double
     free(l);
     return ORACLE_OK;
 }
+
+/*
+ * Rotary position embedding of T rows of dimension d (Methodology §4,
+ * Implementation Details: keys are quantized before RoPE, so attention
+ * rotates the dequantized keys). Reading (the pages do not define RoPE):
+ * the standard rotary embedding with the half-split pairing, channel i with
+ * channel i + d/2 for i < d/2, rotated by the angle pos * base^(-2i/d):
+ *   x'_i       = x_i cos - x_{i+d/2} sin
+ *   x'_{i+d/2} = x_i sin + x_{i+d/2} cos.
+ * pos[t] is the position of row t; the rotation is done in place.
+ */
+int oracle_rope(double* X, int64_t T, int d, const int64_t* pos, double base) {
+    if (d <= 0 || (d & 1) || T < 0 || !(base > 0.0)) return ORACLE_ERR_ARG;
+    const int h = d / 2;
+    for (int64_t t = 0; t < T; ++t) {
+        double* x = X + (size_t)t * d;
+        for (int i = 0; i < h; ++i) {
+            const double theta = pow(base, -2.0 * (double)i / (double)d);
+            const double ang = (double)pos[t] * theta;
+            const double c = cos(ang), s = sin(ang);
+            const double a = x[i], b = x[i + h];
+            x[i] = a * c - b * s;
+            x[i + h] = a * s + b * c;
+        }
+    }
+    return ORACLE_OK;
+}

@@ -37,8 +37,9 @@ def lib():
                                           ctypes.c_int, fp, ctypes.c_int, dp]
         L.oracle_attention_head.argtypes = [dp, ctypes.c_int, dp, dp, ctypes.c_int64,
                                             ctypes.c_int, ctypes.c_double, dp]
+        L.oracle_rope.argtypes = [dp, ctypes.c_int64, ctypes.c_int, i64p, ctypes.c_double]
         for f in ("oracle_hadamard", "oracle_kmeans", "oracle_encode_head",
-                  "oracle_dequant_head", "oracle_attention_head"):
+                  "oracle_dequant_head", "oracle_attention_head", "oracle_rope"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -253,3 +254,29 @@ def decode_with_residual(k_prompt: np.ndarray, v_prompt: np.ndarray, k_new: np.n
                     "s1": np.concatenate(s1[n], axis=2), "s2": np.concatenate(s2[n], axis=2),
                     "o": o[n]}
     return outs, state
+
+
+def rope(x: np.ndarray, positions, base: float = 10000.0) -> np.ndarray:
+    """Rotary embedding of x [..., T, d] at positions [T] (half-split pairing,
+    angle pos * base^(-2i/d)); returns a new fp64 array."""
+    x = np.array(x, dtype=np.float64, copy=True)
+    d = x.shape[-1]
+    T = x.shape[-2]
+    pos = np.ascontiguousarray(np.broadcast_to(np.asarray(positions, dtype=np.int64), (T,)))
+    flat = x.reshape(-1, T, d)
+    for i in range(flat.shape[0]):
+        row = np.ascontiguousarray(flat[i])
+        _check(lib().oracle_rope(_p(row, ctypes.c_double), T, d, _p(pos, ctypes.c_int64),
+                                 float(base)), "rope")
+        flat[i] = row
+    return flat.reshape(x.shape)
+
+
+def attention_rope(q: np.ndarray, Khat: np.ndarray, Vhat: np.ndarray, seq_lens=None,
+                   base: float = 10000.0, scale: Optional[float] = None) -> np.ndarray:
+    """Decode attention with keys quantized before RoPE (Methodology §4,
+    Implementation Details): key t of the cache (dequantized, Khat) is
+    rotated to position t before the dot product; q is the query already
+    rotated at its own position."""
+    T = Khat.shape[2]
+    return attention(q, rope(Khat, np.arange(T), base), Vhat, seq_lens, scale)

@@ -395,3 +395,55 @@ def test_decode_loop_with_a_one_token_window_quantizes_every_token(codebooks):
                        cat(eV, fV, "s2").astype(np.float32), eV["o"].astype(np.float32), C)
         ref = O.attention(qs[s], Kh, Vh)
         assert np.abs(outs[s] - ref).max() < 1e-12
+
+
+# ----------------------------------------------------------------- RoPE --
+def test_rope_matches_the_complex_rotation():
+    """The rotary embedding as complex multiplication: channel pair
+    (x_i, x_{i+64}) as x_i + 1j x_{i+64}, times exp(1j pos base^(-2i/d))
+    (an independent formulation of the same rotation)."""
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal((3, 11, D))
+    pos = np.array([0, 1, 2, 5, 17, 100, 1000, 4095, 32767, 131071, 7])
+    for base in (10000.0, 500000.0):
+        y = O.rope(x, pos, base)
+        i = np.arange(D // 2)
+        ang = pos[:, None] * base ** (-2.0 * i / D)
+        z = (x[..., :D // 2] + 1j * x[..., D // 2:]) * np.exp(1j * ang)
+        ref = np.concatenate([z.real, z.imag], axis=-1)
+        assert np.abs(y - ref).max() < 1e-9 * np.abs(x).max()
+
+
+def test_rope_is_a_rotation_with_relative_positions():
+    """Norm preserved, position 0 is the identity, and the dot product of a
+    query at m with a key at n depends only on m - n."""
+    rng = np.random.default_rng(8)
+    q = rng.standard_normal((1, D))
+    k = rng.standard_normal((1, D))
+    assert np.array_equal(O.rope(k, [0]), k)
+    for m, n in ((5, 3), (1000, 10), (77, 77), (3, 9)):
+        lhs = (O.rope(q, [m]) * O.rope(k, [n])).sum()
+        rhs = (O.rope(q, [m - n]) * k).sum()
+        assert abs(lhs - rhs) < 1e-10 * np.abs(q).sum() * np.abs(k).sum()
+        assert abs(np.linalg.norm(O.rope(k, [n])) - np.linalg.norm(k)) < 1e-12
+
+
+def test_attention_rope_is_sdpa_over_rotated_keys():
+    """Keys quantized before RoPE: attention rotates key t to position t,
+    checked against torch SDPA over keys rotated by the complex formulation."""
+    rng = np.random.default_rng(9)
+    B, Hq, Hkv, T = 2, 4, 2, 40
+    q = rng.standard_normal((B, Hq, D))
+    K = rng.standard_normal((B, Hkv, T, D)) * 1.2
+    V = rng.standard_normal((B, Hkv, T, D))
+    lens = [40, 13]
+    out = O.attention_rope(q, K, V, lens, base=10000.0)
+    i = np.arange(D // 2)
+    ang = np.arange(T)[:, None] * 10000.0 ** (-2.0 * i / D)
+    z = (K[..., :D // 2] + 1j * K[..., D // 2:]) * np.exp(1j * ang)
+    Kr = np.concatenate([z.real, z.imag], axis=-1)
+    G = Hq // Hkv
+    for b in range(B):
+        for h in range(Hq):
+            ref = _sdpa(q[b, h][None], Kr[b, h // G, :lens[b]], V[b, h // G, :lens[b]], 1 / np.sqrt(D))[0]
+            assert np.abs(out[b, h] - ref).max() < 1e-12
