@@ -41,7 +41,7 @@ N_CENTROIDS = 256
 EXPORTED = ("nsnq_status_string", "nsnq_last_error", "nsnq_codebook_index_bytes",
             "nsnq_codebook_index_build", "nsnq_encode_workspace", "nsnq_encode", "nsnq_dequant",
             "nsnq_attn_workspace", "nsnq_attn_decode", "nsnq_attn_decode_res",
-            "nsnq_residual_write", "nsnq_attn_decode_noalloc")
+            "nsnq_attn_decode_rope", "nsnq_residual_write", "nsnq_attn_decode_noalloc")
 
 
 class NSNQError(RuntimeError):
@@ -102,6 +102,10 @@ def load(path: str = LIB_PATH):
                                        _Residual, ci, ci, ci, ci, ctypes.c_float, vp, ci, vp, sz,
                                        vp]
     L.nsnq_attn_decode_res.restype = ci
+    L.nsnq_attn_decode_rope.argtypes = [vp, ci, _Cache, _Cache, _Codebook, _Codebook, vp, i64,
+                                        ctypes.c_double, ci, ci, ci, ci, ctypes.c_float, vp, ci, vp,
+                                        sz, vp]
+    L.nsnq_attn_decode_rope.restype = ci
     L.nsnq_residual_write.argtypes = [vp, ci, ci, ci, i64, ci, i64, i64, i64, i64, vp, ci, i64, vp]
     L.nsnq_residual_write.restype = ci
     L.nsnq_attn_decode_noalloc.argtypes = [vp, ci, _Cache, _Cache, _Codebook, _Codebook, vp, i64,
@@ -407,3 +411,27 @@ class DecodeCache:
         return nsnq_attn_decode_res(q, self.k, self.v, self.k_cb, self.v_cb, self.seq_lens,
                                     self.n_quant, self.Hkv, self.res, softmax_scale, out_dtype,
                                     stream=stream)
+
+
+def nsnq_attn_decode_rope(q: torch.Tensor, k_cache: Cache, v_cache: Cache, k_cb: Codebook,
+                          v_cb: Codebook, seq_lens: torch.Tensor, max_len: int, Hkv: int,
+                          rope_base: float = 10000.0, softmax_scale: float = 0.0,
+                          out_dtype: torch.dtype = torch.bfloat16,
+                          out: Optional[torch.Tensor] = None,
+                          workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Decode step over keys quantized before RoPE: key t is rotated to position t
+    in the kernel; q [B][Hq][D] is already rotated at its own position."""
+    B, Hq, D = q.shape
+    if out is None:
+        out = torch.empty(B, Hq, D, dtype=out_dtype, device=q.device)
+    if workspace is None:
+        workspace = _workspace(nsnq_attn_workspace(B, Hq, Hkv, max_len, D), q.device)
+    if seq_lens.dtype != torch.int32:
+        raise TypeError("seq_lens must be int32")
+    _check(load().nsnq_attn_decode_rope(_ptr(q), _dtype_code(q), k_cache._c(), v_cache._c(),
+                                        k_cb._c(), v_cb._c(), _ptr(seq_lens), max_len,
+                                        float(rope_base), B, Hq, Hkv, D, float(softmax_scale),
+                                        _ptr(out), _dtype_code(out), _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(),
+                                        _stream(stream)))
+    return out

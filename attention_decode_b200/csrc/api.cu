@@ -204,12 +204,15 @@ size_t nsnq_attn_workspace(int B, int Hq, int Hkv, int D, int64_t max_len) {
     return nsnq::plan_attention(B, Hq, Hkv, max_len).total;
 }
 
-nsnq_status nsnq_attn_decode_res(const void* q, nsnq_dtype q_dtype, nsnq_cache k_cache,
-                                 nsnq_cache v_cache, nsnq_codebook k_cb, nsnq_codebook v_cb,
-                                 const int32_t* seq_lens, int64_t max_len, nsnq_residual res,
-                                 int B, int Hq, int Hkv, int D, float softmax_scale, void* out,
-                                 nsnq_dtype out_dtype, void* workspace, size_t workspace_bytes,
-                                 nsnq_stream stream) {
+// Validates a decode-attention call and fills its arguments; *empty is set
+// when there is nothing to launch (B = 0).
+static nsnq_status attn_args(const void* q, nsnq_dtype q_dtype, nsnq_cache k_cache,
+                             nsnq_cache v_cache, nsnq_codebook k_cb, nsnq_codebook v_cb,
+                             const int32_t* seq_lens, int64_t max_len, nsnq_residual res,
+                             int B, int Hq, int Hkv, int D, float softmax_scale, void* out,
+                             nsnq_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                             nsnq::AttnArgs& a, bool* empty) {
+    *empty = false;
     if (D != nsnq::kHeadDim) return fail(NSNQ_ERR_UNSUPPORTED, "D = %d (only 128 is supported)", D);
     if ((q_dtype != NSNQ_F32 && q_dtype != NSNQ_BF16) ||
         (out_dtype != NSNQ_F32 && out_dtype != NSNQ_BF16))
@@ -239,7 +242,10 @@ nsnq_status nsnq_attn_decode_res(const void* q, nsnq_dtype q_dtype, nsnq_cache k
         if (!aligned(res.k, 16) || !aligned(res.v, 16) || !aligned(res.lens, 4))
             return fail(NSNQ_ERR_INVALID_ARG, "res.k and res.v must be 16-byte aligned");
     }
-    if (B == 0) return ok();
+    if (B == 0) {
+        *empty = true;
+        return ok();
+    }
     if (!q || !out || !seq_lens) return fail(NSNQ_ERR_INVALID_ARG, "q, out or seq_lens is NULL");
     if (!aligned(q, 16) || !aligned(out, 16) || !aligned(seq_lens, 4))
         return fail(NSNQ_ERR_INVALID_ARG, "q and out must be 16-byte aligned");
@@ -249,7 +255,7 @@ nsnq_status nsnq_attn_decode_res(const void* q, nsnq_dtype q_dtype, nsnq_cache k
                     workspace ? workspace_bytes : (size_t)0);
     if (!aligned(workspace, nsnq::kWsAlign))
         return fail(NSNQ_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
-    nsnq::AttnArgs a{};
+    a = nsnq::AttnArgs{};
     a.q = q; a.q_bf16 = q_dtype == NSNQ_BF16;
     a.kcodes = k_cache.codes; a.kscales = k_cache.scales; a.kshift = k_cache.shift;
     a.kcap = k_cache.cap; a.kC = k_cb.centroids; a.ksub = k_cb.sub_dim;
@@ -266,8 +272,44 @@ nsnq_status nsnq_attn_decode_res(const void* q, nsnq_dtype q_dtype, nsnq_cache k
         a.rk = res.k; a.rv = res.v; a.r_bf16 = res.dtype == NSNQ_BF16;
         a.res_lens = res.lens; a.rcap = res.cap;
     }
+    return NSNQ_OK;
+}
+
+nsnq_status nsnq_attn_decode_res(const void* q, nsnq_dtype q_dtype, nsnq_cache k_cache,
+                                 nsnq_cache v_cache, nsnq_codebook k_cb, nsnq_codebook v_cb,
+                                 const int32_t* seq_lens, int64_t max_len, nsnq_residual res,
+                                 int B, int Hq, int Hkv, int D, float softmax_scale, void* out,
+                                 nsnq_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                                 nsnq_stream stream) {
+    nsnq::AttnArgs a;
+    bool empty = false;
+    const nsnq_status s = attn_args(q, q_dtype, k_cache, v_cache, k_cb, v_cb, seq_lens, max_len, res, B,
+                                    Hq, Hkv, D, softmax_scale, out, out_dtype, workspace,
+                                    workspace_bytes, a, &empty);
+    if (s != NSNQ_OK || empty) return s;
     cudaError_t e = nsnq::launch_attention(a, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+    return ok();
+}
+
+nsnq_status nsnq_attn_decode_rope(const void* q, nsnq_dtype q_dtype, nsnq_cache k_cache,
+                                  nsnq_cache v_cache, nsnq_codebook k_cb, nsnq_codebook v_cb,
+                                  const int32_t* seq_lens, int64_t max_len, double rope_base,
+                                  int B, int Hq, int Hkv, int D, float softmax_scale, void* out,
+                                  nsnq_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                                  nsnq_stream stream) {
+    if (!isfinite(rope_base) || !(rope_base > 1.0))
+        return fail(NSNQ_ERR_INVALID_ARG, "rope_base = %g must be finite and > 1", rope_base);
+    nsnq::AttnArgs a;
+    bool empty = false;
+    nsnq_residual none{};
+    const nsnq_status s = attn_args(q, q_dtype, k_cache, v_cache, k_cb, v_cb, seq_lens, max_len, none,
+                                    B, Hq, Hkv, D, softmax_scale, out, out_dtype, workspace,
+                                    workspace_bytes, a, &empty);
+    if (s != NSNQ_OK || empty) return s;
+    a.rope_base = rope_base;
+    cudaError_t e = nsnq::launch_attention_rope(a, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "attention (rope) launch");
     return ok();
 }
 

@@ -13,6 +13,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "attn_split.cuh"
 
 namespace nsnq {
 
@@ -74,22 +75,6 @@ __device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
     asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
     return d;
 }
-// Balanced split of the flattened (unit, token) space over the CTAs: CTA c
-// covers virtual tokens [cta_begin(c), cta_begin(c + 1)).
-__host__ __device__ inline int64_t cta_begin(int c, const AttnPlan& p) {
-    const int64_t W = p.units * p.L;
-    return (W / p.ctas) * c + ((W % p.ctas) * c) / p.ctas;
-}
-// The CTA whose range holds virtual token v.
-__host__ __device__ inline int first_cta(int64_t v, const AttnPlan& p) {
-    const int64_t W = p.units * p.L;
-    int c = (int)((double)v * (double)p.ctas / (double)(W > 0 ? W : 1));
-    c = c < 0 ? 0 : (c >= p.ctas ? p.ctas - 1 : c);
-    while (c + 1 < p.ctas && cta_begin(c + 1, p) <= v) ++c;
-    while (c > 0 && cta_begin(c, p) > v) --c;
-    return c;
-}
-
 template <int GC, int KSUB, int VSUB, typename QT>
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a) {
     using S = AttnSmem<GC, KSUB, VSUB>;
@@ -522,6 +507,11 @@ static cudaError_t launch_split_gc(const AttnArgs& a, cudaStream_t s) {
     if (a.plan.gc == 4) return launch_split_sub<4, QT>(a, s);
     if (a.plan.gc == 2) return launch_split_sub<2, QT>(a, s);
     return launch_split_sub<1, QT>(a, s);
+}
+
+cudaError_t launch_attn_combine(const AttnArgs& a, cudaStream_t s) {
+    attn_combine_kernel<<<a.B * a.Hq, kD, 0, s>>>(a);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s) {

@@ -115,8 +115,12 @@ struct AttnArgs {
     int r_bf16;
     const int32_t* res_lens;
     int64_t rcap;
+    // keys quantized before RoPE: rotary base (the split kernel of attention_rope.cu)
+    double rope_base;
 };
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s);
+cudaError_t launch_attn_combine(const AttnArgs& a, cudaStream_t s);
+cudaError_t launch_attention_rope(const AttnArgs& a, cudaStream_t s);
 
 struct ResWriteArgs {
     const void* x;

@@ -359,6 +359,26 @@ def run_attention_bench(args, nsnq, dev, world, barrier, hbm, peak_kind):
     avg = max_over_ranks(sum(ms) / len(ms), world, dev)
     nbytes = B * H * T * attn_bytes_per_token(w.sub_dim, w.sub_dim)
     gbs = nbytes / (avg / 1e3) / 1e9
+    # the same caches read as keys quantized before RoPE (keys rotated in the kernel)
+    for _ in range(args.warmup):
+        nsnq.nsnq_attn_decode_rope(q, kc, vc, cb, cb, seq, T, Hkv=H, out=out, workspace=ws)
+    barrier()
+    torch.cuda.synchronize()
+    for e0, e1 in evs:
+        flush.zero_()
+        e0.record(stream)
+        nsnq.nsnq_attn_decode_rope(q, kc, vc, cb, cb, seq, T, Hkv=H, out=out, workspace=ws)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ravg = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / len(evs), world, dev)
+    rgbs = nbytes / (ravg / 1e3) / 1e9
+    rope = {"ms_per_call": round(ravg, 4), "value": round(rgbs * world, 1), "unit": "GB/s",
+            "roofline": {"bound": "hbm", "achieved": round(rgbs, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(rgbs / hbm, 4), "peak_kind": peak_kind,
+                         "kernel": "nsnq_attn_decode_rope (attn_rope_split + attn_combine)",
+                         "algorithmic_bytes_per_launch": nbytes,
+                         "traffic": measured_traffic("nsnq_attn_decode_rope")}}
     return {"metric": "decode-attn HBM GB/s (algorithmic bytes)", "value": round(gbs * world, 1),
             "unit": "GB/s", "ms_per_call": round(avg, 4),
             "workload": "decode-16x32k-2b (B 16, Hq 32, Hkv 8, T 32768, d 128, 2 bit K and V)",
@@ -367,7 +387,8 @@ def run_attention_bench(args, nsnq, dev, world, barrier, hbm, peak_kind):
                          "kernel": "nsnq_attn_decode (attn_split + attn_combine)",
                          "algorithmic_bytes_per_launch": nbytes,
                          "traffic": measured_traffic("nsnq_attn_decode")},
-            "l2": "flushed before every call (cache 335 MB > L2 anyway)"}
+            "l2": "flushed before every call (cache 335 MB > L2 anyway)",
+            "keys_before_rope": rope}
 
 
 def run_encode1_bench(args, nsnq, dev, world, barrier, hbm, peak_kind, x):

@@ -232,6 +232,26 @@ nsnq_status nsnq_residual_write(const void* x, nsnq_dtype x_dtype, int B, int H,
                                 nsnq_stream stream);
 
 /*
+ * nsnq_attn_decode_rope -- nsnq_attn_decode for keys quantized before the
+ * rotary position embedding (Methodology §4, Implementation Details: NSN is
+ * applied to the keys before RoPE). Key t of a sequence (cache position t)
+ * is dequantized, k_t = s1 (s2 H w_hat + o), rotated to position t and
+ * dotted with q, which the caller passes already rotated at its own
+ * position:
+ *   (k_i, k_{i+D/2}) -> (k_i c - k_{i+D/2} s, k_i s + k_{i+D/2} c),
+ *   c, s = cos, sin of t * rope_base^(-2i/D), i < D/2.
+ *   rope_base  finite, > 1 (10000 in most models).
+ * Values, workspace (nsnq_attn_workspace), outputs and errors are those of
+ * nsnq_attn_decode; there is no residual window here.
+ */
+nsnq_status nsnq_attn_decode_rope(const void* q, nsnq_dtype q_dtype, nsnq_cache k_cache,
+                                  nsnq_cache v_cache, nsnq_codebook k_cb, nsnq_codebook v_cb,
+                                  const int32_t* seq_lens, int64_t max_len, double rope_base,
+                                  int B, int Hq, int Hkv, int D, float softmax_scale, void* out,
+                                  nsnq_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                                  nsnq_stream stream);
+
+/*
  * nsnq_attn_decode_noalloc -- nsnq_attn_decode for callers that cannot
  * allocate device memory (no workspace argument). The method has no
  * counterpart for this: it is a packaging of the same kernels.

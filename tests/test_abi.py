@@ -165,6 +165,24 @@ def test_residual_attention_validation(lib):
     assert _attn_res(lib, R(k=None, v=None, lens=None, cap=0), B=0) == nsnq.NSNQ_OK
 
 
+def test_rope_attention_validation(lib):
+    def f(base=10000.0, **kw):
+        a = dict(q=FAKE, qdt=nsnq.NSNQ_BF16, kc=_cache(), vc=_cache(), kcb=_cb(4), vcb=_cb(8),
+                 lens=FAKE, max_len=100, B=2, Hq=8, Hkv=2, D=128, scale=0.0, out=FAKE,
+                 odt=nsnq.NSNQ_BF16, ws=FAKE, wsb=1 << 24)
+        a.update(kw)
+        return lib.nsnq_attn_decode_rope(a["q"], a["qdt"], a["kc"], a["vc"], a["kcb"], a["vcb"],
+                                         a["lens"], a["max_len"], base, a["B"], a["Hq"], a["Hkv"],
+                                         a["D"], a["scale"], a["out"], a["odt"], a["ws"], a["wsb"],
+                                         None)
+    assert f(base=float("nan")) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert f(base=1.0) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert f(Hq=6, Hkv=4) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert f(wsb=16) == nsnq.NSNQ_ERR_WORKSPACE
+    assert f(qdt=9) == nsnq.NSNQ_ERR_UNSUPPORTED
+    assert f(B=0) == nsnq.NSNQ_OK
+
+
 def test_residual_write_validation(lib):
     def f(**kw):
         a = dict(x=FAKE, dt=nsnq.NSNQ_BF16, B=2, H=2, T=1, D=128, sb=512, sh=256, st=128, off=3,
