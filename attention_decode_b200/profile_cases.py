@@ -11,6 +11,7 @@ Cases (seeded synthetic inputs generated on the device):
   attn-16x32k-2b       decode attention, B 16, Hq 32, Hkv 8, 32768 tokens, 2 bit
   attn-16x32k-1b       the same with 1-bit K and V
   attn-64x8k-gqa8      decode attention, B 64, Hq 64, Hkv 8, 8192 tokens, 2 bit
+  attn-rope-16x32k-2b  attn-16x32k-2b with the keys read as quantized before RoPE
 """
 from __future__ import annotations
 
@@ -57,7 +58,7 @@ def encode_case(B, H, T, reps, dev, sub=4):
           f"{sv} sub-vectors; index mismatch {mism}")
 
 
-def attn_case(B, Hq, Hkv, T, sub, reps, dev):
+def attn_case(B, Hq, Hkv, T, sub, reps, dev, rope=False):
     gen = torch.Generator(device=dev)
     gen.manual_seed(1)
     cb = _codebook(sub, dev)
@@ -72,8 +73,9 @@ def attn_case(B, Hq, Hkv, T, sub, reps, dev):
     seq = torch.full((B,), T, dtype=torch.int32, device=dev)
     ws = torch.empty(nsnq.nsnq_attn_workspace(B, Hq, Hkv, T), dtype=torch.uint8, device=dev)
     out = torch.empty(B, Hq, 128, dtype=torch.bfloat16, device=dev)
+    run = nsnq.nsnq_attn_decode_rope if rope else nsnq.nsnq_attn_decode
     for _ in range(reps):
-        nsnq.nsnq_attn_decode(q, kc, vc, cb, cb, seq, T, Hkv=Hkv, out=out, workspace=ws)
+        run(q, kc, vc, cb, cb, seq, T, Hkv=Hkv, out=out, workspace=ws)
     torch.cuda.synchronize()
 
 
@@ -84,6 +86,7 @@ CASES = {
     "encode1-8x8x4096": lambda r, d: encode_case(8, 8, 4096, r, d, sub=8),
     "attn-16x32k-2b": lambda r, d: attn_case(16, 32, 8, 32768, 4, r, d),
     "attn-16x32k-1b": lambda r, d: attn_case(16, 32, 8, 32768, 8, r, d),
+    "attn-rope-16x32k-2b": lambda r, d: attn_case(16, 32, 8, 32768, 4, r, d, rope=True),
     "attn-64x8k-gqa8": lambda r, d: attn_case(64, 64, 8, 8192, 4, r, d),
 }
 
