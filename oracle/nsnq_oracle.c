@@ -156,11 +156,51 @@ static int nearest_codeword(const double* w, const float* C, int K, int g) {
  * Outputs: codes [T][d/g], s1 [T], s2 [T], o_out [d], and optionally
  * w_out [T][d] (the transformed tokens that were quantized).
  */
+/*
+ * Double quantization (Methodology §3, Double Quantization: the NSN
+ * parameters o and s1 and the codebook entries are quantized to 4 bits).
+ * Reading (the pages give no scheme): 4-bit asymmetric uniform quantization,
+ * 16 levels from the minimum to the maximum of the values (step = range/15,
+ * level = round((x - min) / step), half away from zero); a constant input
+ * keeps its value.
+ */
+int oracle_quantize4(const double* x, int64_t n, double* xq) {
+    if (n < 0 || (n > 0 && (!x || !xq))) return ORACLE_ERR_ARG;
+    if (n == 0) return ORACLE_OK;
+    double lo = x[0], hi = x[0];
+    for (int64_t i = 1; i < n; ++i) {
+        if (x[i] < lo) lo = x[i];
+        if (x[i] > hi) hi = x[i];
+    }
+    const double step = (hi - lo) / 15.0;
+    for (int64_t i = 0; i < n; ++i) {
+        const double q = step > 0.0 ? round((x[i] - lo) / step) : 0.0;
+        xq[i] = lo + q * step;
+    }
+    return ORACLE_OK;
+}
+
+/*
+ * The 4-bit scale grid of one head: s1 is quantized on a grid uniform in
+ * log2 (s1 is a positive scale spanning orders of magnitude), from the
+ * least to the largest log2 s1 of the head's non-zero tokens. The grid
+ * (lo, step) is stored in fp32 and used in that rounding everywhere, so a
+ * later append reproduces the prompt's levels. A zero token keeps s1 = 0.
+ */
+static double s1_level_value(double s1, double lo, double step) {
+    if (!(s1 > 0.0)) return 0.0;
+    double k = step > 0.0 ? round((log2(s1) - lo) / step) : 0.0;
+    if (k < 0.0) k = 0.0;
+    if (k > 15.0) k = 15.0;
+    return exp2(lo + k * step);
+}
+
 int oracle_encode_head(const double* x, int64_t T, int d, int g, const float* C, int K,
-                       int shift_given, const double* o_in, int adaptive_scale, uint8_t* codes,
-                       double* s1, double* s2, double* o_out, double* w_out) {
+                       int shift_given, const double* o_in, int adaptive_scale, int double_quant,
+                       double* s1_grid, uint8_t* codes, double* s1, double* s2, double* o_out,
+                       double* w_out) {
     if (d <= 0 || (d & (d - 1)) != 0 || g <= 0 || d % g != 0 || g > 64 || K <= 0 || K > 256 ||
-        T < 0 || (shift_given && !o_in) || !C || !o_out)
+        T < 0 || (shift_given && !o_in) || !C || !o_out || (double_quant && !s1_grid))
         return ORACLE_ERR_ARG;
     const int J = d / g;
     const double sqrt_d = sqrt((double)d);
@@ -179,8 +219,27 @@ int oracle_encode_head(const double* x, int64_t T, int d, int g, const float* C,
         const double* xt = x + (size_t)t * d;
         double ss = 0.0;
         for (int c = 0; c < d; ++c) ss += xt[c] * xt[c];
-        double s = sqrt(ss) / sqrt_d;
-        s1[t] = s;
+        s1[t] = sqrt(ss) / sqrt_d;
+    }
+    if (double_quant) {  /* s1 on the head's 4-bit log2 grid (given, or from these tokens) */
+        if (!shift_given) {
+            double lo = 0.0, hi = 0.0;
+            int any = 0;
+            for (int64_t t = 0; t < T; ++t) {
+                if (!(s1[t] > 0.0)) continue;
+                const double l = log2(s1[t]);
+                if (!any || l < lo) lo = l;
+                if (!any || l > hi) hi = l;
+                any = 1;
+            }
+            s1_grid[0] = (double)(float)lo;
+            s1_grid[1] = (double)(float)((hi - lo) / 15.0);
+        }
+        for (int64_t t = 0; t < T; ++t) s1[t] = s1_level_value(s1[t], s1_grid[0], s1_grid[1]);
+    }
+    for (int64_t t = 0; t < T; ++t) {
+        const double* xt = x + (size_t)t * d;
+        const double s = s1[t];
         for (int c = 0; c < d; ++c) y[(size_t)t * d + c] = s > 0.0 ? xt[c] / s : 0.0;
     }
     /* Shift (channel-wise): o = mean over the T tokens, or the given o. */
@@ -193,6 +252,7 @@ int oracle_encode_head(const double* x, int64_t T, int d, int g, const float* C,
             o_out[c] = T > 0 ? acc / (double)T : 0.0;
         }
     }
+    if (double_quant && !shift_given) oracle_quantize4(o_out, d, o_out);  /* o on 16 levels */
     for (int64_t t = 0; t < T; ++t) {
         double* yt = y + (size_t)t * d;
         /* z = y - o; Normalize again: s2 = ||z|| / sqrt(d), u = z / s2.

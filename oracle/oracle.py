@@ -31,15 +31,17 @@ def lib():
         L.oracle_kmeans.argtypes = [dp, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                     dp, i64p]
         L.oracle_encode_head.argtypes = [dp, ctypes.c_int64, ctypes.c_int, ctypes.c_int, fp,
-                                         ctypes.c_int, ctypes.c_int, dp, ctypes.c_int, u8p, dp, dp,
-                                         dp, dp]
+                                         ctypes.c_int, ctypes.c_int, dp, ctypes.c_int, ctypes.c_int,
+                                         dp, u8p, dp, dp, dp, dp]
+        L.oracle_quantize4.argtypes = [dp, ctypes.c_int64, dp]
         L.oracle_dequant_head.argtypes = [u8p, fp, fp, fp, ctypes.c_int64, ctypes.c_int,
                                           ctypes.c_int, fp, ctypes.c_int, dp]
         L.oracle_attention_head.argtypes = [dp, ctypes.c_int, dp, dp, ctypes.c_int64,
                                             ctypes.c_int, ctypes.c_double, dp]
         L.oracle_rope.argtypes = [dp, ctypes.c_int64, ctypes.c_int, i64p, ctypes.c_double]
         for f in ("oracle_hadamard", "oracle_kmeans", "oracle_encode_head",
-                  "oracle_dequant_head", "oracle_attention_head", "oracle_rope"):
+                  "oracle_dequant_head", "oracle_attention_head", "oracle_rope",
+                  "oracle_quantize4"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -75,14 +77,18 @@ def kmeans(X: np.ndarray, k: int, iters: int):
 
 
 def encode(x: np.ndarray, codebook: np.ndarray, shift: Optional[np.ndarray] = None,
-           want_w: bool = False, adaptive_scale: bool = False):
+           want_w: bool = False, adaptive_scale: bool = False, double_quant: bool = False,
+           s1_grid: Optional[np.ndarray] = None):
     """Encode x [B][H][T][d] (exact fp64 values of the I/O type).
 
     shift None -> the shift is computed per (b, h) over the T tokens;
     else shift [B][H][d] is used as given. adaptive_scale -> s2 carries the
-    scale adjustment ||w||^2 / (w . w_hat).
+    scale adjustment ||w||^2 / (w . w_hat). double_quant -> s1 on the
+    head's 4-bit log2 grid (s1_grid [B][H][2] = (lo, step), given together
+    with the shift, else computed) and a computed o on 16 uniform levels.
     Returns dict with codes uint8 [B][H][T][d/g], s1, s2 fp64 [B][H][T],
-    o fp64 [B][H][d] and (optionally) w fp64 [B][H][T][d].
+    o fp64 [B][H][d], s1_grid fp64 [B][H][2] and (optionally) w fp64
+    [B][H][T][d].
     """
     x = np.ascontiguousarray(x, dtype=np.float64)
     B, H, T, d = x.shape
@@ -94,11 +100,15 @@ def encode(x: np.ndarray, codebook: np.ndarray, shift: Optional[np.ndarray] = No
     s2 = np.zeros((B, H, T))
     o = np.zeros((B, H, d))
     w = np.zeros((B, H, T, d)) if want_w else None
+    grid = np.zeros((B, H, 2))
+    if s1_grid is not None:
+        grid[...] = np.asarray(s1_grid, dtype=np.float64)
     for b in range(B):
         for h in range(H):
             oin = None
             if shift is not None:
                 oin = np.ascontiguousarray(shift[b, h], dtype=np.float64)
+            gb = np.ascontiguousarray(grid[b, h])
             ob = np.zeros(d)
             cb = np.zeros((T, J), dtype=np.uint8)
             s1b = np.zeros(T)
@@ -107,17 +117,28 @@ def encode(x: np.ndarray, codebook: np.ndarray, shift: Optional[np.ndarray] = No
             _check(lib().oracle_encode_head(
                 _p(np.ascontiguousarray(x[b, h]), ctypes.c_double), T, d, g,
                 _p(C, ctypes.c_float), K, 1 if shift is not None else 0,
-                _p(oin, ctypes.c_double), 1 if adaptive_scale else 0,
-                _p(cb, ctypes.c_uint8), _p(s1b, ctypes.c_double),
+                _p(oin, ctypes.c_double), 1 if adaptive_scale else 0, 1 if double_quant else 0,
+                _p(gb, ctypes.c_double), _p(cb, ctypes.c_uint8), _p(s1b, ctypes.c_double),
                 _p(s2b, ctypes.c_double), _p(ob, ctypes.c_double), _p(wb, ctypes.c_double)),
                 "encode")
             codes[b, h] = cb
             s1[b, h] = s1b
             s2[b, h] = s2b
             o[b, h] = ob
+            grid[b, h] = gb
             if want_w:
                 w[b, h] = wb
-    return {"codes": codes, "s1": s1, "s2": s2, "o": o, "w": w}
+    return {"codes": codes, "s1": s1, "s2": s2, "o": o, "w": w, "s1_grid": grid}
+
+
+def quantize4(x: np.ndarray) -> np.ndarray:
+    """4-bit asymmetric uniform quantization of all entries of x (16 levels
+    from min to max), fp64; for a codebook, its double-quantized entries."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    out = np.empty_like(x)
+    _check(lib().oracle_quantize4(_p(x.reshape(-1), ctypes.c_double), x.size,
+                                  _p(out.reshape(-1), ctypes.c_double)), "quantize4")
+    return out
 
 
 def dequant(codes: np.ndarray, s1: np.ndarray, s2: np.ndarray, o: np.ndarray,

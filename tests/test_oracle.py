@@ -447,3 +447,64 @@ def test_attention_rope_is_sdpa_over_rotated_keys():
         for h in range(Hq):
             ref = _sdpa(q[b, h][None], Kr[b, h // G, :lens[b]], V[b, h // G, :lens[b]], 1 / np.sqrt(D))[0]
             assert np.abs(out[b, h] - ref).max() < 1e-12
+
+
+# ----------------------------------------------------- double quantization --
+def test_quantize4_is_a_16_level_uniform_grid():
+    """Methodology §3 (Double Quantization), 4-bit reading: 16 uniform levels
+    from the minimum to the maximum, each value on its nearest level."""
+    rng = np.random.default_rng(10)
+    x = rng.standard_normal(1000) * 3 + 1
+    xq = O.quantize4(x)
+    lo, hi = x.min(), x.max()
+    step = (hi - lo) / 15
+    k = (xq - lo) / step
+    assert np.abs(k - np.round(k)).max() < 1e-9 and k.min() > -1e-9 and k.max() < 15 + 1e-9
+    assert len(np.unique(np.round(k))) <= 16
+    assert np.abs(x - xq).max() <= step / 2 + 1e-12
+    assert xq.min() == lo and abs(xq.max() - hi) < 1e-12
+    assert np.array_equal(O.quantize4(np.full(7, 2.5)), np.full(7, 2.5))
+    C = np.random.default_rng(11).standard_normal((256, 4)).astype(np.float32)
+    assert len(np.unique(O.quantize4(C))) <= 16
+
+
+@pytest.mark.parametrize("g", [8, 4])
+def test_double_quant_byproducts_and_reconstruction(codebooks, g):
+    """Double quantization: s1 on the head's 16-level log2 grid (the nearest
+    level of log2 of the exact s1, grid from the tokens' least to largest),
+    o on 16 uniform levels, and the byproducts still rebuild the token
+    exactly from the transformed vector (s2 absorbs the quantized s1)."""
+    x = _tiny_keys(T=64)
+    C = codebooks[g]
+    enc = O.encode(x, C, want_w=True, double_quant=True)
+    s1_exact = np.linalg.norm(x[0, 0], axis=1) / np.sqrt(D)
+    lg = np.log2(s1_exact)
+    lo = np.float32(lg.min()).astype(np.float64)
+    step = np.float32((lg.max() - lg.min()) / 15).astype(np.float64)
+    assert np.array_equal(enc["s1_grid"][0, 0], [lo, step])
+    k = np.clip(np.round((lg - lo) / step), 0, 15)
+    assert np.abs(enc["s1"][0, 0] - 2.0 ** (lo + k * step)).max() < 1e-12 * enc["s1"].max()
+    o = enc["o"][0, 0]
+    assert len(np.unique(np.round((o - o.min()) / ((o.max() - o.min()) / 15), 9))) <= 16
+    H = scipy.linalg.hadamard(D) / np.sqrt(D)
+    u = enc["w"][0, 0] @ H
+    rebuilt = enc["s1"][0, 0][:, None] * (enc["s2"][0, 0][:, None] * u + o[None, :])
+    assert np.abs(rebuilt - x[0, 0]).max() < 1e-12 * np.abs(x).max()
+    plain = O.encode(x, C)
+    assert not np.array_equal(plain["s1"], enc["s1"])
+    assert np.array_equal(plain["codes"], O.encode(x, C, double_quant=False)["codes"])
+
+
+def test_double_quant_append_uses_the_stored_grid(codebooks):
+    """Appended tokens (shift given) are quantized on the prompt's stored s1
+    grid, clamped to its 16 levels, with the stored o as the shift."""
+    x = _tiny_keys(T=80)
+    C = codebooks[4]
+    pre = O.encode(x[:, :, :48], C, double_quant=True)
+    new = np.concatenate([x[:, :, 48:], 40 * x[:, :, 48:50]], axis=2)  # two far above the grid
+    app = O.encode(new, C, shift=pre["o"], double_quant=True, s1_grid=pre["s1_grid"])
+    lo, step = pre["s1_grid"][0, 0]
+    k = (np.log2(app["s1"][0, 0]) - lo) / step
+    assert np.abs(k - np.round(k)).max() < 1e-9 and k.min() > -1e-9 and k.max() < 15 + 1e-9
+    assert np.allclose(app["s1"][0, 0, -2:], 2.0 ** (lo + 15 * step))
+    assert np.array_equal(app["o"], pre["o"]) and np.array_equal(app["s1_grid"], pre["s1_grid"])
