@@ -34,7 +34,7 @@ LIB_PATH = os.path.join(_HERE, "_build", "libnsnq.so")
 NSNQ_OK, NSNQ_ERR_INVALID_ARG, NSNQ_ERR_UNSUPPORTED, NSNQ_ERR_WORKSPACE, NSNQ_ERR_CUDA = range(5)
 NSNQ_F32, NSNQ_BF16 = 0, 1
 SHIFT_COMPUTE, SHIFT_GIVEN = 0, 1
-ENCODE_DEFAULT, ENCODE_ADAPTIVE_SCALE = 0, 1
+ENCODE_DEFAULT, ENCODE_ADAPTIVE_SCALE, ENCODE_DOUBLE_QUANT = 0, 1, 2
 HEAD_DIM = 128
 N_CENTROIDS = 256
 
@@ -57,7 +57,8 @@ class _Codebook(ctypes.Structure):
 
 class _Cache(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
-                ("shift", ctypes.c_void_p), ("cap", ctypes.c_int64)]
+                ("shift", ctypes.c_void_p), ("cap", ctypes.c_int64),
+                ("s1_grid", ctypes.c_void_p)]
 
 
 class _Residual(ctypes.Structure):
@@ -176,10 +177,12 @@ class Codebook:
 @dataclasses.dataclass
 class Cache:
     """One quantized tensor (K or V): codes [B][H][cap][D/g] uint8,
-    scales [B][H][cap][2] fp32 (s1, s2), shift [B][H][D] fp32 (o)."""
+    scales [B][H][cap][2] fp32 (s1, s2), shift [B][H][D] fp32 (o) and, for
+    double quantization, s1_grid [B][H][2] fp32 (lo, step of the log2 grid)."""
     codes: torch.Tensor
     scales: torch.Tensor
     shift: torch.Tensor
+    s1_grid: Optional[torch.Tensor] = None
 
     @property
     def cap(self) -> int:
@@ -189,10 +192,12 @@ class Cache:
     def empty(cls, B: int, H: int, cap: int, sub_dim: int, device="cuda", D: int = HEAD_DIM):
         return cls(torch.zeros(B, H, cap, D // sub_dim, dtype=torch.uint8, device=device),
                    torch.zeros(B, H, cap, 2, dtype=torch.float32, device=device),
-                   torch.zeros(B, H, D, dtype=torch.float32, device=device))
+                   torch.zeros(B, H, D, dtype=torch.float32, device=device),
+                   torch.zeros(B, H, 2, dtype=torch.float32, device=device))
 
     def _c(self) -> _Cache:
-        return _Cache(_ptr(self.codes), _ptr(self.scales), _ptr(self.shift), self.cap)
+        return _Cache(_ptr(self.codes), _ptr(self.scales), _ptr(self.shift), self.cap,
+                      _ptr(self.s1_grid))
 
 
 def nsnq_encode_workspace(B: int, H: int, T: int, D: int = HEAD_DIM) -> int:

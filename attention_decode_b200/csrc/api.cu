@@ -120,8 +120,11 @@ nsnq_status nsnq_encode(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t
         return fail(NSNQ_ERR_UNSUPPORTED, "x_dtype = %d", (int)x_dtype);
     if (mode != NSNQ_SHIFT_COMPUTE && mode != NSNQ_SHIFT_GIVEN)
         return fail(NSNQ_ERR_INVALID_ARG, "shift mode = %d", (int)mode);
-    if (flags & ~(unsigned)NSNQ_ENCODE_ADAPTIVE_SCALE)
+    if (flags & ~(unsigned)(NSNQ_ENCODE_ADAPTIVE_SCALE | NSNQ_ENCODE_DOUBLE_QUANT))
         return fail(NSNQ_ERR_INVALID_ARG, "unknown encode flags 0x%x", flags);
+    const bool dq = (flags & NSNQ_ENCODE_DOUBLE_QUANT) != 0;
+    if (dq && (!cache.s1_grid || !aligned(cache.s1_grid, 8)))
+        return fail(NSNQ_ERR_INVALID_ARG, "double quantization needs cache.s1_grid (8-byte aligned)");
     if (B < 0 || H < 0 || T < 0)
         return fail(NSNQ_ERR_INVALID_ARG, "negative size B=%d H=%d T=%lld", B, H, (long long)T);
     if (B > 65535 || H > 65535) return fail(NSNQ_ERR_UNSUPPORTED, "B or H above 65535");
@@ -157,6 +160,8 @@ nsnq_status nsnq_encode(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t
     a.t_offset = t_offset;
     a.given_shift = mode == NSNQ_SHIFT_GIVEN;
     a.adaptive = (flags & NSNQ_ENCODE_ADAPTIVE_SCALE) ? 1 : 0;
+    a.dq = dq ? 1 : 0;
+    a.s1_grid = cache.s1_grid;
     a.C = cb.centroids;
     a.sub = cb.sub_dim;
     a.index = cb.index;
@@ -165,6 +170,7 @@ nsnq_status nsnq_encode(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t
     a.stats = reinterpret_cast<unsigned long long*>(ws);
     a.partial = reinterpret_cast<double*>(ws + plan.partial_off);
     a.o64 = reinterpret_cast<double*>(ws + plan.o64_off);
+    a.minmax = reinterpret_cast<double*>(ws + plan.minmax_off);
     a.nchunk1 = plan.nchunk1;
     a.chunk1 = plan.chunk1;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

@@ -3,6 +3,8 @@
 // Technical Summary, Methodology §1-§3).
 //
 // Three launches per call in shift-compute mode, one in shift-given mode:
+//   nsn_s1minmax_kernel per (b, h, chunk), double quantization only: least and
+//                      largest log2 s1 (the per-head s1 grid)
 //   nsn_stats_kernel   per (b, h, chunk): channel sums of y = x / s1 in fp64
 //   nsn_shift_kernel   per (b, h): o = sum / T (fp64, kept in the workspace
 //                      for the near-tie path) and its fp32 copy in the cache
@@ -12,6 +14,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "dq.cuh"
 #include "internal.h"
 
 namespace nsnq {
@@ -67,7 +70,56 @@ struct Raw16<float> {
     }
 };
 
+// Least and largest log2 s1 of a chunk's non-zero tokens (8 lanes per token,
+// fp64 sum of squares as in the stats kernel).
 template <typename XT>
+__global__ void __launch_bounds__(kStatsThreads) nsn_s1minmax_kernel(EncodeArgs a) {
+    const int chunk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = lane_id();
+    const int tk = lane >> 3, cg = lane & 7;
+    const int64_t t0 = (int64_t)chunk * a.chunk1;
+    const int64_t t1 = min(t0 + a.chunk1, a.T);
+    const XT* xb = reinterpret_cast<const XT*>(a.x) + b * a.sb + h * a.sh + 16 * cg;
+    const double sqrt_d = sqrt((double)kD);
+    constexpr int64_t kStride = 4 * (kStatsThreads / 32);
+    double mn = INFINITY, mx = -INFINITY;
+    for (int64_t t = t0 + warp * 4 + tk; t - tk < t1; t += kStride) {
+        Raw16<XT> r;
+        if (t < t1) r.load(xb + t * a.st); else r.zero();
+        float v[16];
+        r.unpack(v);
+        double ss = 0.0;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) ss = fma((double)v[c], (double)v[c], ss);
+        ss += __shfl_xor_sync(kFull, ss, 1);
+        ss += __shfl_xor_sync(kFull, ss, 2);
+        ss += __shfl_xor_sync(kFull, ss, 4);
+        if (t < t1 && ss > 0.0) {
+            const double l = log2(sqrt(ss) / sqrt_d);
+            mn = fmin(mn, l);
+            mx = fmax(mx, l);
+        }
+    }
+#pragma unroll
+    for (int m = 8; m < 32; m <<= 1) {
+        mn = fmin(mn, __shfl_xor_sync(kFull, mn, m));
+        mx = fmax(mx, __shfl_xor_sync(kFull, mx, m));
+    }
+    __shared__ double red[kStatsThreads / 32][2];
+    if (lane == 0) { red[warp][0] = mn; red[warp][1] = mx; }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < kStatsThreads / 32; ++w) {
+            mn = fmin(mn, red[w][0]);
+            mx = fmax(mx, red[w][1]);
+        }
+        double* out = a.minmax + ((int64_t)(b * a.H + h) * a.nchunk1 + chunk) * 2;
+        out[0] = mn;
+        out[1] = mx;
+    }
+}
+
+template <typename XT, bool DQ>
 __global__ void __launch_bounds__(kStatsThreads) nsn_stats_kernel(EncodeArgs a) {
     const int chunk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = lane_id();
@@ -77,6 +129,9 @@ __global__ void __launch_bounds__(kStatsThreads) nsn_stats_kernel(EncodeArgs a) 
     const XT* xb = reinterpret_cast<const XT*>(a.x) + b * a.sb + h * a.sh + 16 * cg;
     const double sqrt_d = sqrt((double)kD);
     constexpr int64_t kStride = 4 * (kStatsThreads / 32);  // tokens per CTA step
+    double glo = 0.0, gstep = 0.0;
+    if constexpr (DQ)
+        dq_grid_from_chunks(a.minmax + (int64_t)(b * a.H + h) * a.nchunk1 * 2, a.nchunk1, glo, gstep);
     double acc[16];
 #pragma unroll
     for (int c = 0; c < 16; ++c) acc[c] = 0.0;
@@ -101,7 +156,12 @@ __global__ void __launch_bounds__(kStatsThreads) nsn_stats_kernel(EncodeArgs a) 
             ss += __shfl_xor_sync(kFull, ss, 2);
             ss += __shfl_xor_sync(kFull, ss, 4);
             if (ss > 0.0) {
-                const double inv = rsqrt(ss) * sqrt_d;  // 1 / s1
+                double inv;  // 1 / s1
+                if constexpr (DQ) {
+                    inv = 1.0 / dq_s1(sqrt(ss) / sqrt_d, glo, gstep);
+                } else {
+                    inv = rsqrt(ss) * sqrt_d;
+                }
 #pragma unroll
                 for (int c = 0; c < 16; ++c) acc[c] = fma((double)v[c], inv, acc[c]);
             }
@@ -127,12 +187,36 @@ __global__ void __launch_bounds__(kStatsThreads) nsn_stats_kernel(EncodeArgs a) 
     }
 }
 
+template <bool DQ>
 __global__ void __launch_bounds__(kD) nsn_shift_kernel(EncodeArgs a) {
     const int bh = blockIdx.x;
     const int c = threadIdx.x;
     double s = 0.0;
     for (int k = 0; k < a.nchunk1; ++k) s += a.partial[((int64_t)bh * a.nchunk1 + k) * kD + c];
-    const double o = a.T > 0 ? s / (double)a.T : 0.0;
+    double o = a.T > 0 ? s / (double)a.T : 0.0;
+    if constexpr (DQ) {
+        // o on 16 uniform levels between its least and largest channel value
+        __shared__ double red[kD / 32][2];
+        double mn = o, mx = o;
+#pragma unroll
+        for (int m = 1; m < 32; m <<= 1) {
+            mn = fmin(mn, __shfl_xor_sync(kFull, mn, m));
+            mx = fmax(mx, __shfl_xor_sync(kFull, mx, m));
+        }
+        if ((c & 31) == 0) { red[c >> 5][0] = mn; red[c >> 5][1] = mx; }
+        __syncthreads();
+        mn = red[0][0]; mx = red[0][1];
+#pragma unroll
+        for (int w = 1; w < kD / 32; ++w) { mn = fmin(mn, red[w][0]); mx = fmax(mx, red[w][1]); }
+        const double step = (mx - mn) / 15.0;
+        o = mn + (step > 0.0 ? round((o - mn) / step) : 0.0) * step;
+        if (c == 0) {
+            double lo, st;
+            dq_grid_from_chunks(a.minmax + (int64_t)bh * a.nchunk1 * 2, a.nchunk1, lo, st);
+            a.s1_grid[2 * bh] = (float)lo;
+            a.s1_grid[2 * bh + 1] = (float)st;
+        }
+    }
     a.o64[(int64_t)bh * kD + c] = o;
     a.shift[(int64_t)bh * kD + c] = (float)o;
 }
@@ -146,15 +230,23 @@ EncodePlan plan_encode(int B, int H, int64_t T) {
     p.partial_off = align_up(kEncodeStatsBytes, kWsAlign);
     const size_t partial_bytes = (size_t)B * H * p.nchunk1 * kD * sizeof(double);
     p.o64_off = align_up(p.partial_off + partial_bytes, kWsAlign);
-    p.total = align_up(p.o64_off + (size_t)B * H * kD * sizeof(double), kWsAlign);
+    p.minmax_off = align_up(p.o64_off + (size_t)B * H * kD * sizeof(double), kWsAlign);
+    p.total = align_up(p.minmax_off + (size_t)B * H * p.nchunk1 * 2 * sizeof(double), kWsAlign);
     return p;
 }
 
 template <typename XT>
 static cudaError_t launch_encode_t(const EncodeArgs& a, cudaStream_t s) {
     if (!a.given_shift) {
-        nsn_stats_kernel<XT><<<dim3(a.nchunk1, a.H, a.B), kStatsThreads, 0, s>>>(a);
-        nsn_shift_kernel<<<a.B * a.H, kD, 0, s>>>(a);
+        const dim3 grid1(a.nchunk1, a.H, a.B);
+        if (a.dq) {
+            nsn_s1minmax_kernel<XT><<<grid1, kStatsThreads, 0, s>>>(a);
+            nsn_stats_kernel<XT, true><<<grid1, kStatsThreads, 0, s>>>(a);
+            nsn_shift_kernel<true><<<a.B * a.H, kD, 0, s>>>(a);
+        } else {
+            nsn_stats_kernel<XT, false><<<grid1, kStatsThreads, 0, s>>>(a);
+            nsn_shift_kernel<false><<<a.B * a.H, kD, 0, s>>>(a);
+        }
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;

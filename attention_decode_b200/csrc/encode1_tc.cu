@@ -21,6 +21,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "dq.cuh"
 #include "internal.h"
 
 namespace nsnq {
@@ -129,7 +130,8 @@ __device__ __forceinline__ float half_sum(float v) {
 template <typename XT>
 __device__ __noinline__ void exact_warp_tc(const XT* xtok, const double* o64, const float* o32,
                                            const float* C, uint32_t flags, uint4& codes,
-                                           double& s1_out, double& s2_out, double& wq_out) {
+                                           double s1_fixed, double& s1_out, double& s2_out,
+                                           double& wq_out) {
     const int lane = lane_id();
     float xf[4];
     load4(xtok + 4 * lane, xf);
@@ -141,7 +143,7 @@ __device__ __noinline__ void exact_warp_tc(const XT* xtok, const double* o64, co
     }
     const double sqrt_d = sqrt((double)kD);
     const double ss = warp_sum_d(x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3]);
-    const double s1 = sqrt(ss) / sqrt_d;
+    const double s1 = s1_fixed >= 0.0 ? s1_fixed : sqrt(ss) / sqrt_d;  // fixed: quantized s1
     const double inv1 = s1 > 0.0 ? 1.0 / s1 : 0.0;
     double z[4], ss2 = 0.0, yy = 0.0, oo = 0.0;
 #pragma unroll
@@ -205,7 +207,7 @@ __device__ __noinline__ void exact_warp_tc(const XT* xtok, const double* o64, co
     s2_out = s2;
 }
 
-template <typename XT, bool ADAPT>
+template <typename XT, bool ADAPT, bool DQ>
 __global__ void __launch_bounds__(kTcThreads) nsn_encode1_tc_kernel(EncodeArgs a) {
     extern __shared__ __align__(1024) uint8_t smraw[];
     // the base of dynamic shared memory is at least 16-byte aligned; align to 1024
@@ -298,8 +300,21 @@ __global__ void __launch_bounds__(kTcThreads) nsn_encode1_tc_kernel(EncodeArgs a
 #pragma unroll
         for (int k = 0; k < 8; ++k) ss = fmaf(v[k], v[k], ss);
         ss = half_sum(ss);
-        const float s1 = sqrtf(ss * (1.0f / kD));
-        const float inv1 = s1 > 0.f ? 1.0f / s1 : 0.f;
+        float s1 = sqrtf(ss * (1.0f / kD));
+        float inv1 = s1 > 0.f ? 1.0f / s1 : 0.f;
+        double s1dq = -1.0;
+        if constexpr (DQ) {  // s1 on the head's 4-bit log2 grid, level decided in fp64
+            double ss64 = 0.0;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) ss64 = fma((double)v[k], (double)v[k], ss64);
+#pragma unroll
+            for (int m = 1; m < 16; m <<= 1) ss64 += __shfl_xor_sync(kFull, ss64, m);
+            double glo, gstep;
+            dq_grid(a.s1_grid, bh, glo, gstep);
+            s1dq = dq_s1(sqrt(ss64) / sqrt((double)kD), glo, gstep);
+            s1 = (float)s1dq;
+            inv1 = s1dq > 0.0 ? (float)(1.0 / s1dq) : 0.f;
+        }
         const float4* o4 = reinterpret_cast<const float4*>(a.shift + bh * kD + 8 * l16);
         const float4 oa = o4[0], ob = o4[1];
         const float o[8] = {oa.x, oa.y, oa.z, oa.w, ob.x, ob.y, ob.z, ob.w};
@@ -430,8 +445,9 @@ __global__ void __launch_bounds__(kTcThreads) nsn_encode1_tc_kernel(EncodeArgs a
                 uint4 cq = make_uint4(__shfl_sync(kFull, codes.x, 16 * hh), __shfl_sync(kFull, codes.y, 16 * hh),
                                       __shfl_sync(kFull, codes.z, 16 * hh), __shfl_sync(kFull, codes.w, 16 * hh));
                 double s1d, s2d, wq64;
-                exact_warp_tc<XT>(xhead + (t0 + hh) * a.st, o64, a.shift + bh * kD, Cs, flags, cq, s1d,
-                                  s2d, wq64);
+                const double s1f = __shfl_sync(kFull, s1dq, 16 * hh);
+                exact_warp_tc<XT>(xhead + (t0 + hh) * a.st, o64, a.shift + bh * kD, Cs, flags, cq, s1f,
+                                  s1d, s2d, wq64);
                 if (half == hh) {
                     codes = cq;
                     s1o = (float)s1d;
@@ -467,9 +483,9 @@ __global__ void __launch_bounds__(kTcThreads) nsn_encode1_tc_kernel(EncodeArgs a
     }
 }
 
-template <typename XT, bool ADAPT>
+template <typename XT, bool ADAPT, bool DQ>
 cudaError_t launch_tc(const EncodeArgs& a, cudaStream_t s) {
-    auto kern = nsn_encode1_tc_kernel<XT, ADAPT>;
+    auto kern = nsn_encode1_tc_kernel<XT, ADAPT, DQ>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
@@ -486,9 +502,13 @@ cudaError_t launch_tc(const EncodeArgs& a, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_encode1_tc(const EncodeArgs& a, cudaStream_t s) {
-    if (a.adaptive)
-        return a.x_bf16 ? launch_tc<__nv_bfloat16, true>(a, s) : launch_tc<float, true>(a, s);
-    return a.x_bf16 ? launch_tc<__nv_bfloat16, false>(a, s) : launch_tc<float, false>(a, s);
+    if (a.x_bf16) {
+        if (a.dq) return a.adaptive ? launch_tc<__nv_bfloat16, true, true>(a, s)
+                                    : launch_tc<__nv_bfloat16, false, true>(a, s);
+        return a.adaptive ? launch_tc<__nv_bfloat16, true, false>(a, s) : launch_tc<__nv_bfloat16, false, false>(a, s);
+    }
+    if (a.dq) return a.adaptive ? launch_tc<float, true, true>(a, s) : launch_tc<float, false, true>(a, s);
+    return a.adaptive ? launch_tc<float, true, false>(a, s) : launch_tc<float, false, false>(a, s);
 }
 
 }  // namespace nsnq

@@ -15,6 +15,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "dq.cuh"
 #include "vq_index.cuh"
 
 namespace nsnq {
@@ -99,7 +100,8 @@ __device__ __forceinline__ void load64<float>(const float* p, float (&v)[64]) {
 }
 
 // Exact decision for one token-head, by the whole warp: fp64 NSN of the
-// token (lane l holds channels 4l..4l+3), fp64 Hadamard transform across the
+// token (lane l holds channels 4l..4l+3; s1_fixed >= 0 is a given, double-
+// quantized s1), fp64 Hadamard transform across the
 // warp, after which lane l holds sub-vector l of w; each flagged lane scans
 // its cell list in fp64 (the list holds every codeword that can be nearest
 // there; lowest index on exact ties). Returns this lane's code (old_code when
@@ -110,8 +112,8 @@ template <typename XT>
 __device__ __noinline__ int exact_warp(const XT* xtok, const double* o64, const float* o32,
                                        const float4* reps, const uint16_t* offs,
                                        const uint16_t* ents, uint32_t flags, int old_code,
-                                       double& s1_out, double& s2_out, double& wq_all,
-                                       double& wq_delta) {
+                                       double s1_fixed, double& s1_out, double& s2_out,
+                                       double& wq_all, double& wq_delta) {
     const int lane = lane_id();
     float xf[4];
     load4(xtok + 4 * lane, xf);
@@ -123,7 +125,7 @@ __device__ __noinline__ int exact_warp(const XT* xtok, const double* o64, const 
     }
     const double sqrt_d = sqrt((double)kD);
     const double ss = warp_sum_d(x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3]);
-    const double s1 = sqrt(ss) / sqrt_d;
+    const double s1 = s1_fixed >= 0.0 ? s1_fixed : sqrt(ss) / sqrt_d;  // fixed: quantized s1
     const double inv1 = s1 > 0.0 ? 1.0 / s1 : 0.0;
     double z[4], ss2 = 0.0, yy = 0.0, oo = 0.0;
 #pragma unroll
@@ -239,8 +241,9 @@ struct Walk {
 
 // ADAPT: also apply the scale adjustment s2 *= ||w||^2 / (w . w_hat). Since
 // u = z / s2 has ||u||^2 = d and H is orthonormal, ||w||^2 = d; only w . w_hat
-// is accumulated, in the search loop.
-template <typename XT, bool ADAPT>
+// is accumulated, in the search loop. DQ: s1 on the head's 4-bit log2 grid,
+// its level decided from an fp64 sum of squares.
+template <typename XT, bool ADAPT, bool DQ>
 __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(EncodeArgs a) {
     extern __shared__ __align__(16) uint8_t sm[];
     float4* reps = reinterpret_cast<float4*>(sm + kSmReps);
@@ -327,8 +330,20 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
         float2 s01 = upk(add2(acc0, acc1));
         float ss = s01.x + s01.y;
         ss += __shfl_xor_sync(kFull, ss, 1);
-        const float s1 = sqrtf(ss * (1.0f / kD));
-        const float inv1 = s1 > 0.f ? 1.0f / s1 : 0.f;
+        float s1 = sqrtf(ss * (1.0f / kD));
+        float inv1 = s1 > 0.f ? 1.0f / s1 : 0.f;
+        double s1dq = -1.0;
+        if constexpr (DQ) {
+            double ss64 = 0.0;
+#pragma unroll
+            for (int k = 0; k < 64; ++k) ss64 = fma((double)v[k], (double)v[k], ss64);
+            ss64 += __shfl_xor_sync(kFull, ss64, 1);
+            double glo, gstep;
+            dq_grid(a.s1_grid, bh, glo, gstep);
+            s1dq = dq_s1(sqrt(ss64) / sqrt((double)kD), glo, gstep);
+            s1 = (float)s1dq;
+            inv1 = s1dq > 0.0 ? (float)(1.0 / s1dq) : 0.f;
+        }
         const float4* o4 = shift4 + 17 * half;  // upper half stored 4 floats further
         acc0 = 0; acc1 = 0;
         const uint64_t inv2 = pk(inv1, inv1);
@@ -419,9 +434,10 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
                 }
                 const int old_code = (int)((word >> (8 * (lane & 3))) & 0xffu);
                 double s1d, s2d, wq_all, wq_delta;
+                const double s1f = __shfl_sync(kFull, s1dq, src);
                 const int code = exact_warp<XT>(xhead + (t0 + (src >> 1)) * a.st, o64,
                                                 a.shift + bh * kD, reps, offs, ents, flags,
-                                                old_code, s1d, s2d, wq_all, wq_delta);
+                                                old_code, s1f, s1d, s2d, wq_all, wq_delta);
                 const bool mine = (lane >> 1) == (src >> 1);
 #pragma unroll
                 for (int jj = 0; jj < 16; ++jj) {
@@ -455,9 +471,9 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
 
 size_t pruned_smem_bytes() { return kSmBytes; }
 
-template <typename XT, bool ADAPT>
+template <typename XT, bool ADAPT, bool DQ>
 static cudaError_t launch_pruned_t(const EncodeArgs& a, cudaStream_t s) {
-    auto kern = nsn_encode_pruned_kernel<XT, ADAPT>;
+    auto kern = nsn_encode_pruned_kernel<XT, ADAPT, DQ>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmBytes);
     if (e != cudaSuccess) return e;
@@ -472,9 +488,14 @@ static cudaError_t launch_pruned_t(const EncodeArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_encode_pruned(const EncodeArgs& a, cudaStream_t s) {
-    if (a.adaptive)
-        return a.x_bf16 ? launch_pruned_t<__nv_bfloat16, true>(a, s) : launch_pruned_t<float, true>(a, s);
-    return a.x_bf16 ? launch_pruned_t<__nv_bfloat16, false>(a, s) : launch_pruned_t<float, false>(a, s);
+    if (a.x_bf16) {
+        if (a.dq) return a.adaptive ? launch_pruned_t<__nv_bfloat16, true, true>(a, s)
+                                    : launch_pruned_t<__nv_bfloat16, false, true>(a, s);
+        return a.adaptive ? launch_pruned_t<__nv_bfloat16, true, false>(a, s)
+                          : launch_pruned_t<__nv_bfloat16, false, false>(a, s);
+    }
+    if (a.dq) return a.adaptive ? launch_pruned_t<float, true, true>(a, s) : launch_pruned_t<float, false, true>(a, s);
+    return a.adaptive ? launch_pruned_t<float, true, false>(a, s) : launch_pruned_t<float, false, false>(a, s);
 }
 
 }  // namespace nsnq

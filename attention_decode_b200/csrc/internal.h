@@ -29,6 +29,8 @@ struct EncodeArgs {
     int64_t t_offset;
     int given_shift;
     int adaptive;  // scale adjustment folded into s2
+    int dq;        // double quantization of s1 and o
+    float* s1_grid;  // [B][H][2] (lo, step) of the log2 s1 grid
     const float* C;
     int sub;
     const void* index;  // search index (sub == 4)
@@ -40,6 +42,7 @@ struct EncodeArgs {
     unsigned long long* stats;  // [8]
     double* partial;            // [B][H][nchunk1][128]
     double* o64;                // [B][H][128]
+    double* minmax;             // [B][H][nchunk1][2] least / largest log2 s1 per chunk
     int nchunk1;
     int64_t chunk1;
 };
@@ -47,7 +50,7 @@ struct EncodeArgs {
 struct EncodePlan {
     int nchunk1;
     int64_t chunk1;
-    size_t partial_off, o64_off, total;
+    size_t partial_off, o64_off, minmax_off, total;
 };
 
 EncodePlan plan_encode(int B, int H, int64_t T);

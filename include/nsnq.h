@@ -69,7 +69,16 @@ typedef enum {
      * ||w||^2 / (w . w_hat) so that its component along the transformed token w
      * equals w (the error left is orthogonal to w); the factor multiplies the
      * stored s2, so dequant and attention need no change. */
-    NSNQ_ENCODE_ADAPTIVE_SCALE = 1
+    NSNQ_ENCODE_ADAPTIVE_SCALE = 1,
+    /* Double quantization (Methodology §3): s1 takes one of 16 levels of a
+     * per-head grid uniform in log2 (grid = (lo, step), from the least to
+     * the largest log2 s1 of the tokens encoded in shift-compute mode, kept
+     * in cache.s1_grid for later shift-given appends), and a computed o takes
+     * one of 16 uniform levels between its least and largest channel value.
+     * The level values are stored in the usual fp32 fields (the 4-bit level
+     * indices follow from them), so dequant and attention need no change.
+     * Requires cache.s1_grid. */
+    NSNQ_ENCODE_DOUBLE_QUANT = 2
 } nsnq_encode_flags;
 
 typedef struct {
@@ -86,6 +95,8 @@ typedef struct {
     float* scales;    /* device, [B][H][cap][2] = (s1, s2) */
     float* shift;     /* device, [B][H][D] = o */
     int64_t cap;      /* token capacity per (batch, head) */
+    float* s1_grid;   /* device, [B][H][2] = (lo, step) of the double-quantized s1 grid
+                         (log2 domain), or NULL without double quantization */
 } nsnq_cache;
 
 /* Human-readable name of a status code (static string). */
@@ -136,7 +147,8 @@ size_t nsnq_encode_workspace(int B, int H, int64_t T, int D);
  *             dtype x_dtype (fp32 or bf16); 16-byte aligned rows.
  *   mode      NSNQ_SHIFT_COMPUTE: o = mean over the T tokens of x/s1, stored
  *             to cache.shift (fp32); NSNQ_SHIFT_GIVEN: o = cache.shift.
- *   flags     NSNQ_ENCODE_DEFAULT or NSNQ_ENCODE_ADAPTIVE_SCALE.
+ *   flags     NSNQ_ENCODE_DEFAULT, or NSNQ_ENCODE_ADAPTIVE_SCALE and/or
+ *             NSNQ_ENCODE_DOUBLE_QUANT (bitwise or).
  *   cb        codebook; cache: codes/scales written, shift read or written.
  *   workspace device scratch of at least nsnq_encode_workspace(B, H, T, D)
  *             bytes, 256-byte aligned.

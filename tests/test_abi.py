@@ -75,7 +75,8 @@ def test_encode_validation(lib):
     assert _encode(lib, off=95) == nsnq.NSNQ_ERR_INVALID_ARG            # past capacity
     assert _encode(lib, T=-1) == nsnq.NSNQ_ERR_INVALID_ARG
     assert _encode(lib, mode=7) == nsnq.NSNQ_ERR_INVALID_ARG
-    assert _encode(lib, flags=2) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert _encode(lib, flags=4) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert _encode(lib, flags=2) == nsnq.NSNQ_ERR_INVALID_ARG  # double quantization needs s1_grid
     assert _encode(lib, ws=None) == nsnq.NSNQ_ERR_WORKSPACE
     assert _encode(lib, cb=_cb(index=None)) == nsnq.NSNQ_ERR_INVALID_ARG     # 2-bit needs its index
     assert b"nsnq_codebook_index_build" in lib.nsnq_last_error()

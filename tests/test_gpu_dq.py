@@ -1,0 +1,114 @@
+"""GPU parity of double quantization (NSNQuant Technical Summary,
+Methodology §3, Double Quantization): s1 on the head's 4-bit log2 grid, a
+computed o on 16 uniform levels, and a 4-bit codebook, each against the CPU
+oracle on the same seeded inputs."""
+import numpy as np
+import pytest
+import torch
+
+import attention_decode_b200 as nsnq
+import nsnq_synth as S
+from oracle import oracle as O
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+D = 128
+DQ = nsnq.ENCODE_DOUBLE_QUANT
+
+
+def _w(B, H, T, dtype, sub, kdist=S.K_MODERATE, seed=17):
+    return S.Workload("dq", B=B, Hkv=H, Hq=H, T=T, d=D, sub_dim=sub, dtype=dtype, kdist=kdist,
+                      seed=seed)
+
+
+def _check_grid(gpu: np.ndarray, ref: np.ndarray):
+    ulp = np.spacing(np.abs(ref).astype(np.float32)).astype(np.float64)
+    assert (np.abs(gpu.astype(np.float64) - ref) <= ulp).all(), (gpu, ref)
+
+
+@pytest.mark.parametrize("sub,T,dtype,kdist,flags", [
+    (4, 700, "bf16", S.K_MODERATE, DQ),
+    (4, 513, "f32", S.K_STRONG, DQ),
+    (8, 300, "bf16", S.K_MODERATE, DQ),
+    (4, 400, "bf16", S.K_MODERATE, DQ | nsnq.ENCODE_ADAPTIVE_SCALE),
+    (8, 257, "f32", S.K_STRONG, DQ | nsnq.ENCODE_ADAPTIVE_SCALE),
+])
+def test_double_quant_encode_matches_oracle(codebooks, sub, T, dtype, kdist, flags):
+    w = _w(2, 2, T, dtype, sub, kdist)
+    io = S.to_io(S.keys(w), dtype)
+    x64 = S.io_to_f64(io, dtype)
+    C = codebooks[sub]
+    ora = O.encode(x64, C, want_w=True, double_quant=True,
+                   adaptive_scale=bool(flags & nsnq.ENCODE_ADAPTIVE_SCALE))
+    cache = nsnq.Cache.empty(2, 2, T, sub)
+    nsnq.nsnq_encode(P.to_dev(io, dtype), P.codebook(C), cache, flags=flags)
+    torch.cuda.synchronize()
+    _check_grid(cache.s1_grid.cpu().numpy(), ora["s1_grid"])
+    P.check_shift(cache.shift.cpu().numpy(), ora["o"])
+    _, n_bad, worst = P.code_report(cache.codes.cpu().numpy(), ora["codes"], ora["w"], C)
+    assert n_bad == 0, worst
+    P.check_scales(cache.scales.cpu().numpy(), ora)
+
+
+@pytest.mark.parametrize("sub", [4, 8])
+def test_double_quant_append_uses_the_stored_grid(codebooks, sub):
+    """Prompt in shift-compute mode, then appended tokens (some far outside
+    the prompt's s1 range) in shift-given mode on the stored grid and o."""
+    w = _w(1, 2, 600, "bf16", sub)
+    x = S.to_io(S.keys(w), "bf16")
+    x[:, :, 590:] = S.to_io(S.io_to_f64(x[:, :, 590:], "bf16") * 30.0, "bf16")  # above the grid
+    x64 = S.io_to_f64(x, "bf16")
+    C = codebooks[sub]
+    cb = P.codebook(C)
+    cache = nsnq.Cache.empty(1, 2, 600, sub)
+    xd = P.to_dev(x, "bf16")
+    nsnq.nsnq_encode(xd[:, :, :500], cb, cache, flags=DQ)
+    nsnq.nsnq_encode(xd[:, :, 500:], cb, cache, t_offset=500, shift_mode=nsnq.SHIFT_GIVEN, flags=DQ)
+    torch.cuda.synchronize()
+    grid = cache.s1_grid.cpu().numpy().astype(np.float64)
+    o = cache.shift.cpu().numpy().astype(np.float64)
+    pre = O.encode(x64[:, :, :500], C, double_quant=True)
+    _check_grid(grid, pre["s1_grid"])
+    app = O.encode(x64[:, :, 500:], C, shift=o, want_w=True, double_quant=True, s1_grid=grid)
+    _, n_bad, worst = P.code_report(cache.codes[:, :, 500:].cpu().numpy(), app["codes"], app["w"], C)
+    assert n_bad == 0, worst
+    P.check_scales(cache.scales[:, :, 500:].cpu().numpy(), app)
+
+
+@pytest.mark.parametrize("ksub,vsub", [(4, 4), (8, 8)])
+def test_double_quant_codebooks_through_encode_and_attention(codebooks, ksub, vsub):
+    """4-bit codebooks (16 levels over all entries) with double-quantized
+    byproducts: GPU encode, then decode attention over the GPU caches,
+    against the oracle's encode -> dequant -> attention."""
+    B, H, Hq, T = 2, 2, 8, 640
+    w = S.Workload("dqa", B=B, Hkv=H, Hq=Hq, T=T, d=D, sub_dim=4, dtype="bf16",
+                   kdist=S.K_MODERATE, seed=23)
+    Ck = O.quantize4(codebooks[ksub]).astype(np.float32)
+    Cv = O.quantize4(codebooks[vsub]).astype(np.float32)
+    assert len(np.unique(Ck)) <= 16
+    k_io, v_io = S.to_io(S.keys(w), "bf16"), S.to_io(S.values(w), "bf16")
+    ok = O.encode(S.io_to_f64(k_io, "bf16"), Ck, want_w=True, double_quant=True)
+    ov = O.encode(S.io_to_f64(v_io, "bf16"), Cv, want_w=True, double_quant=True)
+    kc, vc = nsnq.Cache.empty(B, H, T, ksub), nsnq.Cache.empty(B, H, T, vsub)
+    kcb, vcb = P.codebook(Ck), P.codebook(Cv)
+    nsnq.nsnq_encode(P.to_dev(k_io, "bf16"), kcb, kc, flags=DQ)
+    nsnq.nsnq_encode(P.to_dev(v_io, "bf16"), vcb, vc, flags=DQ)
+    torch.cuda.synchronize()
+    for cache, ora, C in ((kc, ok, Ck), (vc, ov, Cv)):
+        _, n_bad, worst = P.code_report(cache.codes.cpu().numpy(), ora["codes"], ora["w"], C)
+        assert n_bad == 0, worst
+    q_io = S.to_io(S.queries(w), "bf16")
+    lens = [T, 401]
+    out = nsnq.nsnq_attn_decode(P.to_dev(q_io, "bf16"), kc, vc, kcb, vcb,
+                                torch.tensor(lens, dtype=torch.int32, device="cuda"), T, Hkv=H,
+                                out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    # the oracle's attention over the GPU's stored byproducts (its own codes)
+    Kh = O.dequant(kc.codes.cpu().numpy(), kc.scales[..., 0].cpu().numpy(),
+                   kc.scales[..., 1].cpu().numpy(), kc.shift.cpu().numpy(), Ck)
+    Vh = O.dequant(vc.codes.cpu().numpy(), vc.scales[..., 0].cpu().numpy(),
+                   vc.scales[..., 1].cpu().numpy(), vc.shift.cpu().numpy(), Cv)
+    ref = O.attention(S.io_to_f64(q_io, "bf16"), Kh, Vh, lens)
+    e, _ = P.attn_errors(P.out_to_np(out), ref, False)
+    assert (e <= 1.0).all(), e.max()
