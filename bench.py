@@ -242,10 +242,10 @@ def run_cuda(args):
     tokens_per_step = B * T * world
     value = tokens_per_step / (ms_per_step / 1e3)
 
-    # ---- end to end: pinned host K/V in, result out, through the public API ----
+    # ---- end to end: pinned host K/V/q in, the step's result (the attention
+    #      output) out, through the public API; the quantized cache is device
+    #      state and stays on the GPU ----
     res_host = torch.empty(B, Hq, 128, dtype=torch.bfloat16).pin_memory()
-    codes_host = torch.empty(2, *kc.codes.shape, dtype=torch.uint8).pin_memory()
-    scales_host = torch.empty(2, *kc.scales.shape, dtype=torch.float32).pin_memory()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
@@ -258,17 +258,13 @@ def run_cuda(args):
         q.copy_(host["q"], non_blocking=True)
         step(k, v, q)
         res_host.copy_(out, non_blocking=True)
-        codes_host[0].copy_(kc.codes, non_blocking=True)
-        codes_host[1].copy_(vc.codes, non_blocking=True)
-        scales_host[0].copy_(kc.scales, non_blocking=True)
-        scales_host[1].copy_(vc.scales, non_blocking=True)
         e1.record(stream)
         e1.synchronize()
         e2e_ms += e0.elapsed_time(e1)
     barrier()
     e2e_ms = max_over_ranks(e2e_ms, world, dev)
     h2d = sum(host[n].numel() * host[n].element_size() for n in ("k", "v", "q"))
-    d2h = (res_host.numel() * 2 + codes_host.numel() + scales_host.numel() * 4)
+    d2h = res_host.numel() * res_host.element_size()
     e2e = {"value": tokens_per_step / (e2e_ms / args.steps / 1e3), "unit": "KV tokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
