@@ -171,10 +171,11 @@ nsnq_status nsnq_encode(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t
     a.partial = reinterpret_cast<double*>(ws + plan.partial_off);
     a.o64 = reinterpret_cast<double*>(ws + plan.o64_off);
     a.minmax = reinterpret_cast<double*>(ws + plan.minmax_off);
+    a.head_done = reinterpret_cast<unsigned*>(ws + nsnq::kEncodeStatsBytes);
     a.nchunk1 = plan.nchunk1;
     a.chunk1 = plan.chunk1;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaMemsetAsync(ws, 0, nsnq::kEncodeStatsBytes, st);
+    cudaError_t e = cudaMemsetAsync(ws, 0, plan.reset_bytes, st);
     if (e != cudaSuccess) return cuda_fail(e, "workspace reset");
     e = nsnq::launch_encode(a, st);
     if (e != cudaSuccess) return cuda_fail(e, "encode launch");

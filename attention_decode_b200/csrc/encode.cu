@@ -2,12 +2,14 @@
 // and nearest-codeword vector quantization (gist.science "NSNQuant ...",
 // Technical Summary, Methodology §1-§3).
 //
-// Three launches per call in shift-compute mode, one in shift-given mode:
+// Two launches per call in shift-compute mode (three with double
+// quantization), one in shift-given mode:
 //   nsn_s1minmax_kernel per (b, h, chunk), double quantization only: least and
 //                      largest log2 s1 (the per-head s1 grid)
-//   nsn_stats_kernel   per (b, h, chunk): channel sums of y = x / s1 in fp64
-//   nsn_shift_kernel   per (b, h): o = sum / T (fp64, kept in the workspace
-//                      for the near-tie path) and its fp32 copy in the cache
+//   nsn_stats_kernel   per (b, h, chunk): channel sums of y = x / s1 in fp64;
+//                      the last chunk of a (b, h) to finish computes
+//                      o = sum / T (fp64, kept in the workspace for the
+//                      near-tie path) and its fp32 copy in the cache
 //   pass 2             NSN + FWHT + nearest codeword: encode_pruned.cu
 //                      (2 bit, search index) or encode1_tc.cu (1 bit, all
 //                      codewords scored on the tensor cores)
@@ -22,10 +24,8 @@ namespace nsnq {
 constexpr int kStatsThreads = 256;
 
 // --------------------------------------------------------------- pass 1 --
-// Lane layout: 8 lanes per token (16 channels each), 4 tokens per warp step.
-// Each warp keeps kStatsDepth steps of loads in flight (the kernel streams
-// x once from HBM and needs the bytes in flight to cover the latency).
-constexpr int kStatsDepth = 4;
+// Lane layout of the s1 range kernel: 8 lanes per token (16 channels each),
+// 4 tokens per warp step.
 
 template <typename XT>
 struct Raw16;
@@ -119,42 +119,124 @@ __global__ void __launch_bounds__(kStatsThreads) nsn_s1minmax_kernel(EncodeArgs 
     }
 }
 
+// Pass-1 lane layout: 16 lanes per token (8 channels each, one 16-byte load
+// for bf16), 2 tokens per warp step, stats_depth<XT> steps of loads in
+// flight per warp (64 bytes per lane: the kernel streams x once from HBM and
+// needs the bytes in flight to cover the latency); at most 64 registers so
+// that four CTAs fit on an SM and the usual grids run in one wave.
+template <typename XT>
+constexpr int stats_depth() { return sizeof(XT) == 2 ? 4 : 2; }
+
+template <typename XT>
+struct Raw8;
+template <>
+struct Raw8<__nv_bfloat16> {
+    uint4 u;
+    __device__ __forceinline__ void load(const __nv_bfloat16* p) { u = __ldg(reinterpret_cast<const uint4*>(p)); }
+    __device__ __forceinline__ void zero() { u = make_uint4(0, 0, 0, 0); }
+    __device__ __forceinline__ void unpack(float (&v)[8]) const {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            v[2 * k] = __uint_as_float(w[k] << 16);
+            v[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+        }
+    }
+};
+template <>
+struct Raw8<float> {
+    float4 f[2];
+    __device__ __forceinline__ void load(const float* p) {
+        f[0] = __ldg(reinterpret_cast<const float4*>(p));
+        f[1] = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    }
+    __device__ __forceinline__ void zero() { f[0] = f[1] = make_float4(0.f, 0.f, 0.f, 0.f); }
+    __device__ __forceinline__ void unpack(float (&v)[8]) const {
+        v[0] = f[0].x; v[1] = f[0].y; v[2] = f[0].z; v[3] = f[0].w;
+        v[4] = f[1].x; v[5] = f[1].y; v[6] = f[1].z; v[7] = f[1].w;
+    }
+};
+
+// o of one (b, h) from its chunk partials, by the CTA whose chunk finished
+// last: o = sum / T in fp64 (double quantization: o on 16 uniform levels
+// between its least and largest channel value, and the head's s1 grid).
+template <bool DQ>
+__device__ void shift_of_head(const EncodeArgs& a, int64_t bh, double (*red)[kD]) {
+    const int c = threadIdx.x;
+    double o = 0.0;
+    if (c < kD) {
+        double s = 0.0;
+        for (int k = 0; k < a.nchunk1; ++k) s += __ldcg(a.partial + (bh * a.nchunk1 + k) * kD + c);
+        o = a.T > 0 ? s / (double)a.T : 0.0;
+    }
+    if constexpr (DQ) {
+        double mn = o, mx = o;
+#pragma unroll
+        for (int m = 1; m < 32; m <<= 1) {
+            mn = fmin(mn, __shfl_xor_sync(kFull, mn, m));
+            mx = fmax(mx, __shfl_xor_sync(kFull, mx, m));
+        }
+        __syncthreads();  // red is free again
+        if (c < kD && (c & 31) == 0) { red[0][c >> 5] = mn; red[1][c >> 5] = mx; }
+        __syncthreads();
+        mn = red[0][0]; mx = red[1][0];
+#pragma unroll
+        for (int w = 1; w < kD / 32; ++w) { mn = fmin(mn, red[0][w]); mx = fmax(mx, red[1][w]); }
+        const double step = (mx - mn) / 15.0;
+        o = mn + (step > 0.0 ? round((o - mn) / step) : 0.0) * step;
+        if (c == 0) {
+            double lo, st;
+            dq_grid_from_chunks(a.minmax + bh * a.nchunk1 * 2, a.nchunk1, lo, st);
+            a.s1_grid[2 * bh] = (float)lo;
+            a.s1_grid[2 * bh + 1] = (float)st;
+        }
+    }
+    if (c < kD) {
+        a.o64[bh * kD + c] = o;
+        a.shift[bh * kD + c] = (float)o;
+    }
+}
+
 template <typename XT, bool DQ>
-__global__ void __launch_bounds__(kStatsThreads) nsn_stats_kernel(EncodeArgs a) {
+__global__ void __launch_bounds__(kStatsThreads, 4) nsn_stats_kernel(EncodeArgs a) {
     const int chunk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int64_t bh = (int64_t)b * a.H + h;
     const int warp = threadIdx.x >> 5, lane = lane_id();
-    const int tk = lane >> 3, cg = lane & 7;
+    const int tk = lane >> 4, cg = lane & 15;
     const int64_t t0 = (int64_t)chunk * a.chunk1;
     const int64_t t1 = min(t0 + a.chunk1, a.T);
-    const XT* xb = reinterpret_cast<const XT*>(a.x) + b * a.sb + h * a.sh + 16 * cg;
+    const XT* xb = reinterpret_cast<const XT*>(a.x) + b * a.sb + h * a.sh + 8 * cg;
     const double sqrt_d = sqrt((double)kD);
-    constexpr int64_t kStride = 4 * (kStatsThreads / 32);  // tokens per CTA step
+    constexpr int64_t kStride = 2 * (kStatsThreads / 32);  // tokens per CTA step
     double glo = 0.0, gstep = 0.0;
-    if constexpr (DQ)
-        dq_grid_from_chunks(a.minmax + (int64_t)(b * a.H + h) * a.nchunk1 * 2, a.nchunk1, glo, gstep);
-    double acc[16];
+    if constexpr (DQ) dq_grid_from_chunks(a.minmax + bh * a.nchunk1 * 2, a.nchunk1, glo, gstep);
+    double acc[8];
 #pragma unroll
-    for (int c = 0; c < 16; ++c) acc[c] = 0.0;
-    Raw16<XT> buf[kStatsDepth];
+    for (int c = 0; c < 8; ++c) acc[c] = 0.0;
+    constexpr int kStatsDepth2 = stats_depth<XT>();
+    Raw8<XT> buf[kStatsDepth2];
 #pragma unroll
-    for (int d = 0; d < kStatsDepth; ++d) {
-        const int64_t t = t0 + warp * 4 + d * kStride + tk;
+    for (int d = 0; d < kStatsDepth2; ++d) {
+        const int64_t t = t0 + warp * 2 + d * kStride + tk;
         if (t < t1) buf[d].load(xb + t * a.st); else buf[d].zero();
     }
-    for (int64_t base = t0 + warp * 4; base < t1; base += kStatsDepth * kStride) {
+    for (int64_t base = t0 + warp * 2; base < t1; base += kStatsDepth2 * kStride) {
 #pragma unroll
-        for (int d = 0; d < kStatsDepth; ++d) {
-            float v[16];
+        for (int d = 0; d < kStatsDepth2; ++d) {
+            float v[8];
             buf[d].unpack(v);
-            // refill this slot kStatsDepth steps ahead
-            const int64_t tn = base + (d + kStatsDepth) * kStride + tk;
+            // refill this slot kStatsDepth2 steps ahead
+            const int64_t tn = base + (d + kStatsDepth2) * kStride + tk;
             if (tn < t1) buf[d].load(xb + tn * a.st); else buf[d].zero();
-            double ss = 0.0;
+            double s0 = 0.0, s1 = 0.0;
 #pragma unroll
-            for (int c = 0; c < 16; ++c) ss = fma((double)v[c], (double)v[c], ss);
-            ss += __shfl_xor_sync(kFull, ss, 1);
-            ss += __shfl_xor_sync(kFull, ss, 2);
-            ss += __shfl_xor_sync(kFull, ss, 4);
+            for (int c = 0; c < 8; c += 2) {
+                s0 = fma((double)v[c], (double)v[c], s0);
+                s1 = fma((double)v[c + 1], (double)v[c + 1], s1);
+            }
+            double ss = s0 + s1;
+#pragma unroll
+            for (int m = 1; m < 16; m <<= 1) ss += __shfl_xor_sync(kFull, ss, m);
             if (ss > 0.0) {
                 double inv;  // 1 / s1
                 if constexpr (DQ) {
@@ -163,62 +245,35 @@ __global__ void __launch_bounds__(kStatsThreads) nsn_stats_kernel(EncodeArgs a) 
                     inv = rsqrt(ss) * sqrt_d;
                 }
 #pragma unroll
-                for (int c = 0; c < 16; ++c) acc[c] = fma((double)v[c], inv, acc[c]);
+                for (int c = 0; c < 8; ++c) acc[c] = fma((double)v[c], inv, acc[c]);
             }
         }
     }
-    // Sum the four token slots of each channel group, then the warps.
+    // Sum the two token slots of each channel group, then the warps.
 #pragma unroll
-    for (int c = 0; c < 16; ++c) {
-        acc[c] += __shfl_xor_sync(kFull, acc[c], 8);
-        acc[c] += __shfl_xor_sync(kFull, acc[c], 16);
-    }
+    for (int c = 0; c < 8; ++c) acc[c] += __shfl_xor_sync(kFull, acc[c], 16);
     __shared__ double red[kStatsThreads / 32][kD];
+    __shared__ unsigned last;
     if (tk == 0) {
 #pragma unroll
-        for (int c = 0; c < 16; ++c) red[warp][16 * cg + c] = acc[c];
+        for (int c = 0; c < 8; ++c) red[warp][8 * cg + c] = acc[c];
     }
     __syncthreads();
     if (threadIdx.x < kD) {
         double s = 0.0;
 #pragma unroll
         for (int w = 0; w < kStatsThreads / 32; ++w) s += red[w][threadIdx.x];
-        a.partial[((int64_t)(b * a.H + h) * a.nchunk1 + chunk) * kD + threadIdx.x] = s;
+        a.partial[(bh * a.nchunk1 + chunk) * kD + threadIdx.x] = s;
     }
-}
-
-template <bool DQ>
-__global__ void __launch_bounds__(kD) nsn_shift_kernel(EncodeArgs a) {
-    const int bh = blockIdx.x;
-    const int c = threadIdx.x;
-    double s = 0.0;
-    for (int k = 0; k < a.nchunk1; ++k) s += a.partial[((int64_t)bh * a.nchunk1 + k) * kD + c];
-    double o = a.T > 0 ? s / (double)a.T : 0.0;
-    if constexpr (DQ) {
-        // o on 16 uniform levels between its least and largest channel value
-        __shared__ double red[kD / 32][2];
-        double mn = o, mx = o;
-#pragma unroll
-        for (int m = 1; m < 32; m <<= 1) {
-            mn = fmin(mn, __shfl_xor_sync(kFull, mn, m));
-            mx = fmax(mx, __shfl_xor_sync(kFull, mx, m));
-        }
-        if ((c & 31) == 0) { red[c >> 5][0] = mn; red[c >> 5][1] = mx; }
-        __syncthreads();
-        mn = red[0][0]; mx = red[0][1];
-#pragma unroll
-        for (int w = 1; w < kD / 32; ++w) { mn = fmin(mn, red[w][0]); mx = fmax(mx, red[w][1]); }
-        const double step = (mx - mn) / 15.0;
-        o = mn + (step > 0.0 ? round((o - mn) / step) : 0.0) * step;
-        if (c == 0) {
-            double lo, st;
-            dq_grid_from_chunks(a.minmax + (int64_t)bh * a.nchunk1 * 2, a.nchunk1, lo, st);
-            a.s1_grid[2 * bh] = (float)lo;
-            a.s1_grid[2 * bh + 1] = (float)st;
-        }
+    // The chunk that completes its (b, h) last also derives the shift.
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) last = atomicAdd(a.head_done + bh, 1u) == (unsigned)(a.nchunk1 - 1);
+    __syncthreads();
+    if (last) {
+        __threadfence();
+        shift_of_head<DQ>(a, bh, red);
     }
-    a.o64[(int64_t)bh * kD + c] = o;
-    a.shift[(int64_t)bh * kD + c] = (float)o;
 }
 
 // ---------------------------------------------------------------- host --
@@ -227,7 +282,8 @@ EncodePlan plan_encode(int B, int H, int64_t T) {
     p.chunk1 = 512;
     p.nchunk1 = (int)((T + p.chunk1 - 1) / p.chunk1);
     if (p.nchunk1 < 1) p.nchunk1 = 1;
-    p.partial_off = align_up(kEncodeStatsBytes, kWsAlign);
+    p.reset_bytes = kEncodeStatsBytes + (size_t)B * H * sizeof(unsigned);  // stats + per-head counters
+    p.partial_off = align_up(p.reset_bytes, kWsAlign);
     const size_t partial_bytes = (size_t)B * H * p.nchunk1 * kD * sizeof(double);
     p.o64_off = align_up(p.partial_off + partial_bytes, kWsAlign);
     p.minmax_off = align_up(p.o64_off + (size_t)B * H * kD * sizeof(double), kWsAlign);
@@ -242,10 +298,8 @@ static cudaError_t launch_encode_t(const EncodeArgs& a, cudaStream_t s) {
         if (a.dq) {
             nsn_s1minmax_kernel<XT><<<grid1, kStatsThreads, 0, s>>>(a);
             nsn_stats_kernel<XT, true><<<grid1, kStatsThreads, 0, s>>>(a);
-            nsn_shift_kernel<true><<<a.B * a.H, kD, 0, s>>>(a);
         } else {
             nsn_stats_kernel<XT, false><<<grid1, kStatsThreads, 0, s>>>(a);
-            nsn_shift_kernel<false><<<a.B * a.H, kD, 0, s>>>(a);
         }
     }
     cudaError_t e = cudaGetLastError();

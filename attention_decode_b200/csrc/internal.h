@@ -43,6 +43,7 @@ struct EncodeArgs {
     double* partial;            // [B][H][nchunk1][128]
     double* o64;                // [B][H][128]
     double* minmax;             // [B][H][nchunk1][2] least / largest log2 s1 per chunk
+    unsigned* head_done;        // [B][H] chunks of pass 1 finished (zeroed per call)
     int nchunk1;
     int64_t chunk1;
 };
@@ -50,6 +51,7 @@ struct EncodeArgs {
 struct EncodePlan {
     int nchunk1;
     int64_t chunk1;
+    size_t reset_bytes;  // leading workspace bytes zeroed before each call
     size_t partial_off, o64_off, minmax_off, total;
 };
 
