@@ -275,7 +275,7 @@ def run_cuda(args):
     enc_gbs = enc_bytes / (enc_avg_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(enc_gbs, 1), "peak": hbm, "unit": "GB/s",
                 "frac": round(enc_gbs / hbm, 4), "peak_kind": peak_kind,
-                "kernel": "nsnq_encode (nsn_stats + nsn_shift + nsn_encode, one tensor)",
+                "kernel": "nsnq_encode (nsn_stats + nsn_encode_pruned, one tensor)",
                 "algorithmic_bytes_per_launch": enc_bytes,
                 "traffic": args.traffic if args.traffic is not None else measured_traffic("nsnq_encode")}
 
@@ -417,7 +417,7 @@ def run_encode1_bench(args, nsnq, dev, world, barrier, hbm, peak_kind, x):
             "workload": "encode-8x4096 keys at 1 bit/coord (g = 8), codewords scored on the tensor cores",
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
                          "frac": round(gbs / hbm, 4), "peak_kind": peak_kind,
-                         "kernel": "nsnq_encode at 1 bit (nsn_stats + nsn_shift + nsn_encode1_tc)",
+                         "kernel": "nsnq_encode at 1 bit (nsn_stats + nsn_encode1_tc)",
                          "algorithmic_bytes_per_launch": nbytes,
                          "traffic": measured_traffic("nsnq_encode_1bit")},
             "l2": "flushed before every call"}
