@@ -133,23 +133,36 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a)
         if (lane == 0) gam[warp] = g;
     }
     __syncthreads();
-    for (int e = tid; e < kNC * KJ; e += kAttnThreads) {
-        const int c = e / KJ, j = e % KJ;
-        float ck[KSUB];
+    {
+        // A thread keeps sub-vector j of the rotated queries in registers and
+        // walks the codes c = tid / KJ + k * (threads / KJ): the codeword is
+        // one broadcast read per warp and each warp stores whole LUT rows.
+        static_assert(kAttnThreads % KJ == 0, "threads must tile the sub-vectors");
+        const int j = tid % KJ;
+        float qj[GC][KSUB];
 #pragma unroll
-        for (int r = 0; r < KSUB; ++r) ck[r] = __ldg(a.kC + c * KSUB + r);
-        float sum[GC];
+        for (int h = 0; h < GC; ++h)
 #pragma unroll
-        for (int h = 0; h < GC; ++h) {
-            sum[h] = 0.f;
+            for (int r = 0; r < KSUB; ++r) qj[h][r] = qrot[h * kD + j * KSUB + r];
+#pragma unroll 4
+        for (int c = tid / KJ; c < kNC; c += kAttnThreads / KJ) {
+            float ck[KSUB];
 #pragma unroll
-            for (int r = 0; r < KSUB; ++r) sum[h] = fmaf(qrot[h * kD + j * KSUB + r], ck[r], sum[h]);
-        }
-        if constexpr (GC == 4) {
-            reinterpret_cast<float4*>(lut)[e] = make_float4(sum[0], sum[1], sum[2], sum[3]);
-        } else {
+            for (int r = 0; r < KSUB; ++r) ck[r] = __ldg(a.kC + c * KSUB + r);
+            float sum[GC];
 #pragma unroll
-            for (int h = 0; h < GC; ++h) lut[(size_t)e * GC + h] = sum[h];
+            for (int h = 0; h < GC; ++h) {
+                sum[h] = 0.f;
+#pragma unroll
+                for (int r = 0; r < KSUB; ++r) sum[h] = fmaf(qj[h][r], ck[r], sum[h]);
+            }
+            const int e = c * KJ + j;
+            if constexpr (GC == 4) {
+                reinterpret_cast<float4*>(lut)[e] = make_float4(sum[0], sum[1], sum[2], sum[3]);
+            } else {
+#pragma unroll
+                for (int h = 0; h < GC; ++h) lut[(size_t)e * GC + h] = sum[h];
+            }
         }
     }
     __syncthreads();

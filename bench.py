@@ -54,6 +54,7 @@ def peaks():
         return 6650.0, "fallback"
 
 
+NOMINAL_HBM_GBS = 8000.0  # nominal B200 HBM3e bandwidth (8 TB/s), for the second fraction
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "roofline_traffic.json")
 
 
@@ -205,7 +206,7 @@ def run_cuda(args):
         nsnq.nsnq_encode(vin, cb, vc, workspace=ws_e)
         nsnq.nsnq_attn_decode(qin, kc, vc, cb, cb, seq, T, Hkv=H, out=out, workspace=ws_a)
 
-    LAUNCHES_PER_STEP = 3 + 3 + 2  # (stats, shift, encode) x 2 + (split, combine)
+    LAUNCHES_PER_STEP = 2 + 2 + 2  # (pass 1, pass 2) x 2 + (split, combine)
 
     def barrier():
         if world > 1:
@@ -274,7 +275,7 @@ def run_cuda(args):
     enc_avg_ms = sum(enc_ms) / len(enc_ms)
     enc_gbs = enc_bytes / (enc_avg_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(enc_gbs, 1), "peak": hbm, "unit": "GB/s",
-                "frac": round(enc_gbs / hbm, 4), "peak_kind": peak_kind,
+                "frac": round(enc_gbs / hbm, 4), "frac_vs_8tbs": round(enc_gbs / NOMINAL_HBM_GBS, 4), "peak_kind": peak_kind,
                 "kernel": "nsnq_encode (nsn_stats + nsn_encode_pruned, one tensor)",
                 "algorithmic_bytes_per_launch": enc_bytes,
                 "traffic": args.traffic if args.traffic is not None else measured_traffic("nsnq_encode")}
@@ -282,6 +283,8 @@ def run_cuda(args):
     # ---- decode attention alone at the 32k workload ----
     attention = run_attention_bench(args, nsnq, dev, world, barrier, hbm, peak_kind)
     encode_1bit = run_encode1_bench(args, nsnq, dev, world, barrier, hbm, peak_kind, k)
+    long_context = run_long_context_bench(args, nsnq, dev, world, barrier, hbm)
+    serving = run_serving_bench(args, nsnq, dev, world, barrier, hbm)
     clk.__exit__(None, None, None)
 
     result = {
@@ -296,7 +299,8 @@ def run_cuda(args):
         "stages_ms": {"encode_per_tensor": round(enc_avg_ms, 4),
                       "attention_4k": round(sum(att_small_ms) / len(att_small_ms), 4)},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
-        "roofline": roofline, "attention": attention, "encode_1bit": encode_1bit, "e2e": e2e,
+        "roofline": roofline, "attention": attention, "encode_1bit": encode_1bit,
+        "long_context": long_context, "serving": serving, "e2e": e2e,
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -371,7 +375,7 @@ def run_attention_bench(args, nsnq, dev, world, barrier, hbm, peak_kind):
     rgbs = nbytes / (ravg / 1e3) / 1e9
     rope = {"ms_per_call": round(ravg, 4), "value": round(rgbs * world, 1), "unit": "GB/s",
             "roofline": {"bound": "hbm", "achieved": round(rgbs, 1), "peak": hbm, "unit": "GB/s",
-                         "frac": round(rgbs / hbm, 4), "peak_kind": peak_kind,
+                         "frac": round(rgbs / hbm, 4), "frac_vs_8tbs": round(rgbs / NOMINAL_HBM_GBS, 4), "peak_kind": peak_kind,
                          "kernel": "nsnq_attn_decode_rope (attn_rope_split + attn_combine)",
                          "algorithmic_bytes_per_launch": nbytes,
                          "traffic": measured_traffic("nsnq_attn_decode_rope")}}
@@ -379,7 +383,7 @@ def run_attention_bench(args, nsnq, dev, world, barrier, hbm, peak_kind):
             "unit": "GB/s", "ms_per_call": round(avg, 4),
             "workload": "decode-16x32k-2b (B 16, Hq 32, Hkv 8, T 32768, d 128, 2 bit K and V)",
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
-                         "frac": round(gbs / hbm, 4), "peak_kind": peak_kind,
+                         "frac": round(gbs / hbm, 4), "frac_vs_8tbs": round(gbs / NOMINAL_HBM_GBS, 4), "peak_kind": peak_kind,
                          "kernel": "nsnq_attn_decode (attn_split + attn_combine)",
                          "algorithmic_bytes_per_launch": nbytes,
                          "traffic": measured_traffic("nsnq_attn_decode")},
@@ -416,11 +420,169 @@ def run_encode1_bench(args, nsnq, dev, world, barrier, hbm, peak_kind, x):
             "unit": "KV tokens/s (one tensor)", "ms_per_call": round(avg, 4),
             "workload": "encode-8x4096 keys at 1 bit/coord (g = 8), codewords scored on the tensor cores",
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
-                         "frac": round(gbs / hbm, 4), "peak_kind": peak_kind,
+                         "frac": round(gbs / hbm, 4), "frac_vs_8tbs": round(gbs / NOMINAL_HBM_GBS, 4), "peak_kind": peak_kind,
                          "kernel": "nsnq_encode at 1 bit (nsn_stats + nsn_encode1_tc)",
                          "algorithmic_bytes_per_launch": nbytes,
                          "traffic": measured_traffic("nsnq_encode_1bit")},
             "l2": "flushed before every call"}
+
+
+def _device_kv(w, gen, dev, B, T, which):
+    """Seeded K (outlier channels x LogNormal token scale) or V ~ N(0,1) of the
+    workload's distribution, bf16 [B][Hkv][T][128], drawn on the device."""
+    import torch
+    z = torch.randn(B, w.Hkv, T, 128, generator=gen, device=dev)
+    if which == "v":
+        return z.to(torch.bfloat16)
+    chans, signs = w.kdist.channels(128)
+    bias = torch.zeros(128, device=dev)
+    bias[chans] = torch.tensor(signs, device=dev) * w.kdist.bias
+    s = torch.exp(w.kdist.sigma * torch.randn(B, w.Hkv, T, 1, generator=gen, device=dev))
+    return ((z + bias) * s).to(torch.bfloat16)
+
+
+def _median(xs):
+    return statistics.median(xs) if xs else 0.0
+
+
+def run_long_context_bench(args, nsnq, dev, world, barrier, hbm):
+    """Long context (B 1, Hkv 8, Hq 32, T 131072, strong outliers, 2 bit):
+    the prompt's K and V encoded (shift computed), then decode steps that each
+    encode one new K/V token with the stored shift and attend over the cache."""
+    import torch
+    w = S.WORKLOADS["long-128k"]
+    B, H, Hq, T, n_dec = w.B, w.Hkv, w.Hq, w.T, w.decode_steps
+    cb = nsnq.Codebook(torch.from_numpy(load_codebook(w.sub_dim)).to(dev))
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(4321)
+    k = _device_kv(w, gen, dev, B, T, "k")
+    v = _device_kv(w, gen, dev, B, T, "v")
+    kn = _device_kv(w, gen, dev, B, n_dec, "k")
+    vn = _device_kv(w, gen, dev, B, n_dec, "v")
+    q = torch.randn(n_dec, B, Hq, 128, generator=gen, device=dev).to(torch.bfloat16)
+    cap = T + n_dec
+    kc = nsnq.Cache.empty(B, H, cap, w.sub_dim, device=dev)
+    vc = nsnq.Cache.empty(B, H, cap, w.sub_dim, device=dev)
+    ws_e = torch.empty(nsnq.nsnq_encode_workspace(B, H, T), dtype=torch.uint8, device=dev)
+    ws_a = torch.empty(nsnq.nsnq_attn_workspace(B, Hq, H, cap), dtype=torch.uint8, device=dev)
+    out = torch.empty(B, Hq, 128, dtype=torch.bfloat16, device=dev)
+    seqs = [torch.full((B,), T + i + 1, dtype=torch.int32, device=dev) for i in range(n_dec)]
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def prompt():
+        nsnq.nsnq_encode(k, cb, kc, workspace=ws_e)
+        nsnq.nsnq_encode(v, cb, vc, workspace=ws_e)
+
+    for _ in range(max(1, args.warmup // 2)):
+        prompt()
+    barrier()
+    torch.cuda.synchronize()
+    p_ms = []
+    for _ in range(3):
+        flush.zero_()
+        e0, e1 = ev(), ev()
+        e0.record(stream)
+        prompt()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        p_ms.append(e0.elapsed_time(e1))
+    step_ms, att_ms = [], []
+    for i in range(n_dec):
+        flush.zero_()
+        e0, e1, e2 = ev(), ev(), ev()
+        e0.record(stream)
+        nsnq.nsnq_encode(kn[:, :, i:i + 1], cb, kc, t_offset=T + i, shift_mode=nsnq.SHIFT_GIVEN,
+                         workspace=ws_e)
+        nsnq.nsnq_encode(vn[:, :, i:i + 1], cb, vc, t_offset=T + i, shift_mode=nsnq.SHIFT_GIVEN,
+                         workspace=ws_e)
+        e1.record(stream)
+        nsnq.nsnq_attn_decode(q[i], kc, vc, cb, cb, seqs[i], cap, Hkv=H, out=out, workspace=ws_a)
+        e2.record(stream)
+        torch.cuda.synchronize()
+        step_ms.append(e0.elapsed_time(e2))
+        att_ms.append(e1.elapsed_time(e2))
+    barrier()
+    pm = max_over_ranks(_median(p_ms), world, dev)
+    sm = max_over_ranks(_median(step_ms), world, dev)
+    am = max_over_ranks(_median(att_ms), world, dev)
+    att_bytes = B * H * (T + n_dec // 2) * attn_bytes_per_token(w.sub_dim, w.sub_dim)
+    enc_bytes = 2 * B * H * T * encode_bytes_per_token_head(w.sub_dim)
+    return {"workload": "long-128k (B 1, Hkv 8, Hq 32, T 131072 prompt + 64 decode steps, strong "
+                        "outlier K, 2 bit)",
+            "prompt_encode_ms": round(pm, 4),
+            "prompt_encode_tokens_per_s": round(B * T * world / (pm / 1e3), 1),
+            "prompt_encode_gbs": round(enc_bytes / (pm / 1e3) / 1e9, 1),
+            "decode_step_ms_median": round(sm, 4),
+            "decode_attention_ms_median": round(am, 4),
+            "decode_attention_gbs": round(att_bytes / (am / 1e3) / 1e9, 1),
+            "decode_attention_frac": round(att_bytes / (am / 1e3) / 1e9 / hbm, 4),
+            "steps": n_dec, "l2": "flushed before every timed call"}
+
+
+def run_serving_bench(args, nsnq, dev, world, barrier, hbm):
+    """Serving mix (Hq 64, Hkv 8, 64 resident sequences x 8192 tokens, 2 bit):
+    per step, the 2048-token prompts of 4 new sequences are encoded into 4
+    spare cache slots and one decode query per resident sequence attends."""
+    import torch
+    w = S.WORKLOADS["serving-64x8k"]
+    B, H, Hq, T = w.B, w.Hkv, w.Hq, w.T
+    P, Tp = w.prefill_seqs, w.prefill_len
+    cb = nsnq.Codebook(torch.from_numpy(load_codebook(w.sub_dim)).to(dev))
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(5678)
+    kc = nsnq.Cache.empty(B + P, H, T, w.sub_dim, device=dev)
+    vc = nsnq.Cache.empty(B + P, H, T, w.sub_dim, device=dev)
+    view = lambda c, b0, b1: nsnq.Cache(c.codes[b0:b1], c.scales[b0:b1], c.shift[b0:b1])
+    ws_r = torch.empty(nsnq.nsnq_encode_workspace(1, H, T), dtype=torch.uint8, device=dev)
+    for b in range(B):  # resident sequences, one at a time
+        nsnq.nsnq_encode(_device_kv(w, gen, dev, 1, T, "k"), cb, view(kc, b, b + 1), workspace=ws_r)
+        nsnq.nsnq_encode(_device_kv(w, gen, dev, 1, T, "v"), cb, view(vc, b, b + 1), workspace=ws_r)
+    kp = _device_kv(w, gen, dev, P, Tp, "k")
+    vp = _device_kv(w, gen, dev, P, Tp, "v")
+    q = torch.randn(B, Hq, 128, generator=gen, device=dev).to(torch.bfloat16)
+    seq = torch.full((B,), T, dtype=torch.int32, device=dev)
+    out = torch.empty(B, Hq, 128, dtype=torch.bfloat16, device=dev)
+    ws_e = torch.empty(nsnq.nsnq_encode_workspace(P, H, Tp), dtype=torch.uint8, device=dev)
+    ws_a = torch.empty(nsnq.nsnq_attn_workspace(B, Hq, H, T), dtype=torch.uint8, device=dev)
+    kres, vres = view(kc, 0, B), view(vc, 0, B)
+    kspare, vspare = view(kc, B, B + P), view(vc, B, B + P)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(evs=None):
+        if evs: evs[0].record(stream)
+        nsnq.nsnq_encode(kp, cb, kspare, workspace=ws_e)
+        nsnq.nsnq_encode(vp, cb, vspare, workspace=ws_e)
+        if evs: evs[1].record(stream)
+        nsnq.nsnq_attn_decode(q, kres, vres, cb, cb, seq, T, Hkv=H, out=out, workspace=ws_a)
+        if evs: evs[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    torch.cuda.synchronize()
+    rows = []
+    for _ in range(max(args.steps, 5)):
+        flush.zero_()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        step(evs)
+        rows.append(evs)
+    torch.cuda.synchronize()
+    barrier()
+    st = max_over_ranks(_median([e[0].elapsed_time(e[2]) for e in rows]), world, dev)
+    en = max_over_ranks(_median([e[0].elapsed_time(e[1]) for e in rows]), world, dev)
+    at = max_over_ranks(_median([e[1].elapsed_time(e[2]) for e in rows]), world, dev)
+    att_bytes = B * H * T * attn_bytes_per_token(w.sub_dim, w.sub_dim)
+    return {"workload": "serving-64x8k (Hq 64, Hkv 8, 64 x 8192-token 2-bit caches; per step "
+                        "4 x 2048-token prompts encoded into spare slots + 64 decode queries)",
+            "step_ms_median": round(st, 4), "encode_ms_median": round(en, 4),
+            "encode_tokens_per_s": round(P * Tp * world / (en / 1e3), 1),
+            "attention_ms_median": round(at, 4),
+            "attention_gbs": round(att_bytes / (at / 1e3) / 1e9, 1),
+            "attention_frac": round(att_bytes / (at / 1e3) / 1e9 / hbm, 4),
+            "l2": "flushed before every timed step"}
 
 
 # ------------------------------------------------------------ oracle arm --
