@@ -175,7 +175,10 @@ nsnq_status nsnq_encode(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t
     a.nchunk1 = plan.nchunk1;
     a.chunk1 = plan.chunk1;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaMemsetAsync(ws, 0, plan.reset_bytes, st);
+    // A small shift-given call (a decode step's appends) uses no counter: its
+    // kernel zeroes the stats block itself, which saves the memset.
+    a.zero_stats = a.given_shift && (int64_t)B * H * T <= nsnq::kSmallEncode;
+    cudaError_t e = a.zero_stats ? cudaSuccess : cudaMemsetAsync(ws, 0, plan.reset_bytes, st);
     if (e != cudaSuccess) return cuda_fail(e, "workspace reset");
     e = nsnq::launch_encode(a, st);
     if (e != cudaSuccess) return cuda_fail(e, "encode launch");

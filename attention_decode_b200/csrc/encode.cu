@@ -12,7 +12,9 @@
 //                      near-tie path) and its fp32 copy in the cache
 //   pass 2             NSN + FWHT + nearest codeword: encode_pruned.cu
 //                      (2 bit, search index) or encode1_tc.cu (1 bit, all
-//                      codewords scored on the tensor cores)
+//                      codewords scored on the tensor cores); calls of at
+//                      most kSmallEncode token-heads: encode_small.cu (one
+//                      warp per token-head, fp64)
 #include <math.h>
 
 #include "common.cuh"
@@ -304,6 +306,7 @@ static cudaError_t launch_encode_t(const EncodeArgs& a, cudaStream_t s) {
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    if ((int64_t)a.B * a.H * a.T <= kSmallEncode) return launch_encode_small(a, s);
     return a.sub == 4 ? launch_encode_pruned(a, s) : launch_encode1_tc(a, s);
 }
 

@@ -1,0 +1,157 @@
+// NSNQuant encode pass 2 for small calls (gist.science "NSNQuant ...",
+// Technical Summary, Methodology §1-§3): a decode step appends one token per
+// sequence and kv-head, a few hundred token-heads, where the persistent
+// kernels' fixed costs (staging the search index, one busy warp per tile)
+// dominate. Here one warp takes one token-head and does everything in fp64:
+// NSN with warp sums, the Hadamard transform across the warp (lane l holds
+// coordinates 4l..4l+3), and the nearest codeword of each sub-vector by a
+// full scan of the 256 codewords (lowest index on exact ties), so no near-tie
+// re-decision is needed. Stored s1, s2 are the fp64 values rounded to fp32,
+// as the persistent kernels store them for the tokens they re-decide in fp64.
+#include <math.h>
+
+#include "common.cuh"
+#include "dq.cuh"
+#include "internal.h"
+
+namespace nsnq {
+
+namespace {
+
+constexpr int kSmallThreads = 32;  // one warp (one token-head) per CTA: the CTAs spread over the SMs
+
+template <typename XT, int G, bool ADAPT, bool DQ>
+__global__ void __launch_bounds__(kSmallThreads) nsn_encode_small_kernel(EncodeArgs a) {
+    __shared__ __align__(16) double Cs[kNC * G];  // the codebook, converted once
+    for (int i = threadIdx.x; i < kNC * G; i += kSmallThreads) Cs[i] = (double)a.C[i];
+    __syncthreads();
+    if (a.zero_stats && blockIdx.x == 0 && threadIdx.x < 8) a.stats[threadIdx.x] = 0ull;
+    const int lane = lane_id();
+    const int64_t th = (int64_t)blockIdx.x * (kSmallThreads / 32) + (threadIdx.x >> 5);
+    if (th >= (int64_t)a.B * a.H * a.T) return;  // warp-uniform
+    const int64_t bh = th / a.T, t = th - bh * a.T;
+    const int b = (int)(bh / a.H), h = (int)(bh - (int64_t)b * a.H);
+    const XT* xtok = reinterpret_cast<const XT*>(a.x) + b * a.sb + h * a.sh + t * a.st;
+
+    // ---- NSN in fp64 ----
+    float xf[4];
+    load4(xtok + 4 * lane, xf);
+    double x[4], o[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        x[r] = (double)xf[r];
+        o[r] = a.given_shift ? (double)a.shift[bh * kD + 4 * lane + r] : a.o64[bh * kD + 4 * lane + r];
+    }
+    const double sqrt_d = sqrt((double)kD);
+    const double ss = warp_sum_d(x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3]);
+    double s1 = sqrt(ss) / sqrt_d;
+    if constexpr (DQ) {
+        double glo, gstep;
+        dq_grid(a.s1_grid, bh, glo, gstep);
+        s1 = dq_s1(s1, glo, gstep);
+    }
+    const double inv1 = s1 > 0.0 ? 1.0 / s1 : 0.0;
+    double z[4], ss2 = 0.0, yy = 0.0, oo = 0.0;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const double y = x[r] * inv1;
+        z[r] = y - o[r];
+        ss2 = fma(z[r], z[r], ss2);
+        yy = fma(y, y, yy);
+        oo = fma(o[r], o[r], oo);
+    }
+    ss2 = warp_sum_d(ss2);
+    yy = warp_sum_d(yy);
+    oo = warp_sum_d(oo);
+    // a residual at or below 2^-20 of the token/shift magnitude counts as zero
+    const double s2 = ss2 <= 0x1p-40 * (yy + oo) ? 0.0 : sqrt(ss2) / sqrt_d;
+    const double inv2 = s2 > 0.0 ? 1.0 / s2 : 0.0;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) z[r] *= inv2;
+    fwht128_lane4(z);  // unnormalised: w = z / sqrt(d)
+    const double hs = 1.0 / sqrt_d;
+    double w[G];
+    int j;  // this lane's sub-vector
+    int c0, c1;  // the codewords it scans
+    if constexpr (G == 4) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r) w[r] = z[r] * hs;
+        j = lane;
+        c0 = 0;
+        c1 = kNC;
+    } else {
+        // sub-vector j = coordinates 8j..8j+7 (lanes 2j, 2j+1); the two
+        // halves of the warp scan the two halves of the codebook
+        j = lane & 15;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            w[r] = __shfl_sync(kFull, z[r], 2 * j) * hs;
+            w[4 + r] = __shfl_sync(kFull, z[r], 2 * j + 1) * hs;
+        }
+        c0 = (lane >> 4) * (kNC / 2);
+        c1 = c0 + kNC / 2;
+    }
+    // ---- nearest codeword, fp64: four trackers (codewords c = k mod 4, in
+    //      increasing order, strict <), merged lowest distance then lowest index
+    double bd4[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
+    int bi4[4] = {c0, c0 + 1, c0 + 2, c0 + 3};
+    for (int c = c0; c < c1; c += 4) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            double d = 0.0;
+#pragma unroll
+            for (int r = 0; r < G; ++r) {
+                const double e = w[r] - Cs[(c + k) * G + r];
+                d = fma(e, e, d);
+            }
+            if (d < bd4[k]) { bd4[k] = d; bi4[k] = c + k; }
+        }
+    }
+    double bd = bd4[0];
+    int bi = bi4[0];
+#pragma unroll
+    for (int k = 1; k < 4; ++k)
+        if (bd4[k] < bd || (bd4[k] == bd && bi4[k] < bi)) { bd = bd4[k]; bi = bi4[k]; }
+    if constexpr (G == 8) {  // the lower half wins exact ties (lower index)
+        const double od = __shfl_xor_sync(kFull, bd, 16);
+        const int oi = __shfl_xor_sync(kFull, bi, 16);
+        const bool mine = (lane < 16) ? !(od < bd) : (bd < od);
+        bi = mine ? bi : oi;
+    }
+    float s1o = (float)s1, s2o = (float)s2;
+    if constexpr (ADAPT) {  // s2 * d / (w . w_hat), w . w_hat over all sub-vectors in fp64
+        double q = 0.0;
+        if (G == 4 || lane < 16) {
+#pragma unroll
+            for (int r = 0; r < G; ++r) q = fma(w[r], Cs[bi * G + r], q);
+        }
+        q = warp_sum_d(q);
+        if (q > 0.0) s2o = (float)((double)s2o * ((double)kD / q));
+    }
+    const int64_t orow = bh * a.cap + a.t_offset + t;
+    if (G == 4 || lane < 16) a.codes[orow * (kD / G) + j] = (uint8_t)bi;
+    if (lane == 0) reinterpret_cast<float2*>(a.scales)[orow] = make_float2(s1o, s2o);
+}
+
+template <typename XT, int G>
+cudaError_t launch_small_t(const EncodeArgs& a, cudaStream_t s) {
+    const int64_t n = (int64_t)a.B * a.H * a.T;
+    const int grid = (int)((n + kSmallThreads / 32 - 1) / (kSmallThreads / 32));
+    if (a.dq) {
+        if (a.adaptive) nsn_encode_small_kernel<XT, G, true, true><<<grid, kSmallThreads, 0, s>>>(a);
+        else nsn_encode_small_kernel<XT, G, false, true><<<grid, kSmallThreads, 0, s>>>(a);
+    } else {
+        if (a.adaptive) nsn_encode_small_kernel<XT, G, true, false><<<grid, kSmallThreads, 0, s>>>(a);
+        else nsn_encode_small_kernel<XT, G, false, false><<<grid, kSmallThreads, 0, s>>>(a);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_encode_small(const EncodeArgs& a, cudaStream_t s) {
+    if (a.x_bf16) return a.sub == 4 ? launch_small_t<__nv_bfloat16, 4>(a, s) : launch_small_t<__nv_bfloat16, 8>(a, s);
+    return a.sub == 4 ? launch_small_t<float, 4>(a, s) : launch_small_t<float, 8>(a, s);
+}
+
+}  // namespace nsnq

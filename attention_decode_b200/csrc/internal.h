@@ -44,6 +44,7 @@ struct EncodeArgs {
     double* o64;                // [B][H][128]
     double* minmax;             // [B][H][nchunk1][2] least / largest log2 s1 per chunk
     unsigned* head_done;        // [B][H] chunks of pass 1 finished (zeroed per call)
+    int zero_stats;             // the pass-2 kernel zeroes stats (no memset before the call)
     int nchunk1;
     int64_t chunk1;
 };
@@ -58,6 +59,10 @@ struct EncodePlan {
 EncodePlan plan_encode(int B, int H, int64_t T);
 cudaError_t launch_encode(const EncodeArgs& a, cudaStream_t s);
 cudaError_t launch_encode_pruned(const EncodeArgs& a, cudaStream_t s);
+// Pass 2 of calls with at most kSmallEncode token-heads: one warp per
+// token-head, fp64 throughout (a decode step's appends).
+constexpr int64_t kSmallEncode = 1024;
+cudaError_t launch_encode_small(const EncodeArgs& a, cudaStream_t s);
 cudaError_t launch_encode1_tc(const EncodeArgs& a, cudaStream_t s);
 size_t index_bytes();
 cudaError_t launch_index_build(const float* C, void* index, cudaStream_t s);

@@ -35,6 +35,8 @@ ENCODE_CASES = [
     ("K-1bit-bf16-ragged", 2, 2, 545, "bf16", 8, S.K_MODERATE, "K"),
     ("K-2bit-f32-strong-outliers", 1, 2, 1100, "f32", 4, S.K_STRONG, "K"),
     ("K-2bit-bf16-single-token", 1, 2, 1, "bf16", 4, S.K_MODERATE, "K"),
+    # above the small-call size (1024 token-heads): the tensor-core 1-bit path with fp32 input
+    ("K-1bit-f32-ragged", 2, 2, 300, "f32", 8, S.K_MODERATE, "K"),
 ]
 
 
@@ -274,10 +276,10 @@ def test_encode_detects_index_of_another_codebook(codebooks):
     C = codebooks[4]
     other = P.codebook((C * np.float32(1.01)).astype(np.float32)).prepare()
     good = P.codebook(C)
-    w = _workload(1, 2, 100, "bf16", 4)
+    w = _workload(1, 2, 600, "bf16", 4)  # above the small-call size: the indexed search
     io, _ = _inputs(w, "K")
     x = P.to_dev(io, "bf16")
-    cache = nsnq.Cache.empty(1, 2, 100, 4)
+    cache = nsnq.Cache.empty(1, 2, 600, 4)
     ws = nsnq.nsnq_encode(x, nsnq.Codebook(good.centroids, other.index), cache)
     assert nsnq.encode_stats(ws)[2] != 0
     ws = nsnq.nsnq_encode(x, good, cache)
@@ -306,12 +308,12 @@ def test_encode_adaptive_scale_matches_oracle(codebooks, sub, T, dtype, kdist):
 def test_encode_adaptive_scale_given_shift(codebooks, sub):
     """Scale adjustment with a given shift (the append path), a far-off shift
     included so that some tokens take the fp64 path."""
-    w = _workload(1, 2, 260, "bf16", sub)
+    w = _workload(1, 2, 600, "bf16", sub)  # above the small-call size
     io, x64 = _inputs(w, "K")
     C = codebooks[sub]
     o_given = (np.random.default_rng(3).standard_normal((1, 2, D)) * 0.3).astype(np.float32)
     ora = O.encode(x64, C, shift=o_given.astype(np.float64), want_w=True, adaptive_scale=True)
-    cache = nsnq.Cache.empty(1, 2, 260, sub)
+    cache = nsnq.Cache.empty(1, 2, 600, sub)
     cache.shift.copy_(torch.from_numpy(o_given))
     nsnq.nsnq_encode(P.to_dev(io, "bf16"), P.codebook(C), cache, shift_mode=nsnq.SHIFT_GIVEN,
                      flags=nsnq.ENCODE_ADAPTIVE_SCALE)
@@ -319,3 +321,58 @@ def test_encode_adaptive_scale_given_shift(codebooks, sub):
     _, n_bad, worst = P.code_report(cache.codes.cpu().numpy(), ora["codes"], ora["w"], C)
     assert n_bad == 0, worst
     P.check_scales(cache.scales.cpu().numpy(), ora)
+
+
+ADAPT, DQF = nsnq.ENCODE_ADAPTIVE_SCALE, nsnq.ENCODE_DOUBLE_QUANT
+
+
+@pytest.mark.parametrize("sub,dtype,B,H,T,flags,given", [
+    (4, "bf16", 64, 8, 1, 0, True),        # one decode step's appends, 64 sequences
+    (8, "bf16", 64, 8, 1, 0, True),
+    (4, "f32", 1, 2, 300, 0, False),
+    (8, "f32", 2, 2, 200, ADAPT, False),
+    (4, "bf16", 2, 2, 200, DQF | ADAPT, False),
+    (8, "bf16", 1, 4, 256, DQF, False),
+    (4, "bf16", 4, 8, 32, ADAPT, True),     # exactly the small-call size
+])
+def test_small_call_encode_matches_oracle(codebooks, sub, dtype, B, H, T, flags, given):
+    """Calls of at most 1024 token-heads take the one-warp-per-token-head fp64
+    pass 2; codes, scales and (shift-compute mode) the shift against the
+    oracle, for both bit rates, both input types, the scale adjustment and
+    double quantization."""
+    w = _workload(B, H, T, dtype, sub, S.K_STRONG if sub == 4 else S.K_MODERATE, seed=11)
+    io, x64 = _inputs(w, "K")
+    C = codebooks[sub]
+    o_given = None
+    if given:
+        o_given = (np.random.default_rng(5).standard_normal((B, H, D)) * 0.3).astype(np.float32)
+    ora = O.encode(x64, C, shift=None if o_given is None else o_given.astype(np.float64), want_w=True,
+                   adaptive_scale=bool(flags & ADAPT), double_quant=bool(flags & DQF))
+    cache = nsnq.Cache.empty(B, H, T, sub)
+    if given:
+        cache.shift.copy_(torch.from_numpy(o_given))
+    nsnq.nsnq_encode(P.to_dev(io, dtype), P.codebook(C), cache,
+                     shift_mode=nsnq.SHIFT_GIVEN if given else nsnq.SHIFT_COMPUTE, flags=flags)
+    torch.cuda.synchronize()
+    _, n_bad, worst = P.code_report(cache.codes.cpu().numpy(), ora["codes"], ora["w"], C)
+    assert n_bad == 0, worst
+    P.check_scales(cache.scales.cpu().numpy(), ora)
+    if not given:
+        P.check_shift(cache.shift.cpu().numpy(), ora["o"])
+
+
+def test_small_given_call_resets_the_stats(codebooks):
+    """A small shift-given call (no workspace memset) still leaves the
+    workspace's counters zeroed for encode_stats()."""
+    C = codebooks[4]
+    other = P.codebook((C * np.float32(1.01)).astype(np.float32)).prepare()
+    good = P.codebook(C)
+    w = _workload(1, 2, 600, "bf16", 4)
+    io, _ = _inputs(w, "K")
+    x = P.to_dev(io, "bf16")
+    cache = nsnq.Cache.empty(1, 2, 601, 4)
+    ws = nsnq.nsnq_encode(x, nsnq.Codebook(good.centroids, other.index), cache)
+    assert nsnq.encode_stats(ws)[2] != 0
+    nsnq.nsnq_encode(x[:, :, :1], good, cache, t_offset=600, shift_mode=nsnq.SHIFT_GIVEN, workspace=ws)
+    torch.cuda.synchronize()
+    assert tuple(nsnq.encode_stats(ws)) == (0, 0, 0)
