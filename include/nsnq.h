@@ -154,9 +154,12 @@ size_t nsnq_encode_workspace(int B, int H, int64_t T, int D);
  *             bytes, 256-byte aligned.
  * Codes equal the nearest codeword of the exact (fp64) transformed token;
  * sub-vectors whose two best fp32 distances are within a relative 2e-5
- * (sub_dim 4) or 1e-4 (sub_dim 8) are re-decided in fp64. Stored s1, s2, o are fp32 roundings. A zero-norm
- * token (or a zero residual after the shift) maps to the zero vector with
- * s = 0. T = 0 is a no-op.
+ * (sub_dim 4) or 1e-4 (sub_dim 8) are re-decided in fp64. Calls of at most
+ * 1024 token-heads (B*H*T, e.g. a decode step's appends) compute every
+ * token-head in fp64 with a full codeword scan instead: the index is not
+ * read and the workspace counters stay 0. Stored s1, s2, o are fp32
+ * roundings. A zero-norm token (or a zero residual after the shift) maps to
+ * the zero vector with s = 0. T = 0 is a no-op.
  */
 nsnq_status nsnq_encode(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t T, int D,
                         int64_t stride_b, int64_t stride_h, int64_t stride_t, int64_t t_offset,
