@@ -279,11 +279,21 @@ __global__ void __launch_bounds__(kStatsThreads, 4) nsn_stats_kernel(EncodeArgs 
 }
 
 // ---------------------------------------------------------------- host --
+// Pass 1 splits each head's tokens into nchunk1 chunks so that the grid
+// (B * H * nchunk1 CTAs, four per SM) fills one wave of a 148-SM B200 as
+// evenly as the head count allows; a chunk is at least 64 tokens.
+constexpr int64_t kPass1Slots = 148 * 4;
+
 EncodePlan plan_encode(int B, int H, int64_t T) {
     EncodePlan p{};
-    p.chunk1 = 512;
-    p.nchunk1 = (int)((T + p.chunk1 - 1) / p.chunk1);
-    if (p.nchunk1 < 1) p.nchunk1 = 1;
+    const int64_t heads = (int64_t)B * H > 0 ? (int64_t)B * H : 1;
+    int64_t n = kPass1Slots / heads;
+    const int64_t by_len = (T + 63) / 64;
+    if (n > by_len) n = by_len;
+    if (n < 1) n = 1;
+    p.nchunk1 = (int)n;
+    p.chunk1 = (T + n - 1) / n;
+    if (p.chunk1 < 1) p.chunk1 = 1;
     p.reset_bytes = kEncodeStatsBytes + (size_t)B * H * sizeof(unsigned);  // stats + per-head counters
     p.partial_off = align_up(p.reset_bytes, kWsAlign);
     const size_t partial_bytes = (size_t)B * H * p.nchunk1 * kD * sizeof(double);

@@ -97,10 +97,13 @@ def test_index_build_validation(lib):
     assert lib.nsnq_codebook_index_build(_cb(), FAKE, need - 1, None) == nsnq.NSNQ_ERR_WORKSPACE
 
 
-def test_encode_workspace_grows_with_tokens(lib):
-    a = lib.nsnq_encode_workspace(8, 8, 4096, 128)
-    b = lib.nsnq_encode_workspace(8, 8, 8192, 128)
-    assert 0 < a < b and a % 256 == 0
+def test_encode_workspace_is_bounded(lib):
+    # pass 1 uses at most one wave of chunks: the workspace stops growing with T
+    a = lib.nsnq_encode_workspace(8, 8, 256, 128)
+    b = lib.nsnq_encode_workspace(8, 8, 4096, 128)
+    c = lib.nsnq_encode_workspace(8, 8, 1 << 20, 128)
+    assert 0 < a <= b == c and a % 256 == 0
+    assert lib.nsnq_encode_workspace(1, 1, 10, 128) > 0
     assert lib.nsnq_encode_workspace(8, 8, 4096, 64) == 0
 
 
