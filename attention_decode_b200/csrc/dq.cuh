@@ -17,6 +17,34 @@ __device__ __forceinline__ double dq_s1(double s1, double lo, double step) {
     return exp2(lo + k * step);
 }
 
+// Level tables of a grid, for deciding many tokens of one head without a
+// log2/exp2 per token: lvl[k] = 2^(lo + k step) (k < 16), thr[k] =
+// 2^(lo + (k + 1/2) step) (k < 15), inv[k] = 1 / lvl[k]. Built by threads
+// 0..15 of a block.
+__device__ __forceinline__ void dq_table_build(double lo, double step, double* lvl, double* thr,
+                                               double* inv) {
+    const int k = threadIdx.x;
+    if (k < 16) {
+        lvl[k] = exp2(lo + (double)k * step);
+        inv[k] = 1.0 / lvl[k];
+        if (k < 15) thr[k] = exp2(lo + ((double)k + 0.5) * step);
+    }
+}
+
+// The level dq_s1 picks for s1 > 0, by counting the thresholds at or below
+// s1; -1 when s1 lies within a relative 1e-12 of a threshold, where the
+// rounding of the log2 form decides (the caller then uses dq_s1). Away from
+// the thresholds the two agree exactly: the log2 form's error is ~1e-16.
+__device__ __forceinline__ int dq_level(double s1, double step, const double* thr) {
+    if (!(step > 0.0)) return 0;
+    int k = 0;
+#pragma unroll
+    for (int i = 0; i < 15; ++i) k += s1 >= thr[i] ? 1 : 0;
+    const double lo_t = k > 0 ? thr[k - 1] : 0.0, hi_t = k < 15 ? thr[k] : INFINITY;
+    if (s1 - lo_t <= 1e-12 * s1 || hi_t - s1 <= 1e-12 * s1) return -1;
+    return k;
+}
+
 // The grid of head bh from its fp32 copy.
 __device__ __forceinline__ void dq_grid(const float* s1_grid, int64_t bh, double& lo, double& step) {
     lo = (double)s1_grid[2 * bh];

@@ -73,7 +73,9 @@ struct Raw16<float> {
 };
 
 // Least and largest log2 s1 of a chunk's non-zero tokens (8 lanes per token,
-// fp64 sum of squares as in the stats kernel).
+// fp64 sum of squares as in the stats kernel). log2(sqrt(ss)/sqrt(d)) is
+// increasing in ss, so the chunk keeps the least and largest ss and takes
+// the log2 of those two only.
 template <typename XT>
 __global__ void __launch_bounds__(kStatsThreads) nsn_s1minmax_kernel(EncodeArgs a) {
     const int chunk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -84,7 +86,7 @@ __global__ void __launch_bounds__(kStatsThreads) nsn_s1minmax_kernel(EncodeArgs 
     const XT* xb = reinterpret_cast<const XT*>(a.x) + b * a.sb + h * a.sh + 16 * cg;
     const double sqrt_d = sqrt((double)kD);
     constexpr int64_t kStride = 4 * (kStatsThreads / 32);
-    double mn = INFINITY, mx = -INFINITY;
+    double mn = INFINITY, mx = -INFINITY;  // of ss > 0
     for (int64_t t = t0 + warp * 4 + tk; t - tk < t1; t += kStride) {
         Raw16<XT> r;
         if (t < t1) r.load(xb + t * a.st); else r.zero();
@@ -97,9 +99,8 @@ __global__ void __launch_bounds__(kStatsThreads) nsn_s1minmax_kernel(EncodeArgs 
         ss += __shfl_xor_sync(kFull, ss, 2);
         ss += __shfl_xor_sync(kFull, ss, 4);
         if (t < t1 && ss > 0.0) {
-            const double l = log2(sqrt(ss) / sqrt_d);
-            mn = fmin(mn, l);
-            mx = fmax(mx, l);
+            mn = fmin(mn, ss);
+            mx = fmax(mx, ss);
         }
     }
 #pragma unroll
@@ -116,8 +117,8 @@ __global__ void __launch_bounds__(kStatsThreads) nsn_s1minmax_kernel(EncodeArgs 
             mx = fmax(mx, red[w][1]);
         }
         double* out = a.minmax + ((int64_t)(b * a.H + h) * a.nchunk1 + chunk) * 2;
-        out[0] = mn;
-        out[1] = mx;
+        out[0] = mn <= mx ? log2(sqrt(mn) / sqrt_d) : INFINITY;
+        out[1] = mn <= mx ? log2(sqrt(mx) / sqrt_d) : -INFINITY;
     }
 }
 
@@ -211,7 +212,12 @@ __global__ void __launch_bounds__(kStatsThreads, 4) nsn_stats_kernel(EncodeArgs 
     const double sqrt_d = sqrt((double)kD);
     constexpr int64_t kStride = 2 * (kStatsThreads / 32);  // tokens per CTA step
     double glo = 0.0, gstep = 0.0;
-    if constexpr (DQ) dq_grid_from_chunks(a.minmax + bh * a.nchunk1 * 2, a.nchunk1, glo, gstep);
+    __shared__ double dq_lvl[16], dq_thr[15], dq_inv[16];
+    if constexpr (DQ) {
+        dq_grid_from_chunks(a.minmax + bh * a.nchunk1 * 2, a.nchunk1, glo, gstep);
+        dq_table_build(glo, gstep, dq_lvl, dq_thr, dq_inv);
+        __syncthreads();
+    }
     double acc[8];
 #pragma unroll
     for (int c = 0; c < 8; ++c) acc[c] = 0.0;
@@ -242,7 +248,9 @@ __global__ void __launch_bounds__(kStatsThreads, 4) nsn_stats_kernel(EncodeArgs 
             if (ss > 0.0) {
                 double inv;  // 1 / s1
                 if constexpr (DQ) {
-                    inv = 1.0 / dq_s1(sqrt(ss) / sqrt_d, glo, gstep);
+                    const double st = sqrt(ss) / sqrt_d;
+                    const int k = dq_level(st, gstep, dq_thr);
+                    inv = k >= 0 ? dq_inv[k] : 1.0 / dq_s1(st, glo, gstep);
                 } else {
                     inv = rsqrt(ss) * sqrt_d;
                 }
