@@ -26,102 +26,6 @@ namespace nsnq {
 constexpr int kStatsThreads = 256;
 
 // --------------------------------------------------------------- pass 1 --
-// Lane layout of the s1 range kernel: 8 lanes per token (16 channels each),
-// 4 tokens per warp step.
-
-template <typename XT>
-struct Raw16;
-template <>
-struct Raw16<__nv_bfloat16> {
-    uint4 u[2];
-    __device__ __forceinline__ void load(const __nv_bfloat16* p) {
-        const uint4* q = reinterpret_cast<const uint4*>(p);
-        u[0] = __ldg(q);
-        u[1] = __ldg(q + 1);
-    }
-    __device__ __forceinline__ void zero() { u[0] = u[1] = make_uint4(0, 0, 0, 0); }
-    __device__ __forceinline__ void unpack(float (&v)[16]) const {
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const uint32_t w[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                v[8 * i + 2 * k] = __uint_as_float(w[k] << 16);
-                v[8 * i + 2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
-            }
-        }
-    }
-};
-template <>
-struct Raw16<float> {
-    float4 f[4];
-    __device__ __forceinline__ void load(const float* p) {
-        const float4* q = reinterpret_cast<const float4*>(p);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) f[i] = __ldg(q + i);
-    }
-    __device__ __forceinline__ void zero() {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) f[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    __device__ __forceinline__ void unpack(float (&v)[16]) const {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            v[4 * i] = f[i].x; v[4 * i + 1] = f[i].y; v[4 * i + 2] = f[i].z; v[4 * i + 3] = f[i].w;
-        }
-    }
-};
-
-// Least and largest log2 s1 of a chunk's non-zero tokens (8 lanes per token,
-// fp64 sum of squares as in the stats kernel). log2(sqrt(ss)/sqrt(d)) is
-// increasing in ss, so the chunk keeps the least and largest ss and takes
-// the log2 of those two only.
-template <typename XT>
-__global__ void __launch_bounds__(kStatsThreads) nsn_s1minmax_kernel(EncodeArgs a) {
-    const int chunk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int warp = threadIdx.x >> 5, lane = lane_id();
-    const int tk = lane >> 3, cg = lane & 7;
-    const int64_t t0 = (int64_t)chunk * a.chunk1;
-    const int64_t t1 = min(t0 + a.chunk1, a.T);
-    const XT* xb = reinterpret_cast<const XT*>(a.x) + b * a.sb + h * a.sh + 16 * cg;
-    const double sqrt_d = sqrt((double)kD);
-    constexpr int64_t kStride = 4 * (kStatsThreads / 32);
-    double mn = INFINITY, mx = -INFINITY;  // of ss > 0
-    for (int64_t t = t0 + warp * 4 + tk; t - tk < t1; t += kStride) {
-        Raw16<XT> r;
-        if (t < t1) r.load(xb + t * a.st); else r.zero();
-        float v[16];
-        r.unpack(v);
-        double ss = 0.0;
-#pragma unroll
-        for (int c = 0; c < 16; ++c) ss = fma((double)v[c], (double)v[c], ss);
-        ss += __shfl_xor_sync(kFull, ss, 1);
-        ss += __shfl_xor_sync(kFull, ss, 2);
-        ss += __shfl_xor_sync(kFull, ss, 4);
-        if (t < t1 && ss > 0.0) {
-            mn = fmin(mn, ss);
-            mx = fmax(mx, ss);
-        }
-    }
-#pragma unroll
-    for (int m = 8; m < 32; m <<= 1) {
-        mn = fmin(mn, __shfl_xor_sync(kFull, mn, m));
-        mx = fmax(mx, __shfl_xor_sync(kFull, mx, m));
-    }
-    __shared__ double red[kStatsThreads / 32][2];
-    if (lane == 0) { red[warp][0] = mn; red[warp][1] = mx; }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        for (int w = 1; w < kStatsThreads / 32; ++w) {
-            mn = fmin(mn, red[w][0]);
-            mx = fmax(mx, red[w][1]);
-        }
-        double* out = a.minmax + ((int64_t)(b * a.H + h) * a.nchunk1 + chunk) * 2;
-        out[0] = mn <= mx ? log2(sqrt(mn) / sqrt_d) : INFINITY;
-        out[1] = mn <= mx ? log2(sqrt(mx) / sqrt_d) : -INFINITY;
-    }
-}
-
 // Pass-1 lane layout: 16 lanes per token (8 channels each, one 16-byte load
 // for bf16), 2 tokens per warp step, stats_depth<XT> steps of loads in
 // flight per warp (64 bytes per lane: the kernel streams x once from HBM and
@@ -159,6 +63,66 @@ struct Raw8<float> {
         v[4] = f[1].x; v[5] = f[1].y; v[6] = f[1].z; v[7] = f[1].w;
     }
 };
+
+// Least and largest log2 s1 of a chunk's non-zero tokens (layout and loads
+// as in the stats kernel, fp64 sum of squares). log2(sqrt(ss)/sqrt(d)) is
+// increasing in ss, so the chunk keeps the least and largest ss and takes
+// the log2 of those two only.
+template <typename XT>
+__global__ void __launch_bounds__(kStatsThreads, 4) nsn_s1minmax_kernel(EncodeArgs a) {
+    const int chunk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = lane_id();
+    const int tk = lane >> 4, cg = lane & 15;
+    const int64_t t0 = (int64_t)chunk * a.chunk1;
+    const int64_t t1 = min(t0 + a.chunk1, a.T);
+    const XT* xb = reinterpret_cast<const XT*>(a.x) + b * a.sb + h * a.sh + 8 * cg;
+    constexpr int64_t kStride = 2 * (kStatsThreads / 32);  // tokens per CTA step
+    constexpr int kDepth = stats_depth<XT>();
+    Raw8<XT> buf[kDepth];
+#pragma unroll
+    for (int d = 0; d < kDepth; ++d) {
+        const int64_t t = t0 + warp * 2 + d * kStride + tk;
+        if (t < t1) buf[d].load(xb + t * a.st); else buf[d].zero();
+    }
+    double mn = INFINITY, mx = -INFINITY;  // of ss > 0 (zero-filled slots give 0)
+    for (int64_t base = t0 + warp * 2; base < t1; base += kDepth * kStride) {
+#pragma unroll
+        for (int d = 0; d < kDepth; ++d) {
+            float v[8];
+            buf[d].unpack(v);
+            const int64_t tn = base + (d + kDepth) * kStride + tk;
+            if (tn < t1) buf[d].load(xb + tn * a.st); else buf[d].zero();
+            double s0 = 0.0, s1 = 0.0;
+#pragma unroll
+            for (int c = 0; c < 8; c += 2) {
+                s0 = fma((double)v[c], (double)v[c], s0);
+                s1 = fma((double)v[c + 1], (double)v[c + 1], s1);
+            }
+            double ss = s0 + s1;
+#pragma unroll
+            for (int m = 1; m < 16; m <<= 1) ss += __shfl_xor_sync(kFull, ss, m);
+            if (ss > 0.0) {
+                mn = fmin(mn, ss);
+                mx = fmax(mx, ss);
+            }
+        }
+    }
+    mn = fmin(mn, __shfl_xor_sync(kFull, mn, 16));
+    mx = fmax(mx, __shfl_xor_sync(kFull, mx, 16));
+    __shared__ double red[kStatsThreads / 32][2];
+    if (lane == 0) { red[warp][0] = mn; red[warp][1] = mx; }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < kStatsThreads / 32; ++w) {
+            mn = fmin(mn, red[w][0]);
+            mx = fmax(mx, red[w][1]);
+        }
+        const double sqrt_d = sqrt((double)kD);
+        double* out = a.minmax + ((int64_t)(b * a.H + h) * a.nchunk1 + chunk) * 2;
+        out[0] = mn <= mx ? log2(sqrt(mn) / sqrt_d) : INFINITY;
+        out[1] = mn <= mx ? log2(sqrt(mx) / sqrt_d) : -INFINITY;
+    }
+}
 
 // o of one (b, h) from its chunk partials, by the CTA whose chunk finished
 // last: o = sum / T in fp64 (double quantization: o on 16 uniform levels
