@@ -245,20 +245,43 @@ def run_cuda(args):
 
     # ---- end to end: pinned host K/V/q in, the step's result (the attention
     #      output) out, through the public API; the quantized cache is device
-    #      state and stays on the GPU ----
+    #      state and stays on the GPU. The batch goes over in two halves on a
+    #      copy stream, and each half is encoded as soon as it has arrived (the
+    #      shift is per sequence and head), so the host link and the kernels
+    #      overlap; more, smaller pieces measured slower ----
     res_host = torch.empty(B, Hq, 128, dtype=torch.bfloat16).pin_memory()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    copy_stream = torch.cuda.Stream(device=dev)
+    halves = [(0, (B + 1) // 2), ((B + 1) // 2, B)] if B > 1 else [(0, B)]
+    arrived = [torch.cuda.Event() for _ in halves]
+    cut = lambda c, b0, b1: nsnq.Cache(c.codes[b0:b1], c.scales[b0:b1], c.shift[b0:b1])
+    parts = [(b0, b1, cut(kc, b0, b1), cut(vc, b0, b1)) for b0, b1 in halves]
+    ws_h = torch.empty(nsnq.nsnq_encode_workspace((B + 1) // 2, H, T), dtype=torch.uint8, device=dev)
+
+    def e2e_step():
+        copy_stream.wait_stream(stream)
+        with torch.cuda.stream(copy_stream):
+            for (b0, b1, _, _), ev_ in zip(parts, arrived):
+                k[b0:b1].copy_(host["k"][b0:b1], non_blocking=True)
+                v[b0:b1].copy_(host["v"][b0:b1], non_blocking=True)
+                ev_.record(copy_stream)
+        q.copy_(host["q"], non_blocking=True)
+        for (b0, b1, kh, vh), ev_ in zip(parts, arrived):
+            stream.wait_event(ev_)
+            nsnq.nsnq_encode(k[b0:b1], cb, kh, workspace=ws_h)
+            nsnq.nsnq_encode(v[b0:b1], cb, vh, workspace=ws_h)
+        nsnq.nsnq_attn_decode(q, kc, vc, cb, cb, seq, T, Hkv=H, out=out, workspace=ws_a)
+        res_host.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
     barrier()
     torch.cuda.synchronize()
     e2e_ms = 0.0
     for i in range(args.steps):
         flush.zero_()
         e0.record(stream)
-        k.copy_(host["k"], non_blocking=True)
-        v.copy_(host["v"], non_blocking=True)
-        q.copy_(host["q"], non_blocking=True)
-        step(k, v, q)
-        res_host.copy_(out, non_blocking=True)
+        e2e_step()
         e1.record(stream)
         e1.synchronize()
         e2e_ms += e0.elapsed_time(e1)
@@ -267,7 +290,8 @@ def run_cuda(args):
     h2d = sum(host[n].numel() * host[n].element_size() for n in ("k", "v", "q"))
     d2h = res_host.numel() * res_host.element_size()
     e2e = {"value": tokens_per_step / (e2e_ms / args.steps / 1e3), "unit": "KV tokens/s",
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "overlap": "K/V host copies in two halves on a copy stream, each half encoded on arrival"}
 
     # ---- roofline of the dominant call (encode), algorithmic bytes ----
     hbm, peak_kind = peaks()
