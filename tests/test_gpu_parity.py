@@ -37,6 +37,9 @@ ENCODE_CASES = [
     ("K-2bit-bf16-single-token", 1, 2, 1, "bf16", 4, S.K_MODERATE, "K"),
     # above the small-call size (1024 token-heads): the tensor-core 1-bit path with fp32 input
     ("K-1bit-f32-ragged", 2, 2, 300, "f32", 8, S.K_MODERATE, "K"),
+    # one token-head past the small-call size: the persistent kernels on a single head
+    ("K-2bit-bf16-1025", 1, 1, 1025, "bf16", 4, S.K_STRONG, "K"),
+    ("K-1bit-bf16-1025", 1, 1, 1025, "bf16", 8, S.K_MODERATE, "K"),
 ]
 
 

@@ -508,3 +508,54 @@ def test_double_quant_append_uses_the_stored_grid(codebooks):
     assert np.abs(k - np.round(k)).max() < 1e-9 and k.min() > -1e-9 and k.max() < 15 + 1e-9
     assert np.allclose(app["s1"][0, 0, -2:], 2.0 ** (lo + 15 * step))
     assert np.array_equal(app["o"], pre["o"]) and np.array_equal(app["s1_grid"], pre["s1_grid"])
+
+
+# ------------------------------------------------- rotated-query identities --
+@pytest.mark.parametrize("g", [4, 8])
+def test_lut_scores_equal_dense_scores(codebooks, g):
+    """Methodology §4: with x_hat = s1 (s2 H w_hat + o) and H symmetric
+    orthonormal, q . x_hat = s1 (s2 sum_j L[j][code_j] + q . o) where
+    L[j][c] = (H q)_j . C_c. The left side uses the oracle's dense dequant;
+    the right side is assembled here from the table, so a wrong sign, index
+    or transpose in either form breaks the equality."""
+    w = S.Workload("lut", B=1, Hkv=2, Hq=2, T=64, d=D, sub_dim=g, dtype="f32",
+                   kdist=S.K_MODERATE, seed=31)
+    x = S.keys(w)
+    C = codebooks[g]
+    enc = O.encode(x, C)
+    s1, s2, o = O.stored(enc)
+    xh = O.dequant(enc["codes"], s1, s2, o, C)
+    rng = np.random.default_rng(7)
+    H = scipy.linalg.hadamard(D).astype(np.float64) / np.sqrt(D)
+    for h in range(2):
+        q = rng.standard_normal(D)
+        qr = H @ q
+        L = qr.reshape(D // g, g) @ C.astype(np.float64).T  # [j][c]
+        codes = enc["codes"][0, h].astype(np.int64)           # [T][j]
+        table = L[np.arange(D // g)[None, :], codes].sum(-1)  # [T]
+        lut = s1[0, h].astype(np.float64) * (s2[0, h].astype(np.float64) * table
+                                             + q @ o[0, h].astype(np.float64))
+        dense = xh[0, h] @ q
+        assert np.abs(lut - dense).max() <= 1e-10 * np.abs(dense).max()
+
+
+def test_rotated_domain_value_sum_equals_dense(codebooks):
+    """Methodology §4: sum_t p_t v_hat_t = H (sum_t p_t s1_t s2_t w_hat_t)
+    + (sum_t p_t s1_t) o, i.e. values can be accumulated in the Hadamard
+    domain and rotated once."""
+    g = 4
+    w = S.Workload("vsum", B=1, Hkv=1, Hq=1, T=50, d=D, sub_dim=g, dtype="f32",
+                   kdist=S.K_MODERATE, seed=32)
+    v = S.values(w)
+    C = codebooks[g]
+    enc = O.encode(v, C)
+    s1, s2, o = O.stored(enc)
+    vh = O.dequant(enc["codes"], s1, s2, o, C)[0, 0]
+    p = np.random.default_rng(8).random(50)
+    H = scipy.linalg.hadamard(D).astype(np.float64) / np.sqrt(D)
+    what = C.astype(np.float64)[enc["codes"][0, 0].astype(np.int64)].reshape(50, D)
+    a = (p * s1[0, 0] * s2[0, 0]) @ what
+    beta = (p * s1[0, 0]).sum()
+    rotated = H @ a + beta * o[0, 0].astype(np.float64)
+    dense = p @ vh
+    assert np.abs(rotated - dense).max() <= 1e-10 * np.abs(dense).max()
