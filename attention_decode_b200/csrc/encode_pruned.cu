@@ -281,6 +281,15 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
     if (tid == 0 && blockIdx.x == 0 && a.stats &&
         (*hash_s != hdr->pad[0] || hdr->magic != kIndexMagic || hdr->overflow))
         atomicOr(&a.stats[2], 1ull);
+    // Offsets past the staged entries (an index of other centroids, or not
+    // an index at all: flagged above, its codes are void) are clamped, so
+    // that every walk stays inside shared memory.
+    {
+        uint16_t* offs_w = reinterpret_cast<uint16_t*>(sm + kSmOffsets);
+        for (int i = tid; i <= kCells; i += kPrunedThreads)
+            offs_w[i] = (uint16_t)min((uint32_t)offs_w[i], n_pairs);
+    }
+    __syncthreads();
 
     // Each warp owns tiles of 16 consecutive token-heads of one (batch, head)
     // and keeps its own copy of that head's shift: no CTA barrier in the loop.

@@ -379,3 +379,32 @@ def test_small_given_call_resets_the_stats(codebooks):
     nsnq.nsnq_encode(x[:, :, :1], good, cache, t_offset=600, shift_mode=nsnq.SHIFT_GIVEN, workspace=ws)
     torch.cuda.synchronize()
     assert tuple(nsnq.encode_stats(ws)) == (0, 0, 0)
+
+
+@pytest.mark.parametrize("fill", [0xFF, 0x00, "random"])
+def test_encode_with_a_garbage_index_completes_and_is_flagged(codebooks, fill):
+    """An index buffer that is not an index (offsets past the lists, a wrong
+    magic and hash) must not take the walk outside shared memory: the call
+    completes, the mismatch flag is set, and a later call with the right
+    index is exact again."""
+    C = codebooks[4]
+    good = P.codebook(C)
+    n = int(nsnq.load().nsnq_codebook_index_bytes(4))
+    if fill == "random":
+        junk = torch.randint(0, 256, (n,), dtype=torch.int32, device="cuda",
+                             generator=torch.Generator(device="cuda").manual_seed(9)).to(torch.uint8)
+    else:
+        junk = torch.full((n,), fill, dtype=torch.uint8, device="cuda")
+    w = _workload(1, 2, 600, "bf16", 4)
+    io, x64 = _inputs(w, "K")
+    x = P.to_dev(io, "bf16")
+    cache = nsnq.Cache.empty(1, 2, 600, 4)
+    ws = nsnq.nsnq_encode(x, nsnq.Codebook(good.centroids, junk), cache)
+    torch.cuda.synchronize()
+    assert nsnq.encode_stats(ws)[2] != 0
+    nsnq.nsnq_encode(x, good, cache, workspace=ws)
+    torch.cuda.synchronize()
+    assert nsnq.encode_stats(ws)[2] == 0
+    ora = O.encode(x64, C, want_w=True)
+    _, n_bad, worst = P.code_report(cache.codes.cpu().numpy(), ora["codes"], ora["w"], C)
+    assert n_bad == 0, worst
