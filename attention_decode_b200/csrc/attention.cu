@@ -12,6 +12,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "f32x2.cuh"
 #include "internal.h"
 #include "attn_split.cuh"
 
@@ -50,31 +51,6 @@ __device__ __forceinline__ void load_q4(const void* q, int64_t off, float (&v)[4
     load4(reinterpret_cast<const QT*>(q) + off, v);
 }
 
-__device__ __forceinline__ uint64_t pk2(float a, float b) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-    return r;
-}
-__device__ __forceinline__ float2 upk2(uint64_t u) {
-    float2 r;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(u));
-    return r;
-}
-__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
 template <int GC, int KSUB, int VSUB, typename QT>
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a) {
     using S = AttnSmem<GC, KSUB, VSUB>;
@@ -223,8 +199,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a)
                 const uint32_t word = (t7 & 4) ? kw[(s >> 2) ^ 1] : kw[s >> 2];
                 const uint32_t code = __byte_perm(word, 0u, 0x4440u | (uint32_t)((s ^ t7) & 3));
                 const float4 e = lut4[code * KJ + j];
-                s01 = fadd2(s01, pk2(e.x, e.y));
-                s23 = fadd2(s23, pk2(e.z, e.w));
+                s01 = add2(s01, pk2(e.x, e.y));
+                s23 = add2(s23, pk2(e.z, e.w));
             }
             const float2 a01 = upk2(s01), a23 = upk2(s23);
             sc[0] = a01.x; sc[1] = a01.y; sc[2] = a23.x; sc[3] = a23.y;
@@ -253,7 +229,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a)
             be[h] = fmaf(be[h], alpha, p * v2.x);
             const uint64_t al = pk2(alpha, alpha);
 #pragma unroll
-            for (int r = 0; r < VSUB / 2; ++r) acc[h][r] = fmul2(acc[h][r], al);
+            for (int r = 0; r < VSUB / 2; ++r) acc[h][r] = mul2(acc[h][r], al);
             my_w[lane * GP + h] = p * v2.x * v2.y;
             m[h] = mn;
         }
@@ -281,7 +257,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a)
                 const uint64_t wp = pk2(wv[h], wv[h]);
 #pragma unroll
                 for (int r = 0; r < VSUB / 2; ++r)
-                    acc[h][r] = ffma2(pk2(c[2 * r], c[2 * r + 1]), wp, acc[h][r]);
+                    acc[h][r] = fma2(pk2(c[2 * r], c[2 * r + 1]), wp, acc[h][r]);
             }
         };
         if (nt == 32) {  // full batch: unrolled so that several gathers are in flight

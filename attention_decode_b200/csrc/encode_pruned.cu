@@ -14,6 +14,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "f32x2.cuh"
 #include "internal.h"
 #include "dq.cuh"
 #include "vq_index.cuh"
@@ -34,36 +35,6 @@ constexpr size_t kSmOffsets = kSmBinTab + kBinTabSize;         // uint16 [kCells
 constexpr size_t kSmEntries = kSmOffsets + kIdxSmemOffsetsBytes;
 constexpr size_t kSmBytes = kSmEntries + size_t(kMaxPairs) * 4;
 
-__device__ __forceinline__ uint64_t pk(float a, float b) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-    return r;
-}
-__device__ __forceinline__ float2 upk(uint64_t u) {
-    float2 r;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(u));
-    return r;
-}
-__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
 
 __device__ __forceinline__ uint32_t cb_hash_term(uint32_t bits, uint32_t i) {
     uint32_t h = bits * 0x9E3779B1u ^ (i * 0x85EBCA77u + 0x165667B1u);
@@ -196,8 +167,8 @@ struct Walk {
                          bin_fast(w3, tab);
         p = offs[cell];
         e = offs[cell + 1];
-        w01 = pk(w0, w1);
-        w23 = pk(w2, w3);
+        w01 = pk2(w0, w1);
+        w23 = pk2(w2, w3);
         d1 = INFINITY; d2 = INFINITY; i1 = 0;
     }
 
@@ -218,10 +189,10 @@ struct Walk {
         const bool take1 = (0x4b000000u | (ent1 >> 8)) <= lim;
         const float4 cv0 = myrep[(ent0 & 0xff) * 8];
         const float4 cv1 = myrep[(ent1 & 0xff) * 8];
-        const uint64_t a01 = sub2(w01, pk(cv0.x, cv0.y)), a23 = sub2(w23, pk(cv0.z, cv0.w));
-        const uint64_t b01 = sub2(w01, pk(cv1.x, cv1.y)), b23 = sub2(w23, pk(cv1.z, cv1.w));
-        const float2 da = upk(fma2(a23, a23, mul2(a01, a01)));
-        const float2 db = upk(fma2(b23, b23, mul2(b01, b01)));
+        const uint64_t a01 = sub2(w01, pk2(cv0.x, cv0.y)), a23 = sub2(w23, pk2(cv0.z, cv0.w));
+        const uint64_t b01 = sub2(w01, pk2(cv1.x, cv1.y)), b23 = sub2(w23, pk2(cv1.z, cv1.w));
+        const float2 da = upk2(fma2(a23, a23, mul2(a01, a01)));
+        const float2 db = upk2(fma2(b23, b23, mul2(b01, b01)));
         // Both entries count even past the band: they are listed codewords
         // (or the padding, farther than the nearest by the margin), so they
         // can only tighten d1 or reveal a true near-tie.
@@ -332,11 +303,11 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
         uint64_t acc0 = 0, acc1 = 0;
 #pragma unroll
         for (int k = 0; k < 64; k += 4) {
-            const uint64_t p0 = pk(v[k], v[k + 1]), p1 = pk(v[k + 2], v[k + 3]);
+            const uint64_t p0 = pk2(v[k], v[k + 1]), p1 = pk2(v[k + 2], v[k + 3]);
             acc0 = fma2(p0, p0, acc0);
             acc1 = fma2(p1, p1, acc1);
         }
-        float2 s01 = upk(add2(acc0, acc1));
+        float2 s01 = upk2(add2(acc0, acc1));
         float ss = s01.x + s01.y;
         ss += __shfl_xor_sync(kFull, ss, 1);
         float s1 = sqrtf(ss * (1.0f / kD));
@@ -355,18 +326,18 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
         }
         const float4* o4 = shift4 + 17 * half;  // upper half stored 4 floats further
         acc0 = 0; acc1 = 0;
-        const uint64_t inv2 = pk(inv1, inv1);
+        const uint64_t inv2 = pk2(inv1, inv1);
 #pragma unroll
         for (int k = 0; k < 64; k += 4) {
             const float4 o = o4[k >> 2];
-            const uint64_t z0 = fma2(pk(v[k], v[k + 1]), inv2, pk(o.x, o.y));
-            const uint64_t z1 = fma2(pk(v[k + 2], v[k + 3]), inv2, pk(o.z, o.w));
+            const uint64_t z0 = fma2(pk2(v[k], v[k + 1]), inv2, pk2(o.x, o.y));
+            const uint64_t z1 = fma2(pk2(v[k + 2], v[k + 3]), inv2, pk2(o.z, o.w));
             acc0 = fma2(z0, z0, acc0);
             acc1 = fma2(z1, z1, acc1);
-            const float2 a0 = upk(z0), a1 = upk(z1);
+            const float2 a0 = upk2(z0), a1 = upk2(z1);
             v[k] = a0.x; v[k + 1] = a0.y; v[k + 2] = a1.x; v[k + 3] = a1.y;
         }
-        s01 = upk(add2(acc0, acc1));
+        s01 = upk2(add2(acc0, acc1));
         float ss2 = s01.x + s01.y;
         ss2 += __shfl_xor_sync(kFull, ss2, 1);
         const float s2 = sqrtf(ss2 * (1.0f / kD));
@@ -374,9 +345,9 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
         const float sc = s2 > 0.f ? kRsqrtD / s2 : 0.f;
         // ---- FWHT: bits 0..4 on packed pairs (v[i], v[i+32]), bit 5 in-thread, bit 6 across the pair
         uint64_t P[32];
-        const uint64_t sc2 = pk(sc, sc);
+        const uint64_t sc2 = pk2(sc, sc);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) P[i] = mul2(pk(v[i], v[i + 32]), sc2);
+        for (int i = 0; i < 32; ++i) P[i] = mul2(pk2(v[i], v[i + 32]), sc2);
 #pragma unroll
         for (int bit = 1; bit < 32; bit <<= 1) {
 #pragma unroll
@@ -389,7 +360,7 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
         }
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-            const float2 q = upk(P[i]);
+            const float2 q = upk2(P[i]);
             v[i] = q.x + q.y;
             v[i + 32] = q.x - q.y;
         }
