@@ -5,14 +5,19 @@
 // dominate. Here one warp takes one token-head and does everything in fp64:
 // NSN with warp sums, the Hadamard transform across the warp (lane l holds
 // coordinates 4l..4l+3), and the nearest codeword of each sub-vector by a
-// full scan of the 256 codewords (lowest index on exact ties), so no near-tie
-// re-decision is needed. Stored s1, s2 are the fp64 values rounded to fp32,
-// as the persistent kernels store them for the tokens they re-decide in fp64.
+// full scan of the 256 codewords: in fp32 on the fp64 w rounded to fp32,
+// keeping the best and second-best distance, and again in fp64 (lowest index
+// on exact ties) where the two are within the near-tie band of the indexed
+// search (kTieRel d1 + kTieAbs, far above the fp32 scan's error). Stored s1,
+// s2 are the fp64 values rounded to fp32, as the persistent kernels store
+// them for the tokens they re-decide in fp64.
 #include <math.h>
 
 #include "common.cuh"
 #include "dq.cuh"
+#include "f32x2.cuh"
 #include "internal.h"
+#include "vq_index.cuh"
 
 namespace nsnq {
 
@@ -23,7 +28,11 @@ constexpr int kSmallThreads = 32;  // one warp (one token-head) per CTA: the CTA
 template <typename XT, int G, bool ADAPT, bool DQ>
 __global__ void __launch_bounds__(kSmallThreads) nsn_encode_small_kernel(EncodeArgs a) {
     __shared__ __align__(16) double Cs[kNC * G];  // the codebook, converted once
-    for (int i = threadIdx.x; i < kNC * G; i += kSmallThreads) Cs[i] = (double)a.C[i];
+    __shared__ __align__(16) float Cf[kNC * G];   // and as given
+    for (int i = threadIdx.x; i < kNC * G; i += kSmallThreads) {
+        Cf[i] = a.C[i];
+        Cs[i] = (double)a.C[i];
+    }
     __syncthreads();
     if (a.zero_stats && blockIdx.x == 0 && threadIdx.x < 8) a.stats[threadIdx.x] = 0ull;
     const int lane = lane_id();
@@ -91,32 +100,71 @@ __global__ void __launch_bounds__(kSmallThreads) nsn_encode_small_kernel(EncodeA
         c0 = (lane >> 4) * (kNC / 2);
         c1 = c0 + kNC / 2;
     }
-    // ---- nearest codeword, fp64: four trackers (codewords c = k mod 4, in
-    //      increasing order, strict <), merged lowest distance then lowest index
-    double bd4[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
-    int bi4[4] = {c0, c0 + 1, c0 + 2, c0 + 3};
-    for (int c = c0; c < c1; c += 4) {
+    // ---- nearest codeword: fp32 scan with the best and second best ----
+    uint64_t wp[G / 2];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            double d = 0.0;
+    for (int r = 0; r < G / 2; ++r) wp[r] = pk2((float)w[2 * r], (float)w[2 * r + 1]);
+    float b1 = INFINITY, b2 = INFINITY;
+    int bi = c0;
+#pragma unroll 4
+    for (int c = c0; c < c1; ++c) {
+        const float4* cv = reinterpret_cast<const float4*>(Cf + c * G);
+        uint64_t acc = 0ull;
 #pragma unroll
-            for (int r = 0; r < G; ++r) {
-                const double e = w[r] - Cs[(c + k) * G + r];
-                d = fma(e, e, d);
-            }
-            if (d < bd4[k]) { bd4[k] = d; bi4[k] = c + k; }
+        for (int r = 0; r < G / 4; ++r) {
+            const float4 q = cv[r];
+            const uint64_t e0 = sub2(wp[2 * r], pk2(q.x, q.y)), e1 = sub2(wp[2 * r + 1], pk2(q.z, q.w));
+            acc = fma2(e1, e1, fma2(e0, e0, acc));
         }
+        const float2 dd = upk2(acc);
+        const float d = dd.x + dd.y;
+        b2 = fminf(b2, fmaxf(b1, d));
+        bi = d < b1 ? c : bi;
+        b1 = fminf(b1, d);
     }
-    double bd = bd4[0];
-    int bi = bi4[0];
-#pragma unroll
-    for (int k = 1; k < 4; ++k)
-        if (bd4[k] < bd || (bd4[k] == bd && bi4[k] < bi)) { bd = bd4[k]; bi = bi4[k]; }
-    if constexpr (G == 8) {  // the lower half wins exact ties (lower index)
-        const double od = __shfl_xor_sync(kFull, bd, 16);
+    if constexpr (G == 8) {  // merge the two codebook halves (the lower wins exact ties)
+        const float o1 = __shfl_xor_sync(kFull, b1, 16), o2 = __shfl_xor_sync(kFull, b2, 16);
         const int oi = __shfl_xor_sync(kFull, bi, 16);
-        const bool mine = (lane < 16) ? !(od < bd) : (bd < od);
+        const bool mine = (lane < 16) ? !(o1 < b1) : (b1 < o1);
+        b2 = fminf(fmaxf(b1, o1), fminf(b2, o2));
+        b1 = fminf(b1, o1);
         bi = mine ? bi : oi;
+    }
+    // near ties: the exact decision in fp64 (four trackers over the codewords
+    // c = k mod 4, in increasing order, strict <; merged lowest distance,
+    // then lowest index)
+    const bool tie = (b2 - b1) <= fmaf(kTieRel, b1, kTieAbs);
+    if (__any_sync(kFull, tie)) {  // warp-uniform
+        double bd = INFINITY;
+        int bdi = c0;
+        if (tie) {
+            double bd4[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
+            int bi4[4] = {c0, c0 + 1, c0 + 2, c0 + 3};
+            for (int c = c0; c < c1; c += 4) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    double d = 0.0;
+#pragma unroll
+                    for (int r = 0; r < G; ++r) {
+                        const double e = w[r] - Cs[(c + k) * G + r];
+                        d = fma(e, e, d);
+                    }
+                    if (d < bd4[k]) { bd4[k] = d; bi4[k] = c + k; }
+                }
+            }
+            bd = bd4[0];
+            bdi = bi4[0];
+#pragma unroll
+            for (int k = 1; k < 4; ++k)
+                if (bd4[k] < bd || (bd4[k] == bd && bi4[k] < bdi)) { bd = bd4[k]; bdi = bi4[k]; }
+        }
+        if constexpr (G == 8) {  // both lanes of a sub-vector share its tie flag
+            const double od = __shfl_xor_sync(kFull, bd, 16);
+            const int oi = __shfl_xor_sync(kFull, bdi, 16);
+            const bool mine = (lane < 16) ? !(od < bd) : (bd < od);
+            bdi = mine ? bdi : oi;
+        }
+        if (tie) bi = bdi;
     }
     float s1o = (float)s1, s2o = (float)s2;
     if constexpr (ADAPT) {  // s2 * d / (w . w_hat), w . w_hat over all sub-vectors in fp64

@@ -58,6 +58,24 @@ def encode_case(B, H, T, reps, dev, sub=4):
           f"{sv} sub-vectors; index mismatch {mism}")
 
 
+def append_case(B, H, sub, reps, dev):
+    """A decode step's appends: one token per (sequence, kv-head) encoded with
+    the stored shift (the small-call pass 2) after a 1024-token prompt."""
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(0)
+    cb = _codebook(sub, dev)
+    T = 1024
+    cache = nsnq.Cache.empty(B, H, T + reps, sub, device=dev)
+    ws = torch.empty(nsnq.nsnq_encode_workspace(B, H, T), dtype=torch.uint8, device=dev)
+    cb.prepare()
+    nsnq.nsnq_encode(_keys(gen, B, H, T, dev), cb, cache, workspace=ws)
+    xn = _keys(gen, B, H, reps, dev)
+    for i in range(reps):
+        nsnq.nsnq_encode(xn[:, :, i:i + 1], cb, cache, t_offset=T + i,
+                         shift_mode=nsnq.SHIFT_GIVEN, workspace=ws)
+    torch.cuda.synchronize()
+
+
 def attn_case(B, Hq, Hkv, T, sub, reps, dev, rope=False):
     gen = torch.Generator(device=dev)
     gen.manual_seed(1)
@@ -88,6 +106,7 @@ CASES = {
     "attn-16x32k-1b": lambda r, d: attn_case(16, 32, 8, 32768, 8, r, d),
     "attn-rope-16x32k-2b": lambda r, d: attn_case(16, 32, 8, 32768, 4, r, d, rope=True),
     "attn-64x8k-gqa8": lambda r, d: attn_case(64, 64, 8, 8192, 4, r, d),
+    "append-64x8-2b": lambda r, d: append_case(64, 8, 4, r, d),
 }
 
 
