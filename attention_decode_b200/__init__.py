@@ -21,6 +21,7 @@ the bookkeeping for sequences decoded in lock-step):
 """
 from __future__ import annotations
 
+import collections
 import ctypes
 import dataclasses
 import os
@@ -41,7 +42,8 @@ N_CENTROIDS = 256
 EXPORTED = ("nsnq_status_string", "nsnq_last_error", "nsnq_codebook_index_bytes",
             "nsnq_codebook_index_build", "nsnq_encode_workspace", "nsnq_encode", "nsnq_dequant",
             "nsnq_attn_workspace", "nsnq_attn_decode", "nsnq_attn_decode_res",
-            "nsnq_attn_decode_rope", "nsnq_residual_write", "nsnq_attn_decode_noalloc")
+            "nsnq_attn_decode_rope", "nsnq_residual_write", "nsnq_attn_decode_noalloc",
+            "nsnq_codebook_quantize4")
 
 
 class NSNQError(RuntimeError):
@@ -112,6 +114,8 @@ def load(path: str = LIB_PATH):
     L.nsnq_attn_decode_noalloc.argtypes = [vp, ci, _Cache, _Cache, _Codebook, _Codebook, vp, i64,
                                            ci, ci, ci, ci, ctypes.c_float, vp, ci, vp]
     L.nsnq_attn_decode_noalloc.restype = ci
+    L.nsnq_codebook_quantize4.argtypes = [vp, vp, vp, vp, ci, ci, vp]
+    L.nsnq_codebook_quantize4.restype = ci
     _lib = L
     return L
 
@@ -174,6 +178,21 @@ class Codebook:
                          _ptr(self.index))
 
 
+def codebook_quantize4(centroids: torch.Tensor, stream=None, want_levels: bool = False):
+    """The double-quantized codebook (16 shared uniform levels, Methodology §3):
+    a new [256][g] fp32 tensor, plus (levels [256*g/2] uint8, grid (lo, step)
+    fp64) when want_levels."""
+    if centroids.dtype != torch.float32 or not centroids.is_contiguous():
+        raise TypeError("centroids must be contiguous float32")
+    n, g = int(centroids.shape[0]), int(centroids.shape[1])
+    out = torch.empty_like(centroids)
+    levels = torch.empty(n * g // 2, dtype=torch.uint8, device=centroids.device) if want_levels else None
+    grid = torch.empty(2, dtype=torch.float64, device=centroids.device) if want_levels else None
+    _check(load().nsnq_codebook_quantize4(_ptr(centroids), _ptr(out), _ptr(levels), _ptr(grid), n,
+                                          g, _stream(stream)))
+    return (out, levels, grid) if want_levels else out
+
+
 @dataclasses.dataclass
 class Cache:
     """One quantized tensor (K or V): codes [B][H][cap][D/g] uint8,
@@ -231,11 +250,20 @@ def nsnq_encode(x: torch.Tensor, cb: Codebook, cache: Cache, t_offset: int = 0,
     return workspace
 
 
-def encode_stats(workspace: torch.Tensor):
-    """(token-heads, sub-vectors) decided on the fp64 near-tie path by the last
-    encode, and whether the codebook index did not match the centroids."""
-    v = workspace[:24].cpu().view(torch.int64)
-    return int(v[0]), int(v[1]), int(v[2])
+EncodeStats = collections.namedtuple(
+    "EncodeStats", ("fp64_token_heads", "fp64_subvectors", "index_mismatch", "mma_timeout"))
+EncodeStats.__doc__ = """Counters of the last nsnq_encode that used a workspace (its first 64
+bytes): token-heads and sub-vectors decided on the fp64 near-tie path,
+whether the codebook index did not match the centroids, and whether a
+tensor-core scoring round timed out (that call's codes are then void)."""
+
+
+def encode_stats(workspace: torch.Tensor) -> EncodeStats:
+    """Read the counters of the last encode from its workspace (synchronises
+    with the device): (fp64 token-heads, fp64 sub-vectors, index mismatch,
+    MMA timeout)."""
+    v = workspace[:40].cpu().view(torch.int64)
+    return EncodeStats(int(v[0]), int(v[1]), int(v[2]), int(v[4]))
 
 
 def nsnq_dequant(cache: Cache, cb: Codebook, B: int, H: int, t0: int, T: int,

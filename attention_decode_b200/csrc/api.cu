@@ -106,6 +106,22 @@ nsnq_status nsnq_codebook_index_build(nsnq_codebook cb, void* index, size_t inde
     return ok();
 }
 
+nsnq_status nsnq_codebook_quantize4(const float* centroids, float* out, uint8_t* levels,
+                                    double* grid, int n_centroids, int sub_dim,
+                                    nsnq_stream stream) {
+    if (n_centroids != nsnq::kNCentroids)
+        return fail(NSNQ_ERR_UNSUPPORTED, "n_centroids = %d (only 256 is supported)", n_centroids);
+    if (sub_dim != 4 && sub_dim != 8)
+        return fail(NSNQ_ERR_UNSUPPORTED, "sub_dim = %d (4 or 8 supported)", sub_dim);
+    if (!centroids || !out) return fail(NSNQ_ERR_INVALID_ARG, "centroids or out is NULL");
+    if (!aligned(centroids, 4) || !aligned(out, 4) || (grid && !aligned(grid, 8)))
+        return fail(NSNQ_ERR_INVALID_ARG, "centroids/out must be 4-byte and grid 8-byte aligned");
+    cudaError_t e = nsnq::launch_codebook_q4(centroids, out, levels, grid, n_centroids * sub_dim,
+                                             reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "codebook quantize4 launch");
+    return ok();
+}
+
 size_t nsnq_encode_workspace(int B, int H, int64_t T, int D) {
     if (B < 0 || H < 0 || T < 0 || D != nsnq::kHeadDim) return 0;
     return nsnq::plan_encode(B, H, T).total;

@@ -10,8 +10,8 @@
 // The array is a file-scope __device__ variable: every GPU that loads the
 // library holds its kStaticScratchBytes until the process exits. In host
 // code its name only stands in for the symbol, so the device address is
-// looked up with cudaGetSymbolAddress, once per device, with that device
-// current, on the first call made on that device.
+// looked up with cudaGetSymbolAddress with the device current: on every call
+// whose stream is not capturing (the first call on a device must be one).
 #include <mutex>
 
 #include "../../include/nsnq.h"
@@ -29,18 +29,29 @@ constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
 void* g_device_ptr[kMaxDevices] = {};
 
-// Device address of g_attn_partials on the current device (set up on first use).
-cudaError_t partials_on_current_device(void** out) {
+// Device address of g_attn_partials on the current device. A call whose
+// stream is not capturing looks it up again every time (cheap once the module
+// is loaded), so the address stays right after cudaDeviceReset, which can
+// load the module elsewhere; a capturing call reuses the last address found
+// on this device and sets *need_setup when there is none yet.
+cudaError_t partials_on_current_device(cudaStream_t stream, void** out, bool* need_setup) {
+    *need_setup = false;
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    e = cudaStreamIsCapturing(stream, &cs);
+    if (e != cudaSuccess) return e;
     std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (g_device_ptr[dev] == nullptr) {
+    if (cs == cudaStreamCaptureStatusNone) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_attn_partials);
         if (e != cudaSuccess) return e;
         g_device_ptr[dev] = p;
+    } else if (g_device_ptr[dev] == nullptr) {
+        *need_setup = true;
+        return cudaSuccess;
     }
     *out = g_device_ptr[dev];
     return cudaSuccess;
@@ -66,10 +77,18 @@ extern "C" nsnq_status nsnq_attn_decode_noalloc(const void* q, nsnq_dtype q_dtyp
                                need, kStaticScratchBytes);
     }
     void* partials = nullptr;
-    const cudaError_t e = partials_on_current_device(&partials);
+    bool need_setup = false;
+    const cudaError_t e =
+        partials_on_current_device(reinterpret_cast<cudaStream_t>(stream), &partials, &need_setup);
     if (e != cudaSuccess) {
         return nsnq::set_error(NSNQ_ERR_CUDA, "nsnq_attn_decode_noalloc setup: %s",
                                cudaGetErrorString(e));
+    }
+    if (need_setup) {
+        return nsnq::set_error(NSNQ_ERR_INVALID_ARG,
+                               "nsnq_attn_decode_noalloc: the stream is capturing and this "
+                               "device has no array address yet; make one call on this device "
+                               "before capturing");
     }
     // Every split writes all of its partial rows (empty splits write neutral
     // ones) before the combine reads them, so nothing needs clearing.

@@ -66,6 +66,8 @@ cudaError_t launch_encode_small(const EncodeArgs& a, cudaStream_t s);
 cudaError_t launch_encode1_tc(const EncodeArgs& a, cudaStream_t s);
 size_t index_bytes();
 cudaError_t launch_index_build(const float* C, void* index, cudaStream_t s);
+cudaError_t launch_codebook_q4(const float* in, float* out, uint8_t* levels, double* grid, int n,
+                               cudaStream_t s);
 
 // ----------------------------------------------------------------- dequant --
 struct DequantArgs {

@@ -53,9 +53,9 @@ def encode_case(B, H, T, reps, dev, sub=4):
         nsnq.nsnq_encode(x, cb, cache, workspace=ws)
         e1.record()
     torch.cuda.synchronize()
-    th, sv, mism = nsnq.encode_stats(ws)
+    th, sv, mism, tmo = nsnq.encode_stats(ws)
     print(f"last call {e0.elapsed_time(e1):.3f} ms; fp64 path: {th} of {B * H * T} token-heads, "
-          f"{sv} sub-vectors; index mismatch {mism}")
+          f"{sv} sub-vectors; index mismatch {mism}; MMA timeout {tmo}")
 
 
 def append_case(B, H, sub, reps, dev):

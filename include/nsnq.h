@@ -128,12 +128,40 @@ nsnq_status nsnq_codebook_index_build(nsnq_codebook cb, void* index, size_t inde
                                       nsnq_stream stream);
 
 /*
+ * nsnq_codebook_quantize4 -- the double-quantized form of a codebook
+ * (Methodology §3, Double Quantization: the codebook entries take 4-bit
+ * values). All n_centroids * sub_dim entries share one grid of 16 uniform
+ * levels from their least value lo to their largest value hi:
+ * step = (hi - lo) / 15 and entry e becomes lo + k * step with
+ * k = (e - lo) / step rounded to the nearest integer (halves away from
+ * zero), computed in fp64 and rounded to fp32 (k = 0 for every entry when
+ * hi == lo).
+ *   centroids  device [n_centroids][sub_dim] fp32 (n_centroids 256, sub_dim 4 or 8).
+ *   out        device, same shape: the level values; may equal centroids.
+ *   levels     device [n_centroids * sub_dim / 2] bytes or NULL: the 4-bit k
+ *              of entry i in byte i / 2 (even i in the low nibble).
+ *   grid       device double[2] = (lo, step) or NULL.
+ * The result is a codebook like any other: pass `out` as the centroids of
+ * nsnq_encode (build the index from it for sub_dim 4), nsnq_dequant and the
+ * attention calls. Asynchronous on `stream`.
+ */
+nsnq_status nsnq_codebook_quantize4(const float* centroids, float* out, uint8_t* levels,
+                                    double* grid, int n_centroids, int sub_dim,
+                                    nsnq_stream stream);
+
+/*
  * Workspace bytes nsnq_encode needs for this shape (any shift mode). The
  * first 64 bytes hold counters the call resets and fills:
  *   uint64 [0] token-heads re-encoded on the fp64 near-tie path,
  *   uint64 [1] sub-vectors whose code was decided on that path,
  *   uint64 [2] nonzero if cb.index was not built from cb.centroids,
- *   uint64 [3] used internally (work counter).
+ *   uint64 [3] used internally (work counter),
+ *   uint64 [4] nonzero if a tensor-core scoring round (sub_dim 8) was not
+ *              seen complete within its bounded wait: the CTA that waited
+ *              stopped, so some codes and scales of this call are NOT
+ *              written and the call's result is void. The status returned
+ *              by nsnq_encode cannot report it (the kernel runs after the
+ *              call returns): read this word after the stream has finished.
  */
 size_t nsnq_encode_workspace(int B, int H, int64_t T, int D);
 
@@ -153,12 +181,14 @@ size_t nsnq_encode_workspace(int B, int H, int64_t T, int D);
  *   workspace device scratch of at least nsnq_encode_workspace(B, H, T, D)
  *             bytes, 256-byte aligned.
  * Codes equal the nearest codeword of the exact (fp64) transformed token;
- * sub-vectors whose two best fp32 distances are within a relative 2e-5
- * (sub_dim 4) or 1e-4 (sub_dim 8) are re-decided in fp64. Calls of at most
- * 1024 token-heads (B*H*T, e.g. a decode step's appends) compute every
- * token-head in fp64 with a full codeword scan instead: the index is not
- * read and the workspace counters stay 0. Stored s1, s2, o are fp32
- * roundings. A zero-norm token (or a zero residual after the shift) maps to
+ * sub-vectors whose two best fp32 distances are within the near-tie band
+ * (a bound on the fp32 / three-term tf32 scoring error) are re-decided in
+ * fp64. Calls of at most 1024 token-heads (B*H*T, e.g. a decode step's
+ * appends) take a one-warp-per-token-head path instead: NSN and the
+ * Hadamard transform in fp64, an fp32 scan of all 256 codewords keeping the
+ * best and second best, and an fp64 re-scan of the sub-vectors inside the
+ * near-tie band; the index is not read and the workspace counters stay 0.
+ * Stored s1, s2, o are fp32 roundings. A zero-norm token (or a zero residual after the shift) maps to
  * the zero vector with s = 0. T = 0 is a no-op.
  */
 nsnq_status nsnq_encode(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t T, int D,
@@ -282,9 +312,11 @@ nsnq_status nsnq_attn_decode_rope(const void* q, nsnq_dtype q_dtype, nsnq_cache 
  * Limit: shapes whose partials need more than 4 MiB
  * (nsnq_attn_workspace(B, Hq, Hkv, D, max_len) > 4194304) are rejected with
  * NSNQ_ERR_WORKSPACE before anything is launched.
- * The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress, with that device current); make that first call
- * before any stream capture. The array is shared by all calls and keeps the
+ * Every call whose `stream` is not capturing looks up the array's device
+ * address on the current device (cudaGetSymbolAddress), so the entry point
+ * stays valid after cudaDeviceReset, which can move the array. Make the
+ * first call on each device before any stream capture: a first call on a
+ * capturing stream returns NSNQ_ERR_INVALID_ARG. The array is shared by all calls and keeps the
  * last call's contents; nothing in it needs to start at zero. Calls that
  * overlap on the GPU (different streams, or different host threads on the
  * same device) race on the array: serialise them. Arguments, errors and

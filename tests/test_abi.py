@@ -216,3 +216,13 @@ def test_binding_has_no_fallback(tmp_path):
         mod.load(str(tmp_path / "missing.so"))
     mod._lib = None
     mod.load()
+
+
+def test_codebook_quantize4_validation(lib):
+    q = lib.nsnq_codebook_quantize4
+    assert q(FAKE, FAKE, None, None, 128, 4, None) == nsnq.NSNQ_ERR_UNSUPPORTED
+    assert q(FAKE, FAKE, None, None, 256, 5, None) == nsnq.NSNQ_ERR_UNSUPPORTED
+    assert q(None, FAKE, None, None, 256, 4, None) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert q(FAKE, None, None, None, 256, 8, None) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert q(FAKE + 2, FAKE, None, None, 256, 8, None) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert q(FAKE, FAKE, None, FAKE + 4, 256, 8, None) == nsnq.NSNQ_ERR_INVALID_ARG

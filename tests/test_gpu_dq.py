@@ -84,8 +84,10 @@ def test_double_quant_codebooks_through_encode_and_attention(codebooks, ksub, vs
     B, H, Hq, T = 2, 2, 8, 640
     w = S.Workload("dqa", B=B, Hkv=H, Hq=Hq, T=T, d=D, sub_dim=4, dtype="bf16",
                    kdist=S.K_MODERATE, seed=23)
-    Ck = O.quantize4(codebooks[ksub]).astype(np.float32)
-    Cv = O.quantize4(codebooks[vsub]).astype(np.float32)
+    # the 4-bit codebooks come from the library's own transform (checked
+    # against the oracle's in test_codebook_quantize4_matches_oracle)
+    Ck = nsnq.codebook_quantize4(torch.from_numpy(codebooks[ksub]).cuda()).cpu().numpy()
+    Cv = nsnq.codebook_quantize4(torch.from_numpy(codebooks[vsub]).cuda()).cpu().numpy()
     assert len(np.unique(Ck)) <= 16
     k_io, v_io = S.to_io(S.keys(w), "bf16"), S.to_io(S.values(w), "bf16")
     ok = O.encode(S.io_to_f64(k_io, "bf16"), Ck, want_w=True, double_quant=True)
@@ -112,3 +114,29 @@ def test_double_quant_codebooks_through_encode_and_attention(codebooks, ksub, vs
     ref = O.attention(S.io_to_f64(q_io, "bf16"), Kh, Vh, lens)
     e, _ = P.attn_errors(P.out_to_np(out), ref, False)
     assert (e <= 1.0).all(), e.max()
+
+
+@pytest.mark.parametrize("g", [4, 8])
+def test_codebook_quantize4_matches_oracle(codebooks, g):
+    """The library's 4-bit codebook transform: values equal the oracle's
+    fp64 levels rounded to fp32, the 4-bit indices and the grid rebuild
+    them, and the transform works in place."""
+    C = codebooks[g]
+    ref = O.quantize4(C)
+    dev = torch.from_numpy(C).cuda()
+    out, levels, grid = nsnq.codebook_quantize4(dev, want_levels=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(out.cpu().numpy(), ref.astype(np.float32))
+    lo, step = grid.cpu().numpy()
+    assert lo == C.min() and abs(lo + 15 * step - C.max()) <= 1e-12 * abs(C.max())
+    nib = levels.cpu().numpy()
+    k = np.stack([nib & 15, nib >> 4], -1).reshape(-1).astype(np.float64)
+    assert np.array_equal((lo + k * step).astype(np.float32), out.cpu().numpy().reshape(-1))
+    inplace = dev.clone()
+    nsnq.load().nsnq_codebook_quantize4(inplace.data_ptr(), inplace.data_ptr(), None, None, 256,
+                                        g, torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    assert torch.equal(inplace, out)
+    # a constant codebook keeps its value (step 0)
+    flat = torch.full((256, g), 0.75, device="cuda")
+    assert torch.equal(nsnq.codebook_quantize4(flat), flat)

@@ -156,3 +156,84 @@ def test_fullsize_long_context_encode_and_append(codebooks):
     ref = O.attention(S.io_to_f64(q_io, "bf16")[:, h * G:(h + 1) * G], refs[0], refs[1])
     e, _ = P.attn_errors(P.out_to_np(out)[:, h * G:(h + 1) * G], ref, False)
     assert (e <= 1.0).all(), e.max()
+
+
+def test_fullsize_encode_1bit_tensor_core_loop(codebooks):
+    """8 sequences x 8 kv-heads x 4096 tokens, bf16, 1 bit (g = 8): 32768
+    tiles of the tensor-core kernel, so every CTA of its persistent grid runs
+    dozens of tiles (mbarrier phase, TMEM reuse and A-operand overwrite carried
+    from tile to tile). Sampled heads from the first, middle and last tiles of
+    the grid's loop against the oracle; the MMA-timeout flag must stay 0."""
+    w = S.WORKLOADS["encode-8x4096"]
+    C = codebooks[8]
+    cb = P.codebook(C)
+    for which in ("K", "V"):
+        x64 = S.keys(w) if which == "K" else S.values(w)
+        io = S.to_io(x64, "bf16")
+        x64 = S.io_to_f64(io, "bf16")
+        cache = nsnq.Cache.empty(w.B, w.Hkv, w.T, 8)
+        ws = nsnq.nsnq_encode(P.to_dev(io, "bf16"), cb, cache)
+        torch.cuda.synchronize()
+        st = nsnq.encode_stats(ws)
+        assert st.mma_timeout == 0 and st.index_mismatch == 0, st
+        for b, h in ((0, 0), (3, 6), (7, 7)):
+            _check_encode_slice(cache, b, h, x64[b:b + 1, h:h + 1], C)
+
+
+@pytest.mark.parametrize("name,sub", [("decode-16x32k-1b", 8), ("decode-16x32k-2b", 4)])
+def test_fullsize_attention_over_gpu_encoded_cache(codebooks, name, sub):
+    """decode-16x32k with the cache built by the GPU encode: K and V
+    (16 x 8 kv-heads x 32768 tokens each, drawn on the device) are encoded in
+    one call per tensor (4.2 M token-heads; at 1 bit the tensor-core kernel's
+    full persistent loop), then decode attention runs over them. For sampled
+    (sequence, kv-head) slices the GPU codes, scales and shift are checked
+    against the oracle's encoding of the same bf16 inputs, and the attention
+    output against the oracle's attention over the GPU's own codes, scales
+    and shift."""
+    w = S.WORKLOADS[name]
+    C = codebooks[sub]
+    cb = P.codebook(C)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(w.seed)
+    chans, signs = w.kdist.channels(128)
+    bias = torch.zeros(128, device="cuda")
+    bias[chans] = torch.tensor(signs, device="cuda") * w.kdist.bias
+    samples = [(2, 1), (15, 7)]
+    caches, slices = {}, {}
+    for which in ("K", "V"):
+        z = torch.randn(w.B, w.Hkv, w.T, 128, generator=gen, device="cuda")
+        if which == "K":
+            s = torch.exp(w.kdist.sigma * torch.randn(w.B, w.Hkv, w.T, 1, generator=gen,
+                                                      device="cuda"))
+            z = (z + bias) * s
+        x = z.to(torch.bfloat16)
+        del z
+        cache = nsnq.Cache.empty(w.B, w.Hkv, w.T, sub)
+        ws = nsnq.nsnq_encode(x, cb, cache)
+        torch.cuda.synchronize()
+        st = nsnq.encode_stats(ws)
+        assert st.mma_timeout == 0 and st.index_mismatch == 0, st
+        for b, h in samples:
+            slices[(which, b, h)] = x[b:b + 1, h:h + 1].float().cpu().numpy().astype(np.float64)
+        del x
+        caches[which] = cache
+    q = torch.randn(w.B, w.Hq, 128, generator=gen, device="cuda").to(torch.bfloat16)
+    seq = torch.full((w.B,), w.T, dtype=torch.int32, device="cuda")
+    out = nsnq.nsnq_attn_decode(q, caches["K"], caches["V"], cb, cb, seq, w.T, Hkv=w.Hkv,
+                                out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    got = P.out_to_np(out)
+    q64 = q.float().cpu().numpy().astype(np.float64)
+    G = w.Hq // w.Hkv
+    for b, h in samples:
+        deq = []
+        for which in ("K", "V"):
+            cache = caches[which]
+            _check_encode_slice(cache, b, h, slices[(which, b, h)], C)
+            codes = cache.codes[b:b + 1, h:h + 1].cpu().numpy()
+            sc = cache.scales[b:b + 1, h:h + 1].cpu().numpy()
+            o = cache.shift[b:b + 1, h:h + 1].cpu().numpy()
+            deq.append(O.dequant(codes, sc[..., 0], sc[..., 1], o, C))
+        ref = O.attention(q64[b:b + 1, h * G:(h + 1) * G], deq[0], deq[1])
+        e, _ = P.attn_errors(got[b:b + 1, h * G:(h + 1) * G], ref, True)
+        assert (e <= 1.0).all(), (b, h, e.max())

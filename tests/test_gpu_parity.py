@@ -58,8 +58,8 @@ def test_encode_matches_oracle(codebooks, case):
     assert n_bad == 0, (n_mis, n_bad, worst)
     P.check_scales(cache.scales.cpu().numpy(), ora)
     P.check_shift(cache.shift.cpu().numpy(), ora["o"])
-    th, sv, mismatch = nsnq.encode_stats(ws)
-    assert mismatch == 0
+    th, sv, mismatch, timeout = nsnq.encode_stats(ws)
+    assert mismatch == 0 and timeout == 0
     assert th <= max(4, B * H * T // 50)
 
 
@@ -378,7 +378,7 @@ def test_small_given_call_resets_the_stats(codebooks):
     assert nsnq.encode_stats(ws)[2] != 0
     nsnq.nsnq_encode(x[:, :, :1], good, cache, t_offset=600, shift_mode=nsnq.SHIFT_GIVEN, workspace=ws)
     torch.cuda.synchronize()
-    assert tuple(nsnq.encode_stats(ws)) == (0, 0, 0)
+    assert tuple(nsnq.encode_stats(ws)) == (0, 0, 0, 0)
 
 
 @pytest.mark.parametrize("fill", [0xFF, 0x00, "random"])

@@ -479,11 +479,22 @@ def test_double_quant_byproducts_and_reconstruction(codebooks, g):
     enc = O.encode(x, C, want_w=True, double_quant=True)
     s1_exact = np.linalg.norm(x[0, 0], axis=1) / np.sqrt(D)
     lg = np.log2(s1_exact)
-    lo = np.float32(lg.min()).astype(np.float64)
-    step = np.float32((lg.max() - lg.min()) / 15).astype(np.float64)
-    assert np.array_equal(enc["s1_grid"][0, 0], [lo, step])
-    k = np.clip(np.round((lg - lo) / step), 0, 15)
-    assert np.abs(enc["s1"][0, 0] - 2.0 ** (lo + k * step)).max() < 1e-12 * enc["s1"].max()
+    lo, step = enc["s1_grid"][0, 0]
+    # the grid: fp32 values spanning the tokens' log2 s1 (up to fp32 rounding)
+    assert np.float32(lo) == lo and np.float32(step) == step and step > 0
+    assert abs(lo - lg.min()) <= 2.0 ** -23 * abs(lg.min()) + 1e-30
+    assert abs(lo + 15 * step - lg.max()) <= 16 * 2.0 ** -23 * max(abs(lg.max()), abs(lo))
+    # every stored s1 is one of the 16 levels 2^(lo + j step) ...
+    lq = np.log2(enc["s1"][0, 0])
+    k = (lq - lo) / step
+    assert np.abs(k - np.round(k)).max() < 1e-9 and k.min() > -1e-9 and k.max() < 15 + 1e-9
+    # ... the nearest one in the log2 domain (brute force over the 16 levels)
+    levels = lo + step * np.arange(16)
+    best = np.abs(lg[:, None] - levels[None, :]).min(1)
+    assert (np.abs(lq - lg) <= best + 1e-12).all()
+    assert (np.abs(lq - lg) <= step / 2 + 1e-12).all()
+    # the extreme tokens take the extreme levels
+    assert round(k[np.argmin(lg)]) == 0 and round(k[np.argmax(lg)]) == 15
     o = enc["o"][0, 0]
     assert len(np.unique(np.round((o - o.min()) / ((o.max() - o.min()) / 15), 9))) <= 16
     H = scipy.linalg.hadamard(D) / np.sqrt(D)
