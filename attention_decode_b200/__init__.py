@@ -60,7 +60,7 @@ class _Codebook(ctypes.Structure):
 class _Cache(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
                 ("shift", ctypes.c_void_p), ("cap", ctypes.c_int64),
-                ("s1_grid", ctypes.c_void_p)]
+                ("s1_grid", ctypes.c_void_p), ("s1_levels", ctypes.c_void_p)]
 
 
 class _Residual(ctypes.Structure):
@@ -197,26 +197,44 @@ def codebook_quantize4(centroids: torch.Tensor, stream=None, want_levels: bool =
 class Cache:
     """One quantized tensor (K or V): codes [B][H][cap][D/g] uint8,
     scales [B][H][cap][2] fp32 (s1, s2), shift [B][H][D] fp32 (o) and, for
-    double quantization, s1_grid [B][H][2] fp32 (lo, step of the log2 grid)."""
+    double quantization, s1_grid [B][H][2] fp32 (lo, step of the log2 grid).
+    The packed double-quantized form (Cache.empty(..., packed=True)) keeps s1
+    as 4-bit levels, s1_levels [B][H][(cap+7)/8] int32, and scales holds s2
+    alone, [B][H][cap] fp32 (sign bit set for a token with s1 = 0)."""
     codes: torch.Tensor
     scales: torch.Tensor
     shift: torch.Tensor
     s1_grid: Optional[torch.Tensor] = None
+    s1_levels: Optional[torch.Tensor] = None
 
     @property
     def cap(self) -> int:
         return int(self.codes.shape[2])
 
+    @property
+    def packed(self) -> bool:
+        return self.s1_levels is not None
+
     @classmethod
-    def empty(cls, B: int, H: int, cap: int, sub_dim: int, device="cuda", D: int = HEAD_DIM):
+    def empty(cls, B: int, H: int, cap: int, sub_dim: int, device="cuda", D: int = HEAD_DIM,
+              packed: bool = False):
+        scales = (torch.zeros(B, H, cap, dtype=torch.float32, device=device) if packed else
+                  torch.zeros(B, H, cap, 2, dtype=torch.float32, device=device))
+        levels = (torch.zeros(B, H, (cap + 7) // 8, dtype=torch.int32, device=device)
+                  if packed else None)
         return cls(torch.zeros(B, H, cap, D // sub_dim, dtype=torch.uint8, device=device),
-                   torch.zeros(B, H, cap, 2, dtype=torch.float32, device=device),
-                   torch.zeros(B, H, D, dtype=torch.float32, device=device),
-                   torch.zeros(B, H, 2, dtype=torch.float32, device=device))
+                   scales, torch.zeros(B, H, D, dtype=torch.float32, device=device),
+                   torch.zeros(B, H, 2, dtype=torch.float32, device=device), levels)
+
+    def view(self, b0: int, b1: int) -> "Cache":
+        """The sequences [b0, b1) of this cache (shared storage)."""
+        return Cache(self.codes[b0:b1], self.scales[b0:b1], self.shift[b0:b1],
+                     None if self.s1_grid is None else self.s1_grid[b0:b1],
+                     None if self.s1_levels is None else self.s1_levels[b0:b1])
 
     def _c(self) -> _Cache:
         return _Cache(_ptr(self.codes), _ptr(self.scales), _ptr(self.shift), self.cap,
-                      _ptr(self.s1_grid))
+                      _ptr(self.s1_grid), _ptr(self.s1_levels))
 
 
 def nsnq_encode_workspace(B: int, H: int, T: int, D: int = HEAD_DIM) -> int:

@@ -49,12 +49,32 @@ nsnq_status check_cache(const nsnq_cache& c, const char* name, bool need_shift) 
     if (!aligned(c.codes, 16) || !aligned(c.scales, 16) || (c.shift && !aligned(c.shift, 16)))
         return fail(NSNQ_ERR_INVALID_ARG, "%s buffers must be 16-byte aligned", name);
     if (c.cap < 0) return fail(NSNQ_ERR_INVALID_ARG, "%s.cap = %lld < 0", name, (long long)c.cap);
+    if (c.s1_levels && (!c.s1_grid || !aligned(c.s1_levels, 4) || !aligned(c.s1_grid, 8)))
+        return fail(NSNQ_ERR_INVALID_ARG,
+                    "%s: a packed cache (s1_levels) needs s1_grid; s1_levels 4-byte and s1_grid "
+                    "8-byte aligned", name);
     return NSNQ_OK;
 }
 
 }  // namespace
 
 namespace nsnq {
+int device_sm_count() {
+    static std::atomic<int> cached[64] = {};
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return 148;
+    }
+    if (dev >= 0 && dev < 64 && (n = cached[dev].load(std::memory_order_relaxed)) > 0) return n;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        return 148;
+    }
+    if (dev >= 0 && dev < 64) cached[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+
 nsnq_status set_error(nsnq_status s, const char* fmt, ...) {
     va_list ap;
     va_start(ap, fmt);
@@ -141,6 +161,10 @@ nsnq_status nsnq_encode(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t
     const bool dq = (flags & NSNQ_ENCODE_DOUBLE_QUANT) != 0;
     if (dq && (!cache.s1_grid || !aligned(cache.s1_grid, 8)))
         return fail(NSNQ_ERR_INVALID_ARG, "double quantization needs cache.s1_grid (8-byte aligned)");
+    if (cache.s1_levels && !dq)
+        return fail(NSNQ_ERR_INVALID_ARG,
+                    "a packed cache (s1_levels) holds double-quantized s1 only: pass "
+                    "NSNQ_ENCODE_DOUBLE_QUANT");
     if (B < 0 || H < 0 || T < 0)
         return fail(NSNQ_ERR_INVALID_ARG, "negative size B=%d H=%d T=%lld", B, H, (long long)T);
     if (B > 65535 || H > 65535) return fail(NSNQ_ERR_UNSUPPORTED, "B or H above 65535");
@@ -182,6 +206,7 @@ nsnq_status nsnq_encode(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t
     a.sub = cb.sub_dim;
     a.index = cb.index;
     a.codes = cache.codes; a.scales = cache.scales; a.shift = cache.shift; a.cap = cache.cap;
+    a.s1_levels = cache.s1_levels;
     char* ws = static_cast<char*>(workspace);
     a.stats = reinterpret_cast<unsigned long long*>(ws);
     a.partial = reinterpret_cast<double*>(ws + plan.partial_off);
@@ -217,6 +242,7 @@ nsnq_status nsnq_dequant(nsnq_cache cache, nsnq_codebook cb, int B, int H, int64
     if (!out || !aligned(out, 16)) return fail(NSNQ_ERR_INVALID_ARG, "out NULL or not 16-byte aligned");
     nsnq::DequantArgs a{};
     a.codes = cache.codes; a.scales = cache.scales; a.shift = cache.shift; a.cap = cache.cap;
+    a.s1_levels = cache.s1_levels; a.s1_grid = cache.s1_grid;
     a.C = cb.centroids; a.sub = cb.sub_dim;
     a.B = B; a.H = H; a.t0 = t0; a.T = T;
     a.out = out;
@@ -285,8 +311,10 @@ static nsnq_status attn_args(const void* q, nsnq_dtype q_dtype, nsnq_cache k_cac
     a.q = q; a.q_bf16 = q_dtype == NSNQ_BF16;
     a.kcodes = k_cache.codes; a.kscales = k_cache.scales; a.kshift = k_cache.shift;
     a.kcap = k_cache.cap; a.kC = k_cb.centroids; a.ksub = k_cb.sub_dim;
+    a.klevels = k_cache.s1_levels; a.kgrid = k_cache.s1_grid;
     a.vcodes = v_cache.codes; a.vscales = v_cache.scales; a.vshift = v_cache.shift;
     a.vcap = v_cache.cap; a.vC = v_cb.centroids; a.vsub = v_cb.sub_dim;
+    a.vlevels = v_cache.s1_levels; a.vgrid = v_cache.s1_grid;
     a.seq_lens = seq_lens; a.max_len = max_len;
     a.B = B; a.Hq = Hq; a.Hkv = Hkv;
     const float scale = softmax_scale == 0.f ? 1.0f / sqrtf((float)D) : softmax_scale;

@@ -18,61 +18,84 @@
 
 namespace nsnq {
 
-constexpr int kAttnWarps = 16;
-constexpr int kAttnThreads = kAttnWarps * 32;
-
-// Shared-memory map of the split kernel (bytes):
-//   lut   fp32 [256][KJ][GC]        L[c][j][h] = (H q_h)_j . C^K_c
-//   vrep  fp32 [256][VSUB/4][8] x4  V codewords, 8 interleaved copies of each
-//                                   16-byte piece, so the 8 lanes of a
-//                                   quarter-warp read 8 different bank groups
-//   qrot  fp32 [GC][128], gam fp32 [8]
-//   per warp: V codes [32][VJ] bytes, weights [32][GC padded to 4] fp32
+// Split kernel: warps of a CTA (WARPS of them) stream batches of 32 tokens.
+// Per warp and batch, K and V codes arrive in shared memory by cp.async (16-byte
+// copies issued one batch ahead: K into a single buffer, V into a double buffer),
+// scales by register prefetch. Scores take lane = token (LUT gathers in
+// lane-xor sub-vector order); values take lane = (token of 4, 16-dimension slice)
+// so that a 128-byte row of value codes and the 4 tokens' weights are one
+// shared-memory wavefront each.
 template <int GC, int KSUB, int VSUB>
-struct AttnSmem {
+struct AttnCfg {
     static constexpr int KJ = kD / KSUB, VJ = kD / VSUB;
+    static constexpr int GP = (GC + 3) / 4 * 4;  // weights per token, padded to a float4
     static constexpr size_t lut = (size_t)kNC * KJ * GC * 4;
     static constexpr size_t vrep = (size_t)kNC * (VSUB / 4) * 8 * 16;
     static constexpr size_t qrot = (size_t)GC * kD * 4 + 32;
-    static constexpr size_t wcodes = (size_t)32 * VJ;
-    static constexpr size_t wweights = (size_t)32 * ((GC + 3) / 4) * 16;
-    static constexpr size_t per_warp = wcodes + wweights;
+    static constexpr size_t kbuf = (size_t)32 * KJ;      // K codes of one batch
+    static constexpr size_t vbuf = (size_t)2 * 32 * VJ;  // V codes, two batches
+    static constexpr size_t wts = (size_t)32 * GP * 4;   // value weights of one batch
+    static constexpr size_t per_warp = kbuf + vbuf + wts;
+    static constexpr size_t fixed = lut + vrep + qrot;
+    // as many warps (<= 16) as shared memory allows
+    static constexpr int warps_fit = (int)((232448 - fixed) / per_warp);
+    static constexpr int WARPS = warps_fit >= 16 ? 16 : (warps_fit >= 12 ? 12 : 8);
     static constexpr size_t o_vrep = lut;
     static constexpr size_t o_qrot = o_vrep + vrep;
     static constexpr size_t o_warp = o_qrot + qrot;
-    static constexpr size_t bytes = o_warp + per_warp * kAttnWarps;
-    static constexpr size_t merge = (size_t)kAttnWarps * GC * (3 + kD) * 4;
+    static constexpr size_t bytes = o_warp + per_warp * WARPS;
+    static constexpr size_t merge = (size_t)WARPS * GC * (3 + kD) * 4;
     static_assert(merge <= lut, "merge area must fit in the LUT region");
     static_assert(bytes <= 232448, "shared memory per block");
 };
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+// 16-byte global -> shared copy that bypasses L1; src_bytes = 0 writes zeros.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
 
 template <typename QT>
 __device__ __forceinline__ void load_q4(const void* q, int64_t off, float (&v)[4]) {
     load4(reinterpret_cast<const QT*>(q) + off, v);
 }
 
+// A running max may lag the true max by up to 2^kLazy (log2 units) before the
+// accumulators are rescaled; weights then stay below 2^kLazy, far from the
+// fp32 range.
+constexpr float kLazy = 8.0f;
+
 template <int GC, int KSUB, int VSUB, typename QT>
-__global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a) {
-    using S = AttnSmem<GC, KSUB, VSUB>;
-    constexpr int KJ = S::KJ, VJ = S::VJ;
-    constexpr int KW = KJ / 4;  // 32-bit words per K code row
+__global__ void __launch_bounds__(AttnCfg<GC, KSUB, VSUB>::WARPS * 32, 1) attn_split_kernel(AttnArgs a) {
+    using S = AttnCfg<GC, KSUB, VSUB>;
+    constexpr int WARPS = S::WARPS, THREADS = WARPS * 32;
+    constexpr int KJ = S::KJ, VJ = S::VJ, GP = S::GP;
+    constexpr int KW = KJ / 4;          // 32-bit words per K code row
+    constexpr int SPL = 16 / VSUB;      // value sub-vectors per lane (16 dimensions)
     extern __shared__ __align__(16) uint8_t smb[];
     float* lut = reinterpret_cast<float*>(smb);
     float4* vrep = reinterpret_cast<float4*>(smb + S::o_vrep);
     float* qrot = reinterpret_cast<float*>(smb + S::o_qrot);
     float* gam = qrot + GC * kD;
-    uint8_t* warp_area = smb + S::o_warp;
 
     const int tid = threadIdx.x, lane = lane_id(), warp = tid >> 5;
     const int G = a.Hq / a.Hkv;
     const int cta = blockIdx.x;
     const int64_t L = a.plan.L;
     const int nslot = a.plan.nslot;
-    // This CTA's share of the flattened (unit, token) space; a unit is one
-    // (batch, kv-head, head group) and spans L virtual tokens.
     const int64_t vbeg = cta_begin(cta, a.plan), vend = cta_begin(cta + 1, a.plan);
 
-    for (int i = tid; i < kNC * (VSUB / 4) * 8; i += kAttnThreads)  // [piece][copy]
+    uint8_t* warp_area = smb + S::o_warp + (size_t)warp * S::per_warp;
+    uint8_t* kbuf = warp_area;                       // [32][KJ], 16-byte halves swizzled
+    uint8_t* vbuf = warp_area + S::kbuf;             // [2][32][VJ]
+    float* wts = reinterpret_cast<float*>(warp_area + S::kbuf + S::vbuf);  // [32][GP]
+
+    for (int i = tid; i < kNC * (VSUB / 4) * 8; i += THREADS)  // [piece][copy]
         vrep[i] = reinterpret_cast<const float4*>(a.vC)[i >> 3];
 
   for (int64_t u = vbeg / L; u < a.plan.units && u * L < vend; ++u) {
@@ -89,12 +112,44 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a)
     __syncthreads();  // the previous segment is done with the LUT, qrot and merge area
 
     if (ts >= te) {  // nothing to attend in this segment: neutral partial
-        for (int idx = tid; idx < GC * kPartStride; idx += kAttnThreads) {
+        for (int idx = tid; idx < GC * kPartStride; idx += THREADS) {
             const int h = idx / kPartStride, c = idx % kPartStride;
             float* P = a.part + (((int64_t)b * a.Hq + qh0 + h) * nslot + slot) * kPartStride;
             P[c] = (c == kD) ? -INFINITY : 0.f;
         }
         continue;
+    }
+
+    const uint8_t* kc = a.kcodes + bkv * a.kcap * KJ;
+    const uint8_t* vc = a.vcodes + bkv * a.vcap * VJ;
+    const float lvlK = packed_level_lane(a.klevels, a.kgrid, bkv);
+    const float lvlV = packed_level_lane(a.vlevels, a.vgrid, bkv);
+
+    // Copies of one batch's codes (lane = token): K row with its 16-byte
+    // halves swapped for lanes 4-7 of each group of 8 (conflict-free reads
+    // of whole rows), V row into the batch's buffer.
+    const uint32_t kb_s = smem_u32(kbuf), vb_s = smem_u32(vbuf);
+    auto issue_codes = [&](int64_t base, int parity) {
+        const int64_t t = base + lane;
+        const bool ok = t < te;
+        const int64_t tc = ok ? t : ts;  // any valid row (nothing is read when !ok)
+        const uint32_t nb = ok ? 16u : 0u;
+#pragma unroll
+        for (int p = 0; p < KJ / 16; ++p) {
+            const int ps = (KJ == 32) ? (p ^ ((lane >> 2) & 1)) : p;
+            cp_async16(kb_s + lane * KJ + ps * 16, kc + tc * KJ + p * 16, nb);
+        }
+#pragma unroll
+        for (int p = 0; p < VJ / 16; ++p)
+            cp_async16(vb_s + (parity * 32 + lane) * VJ + p * 16, vc + tc * VJ + p * 16, nb);
+        cp_async_commit();
+    };
+    const int64_t first = ts + warp * 32;
+    if (first < te) issue_codes(first, 0);
+    float2 k2n = make_float2(0.f, 0.f), v2n = make_float2(0.f, 0.f);
+    if (first < te) {  // warp-uniform
+        k2n = load_byproducts(a.kscales, a.klevels, bkv, a.kcap, first + lane, first + lane < te, lvlK);
+        v2n = load_byproducts(a.vscales, a.vlevels, bkv, a.vcap, first + lane, first + lane < te, lvlV);
     }
 
     // ---- segment prologue: rotated queries, q . o_K, LUT ----
@@ -113,7 +168,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a)
         // A thread keeps sub-vector j of the rotated queries in registers and
         // walks the codes c = tid / KJ + k * (threads / KJ): the codeword is
         // one broadcast read per warp and each warp stores whole LUT rows.
-        static_assert(kAttnThreads % KJ == 0, "threads must tile the sub-vectors");
+        static_assert(THREADS % KJ == 0, "threads must tile the sub-vectors");
         const int j = tid % KJ;
         float qj[GC][KSUB];
 #pragma unroll
@@ -121,7 +176,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a)
 #pragma unroll
             for (int r = 0; r < KSUB; ++r) qj[h][r] = qrot[h * kD + j * KSUB + r];
 #pragma unroll 4
-        for (int c = tid / KJ; c < kNC; c += kAttnThreads / KJ) {
+        for (int c = tid / KJ; c < kNC; c += THREADS / KJ) {
             float ck[KSUB];
 #pragma unroll
             for (int r = 0; r < KSUB; ++r) ck[r] = __ldg(a.kC + c * KSUB + r);
@@ -147,48 +202,44 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a)
 #pragma unroll
     for (int h = 0; h < GC; ++h) gm[h] = gam[h];
     float m[GC], l[GC], be[GC];
-    uint64_t acc[GC][VSUB / 2];
+    uint64_t acc[GC][8];  // dims 16 sl + (2r, 2r + 1)
 #pragma unroll
     for (int h = 0; h < GC; ++h) {
         m[h] = -INFINITY; l[h] = 0.f; be[h] = 0.f;
 #pragma unroll
-        for (int r = 0; r < VSUB / 2; ++r) acc[h][r] = 0ull;
+        for (int r = 0; r < 8; ++r) acc[h][r] = 0ull;
     }
-    const uint8_t* kc = a.kcodes + bkv * a.kcap * KJ;
-    const uint8_t* vc = a.vcodes + bkv * a.vcap * VJ;
-    const float2* ks = reinterpret_cast<const float2*>(a.kscales) + bkv * a.kcap;
-    const float2* vs = reinterpret_cast<const float2*>(a.vscales) + bkv * a.vcap;
-    uint8_t* my_codes = warp_area + (size_t)warp * S::per_warp;
-    constexpr int GP = (GC + 3) / 4 * 4;  // weights per token, padded to a float4
-    float* my_w = reinterpret_cast<float*>(my_codes + S::wcodes);  // [32][GP]
-    constexpr int TPI = 32 / VJ;  // tokens per V step (1 at VSUB=4, 2 at VSUB=8)
-    const int jj = lane % VJ, sub_t = lane / VJ;
     const int t7 = lane & 7;
+    const int grp = lane >> 3, sl = lane & 7;  // value phase: token of 4, dimension slice
+    const float4* myrep = vrep + sl;
+    int parity = 0;
 
-    for (int64_t base = ts + warp * 32; base < te; base += kAttnWarps * 32) {
+    for (int64_t base = first; base < te; base += WARPS * 32) {
         const int64_t t = base + lane;
         const bool valid = t < te;
+        const float2 k2 = k2n, v2 = v2n;
+        const int64_t nbase = base + WARPS * 32;
+        cp_async_wait_all();
+        __syncwarp();
+        // ---- this lane's K code row (from the swizzled buffer) ----
+        uint32_t kw[KW];
+        {
+            const uint4* kr = reinterpret_cast<const uint4*>(kbuf + lane * KJ);
+#pragma unroll
+            for (int p = 0; p < KJ / 16; ++p) {
+                const int ps = (KJ == 32) ? (p ^ ((lane >> 2) & 1)) : p;
+                const uint4 w4 = kr[ps];
+                kw[4 * p] = w4.x; kw[4 * p + 1] = w4.y; kw[4 * p + 2] = w4.z; kw[4 * p + 3] = w4.w;
+            }
+        }
+        __syncwarp();  // every lane has its K row: the buffer takes the next batch
+        if (nbase < te) {  // warp-uniform
+            issue_codes(nbase, parity ^ 1);
+            k2n = load_byproducts(a.kscales, a.klevels, bkv, a.kcap, nbase + lane, nbase + lane < te, lvlK);
+            v2n = load_byproducts(a.vscales, a.vlevels, bkv, a.vcap, nbase + lane, nbase + lane < te, lvlV);
+        }
         // ---- scores: lane = token; sub-vector order s ^ (lane & 7) keeps the
         //      eight lanes of a quarter-warp on eight different bank groups
-        uint32_t kw[KW];
-        float2 k2 = make_float2(0.f, 0.f), v2 = make_float2(0.f, 0.f);
-        if (valid) {
-            const uint4* kr = reinterpret_cast<const uint4*>(kc + t * KJ);
-#pragma unroll
-            for (int q4 = 0; q4 < KW / 4; ++q4) {
-                const uint4 w4 = __ldg(kr + q4);
-                kw[4 * q4] = w4.x; kw[4 * q4 + 1] = w4.y; kw[4 * q4 + 2] = w4.z; kw[4 * q4 + 3] = w4.w;
-            }
-            k2 = __ldg(ks + t);
-            v2 = __ldg(vs + t);
-            const uint4* vr = reinterpret_cast<const uint4*>(vc + t * VJ);
-            uint4* dst = reinterpret_cast<uint4*>(my_codes + lane * VJ);
-#pragma unroll
-            for (int q4 = 0; q4 < VJ / 16; ++q4) dst[q4] = __ldg(vr + q4);
-        } else {
-#pragma unroll
-            for (int i = 0; i < KW; ++i) kw[i] = 0u;
-        }
         float sc[GC];
         if constexpr (GC == 4) {
             uint64_t s01 = 0ull, s23 = 0ull;
@@ -217,101 +268,112 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_split_kernel(AttnArgs a)
                 for (int h = 0; h < GC; ++h) sc[h] += e[h];
             }
         }
-        // ---- online softmax (log2 domain) ----
+        // ---- online softmax (log2 domain), lazy rescaling of the accumulators ----
+        float wv[GP];
+#pragma unroll
+        for (int h = 0; h < GP; ++h) wv[h] = 0.f;
 #pragma unroll
         for (int h = 0; h < GC; ++h) {
             const float logit = valid ? k2.x * fmaf(k2.y, sc[h], gm[h]) * a.scale_log2 : -INFINITY;
             const float mx = warp_max(logit);
-            const float mn = fmaxf(m[h], mx);
-            const float alpha = (mn == -INFINITY) ? 1.f : exp2f(m[h] - mn);
-            const float p = valid ? exp2f(logit - mn) : 0.f;
-            l[h] = fmaf(l[h], alpha, p);
-            be[h] = fmaf(be[h], alpha, p * v2.x);
-            const uint64_t al = pk2(alpha, alpha);
+            if (mx > m[h] + kLazy) {  // warp-uniform
+                const float alpha = (m[h] == -INFINITY) ? 0.f : exp2f(m[h] - mx);
+                l[h] *= alpha;
+                be[h] *= alpha;
+                const uint64_t al = pk2(alpha, alpha);
 #pragma unroll
-            for (int r = 0; r < VSUB / 2; ++r) acc[h][r] = mul2(acc[h][r], al);
-            my_w[lane * GP + h] = p * v2.x * v2.y;
-            m[h] = mn;
-        }
-        __syncwarp();
-        // ---- values: lane = sub-vector, fp32 codewords and accumulation ----
-        const int nt = (int)min((int64_t)32, te - base);
-        const float4* myrep = vrep + (lane & 7);
-        // one token's value codewords into the head accumulators (lane = sub-vector)
-        auto vstep = [&](int tt) {
-            const int code = my_codes[tt * VJ + jj];
-            float c[VSUB];
-#pragma unroll
-            for (int k = 0; k < VSUB / 4; ++k) {
-                const float4 cv = myrep[(code * (VSUB / 4) + k) * 8];
-                c[4 * k] = cv.x; c[4 * k + 1] = cv.y; c[4 * k + 2] = cv.z; c[4 * k + 3] = cv.w;
+                for (int r = 0; r < 8; ++r) acc[h][r] = mul2(acc[h][r], al);
+                m[h] = mx;
             }
-            float wv[GP];
+            const float p = valid ? exp2f(logit - m[h]) : 0.f;
+            l[h] += p;
+            be[h] = fmaf(p, v2.x, be[h]);
+            wv[h] = p * v2.x * v2.y;
+        }
+#pragma unroll
+        for (int q4 = 0; q4 < GP / 4; ++q4)
+            reinterpret_cast<float4*>(wts + lane * GP)[q4] =
+                make_float4(wv[4 * q4], wv[4 * q4 + 1], wv[4 * q4 + 2], wv[4 * q4 + 3]);
+        __syncwarp();
+        // ---- values: lane = (token 4i + grp, dimensions 16 sl .. 16 sl + 15) ----
+        const uint8_t* vb = vbuf + (size_t)parity * 32 * VJ;
+        auto vstep = [&](int tt) {
+            uint32_t cw;
+            if constexpr (VSUB == 4) cw = *reinterpret_cast<const uint32_t*>(vb + tt * VJ + 4 * sl);
+            else cw = *reinterpret_cast<const uint16_t*>(vb + tt * VJ + 2 * sl);
+            float wt[GP];
 #pragma unroll
             for (int q4 = 0; q4 < GP / 4; ++q4) {
-                const float4 w4 = reinterpret_cast<const float4*>(my_w + tt * GP)[q4];
-                wv[4 * q4] = w4.x; wv[4 * q4 + 1] = w4.y; wv[4 * q4 + 2] = w4.z; wv[4 * q4 + 3] = w4.w;
+                const float4 w4 = reinterpret_cast<const float4*>(wts + tt * GP)[q4];
+                wt[4 * q4] = w4.x; wt[4 * q4 + 1] = w4.y; wt[4 * q4 + 2] = w4.z; wt[4 * q4 + 3] = w4.w;
             }
 #pragma unroll
-            for (int h = 0; h < GC; ++h) {
-                const uint64_t wp = pk2(wv[h], wv[h]);
+            for (int s = 0; s < SPL; ++s) {
+                const uint32_t code = (cw >> (8 * s)) & 0xffu;
 #pragma unroll
-                for (int r = 0; r < VSUB / 2; ++r)
-                    acc[h][r] = fma2(pk2(c[2 * r], c[2 * r + 1]), wp, acc[h][r]);
+                for (int k = 0; k < VSUB / 4; ++k) {
+                    const float4 cv = myrep[(code * (VSUB / 4) + k) * 8];
+                    const int r0 = (s * VSUB + 4 * k) / 2;  // packed pair index of dims 4k, 4k+1
+                    const uint64_t c01 = pk2(cv.x, cv.y), c23 = pk2(cv.z, cv.w);
+#pragma unroll
+                    for (int h = 0; h < GC; ++h) {
+                        const uint64_t wp = pk2(wt[h], wt[h]);
+                        acc[h][r0] = fma2(c01, wp, acc[h][r0]);
+                        acc[h][r0 + 1] = fma2(c23, wp, acc[h][r0 + 1]);
+                    }
+                }
             }
         };
-        if (nt == 32) {  // full batch: unrolled so that several gathers are in flight
-#pragma unroll 8
-            for (int i = 0; i < 32; i += TPI) vstep(i + sub_t);
-        } else {
-            for (int i = 0; i < nt; i += TPI)
-                if (i + sub_t < nt) vstep(i + sub_t);
-        }
+        // Tokens past the end of a partial batch carry weight 0 and zero-filled
+        // codes, so every batch runs the same eight steps.
+#pragma unroll 4
+        for (int i = 0; i < 8; ++i) vstep(4 * i + grp);
         __syncwarp();
+        parity ^= 1;
     }
 
+    // ---- warp totals: l, beta over lanes; A over the four token groups ----
 #pragma unroll
     for (int h = 0; h < GC; ++h) {
         l[h] = warp_sum(l[h]);
         be[h] = warp_sum(be[h]);
-        if constexpr (TPI == 2) {
 #pragma unroll
-            for (int r = 0; r < VSUB / 2; ++r) {
-                const float2 v = upk2(acc[h][r]);
-                acc[h][r] = pk2(v.x + __shfl_xor_sync(kFull, v.x, 16), v.y + __shfl_xor_sync(kFull, v.y, 16));
-            }
+        for (int r = 0; r < 8; ++r) {
+            float2 v = upk2(acc[h][r]);
+            v.x += __shfl_xor_sync(kFull, v.x, 8);
+            v.y += __shfl_xor_sync(kFull, v.y, 8);
+            v.x += __shfl_xor_sync(kFull, v.x, 16);
+            v.y += __shfl_xor_sync(kFull, v.y, 16);
+            acc[h][r] = pk2(v.x, v.y);
         }
     }
     __syncthreads();  // LUT no longer needed: reuse it for the CTA merge
     float* mw = lut;
-    float* lw = mw + kAttnWarps * GC;
-    float* bw = lw + kAttnWarps * GC;
-    float* Aw = bw + kAttnWarps * GC;  // [warp][h][128]
+    float* lw = mw + WARPS * GC;
+    float* bw = lw + WARPS * GC;
+    float* Aw = bw + WARPS * GC;  // [warp][h][128]
     if (lane == 0) {
 #pragma unroll
         for (int h = 0; h < GC; ++h) {
             mw[warp * GC + h] = m[h]; lw[warp * GC + h] = l[h]; bw[warp * GC + h] = be[h];
         }
     }
-    if (lane < VJ) {
+    if (grp == 0) {
 #pragma unroll
         for (int h = 0; h < GC; ++h)
 #pragma unroll
-            for (int r = 0; r < VSUB / 2; ++r) {
-                const float2 v = upk2(acc[h][r]);
-                Aw[(warp * GC + h) * kD + jj * VSUB + 2 * r] = v.x;
-                Aw[(warp * GC + h) * kD + jj * VSUB + 2 * r + 1] = v.y;
-            }
+            for (int r = 0; r < 8; ++r)
+                reinterpret_cast<float2*>(Aw + (warp * GC + h) * kD + 16 * sl)[r] = upk2(acc[h][r]);
     }
     __syncthreads();
-    for (int idx = tid; idx < GC * (kD + 2); idx += kAttnThreads) {
+    for (int idx = tid; idx < GC * (kD + 2); idx += THREADS) {
         const int h = idx / (kD + 2), c = idx % (kD + 2);
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, mw[w * GC + h]);
+        for (int w = 0; w < WARPS; ++w) M = fmaxf(M, mw[w * GC + h]);
         float accm = 0.f;
 #pragma unroll
-        for (int w = 0; w < kAttnWarps; ++w) {
+        for (int w = 0; w < WARPS; ++w) {
             const float mv = mw[w * GC + h];
             const float f = (mv == -INFINITY) ? 0.f : exp2f(mv - M);
             float v;
@@ -449,16 +511,6 @@ __global__ void __launch_bounds__(kD) attn_combine_kernel(AttnArgs a) {
 }
 
 // ---------------------------------------------------------------- host --
-static int device_sms() {
-    int dev = 0, n = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
-        cudaGetLastError();
-        return 148;
-    }
-    return n;
-}
-
 AttnPlan plan_attention(int B, int Hq, int Hkv, int64_t max_len) {
     AttnPlan p{};
     const int G = Hq / Hkv;
@@ -466,7 +518,7 @@ AttnPlan plan_attention(int B, int Hq, int Hkv, int64_t max_len) {
     p.ngroups = G / p.gc;
     p.units = (int64_t)B * Hkv * p.ngroups;
     p.L = max_len;
-    p.ctas = device_sms();  // one CTA per SM (the tables fill shared memory)
+    p.ctas = device_sm_count();  // one CTA per SM (the tables fill shared memory)
     p.nslot = (int)((p.ctas + p.units - 1) / (p.units > 0 ? p.units : 1)) + 1;
     p.total = align_up((size_t)B * Hq * p.nslot * kPartStride * sizeof(float), kWsAlign);
     return p;
@@ -474,13 +526,10 @@ AttnPlan plan_attention(int B, int Hq, int Hkv, int64_t max_len) {
 
 template <int GC, int KSUB, int VSUB, typename QT>
 static cudaError_t launch_split(const AttnArgs& a, cudaStream_t s) {
-    using S = AttnSmem<GC, KSUB, VSUB>;
-    auto kern = attn_split_kernel<GC, KSUB, VSUB, QT>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)S::bytes);
-    if (e != cudaSuccess) return e;
-    kern<<<a.plan.ctas, kAttnThreads, S::bytes, s>>>(a);
-    return cudaGetLastError();
+    using S = AttnCfg<GC, KSUB, VSUB>;
+    static std::atomic<unsigned long long> ready{0};
+    return launch_smem(attn_split_kernel<GC, KSUB, VSUB, QT>, ready, dim3(a.plan.ctas),
+                       dim3(S::WARPS * 32), S::bytes, s, a);
 }
 
 template <int GC, typename QT>

@@ -150,8 +150,8 @@ __global__ void __launch_bounds__(kRopeThreads, 1) attn_rope_split_kernel(AttnAr
     }
     const uint8_t* kc = a.kcodes + bkv * a.kcap * KJ;
     const uint8_t* vc = a.vcodes + bkv * a.vcap * VJ;
-    const float2* ks = reinterpret_cast<const float2*>(a.kscales) + bkv * a.kcap;
-    const float2* vs = reinterpret_cast<const float2*>(a.vscales) + bkv * a.vcap;
+    const float lvlK = packed_level_lane(a.klevels, a.kgrid, bkv);
+    const float lvlV = packed_level_lane(a.vlevels, a.vgrid, bkv);
 
     for (int64_t base = ts + warp * 32; base < te; base += kRopeWarps * 32) {
         const int64_t t = base + lane;
@@ -166,7 +166,8 @@ __global__ void __launch_bounds__(kRopeThreads, 1) attn_rope_split_kernel(AttnAr
             seed[i] = make_float4((float)cs, (float)sn, (float)-sn, (float)cs);
         }
         uint32_t kw[KW];
-        float2 k2 = make_float2(0.f, 0.f), v2 = make_float2(0.f, 0.f);
+        const float2 k2 = load_byproducts(a.kscales, a.klevels, bkv, a.kcap, t, valid, lvlK);
+        const float2 v2 = load_byproducts(a.vscales, a.vlevels, bkv, a.vcap, t, valid, lvlV);
         if (valid) {
             const uint4* kr = reinterpret_cast<const uint4*>(kc + t * KJ);
 #pragma unroll
@@ -174,8 +175,6 @@ __global__ void __launch_bounds__(kRopeThreads, 1) attn_rope_split_kernel(AttnAr
                 const uint4 w4 = __ldg(kr + q4);
                 kw[4 * q4] = w4.x; kw[4 * q4 + 1] = w4.y; kw[4 * q4 + 2] = w4.z; kw[4 * q4 + 3] = w4.w;
             }
-            k2 = __ldg(ks + t);
-            v2 = __ldg(vs + t);
             const uint4* vr = reinterpret_cast<const uint4*>(vc + t * VJ);
             uint4* dst = reinterpret_cast<uint4*>(my_codes + lane * VJ);
 #pragma unroll
@@ -349,11 +348,9 @@ __global__ void __launch_bounds__(kRopeThreads, 1) attn_rope_split_kernel(AttnAr
 template <int GC, int KSUB, int VSUB, typename QT>
 cudaError_t launch_rope_split(const AttnArgs& a, cudaStream_t s) {
     using S = RopeSmem<GC, KSUB, VSUB>;
-    auto kern = attn_rope_split_kernel<GC, KSUB, VSUB, QT>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::bytes);
-    if (e != cudaSuccess) return e;
-    kern<<<a.plan.ctas, kRopeThreads, S::bytes, s>>>(a);
-    return cudaGetLastError();
+    static std::atomic<unsigned long long> ready{0};
+    return launch_smem(attn_rope_split_kernel<GC, KSUB, VSUB, QT>, ready, dim3(a.plan.ctas),
+                       dim3(kRopeThreads), S::bytes, s, a);
 }
 
 template <int GC, typename QT>

@@ -25,4 +25,34 @@ __host__ __device__ inline int first_cta(int64_t v, const AttnPlan& p) {
     return c;
 }
 
+// (s1, s2) of token t of head bkv in a cache of either form. Packed form
+// (levels != NULL): s2 from scales[t] (sign bit set: s1 = 0) and s1 the
+// head's level value k, taken by shuffle from lane k of `lvl` (lanes 0..15
+// hold the 16 level values), so every lane of the warp must call this
+// together. Invalid lanes read nothing and get (0, 0).
+__device__ __forceinline__ float2 load_byproducts(const float* scales, const uint32_t* levels,
+                                                  int64_t bkv, int64_t cap, int64_t t, bool valid,
+                                                  float lvl) {
+    if (levels) {
+        float s2 = 0.f;
+        uint32_t w = 0u;
+        if (valid) {
+            s2 = __ldg(scales + bkv * cap + t);
+            w = __ldg(levels + bkv * ((cap + 7) >> 3) + (t >> 3));
+        }
+        const float s1 = __shfl_sync(0xffffffffu, lvl, (int)((w >> (4 * (int)(t & 7))) & 15u));
+        return make_float2(signbit(s2) ? 0.f : s1, fabsf(s2));
+    }
+    return valid ? __ldg(reinterpret_cast<const float2*>(scales) + bkv * cap + t)
+                 : make_float2(0.f, 0.f);
+}
+
+// Lane k < 16 of a warp: level k of head bkv's s1 grid (packed caches), else 0.
+__device__ __forceinline__ float packed_level_lane(const uint32_t* levels, const float* grid,
+                                                   int64_t bkv) {
+    const int k = threadIdx.x & 31;
+    if (!levels || k >= 16) return 0.f;
+    return (float)exp2((double)grid[2 * bkv] + (double)k * (double)grid[2 * bkv + 1]);
+}
+
 }  // namespace nsnq

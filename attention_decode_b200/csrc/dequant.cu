@@ -2,6 +2,7 @@
 // (gist.science "NSNQuant ...", Technical Summary, Methodology §1: the
 // byproducts s1, o, s2 reconstruct the tensor; §2: naive Hadamard).
 #include "common.cuh"
+#include "dq.cuh"
 #include "internal.h"
 
 namespace nsnq {
@@ -31,7 +32,14 @@ __global__ void __launch_bounds__(kDequantThreads) nsnq_dequant_kernel(DequantAr
         }
         float v[4] = {cv.x, cv.y, cv.z, cv.w};
         fwht128_lane4(v);
-        const float2 s = reinterpret_cast<const float2*>(a.scales)[row];
+        float2 s;
+        if (a.s1_levels) {  // packed: s2 alone (sign bit: s1 = 0) and the 4-bit s1 level
+            const float s2 = a.scales[row];
+            const int k = dq_packed_level(a.s1_levels, bh, a.cap, a.t0 + (i - bh * a.T));
+            s = make_float2(signbit(s2) ? 0.f : dq_level_value(a.s1_grid, bh, k), fabsf(s2));
+        } else {
+            s = reinterpret_cast<const float2*>(a.scales)[row];
+        }
         const float4 o = reinterpret_cast<const float4*>(a.shift + bh * kD)[lane];
         float4 r;
         r.x = s.x * fmaf(s.y, v[0] * kRsqrtD, o.x);

@@ -10,11 +10,46 @@
 
 namespace nsnq {
 
-__device__ __forceinline__ double dq_s1(double s1, double lo, double step) {
-    if (!(s1 > 0.0)) return 0.0;
+// The level of s1 on the grid (-1 for s1 = 0) and its value 2^(lo + k step).
+__device__ __forceinline__ double dq_s1(double s1, double lo, double step, int* level = nullptr) {
+    if (!(s1 > 0.0)) {
+        if (level) *level = -1;
+        return 0.0;
+    }
     double k = step > 0.0 ? round((log2(s1) - lo) / step) : 0.0;
     k = fmin(fmax(k, 0.0), 15.0);
+    if (level) *level = (int)k;
     return exp2(lo + k * step);
+}
+
+// Level value as every reader of a packed cache evaluates it (fp64, then fp32),
+// equal to the fp32 s1 an encoder stores for that level.
+__device__ __forceinline__ float dq_level_value(const float* s1_grid, int64_t bh, int k) {
+    return (float)exp2((double)s1_grid[2 * bh] + (double)k * (double)s1_grid[2 * bh + 1]);
+}
+
+// The 4-bit s1 level of token position pos in a packed cache's level words.
+__device__ __forceinline__ int dq_packed_level(const uint32_t* levels, int64_t bh, int64_t cap,
+                                               int64_t pos) {
+    return (int)((levels[bh * ((cap + 7) >> 3) + (pos >> 3)] >> (4 * (int)(pos & 7))) & 15u);
+}
+
+// Writes one token's byproducts: the (s1, s2) pair, or in the packed form s2
+// alone (sign bit set for a token with s1 = 0, level < 0) and the 4-bit level.
+// Two atomics keep the neighbouring tokens' nibbles of the word intact.
+__device__ __forceinline__ void store_byproducts(float* scales, uint32_t* levels, int64_t bh,
+                                                 int64_t cap, int64_t pos, float s1, float s2,
+                                                 int level) {
+    const int64_t row = bh * cap + pos;
+    if (levels) {
+        scales[row] = level < 0 ? __int_as_float(__float_as_int(s2) | (int)0x80000000) : s2;
+        uint32_t* w = levels + bh * ((cap + 7) >> 3) + (pos >> 3);
+        const int sh = 4 * (int)(pos & 7);
+        atomicAnd(w, ~(0xFu << sh));
+        atomicOr(w, (uint32_t)(level < 0 ? 0 : level) << sh);
+    } else {
+        reinterpret_cast<float2*>(scales)[row] = make_float2(s1, s2);
+    }
 }
 
 // Level tables of a grid, for deciding many tokens of one head without a

@@ -303,6 +303,7 @@ __global__ void __launch_bounds__(kTcThreads) nsn_encode1_tc_kernel(EncodeArgs a
         float s1 = sqrtf(ss * (1.0f / kD));
         float inv1 = s1 > 0.f ? 1.0f / s1 : 0.f;
         double s1dq = -1.0;
+        int s1lev = 0;
         if constexpr (DQ) {  // s1 on the head's 4-bit log2 grid, level decided in fp64
             double ss64 = 0.0;
 #pragma unroll
@@ -311,7 +312,7 @@ __global__ void __launch_bounds__(kTcThreads) nsn_encode1_tc_kernel(EncodeArgs a
             for (int m = 1; m < 16; m <<= 1) ss64 += __shfl_xor_sync(kFull, ss64, m);
             double glo, gstep;
             dq_grid(a.s1_grid, bh, glo, gstep);
-            s1dq = dq_s1(sqrt(ss64) / sqrt((double)kD), glo, gstep);
+            s1dq = dq_s1(sqrt(ss64) / sqrt((double)kD), glo, gstep, &s1lev);
             s1 = (float)s1dq;
             inv1 = s1dq > 0.0 ? (float)(1.0 / s1dq) : 0.f;
         }
@@ -466,7 +467,7 @@ __global__ void __launch_bounds__(kTcThreads) nsn_encode1_tc_kernel(EncodeArgs a
         if (valid && l16 == 0) {
             const int64_t orow = bh * a.cap + a.t_offset + t;
             reinterpret_cast<uint4*>(a.codes + orow * 16)[0] = codes;
-            reinterpret_cast<float2*>(a.scales)[orow] = make_float2(s1o, s2o);
+            store_byproducts(a.scales, a.s1_levels, bh, a.cap, a.t_offset + t, s1o, s2o, s1lev);
         }
     }
     // ---- release TMEM (after every thread's last read; after the last MMA) ----
@@ -485,18 +486,14 @@ __global__ void __launch_bounds__(kTcThreads) nsn_encode1_tc_kernel(EncodeArgs a
 
 template <typename XT, bool ADAPT, bool DQ>
 cudaError_t launch_tc(const EncodeArgs& a, cudaStream_t s) {
-    auto kern = nsn_encode1_tc_kernel<XT, ADAPT, DQ>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmem);
-    if (e != cudaSuccess) return e;
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    static std::atomic<unsigned long long> ready{0};
+    const int sms = device_sm_count();
     const int64_t npairs = (int64_t)a.B * a.H * ((a.T + 1) / 2);
     const int64_t ntiles = (npairs + 3) / 4;
     const int64_t cap = (int64_t)sms * 4;  // four CTAs per SM: all resident, 512 TMEM columns
     const int grid = (int)(ntiles < cap ? ntiles : cap);
-    kern<<<grid, kTcThreads, kTcSmem, s>>>(a);
-    return cudaGetLastError();
+    return launch_smem(nsn_encode1_tc_kernel<XT, ADAPT, DQ>, ready, dim3(grid), dim3(kTcThreads),
+                       (size_t)kTcSmem, s, a);
 }
 
 }  // namespace

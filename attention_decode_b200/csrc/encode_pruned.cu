@@ -313,6 +313,7 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
         float s1 = sqrtf(ss * (1.0f / kD));
         float inv1 = s1 > 0.f ? 1.0f / s1 : 0.f;
         double s1dq = -1.0;
+        int s1lev = 0;
         if constexpr (DQ) {
             double ss64 = 0.0;
 #pragma unroll
@@ -320,7 +321,7 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
             ss64 += __shfl_xor_sync(kFull, ss64, 1);
             double glo, gstep;
             dq_grid(a.s1_grid, bh, glo, gstep);
-            s1dq = dq_s1(sqrt(ss64) / sqrt((double)kD), glo, gstep);
+            s1dq = dq_s1(sqrt(ss64) / sqrt((double)kD), glo, gstep, &s1lev);
             s1 = (float)s1dq;
             inv1 = s1dq > 0.0 ? (float)(1.0 / s1dq) : 0.f;
         }
@@ -444,7 +445,8 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
             const int64_t row = bh * a.cap + a.t_offset + t;
             reinterpret_cast<uint4*>(a.codes + row * 32)[half] =
                 make_uint4(codes[0], codes[1], codes[2], codes[3]);
-            if (half == 0) reinterpret_cast<float2*>(a.scales)[row] = make_float2(s1o, s2o);
+            if (half == 0)
+                store_byproducts(a.scales, a.s1_levels, bh, a.cap, a.t_offset + t, s1o, s2o, s1lev);
         }
     }
 }
@@ -453,18 +455,13 @@ size_t pruned_smem_bytes() { return kSmBytes; }
 
 template <typename XT, bool ADAPT, bool DQ>
 static cudaError_t launch_pruned_t(const EncodeArgs& a, cudaStream_t s) {
-    auto kern = nsn_encode_pruned_kernel<XT, ADAPT, DQ>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmBytes);
-    if (e != cudaSuccess) return e;
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    static std::atomic<unsigned long long> ready{0};
+    const int sms = device_sm_count();
     const int64_t ntiles = (int64_t)a.B * a.H * ((a.T + kWarpTile - 1) / kWarpTile);
     const int64_t ctas = (ntiles + kWarps - 1) / kWarps;
     const int grid = (int)(ctas < sms ? ctas : sms);
-    kern<<<grid, kPrunedThreads, kSmBytes, s>>>(a);
-    return cudaGetLastError();
+    return launch_smem(nsn_encode_pruned_kernel<XT, ADAPT, DQ>, ready, dim3(grid),
+                       dim3(kPrunedThreads), kSmBytes, s, a);
 }
 
 cudaError_t launch_encode_pruned(const EncodeArgs& a, cudaStream_t s) {

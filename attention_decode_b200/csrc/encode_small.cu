@@ -54,10 +54,11 @@ __global__ void __launch_bounds__(kSmallThreads) nsn_encode_small_kernel(EncodeA
     const double sqrt_d = sqrt((double)kD);
     const double ss = warp_sum_d(x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3]);
     double s1 = sqrt(ss) / sqrt_d;
+    int s1lev = 0;
     if constexpr (DQ) {
         double glo, gstep;
         dq_grid(a.s1_grid, bh, glo, gstep);
-        s1 = dq_s1(s1, glo, gstep);
+        s1 = dq_s1(s1, glo, gstep, &s1lev);
     }
     const double inv1 = s1 > 0.0 ? 1.0 / s1 : 0.0;
     double z[4], ss2 = 0.0, yy = 0.0, oo = 0.0;
@@ -178,7 +179,7 @@ __global__ void __launch_bounds__(kSmallThreads) nsn_encode_small_kernel(EncodeA
     }
     const int64_t orow = bh * a.cap + a.t_offset + t;
     if (G == 4 || lane < 16) a.codes[orow * (kD / G) + j] = (uint8_t)bi;
-    if (lane == 0) reinterpret_cast<float2*>(a.scales)[orow] = make_float2(s1o, s2o);
+    if (lane == 0) store_byproducts(a.scales, a.s1_levels, bh, a.cap, a.t_offset + t, s1o, s2o, s1lev);
 }
 
 template <typename XT, int G>

@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/nsnq.h"
 
 namespace nsnq {
@@ -18,6 +20,43 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Record a printf-style message as the calling thread's nsnq_last_error().
 nsnq_status set_error(nsnq_status s, const char* fmt, ...);
+
+// ---------------------------------------------------- launch set-up cache --
+// Multiprocessor count of the current device, queried once per device.
+int device_sm_count();
+
+// The dynamic shared-memory limit of one kernel, set once per device (one
+// bit per device in `ready`). A device reset drops the attribute; a launch
+// that then fails with cudaErrorInvalidValue is retried once by launch_smem.
+template <typename K>
+cudaError_t ensure_smem(K kern, int bytes, std::atomic<unsigned long long>& ready, bool force) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = (dev >= 0 && dev < 64) ? 1ull << dev : 0ull;
+    if (!force && bit && (ready.load(std::memory_order_relaxed) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && bit) ready.fetch_or(bit, std::memory_order_relaxed);
+    return e;
+}
+
+// Launch kern<<<grid, block, smem, s>>>(args...) with its shared-memory limit
+// set (once per device).
+template <typename... P, typename... A>
+cudaError_t launch_smem(void (*kern)(P...), std::atomic<unsigned long long>& ready, dim3 grid,
+                        dim3 block, size_t smem, cudaStream_t s, A&&... args) {
+    cudaError_t e = ensure_smem(kern, (int)smem, ready, false);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, block, smem, s>>>(args...);
+    e = cudaGetLastError();
+    if (e == cudaErrorInvalidValue) {  // attribute lost (device reset): set it again, once
+        e = ensure_smem(kern, (int)smem, ready, true);
+        if (e != cudaSuccess) return e;
+        kern<<<grid, block, smem, s>>>(args...);
+        e = cudaGetLastError();
+    }
+    return e;
+}
 
 // ------------------------------------------------------------------ encode --
 struct EncodeArgs {
@@ -38,6 +77,7 @@ struct EncodeArgs {
     float* scales;
     float* shift;
     int64_t cap;
+    uint32_t* s1_levels;  // packed double-quantized form: 4-bit s1 levels, scales = s2 only
     // workspace views
     unsigned long long* stats;  // [8]
     double* partial;            // [B][H][nchunk1][128]
@@ -75,6 +115,8 @@ struct DequantArgs {
     const float* scales;
     const float* shift;
     int64_t cap;
+    const uint32_t* s1_levels;  // packed form (scales = s2 only), or NULL
+    const float* s1_grid;
     const float* C;
     int sub;
     int B, H;
@@ -107,12 +149,16 @@ struct AttnArgs {
     int64_t kcap;
     const float* kC;
     int ksub;
+    const uint32_t* klevels;  // packed double-quantized K cache (scales = s2 only), or NULL
+    const float* kgrid;
     const uint8_t* vcodes;
     const float* vscales;
     const float* vshift;
     int64_t vcap;
     const float* vC;
     int vsub;
+    const uint32_t* vlevels;  // packed double-quantized V cache, or NULL
+    const float* vgrid;
     const int32_t* seq_lens;
     int64_t max_len;
     int B, Hq, Hkv;

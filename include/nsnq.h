@@ -34,6 +34,13 @@
  *      codes  uint8 [B][H][cap][D/sub_dim], sub-vector j ascending
  *      scales fp32  [B][H][cap][2] = (s1, s2)
  *      shift  fp32  [B][H][D]      = o
+ *    or, for double-quantized byproducts stored packed (s1_levels != NULL):
+ *      scales    fp32   [B][H][cap]         = s2 (sign bit set: s1 = 0)
+ *      s1_levels uint32 [B][H][(cap+7)/8]   4-bit s1 level of token t in
+ *                                           bits 4(t%8)..4(t%8)+3 of word t/8
+ *      s1_grid   fp32   [B][H][2]           = (lo, step): level k means
+ *                                           s1 = 2^(lo + k step), evaluated in
+ *                                           fp64 and rounded to fp32
  */
 #ifndef NSNQ_H_
 #define NSNQ_H_
@@ -75,9 +82,10 @@ typedef enum {
      * the largest log2 s1 of the tokens encoded in shift-compute mode, kept
      * in cache.s1_grid for later shift-given appends), and a computed o takes
      * one of 16 uniform levels between its least and largest channel value.
-     * The level values are stored in the usual fp32 fields (the 4-bit level
-     * indices follow from them), so dequant and attention need no change.
-     * Requires cache.s1_grid. */
+     * With cache.s1_levels == NULL the level values go to the usual fp32
+     * fields; with cache.s1_levels set, s1 is stored as its 4-bit level and
+     * scales holds s2 alone (the packed form, see nsnq_cache). o stays an
+     * fp32 vector per head (its 16 level values). Requires cache.s1_grid. */
     NSNQ_ENCODE_DOUBLE_QUANT = 2
 } nsnq_encode_flags;
 
@@ -97,6 +105,15 @@ typedef struct {
     int64_t cap;      /* token capacity per (batch, head) */
     float* s1_grid;   /* device, [B][H][2] = (lo, step) of the double-quantized s1 grid
                          (log2 domain), or NULL without double quantization */
+    uint32_t* s1_levels; /* device, [B][H][(cap+7)/8], or NULL. Non-NULL selects the packed
+                         double-quantized form (Methodology §3, Double Quantization: s1
+                         takes 4 bits): s1 is kept only as its 4-bit level on the head's
+                         grid (s1_grid, required), and scales holds s2 alone,
+                         [B][H][cap] fp32; a token with s1 = 0 (an all-zero token) has
+                         level 0 and the sign bit of its stored s2 set. Per token-head this
+                         stores 4.5 bytes of byproducts instead of 8. Only encode calls
+                         with NSNQ_ENCODE_DOUBLE_QUANT may write a packed cache; dequant
+                         and the attention calls read either form. 4-byte aligned. */
 } nsnq_cache;
 
 /* Human-readable name of a status code (static string). */

@@ -207,6 +207,27 @@ def test_residual_write_validation(lib):
     assert f(T=0) == nsnq.NSNQ_OK
 
 
+def test_codebook_quantize4_validation(lib):
+    q = lib.nsnq_codebook_quantize4
+    assert q(FAKE, FAKE, None, None, 128, 4, None) == nsnq.NSNQ_ERR_UNSUPPORTED
+    assert q(FAKE, FAKE, None, None, 256, 5, None) == nsnq.NSNQ_ERR_UNSUPPORTED
+    assert q(None, FAKE, None, None, 256, 4, None) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert q(FAKE, None, None, None, 256, 8, None) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert q(FAKE + 2, FAKE, None, None, 256, 8, None) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert q(FAKE, FAKE, None, FAKE + 4, 256, 8, None) == nsnq.NSNQ_ERR_INVALID_ARG
+
+
+def test_packed_cache_validation(lib):
+    packed = nsnq._Cache(FAKE, FAKE, FAKE, 100, FAKE, FAKE)
+    no_grid = nsnq._Cache(FAKE, FAKE, FAKE, 100, None, FAKE)
+    # a packed cache takes double-quantized s1 only, and needs its grid
+    assert _encode(lib, cache=packed, flags=0) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert _encode(lib, cache=no_grid, flags=2) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert _encode(lib, cache=nsnq._Cache(FAKE, FAKE, FAKE, 100, FAKE, FAKE + 2),
+                   flags=2) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert lib.nsnq_dequant(no_grid, _cb(), 1, 1, 0, 10, 128, FAKE, None) == nsnq.NSNQ_ERR_INVALID_ARG
+
+
 def test_binding_has_no_fallback(tmp_path):
     """The binding raises when the library file is absent; it never computes on the CPU."""
     import importlib
@@ -216,13 +237,3 @@ def test_binding_has_no_fallback(tmp_path):
         mod.load(str(tmp_path / "missing.so"))
     mod._lib = None
     mod.load()
-
-
-def test_codebook_quantize4_validation(lib):
-    q = lib.nsnq_codebook_quantize4
-    assert q(FAKE, FAKE, None, None, 128, 4, None) == nsnq.NSNQ_ERR_UNSUPPORTED
-    assert q(FAKE, FAKE, None, None, 256, 5, None) == nsnq.NSNQ_ERR_UNSUPPORTED
-    assert q(None, FAKE, None, None, 256, 4, None) == nsnq.NSNQ_ERR_INVALID_ARG
-    assert q(FAKE, None, None, None, 256, 8, None) == nsnq.NSNQ_ERR_INVALID_ARG
-    assert q(FAKE + 2, FAKE, None, None, 256, 8, None) == nsnq.NSNQ_ERR_INVALID_ARG
-    assert q(FAKE, FAKE, None, FAKE + 4, 256, 8, None) == nsnq.NSNQ_ERR_INVALID_ARG

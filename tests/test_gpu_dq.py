@@ -140,3 +140,103 @@ def test_codebook_quantize4_matches_oracle(codebooks, g):
     # a constant codebook keeps its value (step 0)
     flat = torch.full((256, g), 0.75, device="cuda")
     assert torch.equal(nsnq.codebook_quantize4(flat), flat)
+
+
+# ------------------------------------------------------------- packed form --
+def unpack(cache):
+    """(s1, s2, level, zero) of a packed cache, read back independently of the
+    library: level k of token t sits in bits 4(t%8).. of word t/8, s1 =
+    2^(lo + k step) evaluated in fp64 and rounded to fp32, and a set sign bit
+    of the stored s2 marks a token with s1 = 0."""
+    lev = cache.s1_levels.cpu().numpy().view(np.uint32)
+    B, H, W = lev.shape
+    nib = (lev[..., None] >> (4 * np.arange(8, dtype=np.uint32))) & np.uint32(15)
+    k = nib.reshape(B, H, W * 8)[:, :, :cache.cap].astype(np.float64)
+    grid = cache.s1_grid.cpu().numpy().astype(np.float64)
+    raw = cache.scales.cpu().numpy()
+    zero = np.signbit(raw)
+    s1 = (2.0 ** (grid[..., 0:1] + k * grid[..., 1:2])).astype(np.float32)
+    return np.where(zero, np.float32(0), s1), np.abs(raw), k, zero
+
+
+@pytest.mark.parametrize("sub,dtype", [(4, "bf16"), (8, "bf16"), (4, "f32")])
+def test_packed_double_quant_encode(codebooks, sub, dtype):
+    """Packed double-quantized caches (4-bit s1 levels, s2 alone): the same
+    codes, grid and shift as the unpacked form, s1 and s2 that unpack to the
+    unpacked cache's values bit for bit, levels equal to the oracle's, and
+    byte-sharing appends (one token at a time at odd positions) that leave
+    their neighbours' levels intact. All-zero tokens (s1 = 0) included."""
+    B, H, T, extra = 2, 2, 501, 5  # odd lengths: partial level words
+    w = _w(B, H, T + extra, dtype, sub)
+    io = S.to_io(S.keys(w), dtype)
+    io[:, :, [3, 17, T + 1]] = 0  # zero tokens in the prompt and among the appends
+    x64 = S.io_to_f64(io, dtype)
+    C = codebooks[sub]
+    cb = P.codebook(C)
+    x = P.to_dev(io, dtype)
+    caches = {}
+    for packed in (True, False):
+        c = nsnq.Cache.empty(B, H, T + extra, sub, packed=packed)
+        nsnq.nsnq_encode(x[:, :, :T], cb, c, flags=DQ)
+        for i in range(extra):
+            nsnq.nsnq_encode(x[:, :, T + i:T + i + 1], cb, c, t_offset=T + i,
+                             shift_mode=nsnq.SHIFT_GIVEN, flags=DQ)
+        caches[packed] = c
+    torch.cuda.synchronize()
+    pk, pl = caches[True], caches[False]
+    assert torch.equal(pk.codes, pl.codes)
+    assert torch.equal(pk.shift, pl.shift) and torch.equal(pk.s1_grid, pl.s1_grid)
+    s1, s2, k, zero = unpack(pk)
+    ref = pl.scales.cpu().numpy()
+    assert np.array_equal(s1, ref[..., 0]) and np.array_equal(s2, ref[..., 1])
+    assert zero[:, :, [3, 17, T + 1]].all() and zero.sum() == 3 * B * H
+    ora = O.encode(x64[:, :, :T], C, want_w=True, double_quant=True)
+    lo, step = pl.s1_grid.cpu().numpy().astype(np.float64)[..., 0], \
+        pl.s1_grid.cpu().numpy().astype(np.float64)[..., 1]
+    with np.errstate(divide="ignore"):
+        k_ora = np.clip(np.round((np.log2(ora["s1"]) - lo[..., None]) / step[..., None]), 0, 15)
+    nz = ora["s1"] > 0
+    assert np.array_equal(k[:, :, :T][nz], k_ora[nz])
+    P.check_scales(np.stack([s1[:, :, :T], s2[:, :, :T]], -1), ora)
+
+
+@pytest.mark.parametrize("sub", [4, 8])
+def test_packed_caches_through_dequant_and_attention(codebooks, sub):
+    """Dequant, decode attention and attention over keys before RoPE read a
+    packed cache exactly as the unpacked one (same values, bit for bit), and
+    agree with the oracle's attention over the unpacked byproducts."""
+    B, H, Hq, T = 2, 2, 8, 640
+    w = S.Workload("dqp", B=B, Hkv=H, Hq=Hq, T=T, d=D, sub_dim=sub, dtype="bf16",
+                   kdist=S.K_MODERATE, seed=29)
+    C = codebooks[sub]
+    cb = P.codebook(C)
+    k_io, v_io = S.to_io(S.keys(w), "bf16"), S.to_io(S.values(w), "bf16")
+    k_io[0, 1, 100] = 0
+    c = {}
+    for packed in (True, False):
+        kc = nsnq.Cache.empty(B, H, T, sub, packed=packed)
+        vc = nsnq.Cache.empty(B, H, T, sub, packed=packed)
+        nsnq.nsnq_encode(P.to_dev(k_io, "bf16"), cb, kc, flags=DQ)
+        nsnq.nsnq_encode(P.to_dev(v_io, "bf16"), cb, vc, flags=DQ)
+        c[packed] = (kc, vc)
+    q = P.to_dev(S.to_io(S.queries(w), "bf16"), "bf16")
+    lens = torch.tensor([T, 333], dtype=torch.int32, device="cuda")
+    outs = {}
+    for packed in (True, False):
+        kc, vc = c[packed]
+        outs[packed] = (
+            nsnq.nsnq_dequant(kc, cb, B, H, 0, T),
+            nsnq.nsnq_attn_decode(q, kc, vc, cb, cb, lens, T, Hkv=H, out_dtype=torch.float32),
+            nsnq.nsnq_attn_decode_rope(q, kc, vc, cb, cb, lens, T, Hkv=H,
+                                       out_dtype=torch.float32))
+    torch.cuda.synchronize()
+    for a, b in zip(outs[True], outs[False]):
+        assert torch.equal(a, b)
+    kc, vc = c[False]
+    Kh = O.dequant(kc.codes.cpu().numpy(), kc.scales[..., 0].cpu().numpy(),
+                   kc.scales[..., 1].cpu().numpy(), kc.shift.cpu().numpy(), C)
+    Vh = O.dequant(vc.codes.cpu().numpy(), vc.scales[..., 0].cpu().numpy(),
+                   vc.scales[..., 1].cpu().numpy(), vc.shift.cpu().numpy(), C)
+    ref = O.attention(S.io_to_f64(S.to_io(S.queries(w), "bf16"), "bf16"), Kh, Vh, [T, 333])
+    e, _ = P.attn_errors(P.out_to_np(outs[True][1]), ref, False)
+    assert (e <= 1.0).all(), e.max()
