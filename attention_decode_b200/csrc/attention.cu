@@ -28,13 +28,12 @@ namespace nsnq {
 template <int GC, int KSUB, int VSUB>
 struct AttnCfg {
     static constexpr int KJ = kD / KSUB, VJ = kD / VSUB;
-    static constexpr int GP = (GC + 3) / 4 * 4;  // weights per token, padded to a float4
     static constexpr size_t lut = (size_t)kNC * KJ * GC * 4;
     static constexpr size_t vrep = (size_t)kNC * (VSUB / 4) * 8 * 16;
     static constexpr size_t qrot = (size_t)GC * kD * 4 + 32;
     static constexpr size_t kbuf = (size_t)32 * KJ;      // K codes of one batch
     static constexpr size_t vbuf = (size_t)2 * 32 * VJ;  // V codes, two batches
-    static constexpr size_t wts = (size_t)32 * GP * 4;   // value weights of one batch
+    static constexpr size_t wts = (size_t)32 * GC * 8;   // value weights (w, w) of one batch
     static constexpr size_t per_warp = kbuf + vbuf + wts;
     static constexpr size_t fixed = lut + vrep + qrot;
     // as many warps (<= 16) as shared memory allows
@@ -74,7 +73,7 @@ template <int GC, int KSUB, int VSUB, typename QT>
 __global__ void __launch_bounds__(AttnCfg<GC, KSUB, VSUB>::WARPS * 32, 1) attn_split_kernel(AttnArgs a) {
     using S = AttnCfg<GC, KSUB, VSUB>;
     constexpr int WARPS = S::WARPS, THREADS = WARPS * 32;
-    constexpr int KJ = S::KJ, VJ = S::VJ, GP = S::GP;
+    constexpr int KJ = S::KJ, VJ = S::VJ;
     constexpr int KW = KJ / 4;          // 32-bit words per K code row
     constexpr int SPL = 16 / VSUB;      // value sub-vectors per lane (16 dimensions)
     extern __shared__ __align__(16) uint8_t smb[];
@@ -93,7 +92,7 @@ __global__ void __launch_bounds__(AttnCfg<GC, KSUB, VSUB>::WARPS * 32, 1) attn_s
     uint8_t* warp_area = smb + S::o_warp + (size_t)warp * S::per_warp;
     uint8_t* kbuf = warp_area;                       // [32][KJ], 16-byte halves swizzled
     uint8_t* vbuf = warp_area + S::kbuf;             // [2][32][VJ]
-    float* wts = reinterpret_cast<float*>(warp_area + S::kbuf + S::vbuf);  // [32][GP]
+    uint64_t* wts = reinterpret_cast<uint64_t*>(warp_area + S::kbuf + S::vbuf);  // [32][GC] (w, w)
 
     for (int i = tid; i < kNC * (VSUB / 4) * 8; i += THREADS)  // [piece][copy]
         vrep[i] = reinterpret_cast<const float4*>(a.vC)[i >> 3];
@@ -169,17 +168,21 @@ __global__ void __launch_bounds__(AttnCfg<GC, KSUB, VSUB>::WARPS * 32, 1) attn_s
         // walks the codes c = tid / KJ + k * (threads / KJ): the codeword is
         // one broadcast read per warp and each warp stores whole LUT rows.
         static_assert(THREADS % KJ == 0, "threads must tile the sub-vectors");
+        // The softmax scale (log2 domain) is folded into the table and gamma.
         const int j = tid % KJ;
         float qj[GC][KSUB];
 #pragma unroll
         for (int h = 0; h < GC; ++h)
 #pragma unroll
-            for (int r = 0; r < KSUB; ++r) qj[h][r] = qrot[h * kD + j * KSUB + r];
+            for (int r = 0; r < KSUB; ++r) qj[h][r] = qrot[h * kD + j * KSUB + r] * a.scale_log2;
 #pragma unroll 4
         for (int c = tid / KJ; c < kNC; c += THREADS / KJ) {
             float ck[KSUB];
 #pragma unroll
-            for (int r = 0; r < KSUB; ++r) ck[r] = __ldg(a.kC + c * KSUB + r);
+            for (int k = 0; k < KSUB / 4; ++k) {
+                const float4 c4 = __ldg(reinterpret_cast<const float4*>(a.kC) + c * (KSUB / 4) + k);
+                ck[4 * k] = c4.x; ck[4 * k + 1] = c4.y; ck[4 * k + 2] = c4.z; ck[4 * k + 3] = c4.w;
+            }
             float sum[GC];
 #pragma unroll
             for (int h = 0; h < GC; ++h) {
@@ -200,7 +203,7 @@ __global__ void __launch_bounds__(AttnCfg<GC, KSUB, VSUB>::WARPS * 32, 1) attn_s
 
     float gm[GC];
 #pragma unroll
-    for (int h = 0; h < GC; ++h) gm[h] = gam[h];
+    for (int h = 0; h < GC; ++h) gm[h] = gam[h] * a.scale_log2;
     float m[GC], l[GC], be[GC];
     uint64_t acc[GC][8];  // dims 16 sl + (2r, 2r + 1)
 #pragma unroll
@@ -213,6 +216,11 @@ __global__ void __launch_bounds__(AttnCfg<GC, KSUB, VSUB>::WARPS * 32, 1) attn_s
     const int grp = lane >> 3, sl = lane & 7;  // value phase: token of 4, dimension slice
     const float4* myrep = vrep + sl;
     int parity = 0;
+    // Score gathers visit sub-vector j = s ^ t7 at step s: its code is byte
+    // (s ^ t7) & 3 of word (s ^ t7) >> 2 of the row. With the row's words
+    // swapped in pairs for t7 >= 4 (kwp), the word index is s >> 2 for every
+    // lane and the byte selector is (s & 3) ^ (t7 & 3).
+    const uint32_t t3 = (uint32_t)(t7 & 3);
 
     for (int64_t base = first; base < te; base += WARPS * 32) {
         const int64_t t = base + lane;
@@ -240,16 +248,17 @@ __global__ void __launch_bounds__(AttnCfg<GC, KSUB, VSUB>::WARPS * 32, 1) attn_s
         }
         // ---- scores: lane = token; sub-vector order s ^ (lane & 7) keeps the
         //      eight lanes of a quarter-warp on eight different bank groups
+        uint32_t kwp[KW];
+#pragma unroll
+        for (int i = 0; i < KW; ++i) kwp[i] = (t7 & 4) ? kw[i ^ 1] : kw[i];
         float sc[GC];
         if constexpr (GC == 4) {
             uint64_t s01 = 0ull, s23 = 0ull;
             const float4* lut4 = reinterpret_cast<const float4*>(lut);
 #pragma unroll
             for (int s = 0; s < KJ; ++s) {
-                const int j = s ^ t7;
-                const uint32_t word = (t7 & 4) ? kw[(s >> 2) ^ 1] : kw[s >> 2];
-                const uint32_t code = __byte_perm(word, 0u, 0x4440u | (uint32_t)((s ^ t7) & 3));
-                const float4 e = lut4[code * KJ + j];
+                const uint32_t code = __byte_perm(kwp[s >> 2], 0u, (0x4440u | (uint32_t)(s & 3)) ^ t3);
+                const float4 e = lut4[(int)code * KJ + (s ^ t7)];
                 s01 = add2(s01, pk2(e.x, e.y));
                 s23 = add2(s23, pk2(e.z, e.w));
             }
@@ -260,23 +269,21 @@ __global__ void __launch_bounds__(AttnCfg<GC, KSUB, VSUB>::WARPS * 32, 1) attn_s
             for (int h = 0; h < GC; ++h) sc[h] = 0.f;
 #pragma unroll
             for (int s = 0; s < KJ; ++s) {
-                const int j = s ^ t7;
-                const uint32_t word = (t7 & 4) ? kw[(s >> 2) ^ 1] : kw[s >> 2];
-                const uint32_t code = __byte_perm(word, 0u, 0x4440u | (uint32_t)((s ^ t7) & 3));
-                const float* e = lut + ((size_t)code * KJ + j) * GC;
+                const uint32_t code = __byte_perm(kwp[s >> 2], 0u, (0x4440u | (uint32_t)(s & 3)) ^ t3);
+                const float* e = lut + ((int)code * KJ + (s ^ t7)) * GC;
 #pragma unroll
                 for (int h = 0; h < GC; ++h) sc[h] += e[h];
             }
         }
-        // ---- online softmax (log2 domain), lazy rescaling of the accumulators ----
-        float wv[GP];
-#pragma unroll
-        for (int h = 0; h < GP; ++h) wv[h] = 0.f;
+        // ---- online softmax (log2 domain). The running max m is raised only
+        //      when a logit exceeds it by more than kLazy (a warp vote); then
+        //      the accumulators are rescaled. Weights stay below 2^kLazy.
+        const float vw = v2.x * v2.y;
 #pragma unroll
         for (int h = 0; h < GC; ++h) {
-            const float logit = valid ? k2.x * fmaf(k2.y, sc[h], gm[h]) * a.scale_log2 : -INFINITY;
-            const float mx = warp_max(logit);
-            if (mx > m[h] + kLazy) {  // warp-uniform
+            const float logit = valid ? k2.x * fmaf(k2.y, sc[h], gm[h]) : -INFINITY;
+            if (__any_sync(kFull, logit > m[h] + kLazy)) {  // warp-uniform, rare
+                const float mx = warp_max(logit);
                 const float alpha = (m[h] == -INFINITY) ? 0.f : exp2f(m[h] - mx);
                 l[h] *= alpha;
                 be[h] *= alpha;
@@ -288,24 +295,29 @@ __global__ void __launch_bounds__(AttnCfg<GC, KSUB, VSUB>::WARPS * 32, 1) attn_s
             const float p = valid ? exp2f(logit - m[h]) : 0.f;
             l[h] += p;
             be[h] = fmaf(p, v2.x, be[h]);
-            wv[h] = p * v2.x * v2.y;
+            const float w = p * vw;
+            wts[lane * GC + h] = pk2(w, w);
         }
-#pragma unroll
-        for (int q4 = 0; q4 < GP / 4; ++q4)
-            reinterpret_cast<float4*>(wts + lane * GP)[q4] =
-                make_float4(wv[4 * q4], wv[4 * q4 + 1], wv[4 * q4 + 2], wv[4 * q4 + 3]);
         __syncwarp();
         // ---- values: lane = (token 4i + grp, dimensions 16 sl .. 16 sl + 15) ----
         const uint8_t* vb = vbuf + (size_t)parity * 32 * VJ;
-        auto vstep = [&](int tt) {
-            uint32_t cw;
-            if constexpr (VSUB == 4) cw = *reinterpret_cast<const uint32_t*>(vb + tt * VJ + 4 * sl);
-            else cw = *reinterpret_cast<const uint16_t*>(vb + tt * VJ + 2 * sl);
-            float wt[GP];
+        uint32_t cws[8];
 #pragma unroll
-            for (int q4 = 0; q4 < GP / 4; ++q4) {
-                const float4 w4 = reinterpret_cast<const float4*>(wts + tt * GP)[q4];
-                wt[4 * q4] = w4.x; wt[4 * q4 + 1] = w4.y; wt[4 * q4 + 2] = w4.z; wt[4 * q4 + 3] = w4.w;
+        for (int i = 0; i < 8; ++i) {
+            const int tt = 4 * i + grp;
+            if constexpr (VSUB == 4) cws[i] = *reinterpret_cast<const uint32_t*>(vb + tt * VJ + 4 * sl);
+            else cws[i] = *reinterpret_cast<const uint16_t*>(vb + tt * VJ + 2 * sl);
+        }
+        auto vstep = [&](int tt, uint32_t cw) {
+            uint64_t wp[GC];
+            if constexpr (GC % 2 == 0) {
+#pragma unroll
+                for (int h2 = 0; h2 < GC / 2; ++h2) {
+                    const ulonglong2 w2 = reinterpret_cast<const ulonglong2*>(wts + tt * GC)[h2];
+                    wp[2 * h2] = w2.x; wp[2 * h2 + 1] = w2.y;
+                }
+            } else {
+                wp[0] = wts[tt];
             }
 #pragma unroll
             for (int s = 0; s < SPL; ++s) {
@@ -317,17 +329,16 @@ __global__ void __launch_bounds__(AttnCfg<GC, KSUB, VSUB>::WARPS * 32, 1) attn_s
                     const uint64_t c01 = pk2(cv.x, cv.y), c23 = pk2(cv.z, cv.w);
 #pragma unroll
                     for (int h = 0; h < GC; ++h) {
-                        const uint64_t wp = pk2(wt[h], wt[h]);
-                        acc[h][r0] = fma2(c01, wp, acc[h][r0]);
-                        acc[h][r0 + 1] = fma2(c23, wp, acc[h][r0 + 1]);
+                        acc[h][r0] = fma2(c01, wp[h], acc[h][r0]);
+                        acc[h][r0 + 1] = fma2(c23, wp[h], acc[h][r0 + 1]);
                     }
                 }
             }
         };
         // Tokens past the end of a partial batch carry weight 0 and zero-filled
         // codes, so every batch runs the same eight steps.
-#pragma unroll 4
-        for (int i = 0; i < 8; ++i) vstep(4 * i + grp);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) vstep(4 * i + grp, cws[i]);
         __syncwarp();
         parity ^= 1;
     }
@@ -511,6 +522,10 @@ __global__ void __launch_bounds__(kD) attn_combine_kernel(AttnArgs a) {
 }
 
 // ---------------------------------------------------------------- host --
+// A CTA pays a fixed cost per segment it attends to (rotated queries, table
+// build, the CTA merge), counted here in streamed tokens.
+constexpr int64_t kSegmentFixedTokens = 1000;
+
 AttnPlan plan_attention(int B, int Hq, int Hkv, int64_t max_len) {
     AttnPlan p{};
     const int G = Hq / Hkv;
@@ -518,7 +533,26 @@ AttnPlan plan_attention(int B, int Hq, int Hkv, int64_t max_len) {
     p.ngroups = G / p.gc;
     p.units = (int64_t)B * Hkv * p.ngroups;
     p.L = max_len;
-    p.ctas = device_sm_count();  // one CTA per SM (the tables fill shared memory)
+    const int sms = device_sm_count();  // one CTA per SM (the tables fill shared memory)
+    p.ctas = sms;
+    // Two ways to cut the (unit, token) space: the balanced split gives every
+    // CTA the same number of tokens, but a CTA whose share crosses a unit
+    // boundary attends to two segments; the unit-aligned split gives each unit
+    // nsplit CTAs of one segment each (padding each unit to nsplit equal parts,
+    // a multiple of 32 tokens), at the price of idle SMs when units * nsplit <
+    // SMs. The cheaper one by the fixed-cost model is taken.
+    if (p.units > 0 && p.units <= sms && max_len > 0) {
+        const int64_t nsplit = sms / p.units;
+        const int64_t seg = (max_len + nsplit - 1) / nsplit;
+        const int64_t seg32 = (seg + 31) / 32 * 32;
+        const int64_t per_cta = (p.units * max_len + sms - 1) / sms;
+        const int64_t balanced = per_cta + (per_cta < max_len ? 2 : 1) * kSegmentFixedTokens;
+        const int64_t aligned = seg32 + kSegmentFixedTokens;
+        if (aligned < balanced) {
+            p.L = nsplit * seg32;
+            p.ctas = (int)(p.units * nsplit);
+        }
+    }
     p.nslot = (int)((p.ctas + p.units - 1) / (p.units > 0 ? p.units : 1)) + 1;
     p.total = align_up((size_t)B * Hq * p.nslot * kPartStride * sizeof(float), kWsAlign);
     return p;
