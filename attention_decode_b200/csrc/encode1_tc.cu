@@ -33,6 +33,21 @@ constexpr int kRows = 128;       // sub-vectors per tile (8 token-heads)
 constexpr int kCols = 128;       // TMEM accumulator columns (one per codeword of a half)
 constexpr float kTieRelTc = 1e-4f;
 constexpr float kTieAbsTc = 1e-6f;
+// Bound on the scoring error of one score s = |C|^2 - 2 w . C, relative to
+// |C|^2 + 2 |w| |C| (the sum of the absolute values of its terms):
+//  - each tf32 x tf32 product is exact in fp32 (11 + 11 significant bits);
+//  - dropping A_lo B_lo and the residuals of the two-term splits of w and
+//    -2C leaves at most 3.001 * 2^-22 of each |w_k| |2 C_k| term;
+//  - |C|^2 is an fp32 chain of 8 fused multiply-adds (8 * 2^-24 relative)
+//    split into two tf32 parts (2^-22 left over);
+//  - the tensor core adds 26 terms (3 split MMAs of K = 8 plus the two |C|^2
+//    parts); with every addition rounding or truncating to fp32 (relative
+//    error <= 2^-23) the sum is off by at most 25 * 2^-23 of the terms'
+//    absolute sum.
+// Together: |s_computed - s| <= 3.71e-6 (|C|^2 + 2 |w| |C|). The near-tie band
+// of a sub-vector is at least the sum of this bound for its best codeword and
+// for the largest codeword (the second best is not tracked by index).
+constexpr float kScoreErrTc = 3.71e-6f;
 constexpr float kCancelTc = 1e-3f;
 constexpr long long kWaitLimit = 1ll << 24;  // spins on the MMA barrier before giving up
 
@@ -264,6 +279,9 @@ __global__ void __launch_bounds__(kTcThreads) nsn_encode1_tc_kernel(EncodeArgs a
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
     const uint32_t tmem = *tmem_slot;
+    float cmax2 = 0.f;  // largest |C|^2 (for the near-tie band)
+    for (int n = 0; n < kNC; ++n) cmax2 = fmaxf(cmax2, n2s[n]);
+    const float cmax = sqrtf(cmax2) * (1.f + 1e-6f);
     const uint64_t dAhi = mat_desc(sbase + kOffAhi, kRows * 16, 128);
     const uint64_t dAlo = mat_desc(sbase + kOffAlo, kRows * 16, 128);
     const uint64_t dAone = mat_desc(sbase + kOffAone, kRows * 16, 128);
@@ -374,8 +392,17 @@ __global__ void __launch_bounds__(kTcThreads) nsn_encode1_tc_kernel(EncodeArgs a
         __syncthreads();  // A written; the previous tile's TMEM reads are done
         // ---- the two halves of the codebook, one MMA round each; best and
         //      second best of this row's scores read back from TMEM ----
-        float b1 = INFINITY, b2 = INFINITY;
-        int i1 = 0;
+        // Scan of the row's 256 scores by groups of 8: the group minimum (no
+        // index), the least and second-least group minimum, and a copy of the
+        // best group's 8 scores. The best score, its index (lowest on ties)
+        // and the second-best score come out exactly as from a full scan: the
+        // second best is the better of the best group's second and the second
+        // group minimum.
+        float gm1 = INFINITY, gm2 = INFINITY;
+        float gs[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) gs[k] = INFINITY;
+        int gcol = 0;
         const uint32_t taddr = tmem + ((uint32_t)(32 * warp) << 16);
 #pragma unroll 1
         for (int hf = 0; hf < 2; ++hf) {
@@ -410,16 +437,34 @@ __global__ void __launch_bounds__(kTcThreads) nsn_encode1_tc_kernel(EncodeArgs a
                 uint32_t r[32];
                 tmem_ld32(taddr + (uint32_t)c0, r);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float s = __uint_as_float(r[j]);
-                    b2 = fminf(b2, fmaxf(b1, s));
-                    i1 = s < b1 ? hf * kCols + c0 + j : i1;
-                    b1 = fminf(b1, s);
+                for (int g = 0; g < 4; ++g) {
+                    float q[8];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) q[k] = __uint_as_float(r[8 * g + k]);
+                    const float m = fminf(fminf(fminf(q[0], q[1]), fminf(q[2], q[3])),
+                                          fminf(fminf(q[4], q[5]), fminf(q[6], q[7])));
+                    const bool better = m < gm1;  // strict: the earlier group keeps ties
+                    gm2 = fminf(gm2, fmaxf(gm1, m));
+                    gm1 = fminf(gm1, m);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) gs[k] = better ? q[k] : gs[k];
+                    gcol = better ? hf * kCols + c0 + 8 * g : gcol;
                 }
             }
         }
         if (failed) break;
-        bool tie = cancel || (b2 - b1) <= fmaf(kTieRelTc, ww + b1, kTieAbsTc);
+        const float b1 = gm1;
+        int k1 = 7;
+#pragma unroll
+        for (int k = 6; k >= 0; --k) k1 = gs[k] == b1 ? k : k1;
+        float bin = INFINITY;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) bin = k == k1 ? bin : fminf(bin, gs[k]);
+        const float b2 = fminf(bin, gm2);
+        const int i1 = gcol + k1;
+        const float wn = sqrtf(ww), c1 = sqrtf(n2s[i1]);
+        const float band_s = kScoreErrTc * (n2s[i1] + cmax * cmax + 2.f * wn * (c1 + cmax));
+        bool tie = cancel || (b2 - b1) <= fmaxf(fmaf(kTieRelTc, ww + b1, kTieAbsTc), band_s);
         if (!valid) tie = false;
         float wq = 0.f;
         if constexpr (ADAPT) wq = half_sum(0.5f * (n2s[i1] - b1));  // w . C[best] = (|C|^2 - s) / 2
