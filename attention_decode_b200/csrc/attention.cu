@@ -145,10 +145,10 @@ __global__ void __launch_bounds__(AttnCfg<GC, KSUB, VSUB>::WARPS * 32, 1) attn_s
     };
     const int64_t first = ts + warp * 32;
     if (first < te) issue_codes(first, 0);
-    float2 k2n = make_float2(0.f, 0.f), v2n = make_float2(0.f, 0.f);
+    RawByproducts k2n{0.f, 0u}, v2n{0.f, 0u};  // next batch's byproducts, still raw
     if (first < te) {  // warp-uniform
-        k2n = load_byproducts(a.kscales, a.klevels, bkv, a.kcap, first + lane, first + lane < te, lvlK);
-        v2n = load_byproducts(a.vscales, a.vlevels, bkv, a.vcap, first + lane, first + lane < te, lvlV);
+        k2n = fetch_byproducts(a.kscales, a.klevels, bkv, a.kcap, first + lane, first + lane < te);
+        v2n = fetch_byproducts(a.vscales, a.vlevels, bkv, a.vcap, first + lane, first + lane < te);
     }
 
     // ---- segment prologue: rotated queries, q . o_K, LUT ----
@@ -225,7 +225,7 @@ __global__ void __launch_bounds__(AttnCfg<GC, KSUB, VSUB>::WARPS * 32, 1) attn_s
     for (int64_t base = first; base < te; base += WARPS * 32) {
         const int64_t t = base + lane;
         const bool valid = t < te;
-        const float2 k2 = k2n, v2 = v2n;
+        const RawByproducts k2r = k2n, v2r = v2n;  // resolved where first needed (softmax)
         const int64_t nbase = base + WARPS * 32;
         cp_async_wait_all();
         __syncwarp();
@@ -243,8 +243,8 @@ __global__ void __launch_bounds__(AttnCfg<GC, KSUB, VSUB>::WARPS * 32, 1) attn_s
         __syncwarp();  // every lane has its K row: the buffer takes the next batch
         if (nbase < te) {  // warp-uniform
             issue_codes(nbase, parity ^ 1);
-            k2n = load_byproducts(a.kscales, a.klevels, bkv, a.kcap, nbase + lane, nbase + lane < te, lvlK);
-            v2n = load_byproducts(a.vscales, a.vlevels, bkv, a.vcap, nbase + lane, nbase + lane < te, lvlV);
+            k2n = fetch_byproducts(a.kscales, a.klevels, bkv, a.kcap, nbase + lane, nbase + lane < te);
+            v2n = fetch_byproducts(a.vscales, a.vlevels, bkv, a.vcap, nbase + lane, nbase + lane < te);
         }
         // ---- scores: lane = token; sub-vector order s ^ (lane & 7) keeps the
         //      eight lanes of a quarter-warp on eight different bank groups
@@ -278,6 +278,8 @@ __global__ void __launch_bounds__(AttnCfg<GC, KSUB, VSUB>::WARPS * 32, 1) attn_s
         // ---- online softmax (log2 domain). The running max m is raised only
         //      when a logit exceeds it by more than kLazy (a warp vote); then
         //      the accumulators are rescaled. Weights stay below 2^kLazy.
+        const float2 k2 = resolve_byproducts(k2r, a.klevels, t, lvlK);
+        const float2 v2 = resolve_byproducts(v2r, a.vlevels, t, lvlV);
         const float vw = v2.x * v2.y;
 #pragma unroll
         for (int h = 0; h < GC; ++h) {

@@ -306,6 +306,7 @@ def run_cuda(args):
 
     # ---- decode attention alone at the 32k workload ----
     attention = run_attention_bench(args, nsnq, dev, world, barrier, hbm, peak_kind)
+    attention_variants = run_attention_variants(args, nsnq, dev, world, barrier, hbm)
     encode_1bit = run_encode1_bench(args, nsnq, dev, world, barrier, hbm, peak_kind, k)
     long_context = run_long_context_bench(args, nsnq, dev, world, barrier, hbm)
     serving = run_serving_bench(args, nsnq, dev, world, barrier, hbm)
@@ -323,7 +324,8 @@ def run_cuda(args):
         "stages_ms": {"encode_per_tensor": round(enc_avg_ms, 4),
                       "attention_4k": round(sum(att_small_ms) / len(att_small_ms), 4)},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
-        "roofline": roofline, "attention": attention, "encode_1bit": encode_1bit,
+        "roofline": roofline, "attention": attention, "attention_variants": attention_variants,
+        "encode_1bit": encode_1bit,
         "long_context": long_context, "serving": serving, "e2e": e2e,
         "clocks": clk.summary(),
     }
@@ -413,6 +415,71 @@ def run_attention_bench(args, nsnq, dev, world, barrier, hbm, peak_kind):
                          "traffic": measured_traffic("nsnq_attn_decode")},
             "l2": "flushed before every call (cache 335 MB > L2 anyway)",
             "keys_before_rope": rope}
+
+
+def _encoded_caches(nsnq, w, cb, dev, sub, packed, flags, seed):
+    """K/V caches of the workload's shape and distributions, encoded on the
+    device one sequence at a time (packed: double-quantized 4-bit s1 levels)."""
+    import torch
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+    B, H, T = w.B, w.Hkv, w.T
+    kc = nsnq.Cache.empty(B, H, T, sub, device=dev, packed=packed)
+    vc = nsnq.Cache.empty(B, H, T, sub, device=dev, packed=packed)
+    for b in range(B):
+        for which, c in (("k", kc), ("v", vc)):
+            nsnq.nsnq_encode(_device_kv(w, gen, dev, 1, T, which), cb, c.view(b, b + 1), flags=flags)
+    return kc, vc
+
+
+def run_attention_variants(args, nsnq, dev, world, barrier, hbm):
+    """Decode attention at 16 x 32k over 1-bit caches, and over packed
+    double-quantized caches (4-bit s1 levels, s2 alone, 4-bit codebook) at 1
+    and 2 bit: 41 and 73 bytes per token instead of 48 and 80."""
+    import torch
+    w = S.WORKLOADS[ATTN_WORKLOAD]
+    B, H, Hq, T = w.B, w.Hkv, w.Hq, w.T
+    q = torch.randn(B, Hq, 128, generator=torch.Generator(device=dev).manual_seed(99), device=dev)
+    q = q.to(torch.bfloat16)
+    seq = torch.full((B,), T, dtype=torch.int32, device=dev)
+    out = torch.empty(B, Hq, 128, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(nsnq.nsnq_attn_workspace(B, Hq, H, T), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    res = {}
+    for name, sub, packed in (("1bit", 8, False), ("dq_packed_1bit", 8, True),
+                              ("dq_packed_2bit", 4, True)):
+        C = torch.from_numpy(load_codebook(sub)).to(dev)
+        if packed:
+            C = nsnq.codebook_quantize4(C)
+        cb = nsnq.Codebook(C)
+        flags = nsnq.ENCODE_DOUBLE_QUANT if packed else 0
+        kc, vc = _encoded_caches(nsnq, w, cb, dev, sub, packed, flags, 4242 + sub)
+        run = lambda: nsnq.nsnq_attn_decode(q, kc, vc, cb, cb, seq, T, Hkv=H, out=out,
+                                             workspace=ws)
+        for _ in range(args.warmup):
+            run()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        barrier()
+        torch.cuda.synchronize()
+        for e0, e1 in evs:
+            flush.zero_()
+            e0.record(stream)
+            run()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        avg = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / len(evs), world, dev)
+        per_tok = 2 * (128 // sub) + (9 if packed else 16)
+        nbytes = B * H * T * per_tok
+        gbs = nbytes / (avg / 1e3) / 1e9
+        res[name] = {"ms_per_call": round(avg, 4), "bytes_per_token": per_tok,
+                     "gbs": round(gbs * world, 1), "frac": round(gbs / hbm, 4)}
+        del kc, vc
+    res["dq_bytes_saved_per_token_head"] = 3.5
+    res["workload"] = "decode-16x32k (B 16, Hq 32, Hkv 8, T 32768), caches encoded on the device"
+    return res
 
 
 def run_encode1_bench(args, nsnq, dev, world, barrier, hbm, peak_kind, x):
