@@ -171,11 +171,20 @@ class Codebook:
             self.index = idx
         return self
 
+    def __setattr__(self, name, value):
+        object.__setattr__(self, name, value)
+        if name != "_cstruct":
+            object.__setattr__(self, "_cstruct", None)  # the C view no longer matches
+
     def _c(self) -> _Codebook:
-        if self.sub_dim == 4 and self.index is None and self.centroids.is_cuda:
-            self.prepare()
-        return _Codebook(_ptr(self.centroids), int(self.centroids.shape[0]), self.sub_dim,
-                         _ptr(self.index))
+        c = getattr(self, "_cstruct", None)
+        if c is None:
+            if self.sub_dim == 4 and self.index is None and self.centroids.is_cuda:
+                self.prepare()
+            c = _Codebook(_ptr(self.centroids), int(self.centroids.shape[0]), self.sub_dim,
+                          _ptr(self.index))
+            object.__setattr__(self, "_cstruct", c)
+        return c
 
 
 def codebook_quantize4(centroids: torch.Tensor, stream=None, want_levels: bool = False):
@@ -232,9 +241,20 @@ class Cache:
                      None if self.s1_grid is None else self.s1_grid[b0:b1],
                      None if self.s1_levels is None else self.s1_levels[b0:b1])
 
+    def __setattr__(self, name, value):
+        object.__setattr__(self, name, value)
+        if name != "_cstruct":
+            object.__setattr__(self, "_cstruct", None)  # the C view no longer matches
+
     def _c(self) -> _Cache:
-        return _Cache(_ptr(self.codes), _ptr(self.scales), _ptr(self.shift), self.cap,
-                      _ptr(self.s1_grid), _ptr(self.s1_levels))
+        # The C view is built once per set of tensors (in-place updates keep
+        # their storage): a decode loop calls the library many times per second.
+        c = getattr(self, "_cstruct", None)
+        if c is None:
+            c = _Cache(_ptr(self.codes), _ptr(self.scales), _ptr(self.shift), self.cap,
+                       _ptr(self.s1_grid), _ptr(self.s1_levels))
+            object.__setattr__(self, "_cstruct", c)
+        return c
 
 
 def nsnq_encode_workspace(B: int, H: int, T: int, D: int = HEAD_DIM) -> int:
@@ -258,9 +278,8 @@ def nsnq_encode(x: torch.Tensor, cb: Codebook, cache: Cache, t_offset: int = 0,
     B, H, T, D = x.shape
     if x.stride(3) != 1:
         raise ValueError("x must have contiguous channels")
-    need = nsnq_encode_workspace(B, H, T, D)
-    if workspace is None:
-        workspace = _workspace(need, x.device)
+    if workspace is None:  # (a given workspace is checked by the library)
+        workspace = _workspace(nsnq_encode_workspace(B, H, T, D), x.device)
     _check(load().nsnq_encode(_ptr(x), _dtype_code(x), B, H, T, D, x.stride(0), x.stride(1),
                               x.stride(2), t_offset, shift_mode, flags, cb._c(), cache._c(),
                               _ptr(workspace), workspace.numel() * workspace.element_size(),

@@ -11,8 +11,9 @@
 //   D  = A_hi B_hi + A_lo B_hi + A_hi B_lo + 1 (|C|^2_hi + |C|^2_lo)
 // with x_hi = tf32(x), x_lo = tf32(x - x_hi) (three-term split, about fp32
 // accuracy) and B = -2C. Each thread then reads its own row of D (its own
-// sub-vector, TMEM lane = row) with tcgen05.ld and keeps the best and
-// second-best score. Near ties (gap within 1e-4 d1 + 1e-6) and tokens with a
+// sub-vector, TMEM lane = row) with tcgen05.ld and finds the best and
+// second-best score by groups of 8. Near ties (gap within the near-tie band,
+// at least the derived scoring-error bound kScoreErrTc) and tokens with a
 // cancelling shift are re-decided in fp64 by the whole warp.
 //
 // Shared-memory operands use the no-swizzle K-major layout: a row's 8 tf32
