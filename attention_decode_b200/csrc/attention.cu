@@ -69,6 +69,14 @@ __device__ __forceinline__ void load_q4(const void* q, int64_t off, float (&v)[4
 // fp32 range.
 constexpr float kLazy = 8.0f;
 
+// 2^x by the hardware approximation (relative error ~2^-22; results below
+// 2^-126 flush to zero, weights far below the softmax's resolution).
+__device__ __forceinline__ float exp2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 template <int GC, int KSUB, int VSUB, typename QT>
 __global__ void __launch_bounds__(AttnCfg<GC, KSUB, VSUB>::WARPS * 32, 1) attn_split_kernel(AttnArgs a) {
     using S = AttnCfg<GC, KSUB, VSUB>;
@@ -123,32 +131,39 @@ __global__ void __launch_bounds__(AttnCfg<GC, KSUB, VSUB>::WARPS * 32, 1) attn_s
     const uint8_t* vc = a.vcodes + bkv * a.vcap * VJ;
     const float lvlK = packed_level_lane(a.klevels, a.kgrid, bkv);
     const float lvlV = packed_level_lane(a.vlevels, a.vgrid, bkv);
+    const ByproductSrc ksrc = byproduct_src(a.kscales, a.klevels, bkv, a.kcap);
+    const ByproductSrc vsrc = byproduct_src(a.vscales, a.vlevels, bkv, a.vcap);
+    // Token indices of the loop are 32-bit: lengths are int32, and a batch
+    // start stays below te + 32 * WARPS < 2^32.
+    const uint32_t ts32 = (uint32_t)ts, te32 = (uint32_t)te;
 
     // Copies of one batch's codes (lane = token): K row with its 16-byte
     // halves swapped for lanes 4-7 of each group of 8 (conflict-free reads
     // of whole rows), V row into the batch's buffer.
     const uint32_t kb_s = smem_u32(kbuf), vb_s = smem_u32(vbuf);
-    auto issue_codes = [&](int64_t base, int parity) {
-        const int64_t t = base + lane;
-        const bool ok = t < te;
-        const int64_t tc = ok ? t : ts;  // any valid row (nothing is read when !ok)
+    const uint32_t kdst = kb_s + lane * KJ, vdst = vb_s + lane * VJ;
+    auto issue_codes = [&](uint32_t base, int parity) {
+        const uint32_t t = base + lane;
+        const bool ok = t < te32;
+        const uint32_t tc = ok ? t : ts32;  // any valid row (nothing is read when !ok)
         const uint32_t nb = ok ? 16u : 0u;
+        const uint8_t* ks = kc + (size_t)tc * KJ;
+        const uint8_t* vs = vc + (size_t)tc * VJ;
 #pragma unroll
         for (int p = 0; p < KJ / 16; ++p) {
             const int ps = (KJ == 32) ? (p ^ ((lane >> 2) & 1)) : p;
-            cp_async16(kb_s + lane * KJ + ps * 16, kc + tc * KJ + p * 16, nb);
+            cp_async16(kdst + ps * 16, ks + p * 16, nb);
         }
 #pragma unroll
-        for (int p = 0; p < VJ / 16; ++p)
-            cp_async16(vb_s + (parity * 32 + lane) * VJ + p * 16, vc + tc * VJ + p * 16, nb);
+        for (int p = 0; p < VJ / 16; ++p) cp_async16(vdst + parity * 32 * VJ + p * 16, vs + p * 16, nb);
         cp_async_commit();
     };
-    const int64_t first = ts + warp * 32;
-    if (first < te) issue_codes(first, 0);
+    const uint32_t first = ts32 + warp * 32;
+    if (first < te32) issue_codes(first, 0);
     RawByproducts k2n{0.f, 0u}, v2n{0.f, 0u};  // next batch's byproducts, still raw
-    if (first < te) {  // warp-uniform
-        k2n = fetch_byproducts(a.kscales, a.klevels, bkv, a.kcap, first + lane, first + lane < te);
-        v2n = fetch_byproducts(a.vscales, a.vlevels, bkv, a.vcap, first + lane, first + lane < te);
+    if (first < te32) {  // warp-uniform
+        k2n = fetch_byproducts(ksrc, first + lane, first + lane < te32);
+        v2n = fetch_byproducts(vsrc, first + lane, first + lane < te32);
     }
 
     // ---- segment prologue: rotated queries, q . o_K, LUT ----
@@ -214,7 +229,8 @@ __global__ void __launch_bounds__(AttnCfg<GC, KSUB, VSUB>::WARPS * 32, 1) attn_s
     }
     const int t7 = lane & 7;
     const int grp = lane >> 3, sl = lane & 7;  // value phase: token of 4, dimension slice
-    const float4* myrep = vrep + sl;
+    // codeword (c0, c1, c2, c3) read as two packed pairs (c0, c1), (c2, c3)
+    const ulonglong2* myrep = reinterpret_cast<const ulonglong2*>(vrep) + sl;
     int parity = 0;
     // Score gathers visit sub-vector j = s ^ t7 at step s: its code is byte
     // (s ^ t7) & 3 of word (s ^ t7) >> 2 of the row. With the row's words
@@ -222,11 +238,11 @@ __global__ void __launch_bounds__(AttnCfg<GC, KSUB, VSUB>::WARPS * 32, 1) attn_s
     // lane and the byte selector is (s & 3) ^ (t7 & 3).
     const uint32_t t3 = (uint32_t)(t7 & 3);
 
-    for (int64_t base = first; base < te; base += WARPS * 32) {
-        const int64_t t = base + lane;
-        const bool valid = t < te;
+    for (uint32_t base = first; base < te32; base += WARPS * 32) {
+        const uint32_t t = base + lane;
+        const bool valid = t < te32;
         const RawByproducts k2r = k2n, v2r = v2n;  // resolved where first needed (softmax)
-        const int64_t nbase = base + WARPS * 32;
+        const uint32_t nbase = base + WARPS * 32;
         cp_async_wait_all();
         __syncwarp();
         // ---- this lane's K code row (from the swizzled buffer) ----
@@ -241,10 +257,10 @@ __global__ void __launch_bounds__(AttnCfg<GC, KSUB, VSUB>::WARPS * 32, 1) attn_s
             }
         }
         __syncwarp();  // every lane has its K row: the buffer takes the next batch
-        if (nbase < te) {  // warp-uniform
+        if (nbase < te32) {  // warp-uniform
             issue_codes(nbase, parity ^ 1);
-            k2n = fetch_byproducts(a.kscales, a.klevels, bkv, a.kcap, nbase + lane, nbase + lane < te);
-            v2n = fetch_byproducts(a.vscales, a.vlevels, bkv, a.vcap, nbase + lane, nbase + lane < te);
+            k2n = fetch_byproducts(ksrc, nbase + lane, nbase + lane < te32);
+            v2n = fetch_byproducts(vsrc, nbase + lane, nbase + lane < te32);
         }
         // ---- scores: lane = token; sub-vector order s ^ (lane & 7) keeps the
         //      eight lanes of a quarter-warp on eight different bank groups
@@ -254,13 +270,14 @@ __global__ void __launch_bounds__(AttnCfg<GC, KSUB, VSUB>::WARPS * 32, 1) attn_s
         float sc[GC];
         if constexpr (GC == 4) {
             uint64_t s01 = 0ull, s23 = 0ull;
-            const float4* lut4 = reinterpret_cast<const float4*>(lut);
+            // a table row is read as two packed pairs: heads (0, 1) and (2, 3)
+            const ulonglong2* lut2 = reinterpret_cast<const ulonglong2*>(lut);
 #pragma unroll
             for (int s = 0; s < KJ; ++s) {
                 const uint32_t code = __byte_perm(kwp[s >> 2], 0u, (0x4440u | (uint32_t)(s & 3)) ^ t3);
-                const float4 e = lut4[(int)code * KJ + (s ^ t7)];
-                s01 = add2(s01, pk2(e.x, e.y));
-                s23 = add2(s23, pk2(e.z, e.w));
+                const ulonglong2 e = lut2[(int)code * KJ + (s ^ t7)];
+                s01 = add2(s01, e.x);
+                s23 = add2(s23, e.y);
             }
             const float2 a01 = upk2(s01), a23 = upk2(s23);
             sc[0] = a01.x; sc[1] = a01.y; sc[2] = a23.x; sc[3] = a23.y;
@@ -278,15 +295,15 @@ __global__ void __launch_bounds__(AttnCfg<GC, KSUB, VSUB>::WARPS * 32, 1) attn_s
         // ---- online softmax (log2 domain). The running max m is raised only
         //      when a logit exceeds it by more than kLazy (a warp vote); then
         //      the accumulators are rescaled. Weights stay below 2^kLazy.
-        const float2 k2 = resolve_byproducts(k2r, a.klevels, t, lvlK);
-        const float2 v2 = resolve_byproducts(v2r, a.vlevels, t, lvlV);
+        const float2 k2 = resolve_byproducts(k2r, ksrc, t, lvlK);
+        const float2 v2 = resolve_byproducts(v2r, vsrc, t, lvlV);
         const float vw = v2.x * v2.y;
 #pragma unroll
         for (int h = 0; h < GC; ++h) {
             const float logit = valid ? k2.x * fmaf(k2.y, sc[h], gm[h]) : -INFINITY;
             if (__any_sync(kFull, logit > m[h] + kLazy)) {  // warp-uniform, rare
                 const float mx = warp_max(logit);
-                const float alpha = (m[h] == -INFINITY) ? 0.f : exp2f(m[h] - mx);
+                const float alpha = (m[h] == -INFINITY) ? 0.f : exp2_approx(m[h] - mx);
                 l[h] *= alpha;
                 be[h] *= alpha;
                 const uint64_t al = pk2(alpha, alpha);
@@ -294,7 +311,7 @@ __global__ void __launch_bounds__(AttnCfg<GC, KSUB, VSUB>::WARPS * 32, 1) attn_s
                 for (int r = 0; r < 8; ++r) acc[h][r] = mul2(acc[h][r], al);
                 m[h] = mx;
             }
-            const float p = valid ? exp2f(logit - m[h]) : 0.f;
+            const float p = valid ? exp2_approx(logit - m[h]) : 0.f;
             l[h] += p;
             be[h] = fmaf(p, v2.x, be[h]);
             const float w = p * vw;
@@ -326,9 +343,9 @@ __global__ void __launch_bounds__(AttnCfg<GC, KSUB, VSUB>::WARPS * 32, 1) attn_s
                 const uint32_t code = (cw >> (8 * s)) & 0xffu;
 #pragma unroll
                 for (int k = 0; k < VSUB / 4; ++k) {
-                    const float4 cv = myrep[(code * (VSUB / 4) + k) * 8];
+                    const ulonglong2 cv = myrep[(code * (VSUB / 4) + k) * 8];
                     const int r0 = (s * VSUB + 4 * k) / 2;  // packed pair index of dims 4k, 4k+1
-                    const uint64_t c01 = pk2(cv.x, cv.y), c23 = pk2(cv.z, cv.w);
+                    const uint64_t c01 = cv.x, c23 = cv.y;
 #pragma unroll
                     for (int h = 0; h < GC; ++h) {
                         acc[h][r0] = fma2(c01, wp[h], acc[h][r0]);

@@ -152,6 +152,8 @@ __global__ void __launch_bounds__(kRopeThreads, 1) attn_rope_split_kernel(AttnAr
     const uint8_t* vc = a.vcodes + bkv * a.vcap * VJ;
     const float lvlK = packed_level_lane(a.klevels, a.kgrid, bkv);
     const float lvlV = packed_level_lane(a.vlevels, a.vgrid, bkv);
+    const ByproductSrc ksrc = byproduct_src(a.kscales, a.klevels, bkv, a.kcap);
+    const ByproductSrc vsrc = byproduct_src(a.vscales, a.vlevels, bkv, a.vcap);
 
     for (int64_t base = ts + warp * 32; base < te; base += kRopeWarps * 32) {
         const int64_t t = base + lane;
@@ -166,8 +168,8 @@ __global__ void __launch_bounds__(kRopeThreads, 1) attn_rope_split_kernel(AttnAr
             seed[i] = make_float4((float)cs, (float)sn, (float)-sn, (float)cs);
         }
         uint32_t kw[KW];
-        const float2 k2 = load_byproducts(a.kscales, a.klevels, bkv, a.kcap, t, valid, lvlK);
-        const float2 v2 = load_byproducts(a.vscales, a.vlevels, bkv, a.vcap, t, valid, lvlV);
+        const float2 k2 = load_byproducts(ksrc, (uint32_t)t, valid, lvlK);
+        const float2 v2 = load_byproducts(vsrc, (uint32_t)t, valid, lvlV);
         if (valid) {
             const uint4* kr = reinterpret_cast<const uint4*>(kc + t * KJ);
 #pragma unroll

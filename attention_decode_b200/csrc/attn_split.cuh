@@ -25,45 +25,60 @@ __host__ __device__ inline int first_cta(int64_t v, const AttnPlan& p) {
     return c;
 }
 
-// (s1, s2) of token t of head bkv in a cache of either form, in two steps so
+// (s1, s2) of token t of one head in a cache of either form, in two steps so
 // that a prefetch does not wait for its loads: fetch_byproducts issues the
 // loads (packed form: s2 from scales[t], sign bit set for s1 = 0, and the
 // word holding t's 4-bit level; otherwise the (s1, s2) pair), and
 // resolve_byproducts, called when the values are needed, turns the level
 // into s1 by a shuffle from lane k of `lvl` (lanes 0..15 hold the 16 level
 // values), so every lane of the warp must call it together. Invalid lanes
-// load nothing and get (0, 0).
+// load nothing and get (0, 0). Token indices are 32-bit (sequence lengths
+// are int32); the head's rows are addressed from ByproductSrc.
 struct RawByproducts {
     float a;     // s2 (packed) or s1
     uint32_t b;  // level word (packed) or the bits of s2
 };
-__device__ __forceinline__ RawByproducts fetch_byproducts(const float* scales,
-                                                          const uint32_t* levels, int64_t bkv,
-                                                          int64_t cap, int64_t t, bool valid) {
+struct ByproductSrc {
+    const float* s;       // head's scales: s2 per token (packed) or (s1, s2) pairs
+    const uint32_t* lv;   // head's level words (packed), else nullptr
+};
+__device__ __forceinline__ ByproductSrc byproduct_src(const float* scales, const uint32_t* levels,
+                                                      int64_t bkv, int64_t cap) {
+    ByproductSrc r;
+    if (levels) {
+        r.s = scales + bkv * cap;
+        r.lv = levels + bkv * ((cap + 7) >> 3);
+    } else {
+        r.s = scales + 2 * bkv * cap;
+        r.lv = nullptr;
+    }
+    return r;
+}
+__device__ __forceinline__ RawByproducts fetch_byproducts(const ByproductSrc& src, uint32_t t,
+                                                          bool valid) {
     RawByproducts r{0.f, 0u};
     if (!valid) return r;
-    if (levels) {
-        r.a = __ldg(scales + bkv * cap + t);
-        r.b = __ldg(levels + bkv * ((cap + 7) >> 3) + (t >> 3));
+    if (src.lv) {
+        r.a = __ldg(src.s + t);
+        r.b = __ldg(src.lv + (t >> 3));
     } else {
-        const float2 v = __ldg(reinterpret_cast<const float2*>(scales) + bkv * cap + t);
+        const float2 v = __ldg(reinterpret_cast<const float2*>(src.s) + t);
         r.a = v.x;
         r.b = __float_as_uint(v.y);
     }
     return r;
 }
-__device__ __forceinline__ float2 resolve_byproducts(RawByproducts r, const uint32_t* levels,
-                                                     int64_t t, float lvl) {
-    if (levels) {
-        const float s1 = __shfl_sync(0xffffffffu, lvl, (int)((r.b >> (4 * (int)(t & 7))) & 15u));
+__device__ __forceinline__ float2 resolve_byproducts(RawByproducts r, const ByproductSrc& src,
+                                                     uint32_t t, float lvl) {
+    if (src.lv) {
+        const float s1 = __shfl_sync(0xffffffffu, lvl, (int)((r.b >> (4 * (t & 7u))) & 15u));
         return make_float2(signbit(r.a) ? 0.f : s1, fabsf(r.a));
     }
     return make_float2(r.a, __uint_as_float(r.b));
 }
-__device__ __forceinline__ float2 load_byproducts(const float* scales, const uint32_t* levels,
-                                                  int64_t bkv, int64_t cap, int64_t t, bool valid,
+__device__ __forceinline__ float2 load_byproducts(const ByproductSrc& src, uint32_t t, bool valid,
                                                   float lvl) {
-    return resolve_byproducts(fetch_byproducts(scales, levels, bkv, cap, t, valid), levels, t, lvl);
+    return resolve_byproducts(fetch_byproducts(src, t, valid), src, t, lvl);
 }
 
 // Lane k < 16 of a warp: level k of head bkv's s1 grid (packed caches), else 0.

@@ -187,10 +187,11 @@ struct Walk {
         const float y = fmaf(d1, (1.0f + kTieRel) * kLbScale, 8388608.0f);
         const uint32_t lim = __float_as_uint(y);
         const bool take1 = (0x4b000000u | (ent1 >> 8)) <= lim;
-        const float4 cv0 = myrep[(ent0 & 0xff) * 8];
-        const float4 cv1 = myrep[(ent1 & 0xff) * 8];
-        const uint64_t a01 = sub2(w01, pk2(cv0.x, cv0.y)), a23 = sub2(w23, pk2(cv0.z, cv0.w));
-        const uint64_t b01 = sub2(w01, pk2(cv1.x, cv1.y)), b23 = sub2(w23, pk2(cv1.z, cv1.w));
+        // codewords read as packed pairs (c0, c1), (c2, c3)
+        const ulonglong2 cv0 = reinterpret_cast<const ulonglong2*>(myrep)[(ent0 & 0xff) * 8];
+        const ulonglong2 cv1 = reinterpret_cast<const ulonglong2*>(myrep)[(ent1 & 0xff) * 8];
+        const uint64_t a01 = sub2(w01, cv0.x), a23 = sub2(w23, cv0.y);
+        const uint64_t b01 = sub2(w01, cv1.x), b23 = sub2(w23, cv1.y);
         const float2 da = upk2(fma2(a23, a23, mul2(a01, a01)));
         const float2 db = upk2(fma2(b23, b23, mul2(b01, b01)));
         // Both entries count even past the band: they are listed codewords
