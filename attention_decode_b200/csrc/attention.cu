@@ -64,18 +64,7 @@ __device__ __forceinline__ void load_q4(const void* q, int64_t off, float (&v)[4
     load4(reinterpret_cast<const QT*>(q) + off, v);
 }
 
-// A running max may lag the true max by up to 2^kLazy (log2 units) before the
-// accumulators are rescaled; weights then stay below 2^kLazy, far from the
-// fp32 range.
-constexpr float kLazy = 8.0f;
 
-// 2^x by the hardware approximation (relative error ~2^-22; results below
-// 2^-126 flush to zero, weights far below the softmax's resolution).
-__device__ __forceinline__ float exp2_approx(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
 
 template <int GC, int KSUB, int VSUB, typename QT>
 __global__ void __launch_bounds__(AttnCfg<GC, KSUB, VSUB>::WARPS * 32, 1) attn_split_kernel(AttnArgs a) {
@@ -298,24 +287,45 @@ __global__ void __launch_bounds__(AttnCfg<GC, KSUB, VSUB>::WARPS * 32, 1) attn_s
         const float2 k2 = resolve_byproducts(k2r, ksrc, t, lvlK);
         const float2 v2 = resolve_byproducts(v2r, vsrc, t, lvlV);
         const float vw = v2.x * v2.y;
+        float logit[GC];
+        bool raise = false;
 #pragma unroll
         for (int h = 0; h < GC; ++h) {
-            const float logit = valid ? k2.x * fmaf(k2.y, sc[h], gm[h]) : -INFINITY;
-            if (__any_sync(kFull, logit > m[h] + kLazy)) {  // warp-uniform, rare
-                const float mx = warp_max(logit);
-                const float alpha = (m[h] == -INFINITY) ? 0.f : exp2_approx(m[h] - mx);
-                l[h] *= alpha;
-                be[h] *= alpha;
-                const uint64_t al = pk2(alpha, alpha);
+            logit[h] = valid ? k2.x * fmaf(k2.y, sc[h], gm[h]) : -INFINITY;
+            raise |= logit[h] > m[h] + kLazy;
+        }
+        if (__any_sync(kFull, raise)) {  // warp-uniform, rare: one vote for all heads
 #pragma unroll
-                for (int r = 0; r < 8; ++r) acc[h][r] = mul2(acc[h][r], al);
-                m[h] = mx;
+            for (int h = 0; h < GC; ++h) {
+                if (__any_sync(kFull, logit[h] > m[h] + kLazy)) {
+                    const float mx = warp_max(logit[h]);
+                    const float alpha = (m[h] == -INFINITY) ? 0.f : exp2_approx(m[h] - mx);
+                    l[h] *= alpha;
+                    be[h] *= alpha;
+                    const uint64_t al = pk2(alpha, alpha);
+#pragma unroll
+                    for (int r = 0; r < 8; ++r) acc[h][r] = mul2(acc[h][r], al);
+                    m[h] = mx;
+                }
             }
-            const float p = valid ? exp2_approx(logit - m[h]) : 0.f;
+        }
+        // Every batch holds a valid token, so m is finite here and an invalid
+        // lane's logit of -inf gives p = 0.
+        uint64_t wpair[GC];
+#pragma unroll
+        for (int h = 0; h < GC; ++h) {
+            const float p = exp2_approx(logit[h] - m[h]);
             l[h] += p;
             be[h] = fmaf(p, v2.x, be[h]);
             const float w = p * vw;
-            wts[lane * GC + h] = pk2(w, w);
+            wpair[h] = pk2(w, w);
+        }
+        if constexpr (GC % 2 == 0) {
+#pragma unroll
+            for (int h2 = 0; h2 < GC / 2; ++h2)
+                reinterpret_cast<ulonglong2*>(wts + lane * GC)[h2] = make_ulonglong2(wpair[2 * h2], wpair[2 * h2 + 1]);
+        } else {
+            wts[lane] = wpair[0];
         }
         __syncwarp();
         // ---- values: lane = (token 4i + grp, dimensions 16 sl .. 16 sl + 15) ----

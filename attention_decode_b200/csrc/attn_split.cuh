@@ -81,6 +81,19 @@ __device__ __forceinline__ float2 load_byproducts(const ByproductSrc& src, uint3
     return resolve_byproducts(fetch_byproducts(src, t, valid), src, t, lvl);
 }
 
+// A running max may lag the true max by up to 2^kLazy (log2 units) before the
+// accumulators are rescaled; weights then stay below 2^kLazy, far from the
+// fp32 range.
+constexpr float kLazy = 8.0f;
+
+// 2^x by the hardware approximation (relative error ~2^-22; results below
+// 2^-126 flush to zero, weights far below the softmax's resolution).
+__device__ __forceinline__ float exp2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // Lane k < 16 of a warp: level k of head bkv's s1 grid (packed caches), else 0.
 __device__ __forceinline__ float packed_level_lane(const uint32_t* levels, const float* grid,
                                                    int64_t bkv) {
