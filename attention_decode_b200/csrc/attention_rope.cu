@@ -38,11 +38,11 @@ constexpr int kHalf = kD / 2;
 //   theta double [64]
 //   qp    float2 [64][GC]: (q_h[i], q_h[i+64])
 //   op    float2 [64]: (o_i, o_{i+64}) of the unit's K shift
-//   per warp: seed float4 [64] (c0, s0, -s0, c0), V codes [32][VJ], weights [32][GP]
+//   per warp: seed float4 [64] (c0, s0, -s0, c0), V codes [32][VJ], weights [32][GC]
+//             as duplicated pairs (w, w)
 template <int GC, int KSUB, int VSUB>
 struct RopeSmem {
     static constexpr int VJ = kD / VSUB;
-    static constexpr int GP = (GC + 3) / 4 * 4;
     static constexpr size_t krep = (size_t)kNC * (KSUB / 4) * 8 * 16;
     static constexpr size_t vrep = (size_t)kNC * (VSUB / 4) * 8 * 16;
     static constexpr size_t rotl = (size_t)kHalf * 32 * 8;
@@ -51,7 +51,7 @@ struct RopeSmem {
     static constexpr size_t op = (size_t)kHalf * 8;
     static constexpr size_t seed = (size_t)kHalf * 16;
     static constexpr size_t wcodes = (size_t)32 * VJ;
-    static constexpr size_t wweights = (size_t)32 * GP * 4;
+    static constexpr size_t wweights = (size_t)32 * GC * 8;
     static constexpr size_t per_warp = seed + wcodes + wweights;
     static constexpr size_t merge = (size_t)kRopeWarps * GC * (3 + kD) * 4;
     static constexpr size_t o_vrep = krep;
@@ -68,7 +68,7 @@ struct RopeSmem {
 template <int GC, int KSUB, int VSUB, typename QT>
 __global__ void __launch_bounds__(kRopeThreads, 1) attn_rope_split_kernel(AttnArgs a) {
     using S = RopeSmem<GC, KSUB, VSUB>;
-    constexpr int KJ = kD / KSUB, VJ = S::VJ, GP = S::GP;
+    constexpr int KJ = kD / KSUB, VJ = S::VJ;
     constexpr int KW = KJ / 4;  // 32-bit words per K code row
     extern __shared__ __align__(16) uint8_t smb[];
     float4* krep = reinterpret_cast<float4*>(smb);
@@ -101,11 +101,11 @@ __global__ void __launch_bounds__(kRopeThreads, 1) attn_rope_split_kernel(AttnAr
     uint8_t* warp_area = smb + S::o_warp + (size_t)warp * S::per_warp;
     float4* seed = reinterpret_cast<float4*>(warp_area);
     uint8_t* my_codes = warp_area + S::seed;
-    float* my_w = reinterpret_cast<float*>(my_codes + S::wcodes);  // [32][GP]
+    uint64_t* my_w = reinterpret_cast<uint64_t*>(my_codes + S::wcodes);  // [32][GC] (w, w)
     constexpr int TPI = 32 / VJ;  // tokens per V step (1 at VSUB=4, 2 at VSUB=8)
     const int jj = lane % VJ, sub_t = lane / VJ;
     const float4* kmy = krep + (lane & 7);
-    const float4* myrep = vrep + (lane & 7);
+    const ulonglong2* myrep = reinterpret_cast<const ulonglong2*>(vrep) + (lane & 7);
 
   for (int64_t u = vbeg / L; u < a.plan.units && u * L < vend; ++u) {
     const int64_t per_b = (int64_t)a.Hkv * a.plan.ngroups;
@@ -220,48 +220,61 @@ __global__ void __launch_bounds__(kRopeThreads, 1) attn_rope_split_kernel(AttnAr
         uint64_t sacc[GC];
 #pragma unroll
         for (int h = 0; h < GC; ++h) sacc[h] = 0ull;
+        // seed read as packed pairs (c0, s0), (-s0, c0); shift and query
+        // pairs (x_i, x_{i+64}) read as one 64-bit word each
         const float2* myL = rotL + lane;
+        const ulonglong2* sd2 = reinterpret_cast<const ulonglong2*>(seed);
+        const uint64_t* op2 = reinterpret_cast<const uint64_t*>(op);
+        const uint64_t* qp2 = reinterpret_cast<const uint64_t*>(qp);
 #pragma unroll
         for (int i = 0; i < kHalf; ++i) {
             const float2 y = upk2(P[i]);
-            const float2 o = op[i];
-            const uint64_t kk = fma2(pk2(y.x + y.y, y.x - y.y), A2, mul2(pk2(o.x, o.y), S1));  // (k_i, k_{i+64})
-            const float4 sd = seed[i];
+            const uint64_t kk = fma2(pk2(y.x + y.y, y.x - y.y), A2, mul2(op2[i], S1));  // (k_i, k_{i+64})
+            const ulonglong2 sd = sd2[i];
             const float2 lr = myL[32 * i];
-            const float2 cs = upk2(fma2(pk2(sd.x, sd.y), pk2(lr.x, lr.x), mul2(pk2(sd.z, sd.w), pk2(lr.y, lr.y))));
+            const float2 cs = upk2(fma2(sd.x, pk2(lr.x, lr.x), mul2(sd.y, pk2(lr.y, lr.y))));  // angle addition
             const float2 kf = upk2(kk);
             // rotated pair: (k_i c - k_{i+64} s, k_i s + k_{i+64} c)
             const uint64_t rk = fma2(pk2(cs.x, cs.x), kk, mul2(pk2(cs.y, cs.y), pk2(-kf.y, kf.x)));
 #pragma unroll
-            for (int h = 0; h < GC; ++h) {
-                const float2 qv = qp[i * GC + h];
-                sacc[h] = fma2(rk, pk2(qv.x, qv.y), sacc[h]);
-            }
+            for (int h = 0; h < GC; ++h) sacc[h] = fma2(rk, qp2[i * GC + h], sacc[h]);
         }
-        // ---- online softmax (log2 domain) ----
-        float wts[GP];
-#pragma unroll
-        for (int h = GC; h < GP; ++h) wts[h] = 0.f;
+        // ---- online softmax (log2 domain), lazy running max as in the plain
+        //      kernel: raised (and the accumulators rescaled) only when a
+        //      logit exceeds it by more than kLazy
+        float logit[GC];
+        bool raise = false;
 #pragma unroll
         for (int h = 0; h < GC; ++h) {
             const float2 sp = upk2(sacc[h]);
-            const float logit = valid ? (sp.x + sp.y) * a.scale_log2 : -INFINITY;
-            const float mx = warp_max(logit);
-            const float mn = fmaxf(m[h], mx);
-            const float alpha = (mn == -INFINITY) ? 1.f : exp2f(m[h] - mn);
-            const float p = valid ? exp2f(logit - mn) : 0.f;
-            l[h] = fmaf(l[h], alpha, p);
-            be[h] = fmaf(be[h], alpha, p * v2.x);
-            const uint64_t al = pk2(alpha, alpha);
-#pragma unroll
-            for (int r = 0; r < VSUB / 2; ++r) acc[h][r] = mul2(acc[h][r], al);
-            wts[h] = p * v2.x * v2.y;
-            m[h] = mn;
+            logit[h] = valid ? (sp.x + sp.y) * a.scale_log2 : -INFINITY;
+            raise |= logit[h] > m[h] + kLazy;
         }
+        if (__any_sync(kFull, raise)) {  // warp-uniform, rare
 #pragma unroll
-        for (int q4 = 0; q4 < GP / 4; ++q4)
-            reinterpret_cast<float4*>(my_w + lane * GP)[q4] =
-                make_float4(wts[4 * q4], wts[4 * q4 + 1], wts[4 * q4 + 2], wts[4 * q4 + 3]);
+            for (int h = 0; h < GC; ++h) {
+                if (__any_sync(kFull, logit[h] > m[h] + kLazy)) {
+                    const float mx = warp_max(logit[h]);
+                    const float alpha = (m[h] == -INFINITY) ? 0.f : exp2_approx(m[h] - mx);
+                    l[h] *= alpha;
+                    be[h] *= alpha;
+                    const uint64_t al = pk2(alpha, alpha);
+#pragma unroll
+                    for (int r = 0; r < VSUB / 2; ++r) acc[h][r] = mul2(acc[h][r], al);
+                    m[h] = mx;
+                }
+            }
+        }
+        // every batch holds a valid token: m is finite and invalid lanes get p = 0
+        const float vw = v2.x * v2.y;
+#pragma unroll
+        for (int h = 0; h < GC; ++h) {
+            const float p = exp2_approx(logit[h] - m[h]);
+            l[h] += p;
+            be[h] = fmaf(p, v2.x, be[h]);
+            const float w = p * vw;
+            my_w[lane * GC + h] = pk2(w, w);
+        }
         __syncwarp();
         // ---- values: lane = sub-vector, fp32 codewords, Hadamard domain ----
         const int nt = (int)min((int64_t)32, te - base);
@@ -269,20 +282,17 @@ __global__ void __launch_bounds__(kRopeThreads, 1) attn_rope_split_kernel(AttnAr
             const int tt = i + sub_t;
             if (tt < nt) {
                 const int code = my_codes[tt * VJ + jj];
-                float c[VSUB];
+                uint64_t c[VSUB / 2];  // codeword as packed pairs
 #pragma unroll
                 for (int k = 0; k < VSUB / 4; ++k) {
-                    const float4 cv = myrep[(code * (VSUB / 4) + k) * 8];
-                    c[4 * k] = cv.x; c[4 * k + 1] = cv.y; c[4 * k + 2] = cv.z; c[4 * k + 3] = cv.w;
+                    const ulonglong2 cv = myrep[(code * (VSUB / 4) + k) * 8];
+                    c[2 * k] = cv.x; c[2 * k + 1] = cv.y;
                 }
-                const float4 w4 = reinterpret_cast<const float4*>(my_w + tt * GP)[0];
-                const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
                 for (int h = 0; h < GC; ++h) {
-                    const uint64_t wp = pk2(wv[h], wv[h]);
+                    const uint64_t wp = my_w[tt * GC + h];
 #pragma unroll
-                    for (int r = 0; r < VSUB / 2; ++r)
-                        acc[h][r] = fma2(pk2(c[2 * r], c[2 * r + 1]), wp, acc[h][r]);
+                    for (int r = 0; r < VSUB / 2; ++r) acc[h][r] = fma2(c[r], wp, acc[h][r]);
                 }
             }
         }
@@ -332,7 +342,7 @@ __global__ void __launch_bounds__(kRopeThreads, 1) attn_rope_split_kernel(AttnAr
 #pragma unroll
         for (int w = 0; w < kRopeWarps; ++w) {
             const float mv = mw[w * GC + h];
-            const float f = (mv == -INFINITY) ? 0.f : exp2f(mv - M);
+            const float f = (mv == -INFINITY) ? 0.f : exp2_approx(mv - M);
             float v;
             if (c < kD) v = Aw[(w * GC + h) * kD + c];
             else if (c == kD) v = lw[w * GC + h];
