@@ -35,7 +35,7 @@ LIB_PATH = os.path.join(_HERE, "_build", "libnsnq.so")
 NSNQ_OK, NSNQ_ERR_INVALID_ARG, NSNQ_ERR_UNSUPPORTED, NSNQ_ERR_WORKSPACE, NSNQ_ERR_CUDA = range(5)
 NSNQ_F32, NSNQ_BF16 = 0, 1
 SHIFT_COMPUTE, SHIFT_GIVEN = 0, 1
-ENCODE_DEFAULT, ENCODE_ADAPTIVE_SCALE, ENCODE_DOUBLE_QUANT = 0, 1, 2
+ENCODE_DEFAULT, ENCODE_ADAPTIVE_SCALE, ENCODE_DOUBLE_QUANT, ENCODE_TC_SEARCH = 0, 1, 2, 4
 HEAD_DIM = 128
 N_CENTROIDS = 256
 
@@ -154,9 +154,11 @@ def _dtype_code(t: torch.Tensor) -> int:
 class Codebook:
     """Global codebook: [256][sub_dim] fp32 on the device. A 2-bit
     (sub_dim 4) codebook also carries its search index, built on first use
-    by nsnq_codebook_index_build."""
+    by nsnq_codebook_index_build, unless no_index is set (then every encode
+    with it must pass ENCODE_TC_SEARCH)."""
     centroids: torch.Tensor
     index: Optional[torch.Tensor] = None
+    no_index: bool = False
 
     @property
     def sub_dim(self) -> int:
@@ -179,7 +181,7 @@ class Codebook:
     def _c(self) -> _Codebook:
         c = getattr(self, "_cstruct", None)
         if c is None:
-            if self.sub_dim == 4 and self.index is None and self.centroids.is_cuda:
+            if self.sub_dim == 4 and self.index is None and self.centroids.is_cuda and not self.no_index:
                 self.prepare()
             c = _Codebook(_ptr(self.centroids), int(self.centroids.shape[0]), self.sub_dim,
                           _ptr(self.index))

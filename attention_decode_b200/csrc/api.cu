@@ -156,7 +156,7 @@ nsnq_status nsnq_encode(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t
         return fail(NSNQ_ERR_UNSUPPORTED, "x_dtype = %d", (int)x_dtype);
     if (mode != NSNQ_SHIFT_COMPUTE && mode != NSNQ_SHIFT_GIVEN)
         return fail(NSNQ_ERR_INVALID_ARG, "shift mode = %d", (int)mode);
-    if (flags & ~(unsigned)(NSNQ_ENCODE_ADAPTIVE_SCALE | NSNQ_ENCODE_DOUBLE_QUANT))
+    if (flags & ~(unsigned)(NSNQ_ENCODE_ADAPTIVE_SCALE | NSNQ_ENCODE_DOUBLE_QUANT | NSNQ_ENCODE_TC_SEARCH))
         return fail(NSNQ_ERR_INVALID_ARG, "unknown encode flags 0x%x", flags);
     const bool dq = (flags & NSNQ_ENCODE_DOUBLE_QUANT) != 0;
     if (dq && (!cache.s1_grid || !aligned(cache.s1_grid, 8)))
@@ -170,6 +170,11 @@ nsnq_status nsnq_encode(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t
     if (B > 65535 || H > 65535) return fail(NSNQ_ERR_UNSUPPORTED, "B or H above 65535");
     nsnq_status s = check_codebook(cb, "cb");
     if (s != NSNQ_OK) return s;
+    const bool tc_search = (flags & NSNQ_ENCODE_TC_SEARCH) != 0;
+    if (cb.sub_dim == 4 && !tc_search && (!cb.index || !aligned(cb.index, 16)))
+        return fail(NSNQ_ERR_INVALID_ARG,
+                    "cb.index is NULL or misaligned: build it with nsnq_codebook_index_build "
+                    "(or pass NSNQ_ENCODE_TC_SEARCH)");
     s = check_cache(cache, "cache", true);
     if (s != NSNQ_OK) return s;
     if (t_offset < 0 || t_offset > cache.cap || T > cache.cap - t_offset)
@@ -188,9 +193,6 @@ nsnq_status nsnq_encode(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t
                     workspace ? workspace_bytes : (size_t)0);
     if (!aligned(workspace, nsnq::kWsAlign))
         return fail(NSNQ_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
-    if (cb.sub_dim == 4 && (!cb.index || !aligned(cb.index, 16)))
-        return fail(NSNQ_ERR_INVALID_ARG,
-                    "cb.index is NULL or misaligned: build it with nsnq_codebook_index_build");
 
     nsnq::EncodeArgs a{};
     a.x = x;
@@ -205,6 +207,7 @@ nsnq_status nsnq_encode(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t
     a.C = cb.centroids;
     a.sub = cb.sub_dim;
     a.index = cb.index;
+    a.tc_search = tc_search ? 1 : 0;
     a.codes = cache.codes; a.scales = cache.scales; a.shift = cache.shift; a.cap = cache.cap;
     a.s1_levels = cache.s1_levels;
     char* ws = static_cast<char*>(workspace);

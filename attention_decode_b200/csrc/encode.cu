@@ -289,7 +289,7 @@ static cudaError_t launch_encode_t(const EncodeArgs& a, cudaStream_t s) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if ((int64_t)a.B * a.H * a.T <= kSmallEncode) return launch_encode_small(a, s);
-    return a.sub == 4 ? launch_encode_pruned(a, s) : launch_encode1_tc(a, s);
+    return (a.sub == 4 && !a.tc_search) ? launch_encode_pruned(a, s) : launch_encode_tc(a, s);
 }
 
 cudaError_t launch_encode(const EncodeArgs& a, cudaStream_t s) {

@@ -1,13 +1,19 @@
-// Pass 2 of the 1-bit encode on the 5th-generation tensor cores (gist.science
-// "NSNQuant ...", Technical Summary, Methodology §1-§3).
+// Pass 2 of the encode with every codeword scored on the 5th-generation
+// tensor cores (gist.science "NSNQuant ...", Technical Summary, Methodology
+// §1-§3): the 1-bit encode (8-dimensional sub-vectors), and the 2-bit encode
+// when the caller asks for the tensor-core search (4-dimensional
+// sub-vectors, no search index; slower than the index walk of
+// encode_pruned.cu, kept as the index-free path and for comparison).
 //
-// With 8-dimensional sub-vectors every codeword is scored, so the scoring is
-// a dense contraction: for a tile of 128 sub-vectors (8 token-heads) and the
-// 256 codewords, s[m][n] = |C_n|^2 - 2 w_m . C_n, and the nearest codeword
-// has the least s (d = |w|^2 + s). The CTA computes w by NSN and the Hadamard
-// transform (two token-heads per warp, one sub-vector per lane), writes it as
-// the A operand, and one thread issues tcgen05.mma (kind::tf32, M 128, N 128,
-// K 8) into a 128-column TMEM accumulator, once for each half of the codebook:
+// Every codeword is scored, so the scoring is a dense contraction: for a
+// tile of 128 sub-vectors and the 256 codewords, s[m][n] = |C_n|^2 - 2 w_m .
+// C_n, and the nearest codeword has the least s (d = |w|^2 + s). The CTA
+// computes w by NSN and the Hadamard transform (two token-heads per warp,
+// 8 coordinates per lane: one 8-dimensional sub-vector, or two 4-dimensional
+// ones taken in two rounds), writes it as the A operand (a 4-dimensional
+// sub-vector padded with zeros to K = 8), and one thread issues tcgen05.mma
+// (kind::tf32, M 128, N 128, K 8) into a 128-column TMEM accumulator, once
+// for each half of the codebook:
 //   D  = A_hi B_hi + A_lo B_hi + A_hi B_lo + 1 (|C|^2_hi + |C|^2_lo)
 // with x_hi = tf32(x), x_lo = tf32(x - x_hi) (three-term split, about fp32
 // accuracy) and B = -2C. Each thread then reads its own row of D (its own
@@ -39,12 +45,12 @@ constexpr float kTieAbsTc = 1e-6f;
 //  - each tf32 x tf32 product is exact in fp32 (11 + 11 significant bits);
 //  - dropping A_lo B_lo and the residuals of the two-term splits of w and
 //    -2C leaves at most 3.001 * 2^-22 of each |w_k| |2 C_k| term;
-//  - |C|^2 is an fp32 chain of 8 fused multiply-adds (8 * 2^-24 relative)
-//    split into two tf32 parts (2^-22 left over);
-//  - the tensor core adds 26 terms (3 split MMAs of K = 8 plus the two |C|^2
-//    parts); with every addition rounding or truncating to fp32 (relative
-//    error <= 2^-23) the sum is off by at most 25 * 2^-23 of the terms'
-//    absolute sum.
+//  - |C|^2 is an fp32 chain of at most 8 fused multiply-adds (8 * 2^-24
+//    relative) split into two tf32 parts (2^-22 left over);
+//  - the tensor core adds at most 26 terms (3 split MMAs of K = 8 plus the
+//    two |C|^2 parts; zero padding adds exact zeros); with every addition
+//    rounding or truncating to fp32 (relative error <= 2^-23) the sum is off
+//    by at most 25 * 2^-23 of the terms' absolute sum.
 // Together: |s_computed - s| <= 3.71e-6 (|C|^2 + 2 |w| |C|). The near-tie band
 // of a sub-vector is at least the sum of this bound for its best codeword and
 // for the largest codeword (the second best is not tracked by index).
@@ -59,7 +65,7 @@ constexpr uint32_t kOffAone = 8192;
 constexpr uint32_t kOffBhi = 12288;    // [2 pieces][256 rows][16 B]
 constexpr uint32_t kOffBlo = 20480;
 constexpr uint32_t kOffBn2 = 28672;
-constexpr uint32_t kOffC = 36864;      // fp32 codebook [256][8] (fp64 path)
+constexpr uint32_t kOffC = 36864;      // fp32 codebook [256][SUB] (fp64 path)
 constexpr uint32_t kOffN2 = 45056;     // fp32 |C|^2 [256]
 constexpr uint32_t kOffBar = 46080;    // mbarrier (8 B) + TMEM address (4 B)
 // Dynamic shared memory per CTA: above 46 KB so that at most four CTAs share
@@ -140,14 +146,15 @@ __device__ __forceinline__ float half_sum(float v) {
 
 // Exact decision for one token-head by the whole warp (see the fp64 path of
 // the 2-bit encode): fp64 NSN and Hadamard transform, lane l holding
-// coordinates 4l..4l+3; each flagged sub-vector j (lanes 2j, 2j+1) is scored
-// against all 256 codewords in fp64, split over the lanes, with a warp argmin
-// (lowest index on exact ties). codes: byte j = code of sub-vector j.
-template <typename XT>
+// coordinates 4l..4l+3; each flagged sub-vector j (lanes (SUB/4) j ..) is
+// scored against all 256 codewords in fp64, split over the lanes, with a
+// warp argmin (lowest index on exact ties). cw: byte j = code of sub-vector j.
+template <typename XT, int SUB>
 __device__ __noinline__ void exact_warp_tc(const XT* xtok, const double* o64, const float* o32,
-                                           const float* C, uint32_t flags, uint4& codes,
+                                           const float* C, uint32_t flags, uint32_t* cw,
                                            double s1_fixed, double& s1_out, double& s2_out,
                                            double& wq_out) {
+    constexpr int LPS = SUB / 4;  // lanes per sub-vector
     const int lane = lane_id();
     float xf[4];
     load4(xtok + 4 * lane, xf);
@@ -182,14 +189,13 @@ __device__ __noinline__ void exact_warp_tc(const XT* xtok, const double* o64, co
     const double hs = 1.0 / sqrt_d;
 #pragma unroll
     for (int r = 0; r < 4; ++r) z[r] *= hs;
-    uint32_t cw[4] = {codes.x, codes.y, codes.z, codes.w};
     uint32_t todo = flags;
     while (todo) {  // warp-uniform
         const int j = __ffs(todo) - 1;
         todo &= todo - 1;
-        double f[8];
+        double f[SUB];
 #pragma unroll
-        for (int r = 0; r < 8; ++r) f[r] = __shfl_sync(kFull, z[r & 3], 2 * j + (r >> 2));
+        for (int r = 0; r < SUB; ++r) f[r] = __shfl_sync(kFull, z[r & 3], LPS * j + (r >> 2));
         double bd = INFINITY;
         int bi = 0;
 #pragma unroll 2
@@ -197,8 +203,8 @@ __device__ __noinline__ void exact_warp_tc(const XT* xtok, const double* o64, co
             const int c = lane + 32 * k;
             double d = 0.0;
 #pragma unroll
-            for (int r = 0; r < 8; ++r) {
-                const double e = f[r] - (double)C[c * 8 + r];
+            for (int r = 0; r < SUB; ++r) {
+                const double e = f[r] - (double)C[c * SUB + r];
                 d = fma(e, e, d);
             }
             if (d < bd) { bd = d; bi = c; }  // c rises with k: ties keep the lower index
@@ -212,19 +218,22 @@ __device__ __noinline__ void exact_warp_tc(const XT* xtok, const double* o64, co
         const int sh = 8 * (j & 3);
         cw[j >> 2] = (cw[j >> 2] & ~(0xffu << sh)) | ((uint32_t)bi << sh);
     }
-    const int j = lane >> 1;
+    const int j = lane / LPS;
     const int code = (int)((cw[j >> 2] >> (8 * (j & 3))) & 0xffu);
     double q = 0.0;
 #pragma unroll
-    for (int r = 0; r < 4; ++r) q = fma(z[r], (double)C[code * 8 + 4 * (lane & 1) + r], q);
+    for (int r = 0; r < 4; ++r) q = fma(z[r], (double)C[code * SUB + 4 * (lane % LPS) + r], q);
     wq_out = warp_sum_d(q);
-    codes = make_uint4(cw[0], cw[1], cw[2], cw[3]);
     s1_out = s1;
     s2_out = s2;
 }
 
-template <typename XT, bool ADAPT, bool DQ>
-__global__ void __launch_bounds__(kTcThreads) nsn_encode1_tc_kernel(EncodeArgs a) {
+// SUB = 8: one sub-vector per lane (1 bit/coordinate); SUB = 4: two per
+// lane, scored in two rounds (2 bits/coordinate, the tensor-core search).
+template <typename XT, bool ADAPT, bool DQ, int SUB>
+__global__ void __launch_bounds__(kTcThreads) nsn_encode_tc_kernel(EncodeArgs a) {
+    constexpr int RPL = 8 / SUB;        // rounds (sub-vectors) per lane
+    constexpr int NW = 32 / SUB;        // 32-bit code words per token-head
     extern __shared__ __align__(1024) uint8_t smraw[];
     // the base of dynamic shared memory is at least 16-byte aligned; align to 1024
     uint8_t* sm = smraw + ((1024u - (smem_addr(smraw) & 1023u)) & 1023u);
@@ -235,18 +244,19 @@ __global__ void __launch_bounds__(kTcThreads) nsn_encode1_tc_kernel(EncodeArgs a
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kOffBar + 8);
     const int tid = threadIdx.x, lane = lane_id(), warp = tid >> 5;
 
-    // ---- constant operands: B = -2C (hi, lo), |C|^2 column, ones column ----
-    for (int i = tid; i < kNC * 8; i += kTcThreads) Cs[i] = a.C[i];
+    // ---- constant operands: B = -2C (hi, lo; zero-padded to K = 8), |C|^2
+    //      column, ones column ----
+    for (int i = tid; i < kNC * SUB; i += kTcThreads) Cs[i] = a.C[i];
     __syncthreads();
     for (int n = tid; n < kNC; n += kTcThreads) {
         float nn = 0.f;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) nn = fmaf(Cs[n * 8 + k], Cs[n * 8 + k], nn);
+        for (int k = 0; k < SUB; ++k) nn = fmaf(Cs[n * SUB + k], Cs[n * SUB + k], nn);
         n2s[n] = nn;
         uint32_t hi[8], lo[8], q2[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-            const float c = -2.0f * Cs[n * 8 + k];
+            const float c = k < SUB ? -2.0f * Cs[n * SUB + k] : 0.f;
             hi[k] = to_tf32(c);
             lo[k] = to_tf32(c - __uint_as_float(hi[k]));
             q2[k] = 0u;
@@ -370,133 +380,159 @@ __global__ void __launch_bounds__(kTcThreads) nsn_encode1_tc_kernel(EncodeArgs a
                 v[k] = fmaf(v[k], sg, p);  // lower index a + b, upper index b - a
             }
         }
-        float ww = 0.f;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) ww = fmaf(v[k], v[k], ww);
-        // ---- A operand (this thread's row), then the MMAs ----
-        {
-            uint32_t hi[8], lo[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                hi[k] = to_tf32(v[k]);
-                lo[k] = to_tf32(v[k] - __uint_as_float(hi[k]));
-            }
-#pragma unroll
-            for (int p = 0; p < 2; ++p) {
-                const uint32_t off = (uint32_t)p * (kRows * 16) + (uint32_t)row * 16;
-                *reinterpret_cast<uint4*>(sm + kOffAhi + off) = make_uint4(hi[4 * p], hi[4 * p + 1], hi[4 * p + 2], hi[4 * p + 3]);
-                *reinterpret_cast<uint4*>(sm + kOffAlo + off) = make_uint4(lo[4 * p], lo[4 * p + 1], lo[4 * p + 2], lo[4 * p + 3]);
-            }
-        }
-        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-        asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
-        __syncthreads();  // A written; the previous tile's TMEM reads are done
-        // ---- the two halves of the codebook, one MMA round each; best and
-        //      second best of this row's scores read back from TMEM ----
-        // Scan of the row's 256 scores by groups of 8: the group minimum (no
-        // index), the least and second-least group minimum, and a copy of the
-        // best group's 8 scores. The best score, its index (lowest on ties)
-        // and the second-best score come out exactly as from a full scan: the
-        // second best is the better of the best group's second and the second
-        // group minimum.
-        float gm1 = INFINITY, gm2 = INFINITY;
-        float gs[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) gs[k] = INFINITY;
-        int gcol = 0;
+        // ---- per round: this thread's sub-vector as the A row, the MMAs over
+        //      both halves of the codebook, and the scan of its 256 scores ----
+        int i1r[RPL];
+        bool tier[RPL];
+        float wq = 0.f;
         const uint32_t taddr = tmem + ((uint32_t)(32 * warp) << 16);
-#pragma unroll 1
-        for (int hf = 0; hf < 2; ++hf) {
-            if (hf) {  // this half reuses the accumulator: every read of the first is done
-                asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
-                __syncthreads();
-            }
-            if (tid == 0) {
-                asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-                const uint64_t bo = (uint64_t)((hf * kCols * 16) >> 4);  // rows 128 hf.. of B
-                mma_tf32(tmem, dAhi, dBhi + bo, 0u);
-                mma_tf32(tmem, dAlo, dBhi + bo, 1u);
-                mma_tf32(tmem, dAhi, dBlo + bo, 1u);
-                mma_tf32(tmem, dAone, dBn2 + bo, 1u);
-                asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
-                                 smem_addr(bar))
-                             : "memory");
-            }
-            long long spins = 0;
-            while (!mbar_try_wait(smem_addr(bar), phase) && ++spins < kWaitLimit) {
-            }
-            const bool done = spins < kWaitLimit;
-            if (__syncthreads_and(done) == 0) {  // MMA not seen complete: flag and stop
-                if (tid == 0 && a.stats) atomicOr(&a.stats[4], 1ull);
-                failed = true;
-                break;
-            }
-            phase ^= 1u;
-            asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-#pragma unroll 1
-            for (int c0 = 0; c0 < kCols; c0 += 32) {
-                uint32_t r[32];
-                tmem_ld32(taddr + (uint32_t)c0, r);
 #pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    float q[8];
+        for (int rd = 0; rd < RPL; ++rd) {
+            float ws[8];
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) q[k] = __uint_as_float(r[8 * g + k]);
-                    const float m = fminf(fminf(fminf(q[0], q[1]), fminf(q[2], q[3])),
-                                          fminf(fminf(q[4], q[5]), fminf(q[6], q[7])));
-                    const bool better = m < gm1;  // strict: the earlier group keeps ties
-                    gm2 = fminf(gm2, fmaxf(gm1, m));
-                    gm1 = fminf(gm1, m);
+            for (int k = 0; k < 8; ++k) ws[k] = k < SUB ? v[SUB * rd + k] : 0.f;
+            float ww = 0.f;
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) gs[k] = better ? q[k] : gs[k];
-                    gcol = better ? hf * kCols + c0 + 8 * g : gcol;
+            for (int k = 0; k < SUB; ++k) ww = fmaf(ws[k], ws[k], ww);
+            {
+                uint32_t hi[8], lo[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    hi[k] = to_tf32(ws[k]);
+                    lo[k] = to_tf32(ws[k] - __uint_as_float(hi[k]));
+                }
+#pragma unroll
+                for (int p = 0; p < 2; ++p) {
+                    const uint32_t off = (uint32_t)p * (kRows * 16) + (uint32_t)row * 16;
+                    *reinterpret_cast<uint4*>(sm + kOffAhi + off) = make_uint4(hi[4 * p], hi[4 * p + 1], hi[4 * p + 2], hi[4 * p + 3]);
+                    *reinterpret_cast<uint4*>(sm + kOffAlo + off) = make_uint4(lo[4 * p], lo[4 * p + 1], lo[4 * p + 2], lo[4 * p + 3]);
                 }
             }
+            asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+            asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+            __syncthreads();  // A written; the previous round's TMEM reads are done
+            // Scan of the row's 256 scores by groups of 8: the group minimum (no
+            // index), the least and second-least group minimum, and a copy of the
+            // best group's 8 scores. The best score, its index (lowest on ties)
+            // and the second-best score come out exactly as from a full scan: the
+            // second best is the better of the best group's second and the second
+            // group minimum.
+            float gm1 = INFINITY, gm2 = INFINITY;
+            float gs[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) gs[k] = INFINITY;
+            int gcol = 0;
+#pragma unroll 1
+            for (int hf = 0; hf < 2; ++hf) {
+                if (hf) {  // this half reuses the accumulator: every read of the first is done
+                    asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+                    __syncthreads();
+                }
+                if (tid == 0) {
+                    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+                    const uint64_t bo = (uint64_t)((hf * kCols * 16) >> 4);  // rows 128 hf.. of B
+                    mma_tf32(tmem, dAhi, dBhi + bo, 0u);
+                    mma_tf32(tmem, dAlo, dBhi + bo, 1u);
+                    mma_tf32(tmem, dAhi, dBlo + bo, 1u);
+                    mma_tf32(tmem, dAone, dBn2 + bo, 1u);
+                    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
+                                     smem_addr(bar))
+                                 : "memory");
+                }
+                long long spins = 0;
+                while (!mbar_try_wait(smem_addr(bar), phase) && ++spins < kWaitLimit) {
+                }
+                const bool done = spins < kWaitLimit;
+                if (__syncthreads_and(done) == 0) {  // MMA not seen complete: flag and stop
+                    if (tid == 0 && a.stats) atomicOr(&a.stats[4], 1ull);
+                    failed = true;
+                    break;
+                }
+                phase ^= 1u;
+                asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+#pragma unroll 1
+                for (int c0 = 0; c0 < kCols; c0 += 32) {
+                    uint32_t r[32];
+                    tmem_ld32(taddr + (uint32_t)c0, r);
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+                        float q[8];
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) q[k] = __uint_as_float(r[8 * g + k]);
+                        const float m = fminf(fminf(fminf(q[0], q[1]), fminf(q[2], q[3])),
+                                              fminf(fminf(q[4], q[5]), fminf(q[6], q[7])));
+                        const bool better = m < gm1;  // strict: the earlier group keeps ties
+                        gm2 = fminf(gm2, fmaxf(gm1, m));
+                        gm1 = fminf(gm1, m);
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) gs[k] = better ? q[k] : gs[k];
+                        gcol = better ? hf * kCols + c0 + 8 * g : gcol;
+                    }
+                }
+            }
+            if (failed) break;
+            const float b1 = gm1;
+            int k1 = 7;
+#pragma unroll
+            for (int k = 6; k >= 0; --k) k1 = gs[k] == b1 ? k : k1;
+            float bin = INFINITY;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) bin = k == k1 ? bin : fminf(bin, gs[k]);
+            const float b2 = fminf(bin, gm2);
+            const int i1 = gcol + k1;
+            const float wn = sqrtf(ww), c1 = sqrtf(n2s[i1]);
+            const float band_s = kScoreErrTc * (n2s[i1] + cmax * cmax + 2.f * wn * (c1 + cmax));
+            tier[rd] = valid && (cancel || (b2 - b1) <= fmaxf(fmaf(kTieRelTc, ww + b1, kTieAbsTc), band_s));
+            i1r[rd] = i1;
+            if constexpr (ADAPT) wq += 0.5f * (n2s[i1] - b1);  // w . C[best] = (|C|^2 - s) / 2
         }
         if (failed) break;
-        const float b1 = gm1;
-        int k1 = 7;
+        if constexpr (ADAPT) wq = half_sum(wq);
+        // ---- codes of the warp's two token-heads (lane l16 holds sub-vectors
+        //      RPL l16 .. RPL l16 + RPL - 1 of its token), then the exact path ----
+        uint32_t mine = 0u;  // this lane's codes, one byte per round
 #pragma unroll
-        for (int k = 6; k >= 0; --k) k1 = gs[k] == b1 ? k : k1;
-        float bin = INFINITY;
+        for (int rd = 0; rd < RPL; ++rd) mine |= (uint32_t)i1r[rd] << (8 * rd);
+        constexpr int LPW = 4 / RPL;  // lanes per code word
+        uint32_t cw[NW];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) bin = k == k1 ? bin : fminf(bin, gs[k]);
-        const float b2 = fminf(bin, gm2);
-        const int i1 = gcol + k1;
-        const float wn = sqrtf(ww), c1 = sqrtf(n2s[i1]);
-        const float band_s = kScoreErrTc * (n2s[i1] + cmax * cmax + 2.f * wn * (c1 + cmax));
-        bool tie = cancel || (b2 - b1) <= fmaxf(fmaf(kTieRelTc, ww + b1, kTieAbsTc), band_s);
-        if (!valid) tie = false;
-        float wq = 0.f;
-        if constexpr (ADAPT) wq = half_sum(0.5f * (n2s[i1] - b1));  // w . C[best] = (|C|^2 - s) / 2
-        // ---- codes of the warp's two token-heads, then the exact path ----
-        uint32_t cw[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
+        for (int k = 0; k < NW; ++k) {
             uint32_t word = 0u;
 #pragma unroll
-            for (int r = 0; r < 4; ++r)
-                word |= (uint32_t)__shfl_sync(kFull, i1, 16 * half + 4 * k + r) << (8 * r);
+            for (int r = 0; r < LPW; ++r)
+                word |= __shfl_sync(kFull, mine, 16 * half + LPW * k + r) << (8 * RPL * r);
             cw[k] = word;
         }
-        uint4 codes = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        // near-tie flags of the warp's token-heads: bit j of half hh = sub-vector j
+        uint32_t tflag[2] = {0u, 0u};
+#pragma unroll
+        for (int rd = 0; rd < RPL; ++rd) {
+            const uint32_t m = __ballot_sync(kFull, tier[rd]);
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const uint32_t f = (m >> (16 * hh)) & 0xffffu;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) tflag[hh] |= ((f >> i) & 1u) << (RPL * i + rd);
+            }
+        }
         float s1o = s1, s2o = s2;
         double wqd = (double)wq;
-        const uint32_t tmask = __ballot_sync(kFull, tie);
-        if (tmask) {
+        if (tflag[0] | tflag[1]) {  // warp-uniform
             const double* o64 = a.given_shift ? nullptr : a.o64 + bh * kD;
 #pragma unroll 1
             for (int hh = 0; hh < 2; ++hh) {
-                const uint32_t flags = (tmask >> (16 * hh)) & 0xffffu;  // bit j: sub-vector j
+                const uint32_t flags = tflag[hh];
                 if (!flags) continue;  // warp-uniform
-                uint4 cq = make_uint4(__shfl_sync(kFull, codes.x, 16 * hh), __shfl_sync(kFull, codes.y, 16 * hh),
-                                      __shfl_sync(kFull, codes.z, 16 * hh), __shfl_sync(kFull, codes.w, 16 * hh));
+                uint32_t cq[NW];
+#pragma unroll
+                for (int k = 0; k < NW; ++k) cq[k] = __shfl_sync(kFull, cw[k], 16 * hh);
                 double s1d, s2d, wq64;
                 const double s1f = __shfl_sync(kFull, s1dq, 16 * hh);
-                exact_warp_tc<XT>(xhead + (t0 + hh) * a.st, o64, a.shift + bh * kD, Cs, flags, cq, s1f,
-                                  s1d, s2d, wq64);
+                exact_warp_tc<XT, SUB>(xhead + (t0 + hh) * a.st, o64, a.shift + bh * kD, Cs, flags, cq, s1f,
+                                       s1d, s2d, wq64);
                 if (half == hh) {
-                    codes = cq;
+#pragma unroll
+                    for (int k = 0; k < NW; ++k) cw[k] = cq[k];
                     s1o = (float)s1d;
                     s2o = (float)s2d;
                     wqd = wq64;
@@ -512,7 +548,9 @@ __global__ void __launch_bounds__(kTcThreads) nsn_encode1_tc_kernel(EncodeArgs a
         }
         if (valid && l16 == 0) {
             const int64_t orow = bh * a.cap + a.t_offset + t;
-            reinterpret_cast<uint4*>(a.codes + orow * 16)[0] = codes;
+            uint4* dst = reinterpret_cast<uint4*>(a.codes + orow * (4 * NW));
+#pragma unroll
+            for (int k = 0; k < NW / 4; ++k) dst[k] = make_uint4(cw[4 * k], cw[4 * k + 1], cw[4 * k + 2], cw[4 * k + 3]);
             store_byproducts(a.scales, a.s1_levels, bh, a.cap, a.t_offset + t, s1o, s2o, s1lev);
         }
     }
@@ -530,7 +568,7 @@ __global__ void __launch_bounds__(kTcThreads) nsn_encode1_tc_kernel(EncodeArgs a
     }
 }
 
-template <typename XT, bool ADAPT, bool DQ>
+template <typename XT, bool ADAPT, bool DQ, int SUB>
 cudaError_t launch_tc(const EncodeArgs& a, cudaStream_t s) {
     static std::atomic<unsigned long long> ready{0};
     const int sms = device_sm_count();
@@ -538,20 +576,26 @@ cudaError_t launch_tc(const EncodeArgs& a, cudaStream_t s) {
     const int64_t ntiles = (npairs + 3) / 4;
     const int64_t cap = (int64_t)sms * 4;  // four CTAs per SM: all resident, 512 TMEM columns
     const int grid = (int)(ntiles < cap ? ntiles : cap);
-    return launch_smem(nsn_encode1_tc_kernel<XT, ADAPT, DQ>, ready, dim3(grid), dim3(kTcThreads),
+    return launch_smem(nsn_encode_tc_kernel<XT, ADAPT, DQ, SUB>, ready, dim3(grid), dim3(kTcThreads),
                        (size_t)kTcSmem, s, a);
+}
+
+template <int SUB>
+cudaError_t launch_tc_sub(const EncodeArgs& a, cudaStream_t s) {
+    if (a.x_bf16) {
+        if (a.dq) return a.adaptive ? launch_tc<__nv_bfloat16, true, true, SUB>(a, s)
+                                    : launch_tc<__nv_bfloat16, false, true, SUB>(a, s);
+        return a.adaptive ? launch_tc<__nv_bfloat16, true, false, SUB>(a, s)
+                          : launch_tc<__nv_bfloat16, false, false, SUB>(a, s);
+    }
+    if (a.dq) return a.adaptive ? launch_tc<float, true, true, SUB>(a, s) : launch_tc<float, false, true, SUB>(a, s);
+    return a.adaptive ? launch_tc<float, true, false, SUB>(a, s) : launch_tc<float, false, false, SUB>(a, s);
 }
 
 }  // namespace
 
-cudaError_t launch_encode1_tc(const EncodeArgs& a, cudaStream_t s) {
-    if (a.x_bf16) {
-        if (a.dq) return a.adaptive ? launch_tc<__nv_bfloat16, true, true>(a, s)
-                                    : launch_tc<__nv_bfloat16, false, true>(a, s);
-        return a.adaptive ? launch_tc<__nv_bfloat16, true, false>(a, s) : launch_tc<__nv_bfloat16, false, false>(a, s);
-    }
-    if (a.dq) return a.adaptive ? launch_tc<float, true, true>(a, s) : launch_tc<float, false, true>(a, s);
-    return a.adaptive ? launch_tc<float, true, false>(a, s) : launch_tc<float, false, false>(a, s);
+cudaError_t launch_encode_tc(const EncodeArgs& a, cudaStream_t s) {
+    return a.sub == 4 ? launch_tc_sub<4>(a, s) : launch_tc_sub<8>(a, s);
 }
 
 }  // namespace nsnq

@@ -72,7 +72,8 @@ struct EncodeArgs {
     float* s1_grid;  // [B][H][2] (lo, step) of the log2 s1 grid
     const float* C;
     int sub;
-    const void* index;  // search index (sub == 4)
+    const void* index;  // search index (sub == 4, walk search)
+    int tc_search;      // sub == 4: score every codeword on the tensor cores (no index)
     uint8_t* codes;
     float* scales;
     float* shift;
@@ -103,7 +104,9 @@ cudaError_t launch_encode_pruned(const EncodeArgs& a, cudaStream_t s);
 // token-head, fp64 throughout (a decode step's appends).
 constexpr int64_t kSmallEncode = 1024;
 cudaError_t launch_encode_small(const EncodeArgs& a, cudaStream_t s);
-cudaError_t launch_encode1_tc(const EncodeArgs& a, cudaStream_t s);
+// Pass 2 with every codeword scored on the tensor cores: sub == 8, or sub == 4
+// with tc_search (encode1_tc.cu).
+cudaError_t launch_encode_tc(const EncodeArgs& a, cudaStream_t s);
 size_t index_bytes();
 cudaError_t launch_index_build(const float* C, void* index, cudaStream_t s);
 cudaError_t launch_codebook_q4(const float* in, float* out, uint8_t* levels, double* grid, int n,

@@ -6,6 +6,7 @@ Cases (seeded synthetic inputs generated on the device):
   encode-16x8x4096     encode one bf16 tensor, 16 x 8 kv-heads x 4096 tokens, 2 bit
                        (134 MB of input: larger than L2)
   encode-8x8x4096      the benchmark's per-tensor encode (67 MB)
+  encode-tc-8x8x4096   the same with the tensor-core search (ENCODE_TC_SEARCH, no index)
   encode1-16x8x4096    1-bit encode (tensor-core scoring), 16 x 8 kv-heads x 4096 tokens
   encode1-8x8x4096     1-bit encode, 8 x 8 kv-heads x 4096 tokens
   attn-16x32k-2b       decode attention, B 16, Hq 32, Hkv 8, 32768 tokens, 2 bit
@@ -40,18 +41,20 @@ def _keys(gen, B, H, T, dev):
     return ((z + bias) * s).to(torch.bfloat16)
 
 
-def encode_case(B, H, T, reps, dev, sub=4):
+def encode_case(B, H, T, reps, dev, sub=4, flags=nsnq.ENCODE_DEFAULT):
     gen = torch.Generator(device=dev)
     gen.manual_seed(0)
     cb = _codebook(sub, dev)
+    cb.no_index = bool(flags & nsnq.ENCODE_TC_SEARCH)
     x = _keys(gen, B, H, T, dev)
     cache = nsnq.Cache.empty(B, H, T, sub, device=dev)
     ws = torch.empty(nsnq.nsnq_encode_workspace(B, H, T), dtype=torch.uint8, device=dev)
-    cb.prepare()
+    if not cb.no_index:
+        cb.prepare()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     for _ in range(reps):
         e0.record()
-        nsnq.nsnq_encode(x, cb, cache, workspace=ws)
+        nsnq.nsnq_encode(x, cb, cache, workspace=ws, flags=flags)
         e1.record()
     torch.cuda.synchronize()
     th, sv, mism, tmo = nsnq.encode_stats(ws)
@@ -101,6 +104,7 @@ def attn_case(B, Hq, Hkv, T, sub, reps, dev, rope=False):
 CASES = {
     "encode-16x8x4096": lambda r, d: encode_case(16, 8, 4096, r, d),
     "encode-8x8x4096": lambda r, d: encode_case(8, 8, 4096, r, d),
+    "encode-tc-8x8x4096": lambda r, d: encode_case(8, 8, 4096, r, d, flags=nsnq.ENCODE_TC_SEARCH),
     "encode1-16x8x4096": lambda r, d: encode_case(16, 8, 4096, r, d, sub=8),
     "encode1-8x8x4096": lambda r, d: encode_case(8, 8, 4096, r, d, sub=8),
     "attn-16x32k-2b": lambda r, d: attn_case(16, 32, 8, 32768, 4, r, d),

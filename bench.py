@@ -308,6 +308,7 @@ def run_cuda(args):
     attention = run_attention_bench(args, nsnq, dev, world, barrier, hbm, peak_kind)
     attention_variants = run_attention_variants(args, nsnq, dev, world, barrier, hbm)
     encode_1bit = run_encode1_bench(args, nsnq, dev, world, barrier, hbm, peak_kind, k)
+    encode_tc_search = run_encode1_bench(args, nsnq, dev, world, barrier, hbm, peak_kind, k, sub=4)
     long_context = run_long_context_bench(args, nsnq, dev, world, barrier, hbm)
     serving = run_serving_bench(args, nsnq, dev, world, barrier, hbm)
     clk.__exit__(None, None, None)
@@ -325,7 +326,7 @@ def run_cuda(args):
                       "attention_4k": round(sum(att_small_ms) / len(att_small_ms), 4)},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "roofline": roofline, "attention": attention, "attention_variants": attention_variants,
-        "encode_1bit": encode_1bit,
+        "encode_1bit": encode_1bit, "encode_2bit_tc_search": encode_tc_search,
         "long_context": long_context, "serving": serving, "e2e": e2e,
         "clocks": clk.summary(),
     }
@@ -482,16 +483,19 @@ def run_attention_variants(args, nsnq, dev, world, barrier, hbm):
     return res
 
 
-def run_encode1_bench(args, nsnq, dev, world, barrier, hbm, peak_kind, x):
-    """The 1-bit encode (tensor-core scoring) of the step's K tensor."""
+def run_encode1_bench(args, nsnq, dev, world, barrier, hbm, peak_kind, x, sub=8):
+    """Encode of the step's K tensor with every codeword scored on the tensor
+    cores: at 1 bit (sub 8), or at 2 bits with the tensor-core search (sub 4,
+    ENCODE_TC_SEARCH, no index: the comparison with the index walk)."""
     import torch
     B, H, T = x.shape[0], x.shape[1], x.shape[2]
-    cb = nsnq.Codebook(torch.from_numpy(load_codebook(8)).to(dev))
-    cache = nsnq.Cache.empty(B, H, T, 8, device=dev)
+    flags = nsnq.ENCODE_TC_SEARCH if sub == 4 else nsnq.ENCODE_DEFAULT
+    cb = nsnq.Codebook(torch.from_numpy(load_codebook(sub)).to(dev), no_index=sub == 4)
+    cache = nsnq.Cache.empty(B, H, T, sub, device=dev)
     ws = torch.empty(nsnq.nsnq_encode_workspace(B, H, T), dtype=torch.uint8, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
-        nsnq.nsnq_encode(x, cb, cache, workspace=ws)
+        nsnq.nsnq_encode(x, cb, cache, workspace=ws, flags=flags)
     stream = torch.cuda.current_stream()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
@@ -500,21 +504,24 @@ def run_encode1_bench(args, nsnq, dev, world, barrier, hbm, peak_kind, x):
     for e0, e1 in evs:
         flush.zero_()
         e0.record(stream)
-        nsnq.nsnq_encode(x, cb, cache, workspace=ws)
+        nsnq.nsnq_encode(x, cb, cache, workspace=ws, flags=flags)
         e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     avg = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / len(evs), world, dev)
-    nbytes = B * H * T * encode_bytes_per_token_head(8)
+    nbytes = B * H * T * encode_bytes_per_token_head(sub)
     gbs = nbytes / (avg / 1e3) / 1e9
-    return {"metric": "KV tokens/s encoded at 1 bit", "value": round(B * T * world / (avg / 1e3), 1),
+    what = ("1 bit/coord (g = 8), codewords scored on the tensor cores" if sub == 8 else
+            "2 bits/coord (g = 4), all 256 codewords scored on the tensor cores (no index)")
+    return {"metric": f"KV tokens/s encoded at {8 // sub} bit" + ("" if sub == 8 else "s, tensor-core search"),
+            "value": round(B * T * world / (avg / 1e3), 1),
             "unit": "KV tokens/s (one tensor)", "ms_per_call": round(avg, 4),
-            "workload": "encode-8x4096 keys at 1 bit/coord (g = 8), codewords scored on the tensor cores",
+            "workload": f"encode-8x4096 keys at {what}",
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
                          "frac": round(gbs / hbm, 4), "frac_vs_8tbs": round(gbs / NOMINAL_HBM_GBS, 4), "peak_kind": peak_kind,
-                         "kernel": "nsnq_encode at 1 bit (nsn_stats + nsn_encode1_tc)",
+                         "kernel": f"nsnq_encode at {8 // sub} bit (nsn_stats + nsn_encode_tc)",
                          "algorithmic_bytes_per_launch": nbytes,
-                         "traffic": measured_traffic("nsnq_encode_1bit")},
+                         "traffic": measured_traffic("nsnq_encode_1bit") if sub == 8 else None},
             "l2": "flushed before every call"}
 
 

@@ -86,7 +86,15 @@ typedef enum {
      * fields; with cache.s1_levels set, s1 is stored as its 4-bit level and
      * scales holds s2 alone (the packed form, see nsnq_cache). o stays an
      * fp32 vector per head (its 16 level values). Requires cache.s1_grid. */
-    NSNQ_ENCODE_DOUBLE_QUANT = 2
+    NSNQ_ENCODE_DOUBLE_QUANT = 2,
+    /* sub_dim 4: find the nearest codeword by scoring all 256 on the tensor
+     * cores (|C|^2 - 2 w.C, as for sub_dim 8) instead of walking the search
+     * index; cb.index is then not needed. Same codes (exact up to the
+     * near-tie rule), slower than the index walk: it serves codebooks whose
+     * index does not fit (nsnq_codebook_index_build returns
+     * NSNQ_ERR_UNSUPPORTED) and comparison. Calls of at most 1024
+     * token-heads use the small-call path either way. No effect at sub_dim 8. */
+    NSNQ_ENCODE_TC_SEARCH = 4
 } nsnq_encode_flags;
 
 typedef struct {
@@ -95,7 +103,8 @@ typedef struct {
     int sub_dim;             /* 4 (2 bits/coordinate) or 8 (1 bit/coordinate) */
     const void* index;       /* device search index built from these centroids by
                                 nsnq_codebook_index_build; required by nsnq_encode when
-                                sub_dim == 4, ignored otherwise (may be NULL) */
+                                sub_dim == 4 unless NSNQ_ENCODE_TC_SEARCH is passed,
+                                ignored otherwise (may be NULL) */
 } nsnq_codebook;
 
 typedef struct {
@@ -192,8 +201,9 @@ size_t nsnq_encode_workspace(int B, int H, int64_t T, int D);
  *             dtype x_dtype (fp32 or bf16); 16-byte aligned rows.
  *   mode      NSNQ_SHIFT_COMPUTE: o = mean over the T tokens of x/s1, stored
  *             to cache.shift (fp32); NSNQ_SHIFT_GIVEN: o = cache.shift.
- *   flags     NSNQ_ENCODE_DEFAULT, or NSNQ_ENCODE_ADAPTIVE_SCALE and/or
- *             NSNQ_ENCODE_DOUBLE_QUANT (bitwise or).
+ *   flags     NSNQ_ENCODE_DEFAULT, or any of NSNQ_ENCODE_ADAPTIVE_SCALE,
+ *             NSNQ_ENCODE_DOUBLE_QUANT, NSNQ_ENCODE_TC_SEARCH (bitwise or);
+ *             other bits: NSNQ_ERR_INVALID_ARG.
  *   cb        codebook; cache: codes/scales written, shift read or written.
  *   workspace device scratch of at least nsnq_encode_workspace(B, H, T, D)
  *             bytes, 256-byte aligned.

@@ -75,12 +75,16 @@ def test_encode_validation(lib):
     assert _encode(lib, off=95) == nsnq.NSNQ_ERR_INVALID_ARG            # past capacity
     assert _encode(lib, T=-1) == nsnq.NSNQ_ERR_INVALID_ARG
     assert _encode(lib, mode=7) == nsnq.NSNQ_ERR_INVALID_ARG
-    assert _encode(lib, flags=4) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert _encode(lib, flags=8) == nsnq.NSNQ_ERR_INVALID_ARG            # unknown flag bit
     assert _encode(lib, flags=2) == nsnq.NSNQ_ERR_INVALID_ARG  # double quantization needs s1_grid
     assert _encode(lib, ws=None) == nsnq.NSNQ_ERR_WORKSPACE
     assert _encode(lib, cb=_cb(index=None)) == nsnq.NSNQ_ERR_INVALID_ARG     # 2-bit needs its index
     assert b"nsnq_codebook_index_build" in lib.nsnq_last_error()
     assert _encode(lib, cb=_cb(sub=8, index=None), T=0) == nsnq.NSNQ_OK
+    # the tensor-core search needs no index: the index check passes and the
+    # workspace check (later) fails; without the flag the index check fails
+    assert _encode(lib, cb=_cb(index=None), wsb=16) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert _encode(lib, cb=_cb(index=None), flags=nsnq.ENCODE_TC_SEARCH, wsb=16) == nsnq.NSNQ_ERR_WORKSPACE
     need = lib.nsnq_encode_workspace(1, 1, 10, 128)
     assert need > 0
     assert _encode(lib, wsb=need - 1) == nsnq.NSNQ_ERR_WORKSPACE

@@ -4,7 +4,8 @@ allocation is not allowed, a C caller without an allocator). Its split
 partials live in the library's fixed 4 MiB device array instead of a
 caller workspace. Checked through the C ABI against nsnq_attn_decode on
 two calls in a row (the array is shared and keeps the previous call's
-contents), and for the rejection of shapes that do not fit.
+contents), for the rejection of shapes that do not fit, and for a call
+captured into a CUDA graph after a warm-up call.
 
 Kept in a file of its own that is collected last."""
 import os
@@ -62,3 +63,29 @@ def test_noalloc_rejects_shapes_beyond_its_array():
         nsnq.nsnq_attn_decode_noalloc(q, kc, vc, cb, cb, lens, T, Hkv=Hkv)
     assert ei.value.status == nsnq.NSNQ_ERR_WORKSPACE
     assert "fixed device array" in str(ei.value)
+
+
+def test_noalloc_call_captured_in_a_cuda_graph():
+    """The documented use: one call outside capture (it looks up the array),
+    then calls captured into a CUDA graph; a replay reads the inputs' current
+    contents and matches nsnq_attn_decode on them."""
+    nbuild.build()
+    cb = nsnq.Codebook(torch.from_numpy(load_codebook(4)).cuda())
+    B, Hq, Hkv, T = 4, 32, 8, 2000
+    (kc, vc), q, lens = _random_inputs(B, Hq, Hkv, T, 4, 5)
+    out = torch.empty(B, Hq, 128, dtype=torch.float32, device="cuda")
+    nsnq.nsnq_attn_decode_noalloc(q, kc, vc, cb, cb, lens, T, Hkv=Hkv, out=out)  # warm-up
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        nsnq.nsnq_attn_decode_noalloc(q, kc, vc, cb, cb, lens, T, Hkv=Hkv, out=out)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(6)
+    q.copy_(torch.randn(q.shape, generator=gen, device="cuda").to(q.dtype))  # new query, same buffer
+    out.zero_()
+    graph.replay()
+    ref = nsnq.nsnq_attn_decode(q, kc, vc, cb, cb, lens, T, Hkv=Hkv, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    e, _ = P.attn_errors(out.cpu().numpy(), ref.cpu().numpy().astype(np.float64), False)
+    assert (e <= 1.0).all(), e.max()
+    del graph
