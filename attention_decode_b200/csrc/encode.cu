@@ -166,6 +166,9 @@ __device__ void shift_of_head(const EncodeArgs& a, int64_t bh, double (*red)[kD]
 
 template <typename XT, bool DQ>
 __global__ void __launch_bounds__(kStatsThreads, 4) nsn_stats_kernel(EncodeArgs a) {
+    // pass 2 is a programmatic dependent: it may be scheduled as this grid's
+    // CTAs retire (it waits for the whole grid before reading the shift)
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
     const int chunk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int64_t bh = (int64_t)b * a.H + h;
     const int warp = threadIdx.x >> 5, lane = lane_id();

@@ -300,6 +300,9 @@ __global__ void __launch_bounds__(kTcThreads) nsn_encode_tc_kernel(EncodeArgs a)
     const uint64_t dBlo = mat_desc(sbase + kOffBlo, kNC * 16, 128);
     const uint64_t dBn2 = mat_desc(sbase + kOffBn2, kNC * 16, 128);
 
+    // Launched as a programmatic dependent of pass 1: the setup above
+    // overlaps its end; the shift it derives is read only after this wait.
+    asm volatile("griddepcontrol.wait;\n" ::: "memory");
     const int l16 = lane & 15, half = lane >> 4;
     const int row = tid;  // = 32 * warp + lane: this thread's sub-vector row and TMEM lane
     const int64_t pairs_per_head = (a.T + 1) / 2;
@@ -576,8 +579,8 @@ cudaError_t launch_tc(const EncodeArgs& a, cudaStream_t s) {
     const int64_t ntiles = (npairs + 3) / 4;
     const int64_t cap = (int64_t)sms * 4;  // four CTAs per SM: all resident, 512 TMEM columns
     const int grid = (int)(ntiles < cap ? ntiles : cap);
-    return launch_smem(nsn_encode_tc_kernel<XT, ADAPT, DQ, SUB>, ready, dim3(grid), dim3(kTcThreads),
-                       (size_t)kTcSmem, s, a);
+    return launch_smem_pdl(nsn_encode_tc_kernel<XT, ADAPT, DQ, SUB>, ready, dim3(grid), dim3(kTcThreads),
+                           (size_t)kTcSmem, s, a);
 }
 
 template <int SUB>

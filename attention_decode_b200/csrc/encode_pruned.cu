@@ -262,6 +262,9 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
             offs_w[i] = (uint16_t)min((uint32_t)offs_w[i], n_pairs);
     }
     __syncthreads();
+    // Launched as a programmatic dependent of pass 1: the staging above
+    // overlaps its end; the shift it derives is read only after this wait.
+    asm volatile("griddepcontrol.wait;\n" ::: "memory");
 
     // Each warp owns tiles of 16 consecutive token-heads of one (batch, head)
     // and keeps its own copy of that head's shift: no CTA barrier in the loop.
@@ -461,8 +464,8 @@ static cudaError_t launch_pruned_t(const EncodeArgs& a, cudaStream_t s) {
     const int64_t ntiles = (int64_t)a.B * a.H * ((a.T + kWarpTile - 1) / kWarpTile);
     const int64_t ctas = (ntiles + kWarps - 1) / kWarps;
     const int grid = (int)(ctas < sms ? ctas : sms);
-    return launch_smem(nsn_encode_pruned_kernel<XT, ADAPT, DQ>, ready, dim3(grid),
-                       dim3(kPrunedThreads), kSmBytes, s, a);
+    return launch_smem_pdl(nsn_encode_pruned_kernel<XT, ADAPT, DQ>, ready, dim3(grid),
+                           dim3(kPrunedThreads), kSmBytes, s, a);
 }
 
 cudaError_t launch_encode_pruned(const EncodeArgs& a, cudaStream_t s) {

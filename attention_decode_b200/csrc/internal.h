@@ -58,6 +58,33 @@ cudaError_t launch_smem(void (*kern)(P...), std::atomic<unsigned long long>& rea
     return e;
 }
 
+// launch_smem as a programmatic dependent launch: the kernel may start while
+// the previous kernel in the stream finishes, and must execute
+// griddepcontrol.wait before it reads what that kernel wrote.
+template <typename... P, typename... A>
+cudaError_t launch_smem_pdl(void (*kern)(P...), std::atomic<unsigned long long>& ready, dim3 grid,
+                            dim3 block, size_t smem, cudaStream_t s, A&&... args) {
+    cudaError_t e = ensure_smem(kern, (int)smem, ready, false);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, args...);
+    if (e == cudaErrorInvalidValue) {  // attribute lost (device reset): set it again, once
+        e = ensure_smem(kern, (int)smem, ready, true);
+        if (e != cudaSuccess) return e;
+        e = cudaLaunchKernelEx(&cfg, kern, args...);
+    }
+    return e;
+}
+
 // ------------------------------------------------------------------ encode --
 struct EncodeArgs {
     const void* x;

@@ -13,6 +13,7 @@ Cases (seeded synthetic inputs generated on the device):
   attn-16x32k-1b       the same with 1-bit K and V
   attn-64x8k-gqa8      decode attention, B 64, Hq 64, Hkv 8, 8192 tokens, 2 bit
   attn-8x4k-2b         decode attention of the benchmark step: B 8, Hq 32, Hkv 8, 4096 tokens
+  attn-1x128k-2b       long-context decode attention: B 1, Hq 32, Hkv 8, 131072 tokens, 2 bit
   attn-rope-16x32k-2b  attn-16x32k-2b with the keys read as quantized before RoPE
 """
 from __future__ import annotations
@@ -112,6 +113,7 @@ CASES = {
     "attn-rope-16x32k-2b": lambda r, d: attn_case(16, 32, 8, 32768, 4, r, d, rope=True),
     "attn-64x8k-gqa8": lambda r, d: attn_case(64, 64, 8, 8192, 4, r, d),
     "attn-8x4k-2b": lambda r, d: attn_case(8, 32, 8, 4096, 4, r, d),
+    "attn-1x128k-2b": lambda r, d: attn_case(1, 32, 8, 131072, 4, r, d),
     "append-64x8-2b": lambda r, d: append_case(64, 8, 4, r, d),
 }
 
