@@ -147,13 +147,6 @@ __global__ void __launch_bounds__(AttnCfg<GC, KSUB, VSUB>::WARPS * 32, 1) attn_s
         for (int p = 0; p < VJ / 16; ++p) cp_async16(vdst + parity * 32 * VJ + p * 16, vs + p * 16, nb);
         cp_async_commit();
     };
-    const uint32_t first = ts32 + warp * 32;
-    if (first < te32) issue_codes(first, 0);
-    RawByproducts k2n{0.f, 0u}, v2n{0.f, 0u};  // next batch's byproducts, still raw
-    if (first < te32) {  // warp-uniform
-        k2n = fetch_byproducts(ksrc, first + lane, first + lane < te32);
-        v2n = fetch_byproducts(vsrc, first + lane, first + lane < te32);
-    }
 
     // ---- segment prologue: rotated queries, q . o_K, LUT ----
     if (warp < GC) {
@@ -204,6 +197,18 @@ __global__ void __launch_bounds__(AttnCfg<GC, KSUB, VSUB>::WARPS * 32, 1) attn_s
         }
     }
     __syncthreads();
+    // Launched as a programmatic dependent (of the encode that appended to
+    // the caches, in a decode step): the prologue above reads only q, o_K and
+    // the codebook, so it overlaps that kernel; codes and scales are read
+    // after this wait.
+    asm volatile("griddepcontrol.wait;\n" ::: "memory");
+    const uint32_t first = ts32 + warp * 32;
+    if (first < te32) issue_codes(first, 0);
+    RawByproducts k2n{0.f, 0u}, v2n{0.f, 0u};  // next batch's byproducts, still raw
+    if (first < te32) {  // warp-uniform
+        k2n = fetch_byproducts(ksrc, first + lane, first + lane < te32);
+        v2n = fetch_byproducts(vsrc, first + lane, first + lane < te32);
+    }
 
     float gm[GC];
 #pragma unroll
@@ -591,8 +596,8 @@ template <int GC, int KSUB, int VSUB, typename QT>
 static cudaError_t launch_split(const AttnArgs& a, cudaStream_t s) {
     using S = AttnCfg<GC, KSUB, VSUB>;
     static std::atomic<unsigned long long> ready{0};
-    return launch_smem(attn_split_kernel<GC, KSUB, VSUB, QT>, ready, dim3(a.plan.ctas),
-                       dim3(S::WARPS * 32), S::bytes, s, a);
+    return launch_smem_pdl(attn_split_kernel<GC, KSUB, VSUB, QT>, ready, dim3(a.plan.ctas),
+                           dim3(S::WARPS * 32), S::bytes, s, a);
 }
 
 template <int GC, typename QT>

@@ -302,7 +302,10 @@ __global__ void __launch_bounds__(kTcThreads) nsn_encode_tc_kernel(EncodeArgs a)
 
     // Launched as a programmatic dependent of pass 1: the setup above
     // overlaps its end; the shift it derives is read only after this wait.
+    // A dependent attention kernel may then be scheduled (it waits for this
+    // grid before reading the codes).
     asm volatile("griddepcontrol.wait;\n" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
     const int l16 = lane & 15, half = lane >> 4;
     const int row = tid;  // = 32 * warp + lane: this thread's sub-vector row and TMEM lane
     const int64_t pairs_per_head = (a.T + 1) / 2;

@@ -264,7 +264,10 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
     __syncthreads();
     // Launched as a programmatic dependent of pass 1: the staging above
     // overlaps its end; the shift it derives is read only after this wait.
+    // The next kernel (decode attention over these caches) may then be
+    // scheduled; it waits for this grid before reading the codes.
     asm volatile("griddepcontrol.wait;\n" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
 
     // Each warp owns tiles of 16 consecutive token-heads of one (batch, head)
     // and keeps its own copy of that head's shift: no CTA barrier in the loop.

@@ -27,6 +27,9 @@ constexpr int kSmallThreads = 32;  // one warp (one token-head) per CTA: the CTA
 
 template <typename XT, int G, bool ADAPT, bool DQ>
 __global__ void __launch_bounds__(kSmallThreads) nsn_encode_small_kernel(EncodeArgs a) {
+    // a dependent attention kernel (a decode step's) may be scheduled now;
+    // it waits for this grid before reading the codes
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
     __shared__ __align__(16) double Cs[kNC * G];  // the codebook, converted once
     __shared__ __align__(16) float Cf[kNC * G];   // and as given
     for (int i = threadIdx.x; i < kNC * G; i += kSmallThreads) {
