@@ -182,7 +182,8 @@ nsnq_status nsnq_codebook_quantize4(const float* centroids, float* out, uint8_t*
  *   uint64 [1] sub-vectors whose code was decided on that path,
  *   uint64 [2] nonzero if cb.index was not built from cb.centroids,
  *   uint64 [3] used internally (work counter),
- *   uint64 [4] nonzero if a tensor-core scoring round (sub_dim 8) was not
+ *   uint64 [4] nonzero if a tensor-core scoring round (sub_dim 8, or 4 with
+ *              NSNQ_ENCODE_TC_SEARCH) was not
  *              seen complete within its bounded wait: the CTA that waited
  *              stopped, so some codes and scales of this call are NOT
  *              written and the call's result is void. The status returned
