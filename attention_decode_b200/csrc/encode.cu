@@ -11,10 +11,13 @@
 //                      o = sum / T (fp64, kept in the workspace for the
 //                      near-tie path) and its fp32 copy in the cache
 //   pass 2             NSN + FWHT + nearest codeword: encode_pruned.cu
-//                      (2 bit, search index) or encode1_tc.cu (1 bit, all
-//                      codewords scored on the tensor cores); calls of at
-//                      most kSmallEncode token-heads: encode_small.cu (one
-//                      warp per token-head, fp64)
+//                      (2 bit, search index) or encode1_tc.cu (1 bit, and
+//                      2 bit with the tensor-core search: all codewords
+//                      scored on the tensor cores); calls of at most
+//                      kSmallEncode token-heads: encode_small.cu (one warp
+//                      per token-head, fp32 scan, fp64 near ties)
+// Pass 2 is a programmatic dependent launch of pass 1 (pass 1 triggers its
+// dependents first; pass 2 stages its tables, then waits for the shift).
 #include <math.h>
 
 #include "common.cuh"
