@@ -76,3 +76,29 @@ def test_captured_step_equals_eager(codebooks, kind):
     assert torch.equal(ke.scales, kg.scales) and torch.equal(ve.scales, vg.scales)
     assert torch.equal(ke.shift, kg.shift) and torch.equal(ve.shift, vg.shift)
     assert torch.equal(outs["eager"], outs["graph"])
+
+
+@pytest.mark.parametrize("order,T", [("vk", 3000), ("vk", 100), ("kv", 100)])
+def test_attention_right_after_either_encode(codebooks, order, T):
+    """Attention launched right after the encode of K (V encoded before it),
+    or after a small-call encode: the attention kernel starts under the
+    encode (programmatic dependent launch) and must still read the finished
+    caches. Compared with the same attention after a device synchronize."""
+    B, H = 2, 4
+    cb = P.codebook(codebooks[4])
+    k, v = _kv(B, H, T, seed=31)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(32)
+    q = torch.randn(B, 4 * H, D, generator=gen, device="cuda").to(torch.bfloat16)
+    seq = torch.full((B,), T, dtype=torch.int32, device="cuda")
+    kc = nsnq.Cache.empty(B, H, T, 4)
+    vc = nsnq.Cache.empty(B, H, T, 4)
+    cb._c()
+    first, second = ((v, vc), (k, kc)) if order == "vk" else ((k, kc), (v, vc))
+    nsnq.nsnq_encode(first[0], cb, first[1])
+    nsnq.nsnq_encode(second[0], cb, second[1])
+    out = nsnq.nsnq_attn_decode(q, kc, vc, cb, cb, seq, T, Hkv=H, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    ref = nsnq.nsnq_attn_decode(q, kc, vc, cb, cb, seq, T, Hkv=H, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
