@@ -10,7 +10,7 @@ GPU codes must equal the oracle's fp64 argmin of the same fp32 input except
 where the oracle's own relative gap is below the 1e-6 tie rule; with offsets
 on both sides of that rule this exercises the fp32 decision, the near-tie
 band and the fp64 re-decision of every encode path (small calls, the 2-bit
-indexed walk, the 1-bit tensor-core scores)."""
+indexed walk, the 1-bit and 2-bit tensor-core scores)."""
 import numpy as np
 import pytest
 import scipy.linalg
@@ -79,11 +79,12 @@ def _near_tie_tokens(C: np.ndarray, n_tok: int, seed: int):
     return np.asarray(xs, dtype=np.float32), o.astype(np.float32)
 
 
-@pytest.mark.parametrize("g", [4, 8])
-@pytest.mark.parametrize("T", [1, 1500])
-def test_encode_near_voronoi_boundaries(codebooks, g, T):
+@pytest.mark.parametrize("g,tc,T", [(4, False, 1), (8, False, 1), (4, False, 1500),
+                                      (8, False, 1500), (4, True, 1500)])
+def test_encode_near_voronoi_boundaries(codebooks, g, tc, T):
     """T = 1: one token per (sequence, head), a decode step's appends (small
-    calls); T = 1500: the persistent 2-bit walk or 1-bit tensor-core kernel."""
+    calls); T = 1500: the persistent 2-bit walk, the 1-bit tensor-core kernel
+    or (tc) the 2-bit tensor-core search."""
     C = codebooks[g]
     B, H = (1, 512) if T == 1 else (1, 2)
     n = B * H * T
@@ -93,7 +94,8 @@ def test_encode_near_voronoi_boundaries(codebooks, g, T):
     ora = O.encode(x.astype(np.float64), C, shift=shift.astype(np.float64), want_w=True)
     cache = nsnq.Cache.empty(B, H, T, g)
     cache.shift.copy_(torch.from_numpy(shift))
-    ws = nsnq.nsnq_encode(P.to_dev(x, "f32"), P.codebook(C), cache, shift_mode=nsnq.SHIFT_GIVEN)
+    ws = nsnq.nsnq_encode(P.to_dev(x, "f32"), P.codebook(C), cache, shift_mode=nsnq.SHIFT_GIVEN,
+                          flags=nsnq.ENCODE_TC_SEARCH if tc else nsnq.ENCODE_DEFAULT)
     torch.cuda.synchronize()
     n_mis, n_bad, worst = P.code_report(cache.codes.cpu().numpy(), ora["codes"], ora["w"], C)
     assert n_bad == 0, (n_mis, worst)
