@@ -9,6 +9,7 @@ CPU fallback: if the library is missing, loading raises.
     cache = Cache.empty(B, H, cap, sub_dim=cb.sub_dim, device="cuda")
     nsnq_encode(x, cb, cache)                      # prompt: shift computed
     nsnq_encode(x_new, cb, cache, t_offset=T, shift_mode=SHIFT_GIVEN)
+    nsnq_encode_kv(k, v, cb, k_cache, v_cache)     # keys and values in one call
     out = nsnq_attn_decode(q, k_cache, v_cache, k_cb, v_cb, seq_lens, max_len)
 
 With a full-precision residual window of R recent tokens (DecodeCache does
@@ -43,7 +44,7 @@ EXPORTED = ("nsnq_status_string", "nsnq_last_error", "nsnq_codebook_index_bytes"
             "nsnq_codebook_index_build", "nsnq_encode_workspace", "nsnq_encode", "nsnq_dequant",
             "nsnq_attn_workspace", "nsnq_attn_decode", "nsnq_attn_decode_res",
             "nsnq_attn_decode_rope", "nsnq_residual_write", "nsnq_attn_decode_noalloc",
-            "nsnq_codebook_quantize4")
+            "nsnq_codebook_quantize4", "nsnq_encode_kv_workspace", "nsnq_encode_kv")
 
 
 class NSNQError(RuntimeError):
@@ -94,6 +95,11 @@ def load(path: str = LIB_PATH):
     L.nsnq_encode.argtypes = [vp, ci, ci, ci, i64, ci, i64, i64, i64, i64, ci, ctypes.c_uint,
                               _Codebook, _Cache, vp, sz, vp]
     L.nsnq_encode.restype = ci
+    L.nsnq_encode_kv_workspace.argtypes = [ci, ci, i64, ci]
+    L.nsnq_encode_kv_workspace.restype = sz
+    L.nsnq_encode_kv.argtypes = [vp, vp, ci, ci, ci, i64, ci, i64, i64, i64, i64, ci, ctypes.c_uint,
+                                 _Codebook, _Cache, _Cache, vp, sz, vp]
+    L.nsnq_encode_kv.restype = ci
     L.nsnq_dequant.argtypes = [_Cache, _Codebook, ci, ci, i64, i64, ci, vp, vp]
     L.nsnq_dequant.restype = ci
     L.nsnq_attn_workspace.argtypes = [ci, ci, ci, ci, i64]
@@ -289,6 +295,31 @@ def nsnq_encode(x: torch.Tensor, cb: Codebook, cache: Cache, t_offset: int = 0,
     return workspace
 
 
+def nsnq_encode_kv_workspace(B: int, H: int, T: int, D: int = HEAD_DIM) -> int:
+    return int(load().nsnq_encode_kv_workspace(B, H, T, D))
+
+
+def nsnq_encode_kv(k: torch.Tensor, v: torch.Tensor, cb: Codebook, k_cache: Cache, v_cache: Cache,
+                   t_offset: int = 0, shift_mode: int = SHIFT_COMPUTE,
+                   workspace: Optional[torch.Tensor] = None, stream=None,
+                   flags: int = ENCODE_DEFAULT) -> torch.Tensor:
+    """nsnq_encode of keys k and values v (same shape, dtype and strides) with
+    one codebook, in one call: both tensors share the call's launches.
+    Returns the workspace (its counters cover both tensors)."""
+    B, H, T, D = k.shape
+    if tuple(v.shape) != (B, H, T, D) or v.dtype != k.dtype or v.stride() != k.stride():
+        raise ValueError("k and v must have the same shape, dtype and strides")
+    if k.stride(3) != 1:
+        raise ValueError("k and v must have contiguous channels")
+    if workspace is None:
+        workspace = _workspace(nsnq_encode_kv_workspace(B, H, T, D), k.device)
+    _check(load().nsnq_encode_kv(_ptr(k), _ptr(v), _dtype_code(k), B, H, T, D, k.stride(0),
+                                 k.stride(1), k.stride(2), t_offset, shift_mode, flags, cb._c(),
+                                 k_cache._c(), v_cache._c(), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream)))
+    return workspace
+
+
 EncodeStats = collections.namedtuple(
     "EncodeStats", ("fp64_token_heads", "fp64_subvectors", "index_mismatch", "mma_timeout"))
 EncodeStats.__doc__ = """Counters of the last nsnq_encode that used a workspace (its first 64
@@ -443,11 +474,21 @@ class DecodeCache:
         if self._prefilled:
             raise RuntimeError("prefill() was already called")
         T = int(k.shape[2])
-        nsnq_encode(k, self.k_cb, self.k, stream=stream, flags=self.flags)
-        nsnq_encode(v, self.v_cb, self.v, stream=stream, flags=self.flags)
+        self._encode(k, v, 0, SHIFT_COMPUTE, stream)
         self.n_quant = T
         self.seq_lens.fill_(T)
         self._prefilled = True
+
+    def _encode(self, k: torch.Tensor, v: torch.Tensor, t_offset: int, mode: int, stream):
+        # one call for both caches when they share a codebook and the inputs a layout
+        if self.k_cb is self.v_cb and v.dtype == k.dtype and v.stride() == k.stride():
+            nsnq_encode_kv(k, v, self.k_cb, self.k, self.v, t_offset=t_offset, shift_mode=mode,
+                           stream=stream, flags=self.flags)
+        else:
+            nsnq_encode(k, self.k_cb, self.k, t_offset=t_offset, shift_mode=mode, stream=stream,
+                        flags=self.flags)
+            nsnq_encode(v, self.v_cb, self.v, t_offset=t_offset, shift_mode=mode, stream=stream,
+                        flags=self.flags)
 
     def append(self, k_new: torch.Tensor, v_new: torch.Tensor, stream=None):
         """k_new, v_new [B][Hkv][D] or [B][Hkv][1][D]: one token per sequence."""
@@ -469,10 +510,7 @@ class DecodeCache:
         if self.n_quant + self.n_res > self.k.cap:
             raise RuntimeError("quantized cache is full")
         n = self.n_res
-        nsnq_encode(self.res.k[:, :, :n], self.k_cb, self.k, t_offset=self.n_quant,
-                    shift_mode=SHIFT_GIVEN, stream=stream, flags=self.flags)
-        nsnq_encode(self.res.v[:, :, :n], self.v_cb, self.v, t_offset=self.n_quant,
-                    shift_mode=SHIFT_GIVEN, stream=stream, flags=self.flags)
+        self._encode(self.res.k[:, :, :n], self.res.v[:, :, :n], self.n_quant, SHIFT_GIVEN, stream)
         self.n_quant += n
         self.n_res = 0
         self.seq_lens.fill_(self.n_quant)

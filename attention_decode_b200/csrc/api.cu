@@ -147,10 +147,33 @@ size_t nsnq_encode_workspace(int B, int H, int64_t T, int D) {
     return nsnq::plan_encode(B, H, T).total;
 }
 
-nsnq_status nsnq_encode(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t T, int D,
-                        int64_t stride_b, int64_t stride_h, int64_t stride_t, int64_t t_offset,
-                        nsnq_shift_mode mode, unsigned flags, nsnq_codebook cb, nsnq_cache cache,
-                        void* workspace, size_t workspace_bytes, nsnq_stream stream) {
+namespace {
+
+// Checks of one tensor's cache for an encode call (shared by both entry points).
+nsnq_status check_encode_cache(const nsnq_cache& cache, const char* name, bool dq, int64_t T,
+                               int64_t t_offset) {
+    if (dq && (!cache.s1_grid || !aligned(cache.s1_grid, 8)))
+        return fail(NSNQ_ERR_INVALID_ARG, "double quantization needs %s.s1_grid (8-byte aligned)", name);
+    if (cache.s1_levels && !dq)
+        return fail(NSNQ_ERR_INVALID_ARG,
+                    "a packed cache (%s.s1_levels) holds double-quantized s1 only: pass "
+                    "NSNQ_ENCODE_DOUBLE_QUANT", name);
+    nsnq_status s = check_cache(cache, name, true);
+    if (s != NSNQ_OK) return s;
+    if (t_offset < 0 || t_offset > cache.cap || T > cache.cap - t_offset)
+        return fail(NSNQ_ERR_INVALID_ARG, "positions [%lld, %lld) exceed %s capacity %lld",
+                    (long long)t_offset, (long long)(t_offset + T), name, (long long)cache.cap);
+    return NSNQ_OK;
+}
+
+// One tensor (x2 == NULL) or two of one shape sharing every launch: the
+// second tensor's heads follow the first's as batches [B, 2B) of the grid.
+nsnq_status encode_impl(const void* x, const void* x2, nsnq_dtype x_dtype, int B, int H, int64_t T,
+                        int D, int64_t stride_b, int64_t stride_h, int64_t stride_t,
+                        int64_t t_offset, nsnq_shift_mode mode, unsigned flags, nsnq_codebook cb,
+                        const nsnq_cache& cache, const nsnq_cache* cache2, void* workspace,
+                        size_t workspace_bytes, nsnq_stream stream) {
+    const bool pair = cache2 != nullptr;
     if (D != nsnq::kHeadDim) return fail(NSNQ_ERR_UNSUPPORTED, "D = %d (only 128 is supported)", D);
     if (x_dtype != NSNQ_F32 && x_dtype != NSNQ_BF16)
         return fail(NSNQ_ERR_UNSUPPORTED, "x_dtype = %d", (int)x_dtype);
@@ -159,15 +182,10 @@ nsnq_status nsnq_encode(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t
     if (flags & ~(unsigned)(NSNQ_ENCODE_ADAPTIVE_SCALE | NSNQ_ENCODE_DOUBLE_QUANT | NSNQ_ENCODE_TC_SEARCH))
         return fail(NSNQ_ERR_INVALID_ARG, "unknown encode flags 0x%x", flags);
     const bool dq = (flags & NSNQ_ENCODE_DOUBLE_QUANT) != 0;
-    if (dq && (!cache.s1_grid || !aligned(cache.s1_grid, 8)))
-        return fail(NSNQ_ERR_INVALID_ARG, "double quantization needs cache.s1_grid (8-byte aligned)");
-    if (cache.s1_levels && !dq)
-        return fail(NSNQ_ERR_INVALID_ARG,
-                    "a packed cache (s1_levels) holds double-quantized s1 only: pass "
-                    "NSNQ_ENCODE_DOUBLE_QUANT");
     if (B < 0 || H < 0 || T < 0)
         return fail(NSNQ_ERR_INVALID_ARG, "negative size B=%d H=%d T=%lld", B, H, (long long)T);
-    if (B > 65535 || H > 65535) return fail(NSNQ_ERR_UNSUPPORTED, "B or H above 65535");
+    if (B > (pair ? 32767 : 65535) || H > 65535)
+        return fail(NSNQ_ERR_UNSUPPORTED, "B or H above %s", pair ? "32767 / 65535" : "65535");
     nsnq_status s = check_codebook(cb, "cb");
     if (s != NSNQ_OK) return s;
     const bool tc_search = (flags & NSNQ_ENCODE_TC_SEARCH) != 0;
@@ -175,19 +193,27 @@ nsnq_status nsnq_encode(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t
         return fail(NSNQ_ERR_INVALID_ARG,
                     "cb.index is NULL or misaligned: build it with nsnq_codebook_index_build "
                     "(or pass NSNQ_ENCODE_TC_SEARCH)");
-    s = check_cache(cache, "cache", true);
+    s = check_encode_cache(cache, pair ? "cache_k" : "cache", dq, T, t_offset);
     if (s != NSNQ_OK) return s;
-    if (t_offset < 0 || t_offset > cache.cap || T > cache.cap - t_offset)
-        return fail(NSNQ_ERR_INVALID_ARG, "positions [%lld, %lld) exceed cache capacity %lld",
-                    (long long)t_offset, (long long)(t_offset + T), (long long)cache.cap);
+    if (pair) {
+        s = check_encode_cache(*cache2, "cache_v", dq, T, t_offset);
+        if (s != NSNQ_OK) return s;
+        if (cache2->cap != cache.cap)
+            return fail(NSNQ_ERR_INVALID_ARG, "cache_k.cap = %lld and cache_v.cap = %lld differ",
+                        (long long)cache.cap, (long long)cache2->cap);
+        if ((cache2->s1_levels != nullptr) != (cache.s1_levels != nullptr))
+            return fail(NSNQ_ERR_INVALID_ARG, "cache_k and cache_v must both be packed or both not");
+    }
     if (B == 0 || H == 0 || T == 0) return ok();
-    if (!x) return fail(NSNQ_ERR_INVALID_ARG, "x is NULL");
+    if (!x || (pair && !x2)) return fail(NSNQ_ERR_INVALID_ARG, "%s is NULL", pair ? "x_k or x_v" : "x");
     const int64_t esz = x_dtype == NSNQ_BF16 ? 2 : 4;
-    if (!aligned(x, 16) || (stride_b * esz) % 16 || (stride_h * esz) % 16 || (stride_t * esz) % 16)
+    if (!aligned(x, 16) || (pair && !aligned(x2, 16)) || (stride_b * esz) % 16 || (stride_h * esz) % 16 ||
+        (stride_t * esz) % 16)
         return fail(NSNQ_ERR_INVALID_ARG, "x and its strides must be 16-byte aligned");
     if (stride_b < 0 || stride_h < 0 || stride_t < D)
         return fail(NSNQ_ERR_INVALID_ARG, "strides must be non-negative with stride_t >= D");
-    const nsnq::EncodePlan plan = nsnq::plan_encode(B, H, T);
+    const int Bg = pair ? 2 * B : B;  // batches of the grid
+    const nsnq::EncodePlan plan = nsnq::plan_encode(Bg, H, T);
     if (!workspace || workspace_bytes < plan.total)
         return fail(NSNQ_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", plan.total,
                     workspace ? workspace_bytes : (size_t)0);
@@ -197,7 +223,7 @@ nsnq_status nsnq_encode(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t
     nsnq::EncodeArgs a{};
     a.x = x;
     a.x_bf16 = x_dtype == NSNQ_BF16;
-    a.B = B; a.H = H; a.T = T;
+    a.B = Bg; a.H = H; a.T = T;
     a.sb = stride_b; a.sh = stride_h; a.st = stride_t;
     a.t_offset = t_offset;
     a.given_shift = mode == NSNQ_SHIFT_GIVEN;
@@ -210,6 +236,11 @@ nsnq_status nsnq_encode(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t
     a.tc_search = tc_search ? 1 : 0;
     a.codes = cache.codes; a.scales = cache.scales; a.shift = cache.shift; a.cap = cache.cap;
     a.s1_levels = cache.s1_levels;
+    a.B1 = B;
+    const nsnq_cache& c2 = pair ? *cache2 : cache;
+    a.x2 = pair ? x2 : x;
+    a.codes2 = c2.codes; a.scales2 = c2.scales; a.shift2 = c2.shift;
+    a.s1_levels2 = c2.s1_levels; a.s1_grid2 = c2.s1_grid;
     char* ws = static_cast<char*>(workspace);
     a.stats = reinterpret_cast<unsigned long long*>(ws);
     a.partial = reinterpret_cast<double*>(ws + plan.partial_off);
@@ -221,12 +252,36 @@ nsnq_status nsnq_encode(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     // A small shift-given call (a decode step's appends) uses no counter: its
     // kernel zeroes the stats block itself, which saves the memset.
-    a.zero_stats = a.given_shift && (int64_t)B * H * T <= nsnq::kSmallEncode;
+    a.zero_stats = a.given_shift && (int64_t)Bg * H * T <= nsnq::kSmallEncode;
     cudaError_t e = a.zero_stats ? cudaSuccess : cudaMemsetAsync(ws, 0, plan.reset_bytes, st);
     if (e != cudaSuccess) return cuda_fail(e, "workspace reset");
     e = nsnq::launch_encode(a, st);
     if (e != cudaSuccess) return cuda_fail(e, "encode launch");
     return ok();
+}
+
+}  // namespace
+
+nsnq_status nsnq_encode(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t T, int D,
+                        int64_t stride_b, int64_t stride_h, int64_t stride_t, int64_t t_offset,
+                        nsnq_shift_mode mode, unsigned flags, nsnq_codebook cb, nsnq_cache cache,
+                        void* workspace, size_t workspace_bytes, nsnq_stream stream) {
+    return encode_impl(x, nullptr, x_dtype, B, H, T, D, stride_b, stride_h, stride_t, t_offset, mode,
+                       flags, cb, cache, nullptr, workspace, workspace_bytes, stream);
+}
+
+size_t nsnq_encode_kv_workspace(int B, int H, int64_t T, int D) {
+    if (B < 0 || B > 32767 || H < 0 || T < 0 || D != nsnq::kHeadDim) return 0;
+    return nsnq::plan_encode(2 * B, H, T).total;
+}
+
+nsnq_status nsnq_encode_kv(const void* x_k, const void* x_v, nsnq_dtype x_dtype, int B, int H,
+                           int64_t T, int D, int64_t stride_b, int64_t stride_h, int64_t stride_t,
+                           int64_t t_offset, nsnq_shift_mode mode, unsigned flags, nsnq_codebook cb,
+                           nsnq_cache cache_k, nsnq_cache cache_v, void* workspace,
+                           size_t workspace_bytes, nsnq_stream stream) {
+    return encode_impl(x_k, x_v, x_dtype, B, H, T, D, stride_b, stride_h, stride_t, t_offset, mode,
+                       flags, cb, cache_k, &cache_v, workspace, workspace_bytes, stream);
 }
 
 nsnq_status nsnq_dequant(nsnq_cache cache, nsnq_codebook cb, int B, int H, int64_t t0, int64_t T,

@@ -78,7 +78,7 @@ __global__ void __launch_bounds__(kStatsThreads, 4) nsn_s1minmax_kernel(EncodeAr
     const int tk = lane >> 4, cg = lane & 15;
     const int64_t t0 = (int64_t)chunk * a.chunk1;
     const int64_t t1 = min(t0 + a.chunk1, a.T);
-    const XT* xb = reinterpret_cast<const XT*>(a.x) + b * a.sb + h * a.sh + 8 * cg;
+    const XT* xb = enc_head<XT>(a, b, h) + 8 * cg;
     constexpr int64_t kStride = 2 * (kStatsThreads / 32);  // tokens per CTA step
     constexpr int kDepth = stats_depth<XT>();
     Raw8<XT> buf[kDepth];
@@ -133,6 +133,8 @@ __global__ void __launch_bounds__(kStatsThreads, 4) nsn_s1minmax_kernel(EncodeAr
 template <bool DQ>
 __device__ void shift_of_head(const EncodeArgs& a, int64_t bh, double (*red)[kD]) {
     const int c = threadIdx.x;
+    const bool sec = enc_second(a, bh);
+    const int64_t cbh = enc_cbh(a, bh);
     double o = 0.0;
     if (c < kD) {
         double s = 0.0;
@@ -157,13 +159,14 @@ __device__ void shift_of_head(const EncodeArgs& a, int64_t bh, double (*red)[kD]
         if (c == 0) {
             double lo, st;
             dq_grid_from_chunks(a.minmax + bh * a.nchunk1 * 2, a.nchunk1, lo, st);
-            a.s1_grid[2 * bh] = (float)lo;
-            a.s1_grid[2 * bh + 1] = (float)st;
+            float* grid = enc_s1_grid(a, sec);
+            grid[2 * cbh] = (float)lo;
+            grid[2 * cbh + 1] = (float)st;
         }
     }
     if (c < kD) {
         a.o64[bh * kD + c] = o;
-        a.shift[bh * kD + c] = (float)o;
+        enc_shift(a, sec)[cbh * kD + c] = (float)o;
     }
 }
 
@@ -178,7 +181,7 @@ __global__ void __launch_bounds__(kStatsThreads, 4) nsn_stats_kernel(EncodeArgs 
     const int tk = lane >> 4, cg = lane & 15;
     const int64_t t0 = (int64_t)chunk * a.chunk1;
     const int64_t t1 = min(t0 + a.chunk1, a.T);
-    const XT* xb = reinterpret_cast<const XT*>(a.x) + b * a.sb + h * a.sh + 8 * cg;
+    const XT* xb = enc_head<XT>(a, b, h) + 8 * cg;
     const double sqrt_d = sqrt((double)kD);
     constexpr int64_t kStride = 2 * (kStatsThreads / 32);  // tokens per CTA step
     double glo = 0.0, gstep = 0.0;

@@ -322,7 +322,7 @@ __global__ void __launch_bounds__(kTcThreads) nsn_encode_tc_kernel(EncodeArgs a)
         const int64_t t = t0 + half;
         const int b = (int)(bh / a.H), h = (int)(bh - (int64_t)b * a.H);
         const bool valid = wvalid && t < a.T;
-        const XT* xhead = reinterpret_cast<const XT*>(a.x) + b * a.sb + h * a.sh;
+        const XT* xhead = enc_head<XT>(a, b, h);
         float v[8];
         if (valid) {
             load8<XT>(xhead + t * a.st + 8 * l16, v);
@@ -346,12 +346,13 @@ __global__ void __launch_bounds__(kTcThreads) nsn_encode_tc_kernel(EncodeArgs a)
 #pragma unroll
             for (int m = 1; m < 16; m <<= 1) ss64 += __shfl_xor_sync(kFull, ss64, m);
             double glo, gstep;
-            dq_grid(a.s1_grid, bh, glo, gstep);
+            dq_grid(enc_s1_grid(a, enc_second(a, bh)), enc_cbh(a, bh), glo, gstep);
             s1dq = dq_s1(sqrt(ss64) / sqrt((double)kD), glo, gstep, &s1lev);
             s1 = (float)s1dq;
             inv1 = s1dq > 0.0 ? (float)(1.0 / s1dq) : 0.f;
         }
-        const float4* o4 = reinterpret_cast<const float4*>(a.shift + bh * kD + 8 * l16);
+        const float* shift_h = enc_shift(a, enc_second(a, bh)) + enc_cbh(a, bh) * kD;
+        const float4* o4 = reinterpret_cast<const float4*>(shift_h + 8 * l16);
         const float4 oa = o4[0], ob = o4[1];
         const float o[8] = {oa.x, oa.y, oa.z, oa.w, ob.x, ob.y, ob.z, ob.w};
         float ss2 = 0.f;
@@ -534,8 +535,9 @@ __global__ void __launch_bounds__(kTcThreads) nsn_encode_tc_kernel(EncodeArgs a)
                 for (int k = 0; k < NW; ++k) cq[k] = __shfl_sync(kFull, cw[k], 16 * hh);
                 double s1d, s2d, wq64;
                 const double s1f = __shfl_sync(kFull, s1dq, 16 * hh);
-                exact_warp_tc<XT, SUB>(xhead + (t0 + hh) * a.st, o64, a.shift + bh * kD, Cs, flags, cq, s1f,
-                                       s1d, s2d, wq64);
+                exact_warp_tc<XT, SUB>(xhead + (t0 + hh) * a.st, o64,
+                                       enc_shift(a, enc_second(a, bh)) + enc_cbh(a, bh) * kD, Cs, flags,
+                                       cq, s1f, s1d, s2d, wq64);
                 if (half == hh) {
 #pragma unroll
                     for (int k = 0; k < NW; ++k) cw[k] = cq[k];
@@ -553,11 +555,14 @@ __global__ void __launch_bounds__(kTcThreads) nsn_encode_tc_kernel(EncodeArgs a)
             if (wqd > 0.0) s2o = (float)((double)s2o * ((double)kD / wqd));
         }
         if (valid && l16 == 0) {
-            const int64_t orow = bh * a.cap + a.t_offset + t;
-            uint4* dst = reinterpret_cast<uint4*>(a.codes + orow * (4 * NW));
+            const bool sec = enc_second(a, bh);
+            const int64_t cbh = enc_cbh(a, bh);
+            const int64_t orow = cbh * a.cap + a.t_offset + t;
+            uint4* dst = reinterpret_cast<uint4*>(enc_codes(a, sec) + orow * (4 * NW));
 #pragma unroll
             for (int k = 0; k < NW / 4; ++k) dst[k] = make_uint4(cw[4 * k], cw[4 * k + 1], cw[4 * k + 2], cw[4 * k + 3]);
-            store_byproducts(a.scales, a.s1_levels, bh, a.cap, a.t_offset + t, s1o, s2o, s1lev);
+            store_byproducts(enc_scales(a, sec), enc_s1_levels(a, sec), cbh, a.cap, a.t_offset + t, s1o,
+                             s2o, s1lev);
         }
     }
     // ---- release TMEM (after every thread's last read; after the last MMA) ----

@@ -290,15 +290,15 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
         const int b = (int)(bh / a.H), h = (int)(bh - (int64_t)b * a.H);
         if (bh != cur_bh) {  // warp-uniform
             __syncwarp();
-            const float4 o = reinterpret_cast<const float4*>(a.shift + bh * kD)[lane];
+            const float4 o =
+                reinterpret_cast<const float4*>(enc_shift(a, enc_second(a, bh)) + enc_cbh(a, bh) * kD)[lane];
             reinterpret_cast<float4*>(wshift)[lane + (lane >= 16 ? 1 : 0)] =
                 make_float4(-o.x, -o.y, -o.z, -o.w);  // -o: the shift is subtracted
             __syncwarp();
             cur_bh = bh;
         }
         const bool valid = t < a.T;
-        const XT* xrow = reinterpret_cast<const XT*>(a.x) + b * a.sb + h * a.sh +
-                         (valid ? t : 0) * a.st;
+        const XT* xrow = enc_head<XT>(a, b, h) + (valid ? t : 0) * a.st;
         float v[64];
         if (valid) {
             load64<XT>(xrow + 64 * half, v);
@@ -327,7 +327,7 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
             for (int k = 0; k < 64; ++k) ss64 = fma((double)v[k], (double)v[k], ss64);
             ss64 += __shfl_xor_sync(kFull, ss64, 1);
             double glo, gstep;
-            dq_grid(a.s1_grid, bh, glo, gstep);
+            dq_grid(enc_s1_grid(a, enc_second(a, bh)), enc_cbh(a, bh), glo, gstep);
             s1dq = dq_s1(sqrt(ss64) / sqrt((double)kD), glo, gstep, &s1lev);
             s1 = (float)s1dq;
             inv1 = s1dq > 0.0 ? (float)(1.0 / s1dq) : 0.f;
@@ -407,7 +407,7 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
         uint32_t pending = __ballot_sync(kFull, both != 0u && half == 0);
         if (pending) {
             const double* o64 = a.given_shift ? nullptr : a.o64 + bh * kD;
-            const XT* xhead = reinterpret_cast<const XT*>(a.x) + b * a.sb + h * a.sh;
+            const XT* xhead = enc_head<XT>(a, b, h);
             const int64_t t0 = t - (lane >> 1);  // first token of the tile
             while (pending) {
                 const int src = __ffs(pending) - 1;  // even lane of the token-head's pair
@@ -424,7 +424,8 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
                 double s1d, s2d, wq_all, wq_delta;
                 const double s1f = __shfl_sync(kFull, s1dq, src);
                 const int code = exact_warp<XT>(xhead + (t0 + (src >> 1)) * a.st, o64,
-                                                a.shift + bh * kD, reps, offs, ents, flags,
+                                                enc_shift(a, enc_second(a, bh)) + enc_cbh(a, bh) * kD,
+                                                reps, offs, ents, flags,
                                                 old_code, s1f, s1d, s2d, wq_all, wq_delta);
                 const bool mine = (lane >> 1) == (src >> 1);
 #pragma unroll
@@ -449,11 +450,14 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
             if (wqd > 0.0) s2o = (float)((double)s2o * ((double)kD / wqd));
         }
         if (valid) {
-            const int64_t row = bh * a.cap + a.t_offset + t;
-            reinterpret_cast<uint4*>(a.codes + row * 32)[half] =
+            const bool sec = enc_second(a, bh);
+            const int64_t cbh = enc_cbh(a, bh);
+            const int64_t row = cbh * a.cap + a.t_offset + t;
+            reinterpret_cast<uint4*>(enc_codes(a, sec) + row * 32)[half] =
                 make_uint4(codes[0], codes[1], codes[2], codes[3]);
             if (half == 0)
-                store_byproducts(a.scales, a.s1_levels, bh, a.cap, a.t_offset + t, s1o, s2o, s1lev);
+                store_byproducts(enc_scales(a, sec), enc_s1_levels(a, sec), cbh, a.cap, a.t_offset + t,
+                                 s1o, s2o, s1lev);
         }
     }
 }

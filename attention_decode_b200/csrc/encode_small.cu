@@ -43,7 +43,9 @@ __global__ void __launch_bounds__(kSmallThreads) nsn_encode_small_kernel(EncodeA
     if (th >= (int64_t)a.B * a.H * a.T) return;  // warp-uniform
     const int64_t bh = th / a.T, t = th - bh * a.T;
     const int b = (int)(bh / a.H), h = (int)(bh - (int64_t)b * a.H);
-    const XT* xtok = reinterpret_cast<const XT*>(a.x) + b * a.sb + h * a.sh + t * a.st;
+    const bool sec = enc_second(a, bh);
+    const int64_t cbh = enc_cbh(a, bh);
+    const XT* xtok = enc_head<XT>(a, b, h) + t * a.st;
 
     // ---- NSN in fp64 ----
     float xf[4];
@@ -52,7 +54,8 @@ __global__ void __launch_bounds__(kSmallThreads) nsn_encode_small_kernel(EncodeA
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
         x[r] = (double)xf[r];
-        o[r] = a.given_shift ? (double)a.shift[bh * kD + 4 * lane + r] : a.o64[bh * kD + 4 * lane + r];
+        o[r] = a.given_shift ? (double)enc_shift(a, sec)[cbh * kD + 4 * lane + r]
+                             : a.o64[bh * kD + 4 * lane + r];
     }
     const double sqrt_d = sqrt((double)kD);
     const double ss = warp_sum_d(x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3]);
@@ -60,7 +63,7 @@ __global__ void __launch_bounds__(kSmallThreads) nsn_encode_small_kernel(EncodeA
     int s1lev = 0;
     if constexpr (DQ) {
         double glo, gstep;
-        dq_grid(a.s1_grid, bh, glo, gstep);
+        dq_grid(enc_s1_grid(a, sec), cbh, glo, gstep);
         s1 = dq_s1(s1, glo, gstep, &s1lev);
     }
     const double inv1 = s1 > 0.0 ? 1.0 / s1 : 0.0;
@@ -180,9 +183,11 @@ __global__ void __launch_bounds__(kSmallThreads) nsn_encode_small_kernel(EncodeA
         q = warp_sum_d(q);
         if (q > 0.0) s2o = (float)((double)s2o * ((double)kD / q));
     }
-    const int64_t orow = bh * a.cap + a.t_offset + t;
-    if (G == 4 || lane < 16) a.codes[orow * (kD / G) + j] = (uint8_t)bi;
-    if (lane == 0) store_byproducts(a.scales, a.s1_levels, bh, a.cap, a.t_offset + t, s1o, s2o, s1lev);
+    const int64_t orow = cbh * a.cap + a.t_offset + t;
+    if (G == 4 || lane < 16) enc_codes(a, sec)[orow * (kD / G) + j] = (uint8_t)bi;
+    if (lane == 0)
+        store_byproducts(enc_scales(a, sec), enc_s1_levels(a, sec), cbh, a.cap,
+                         a.t_offset + t, s1o, s2o, s1lev);
 }
 
 template <typename XT, int G>

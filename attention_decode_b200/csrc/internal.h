@@ -115,7 +115,52 @@ struct EncodeArgs {
     int zero_stats;             // the pass-2 kernel zeroes stats (no memset before the call)
     int nchunk1;
     int64_t chunk1;
+    // Two tensors in one call (keys and values, nsnq_encode_kv): batches
+    // [0, B1) of the grid are the first tensor (x, codes, ...), [B1, B) the
+    // second (x2, codes2, ...), B = 2 B1. The workspace is indexed by the
+    // grid's (b, h); the caches by the tensor's own. One tensor: B1 = B.
+    int B1;
+    const void* x2;
+    uint8_t* codes2;
+    float* scales2;
+    float* shift2;
+    uint32_t* s1_levels2;
+    float* s1_grid2;
 };
+
+#ifdef __CUDACC__
+// Grid head bh = b * H + h (b < B) belongs to the second tensor when
+// b >= B1; its cache row block is then bh - B1 * H.
+__device__ __forceinline__ bool enc_second(const EncodeArgs& a, int64_t bh) {
+    return bh >= (int64_t)a.B1 * a.H;
+}
+__device__ __forceinline__ int64_t enc_cbh(const EncodeArgs& a, int64_t bh) {
+    return enc_second(a, bh) ? bh - (int64_t)a.B1 * a.H : bh;
+}
+// First element of head (b, h) of the tensor that grid batch b belongs to.
+template <typename XT>
+__device__ __forceinline__ const XT* enc_head(const EncodeArgs& a, int b, int h) {
+    const bool sec = b >= a.B1;
+    return reinterpret_cast<const XT*>(sec ? a.x2 : a.x) + (int64_t)(sec ? b - a.B1 : b) * a.sb +
+           (int64_t)h * a.sh;
+}
+// The cache arrays of the tensor selected by `sec`.
+__device__ __forceinline__ uint8_t* enc_codes(const EncodeArgs& a, bool sec) {
+    return sec ? a.codes2 : a.codes;
+}
+__device__ __forceinline__ float* enc_scales(const EncodeArgs& a, bool sec) {
+    return sec ? a.scales2 : a.scales;
+}
+__device__ __forceinline__ float* enc_shift(const EncodeArgs& a, bool sec) {
+    return sec ? a.shift2 : a.shift;
+}
+__device__ __forceinline__ uint32_t* enc_s1_levels(const EncodeArgs& a, bool sec) {
+    return sec ? a.s1_levels2 : a.s1_levels;
+}
+__device__ __forceinline__ float* enc_s1_grid(const EncodeArgs& a, bool sec) {
+    return sec ? a.s1_grid2 : a.s1_grid;
+}
+#endif
 
 struct EncodePlan {
     int nchunk1;

@@ -6,6 +6,8 @@ Cases (seeded synthetic inputs generated on the device):
   encode-16x8x4096     encode one bf16 tensor, 16 x 8 kv-heads x 4096 tokens, 2 bit
                        (134 MB of input: larger than L2)
   encode-8x8x4096      the benchmark's per-tensor encode (67 MB)
+  encode-kv-8x8x4096   the benchmark step's encode: keys and values of 8 x 8 kv-heads x
+                       4096 tokens in one nsnq_encode_kv call (134 MB)
   encode-tc-8x8x4096   the same with the tensor-core search (ENCODE_TC_SEARCH, no index)
   encode1-16x8x4096    1-bit encode (tensor-core scoring), 16 x 8 kv-heads x 4096 tokens
   encode1-8x8x4096     1-bit encode, 8 x 8 kv-heads x 4096 tokens
@@ -63,6 +65,26 @@ def encode_case(B, H, T, reps, dev, sub=4, flags=nsnq.ENCODE_DEFAULT):
           f"{sv} sub-vectors; index mismatch {mism}; MMA timeout {tmo}")
 
 
+def encode_kv_case(B, H, T, reps, dev, sub=4):
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(0)
+    cb = _codebook(sub, dev).prepare()
+    k = _keys(gen, B, H, T, dev)
+    v = torch.randn(B, H, T, 128, generator=gen, device=dev).to(torch.bfloat16)
+    kc = nsnq.Cache.empty(B, H, T, sub, device=dev)
+    vc = nsnq.Cache.empty(B, H, T, sub, device=dev)
+    ws = torch.empty(nsnq.nsnq_encode_kv_workspace(B, H, T), dtype=torch.uint8, device=dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(reps):
+        e0.record()
+        nsnq.nsnq_encode_kv(k, v, cb, kc, vc, workspace=ws)
+        e1.record()
+    torch.cuda.synchronize()
+    th, sv, mism, tmo = nsnq.encode_stats(ws)
+    print(f"last call {e0.elapsed_time(e1):.3f} ms; fp64 path: {th} of {2 * B * H * T} token-heads, "
+          f"{sv} sub-vectors; index mismatch {mism}; MMA timeout {tmo}")
+
+
 def append_case(B, H, sub, reps, dev):
     """A decode step's appends: one token per (sequence, kv-head) encoded with
     the stored shift (the small-call pass 2) after a 1024-token prompt."""
@@ -105,6 +127,7 @@ def attn_case(B, Hq, Hkv, T, sub, reps, dev, rope=False):
 CASES = {
     "encode-16x8x4096": lambda r, d: encode_case(16, 8, 4096, r, d),
     "encode-8x8x4096": lambda r, d: encode_case(8, 8, 4096, r, d),
+    "encode-kv-8x8x4096": lambda r, d: encode_kv_case(8, 8, 4096, r, d),
     "encode-tc-8x8x4096": lambda r, d: encode_case(8, 8, 4096, r, d, flags=nsnq.ENCODE_TC_SEARCH),
     "encode1-16x8x4096": lambda r, d: encode_case(16, 8, 4096, r, d, sub=8),
     "encode1-8x8x4096": lambda r, d: encode_case(8, 8, 4096, r, d, sub=8),

@@ -194,7 +194,7 @@ def run_cuda(args):
     q = host["q"].to(dev)
     kc = nsnq.Cache.empty(B, H, T, w.sub_dim, device=dev)
     vc = nsnq.Cache.empty(B, H, T, w.sub_dim, device=dev)
-    ws_e = torch.empty(nsnq.nsnq_encode_workspace(B, H, T), dtype=torch.uint8, device=dev)
+    ws_e = torch.empty(nsnq.nsnq_encode_kv_workspace(B, H, T), dtype=torch.uint8, device=dev)
     ws_a = torch.empty(max(256, nsnq.nsnq_attn_workspace(B, Hq, H, T)), dtype=torch.uint8, device=dev)
     seq = torch.full((B,), T, dtype=torch.int32, device=dev)
     out = torch.empty(B, Hq, 128, dtype=torch.bfloat16, device=dev)
@@ -202,11 +202,10 @@ def run_cuda(args):
     stream = torch.cuda.current_stream()
 
     def step(kin, vin, qin):
-        nsnq.nsnq_encode(kin, cb, kc, workspace=ws_e)
-        nsnq.nsnq_encode(vin, cb, vc, workspace=ws_e)
+        nsnq.nsnq_encode_kv(kin, vin, cb, kc, vc, workspace=ws_e)
         nsnq.nsnq_attn_decode(qin, kc, vc, cb, cb, seq, T, Hkv=H, out=out, workspace=ws_a)
 
-    LAUNCHES_PER_STEP = 2 + 2 + 2  # (pass 1, pass 2) x 2 + (split, combine)
+    LAUNCHES_PER_STEP = 2 + 2  # encode of K and V (pass 1, pass 2) + attention (split, combine)
 
     def barrier():
         if world > 1:
@@ -219,7 +218,7 @@ def run_cuda(args):
     torch.cuda.synchronize()
 
     # ---- timed device-resident steps (L2 flushed before each step) ----
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
     if True:
@@ -227,17 +226,15 @@ def run_cuda(args):
             flush.zero_()
             e = ev[i]
             e[0].record(stream)
-            nsnq.nsnq_encode(k, cb, kc, workspace=ws_e)
+            nsnq.nsnq_encode_kv(k, v, cb, kc, vc, workspace=ws_e)
             e[1].record(stream)
-            nsnq.nsnq_encode(v, cb, vc, workspace=ws_e)
-            e[2].record(stream)
             nsnq.nsnq_attn_decode(q, kc, vc, cb, cb, seq, T, Hkv=H, out=out, workspace=ws_a)
-            e[3].record(stream)
+            e[2].record(stream)
         torch.cuda.synchronize()
     barrier()
-    step_ms = [e[0].elapsed_time(e[3]) for e in ev]
-    enc_ms = [e[0].elapsed_time(e[1]) for e in ev] + [e[1].elapsed_time(e[2]) for e in ev]
-    att_small_ms = [e[2].elapsed_time(e[3]) for e in ev]
+    step_ms = [e[0].elapsed_time(e[2]) for e in ev]
+    enc_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    att_small_ms = [e[1].elapsed_time(e[2]) for e in ev]
     total_ms = max_over_ranks(sum(step_ms), world, dev)
     ms_per_step = total_ms / args.steps
     tokens_per_step = B * T * world
@@ -261,7 +258,7 @@ def run_cuda(args):
     cut = lambda c, b0, b1: nsnq.Cache(c.codes[b0:b1], c.scales[b0:b1], c.shift[b0:b1])
     parts = [(b0, b1, cut(kc, b0, b1), cut(vc, b0, b1)) for b0, b1 in halves]
     # (a smaller piece can need more workspace: more pass-1 chunks per head)
-    ws_h = torch.empty(max(nsnq.nsnq_encode_workspace(b1 - b0, H, T) for b0, b1 in halves),
+    ws_h = torch.empty(max(nsnq.nsnq_encode_kv_workspace(b1 - b0, H, T) for b0, b1 in halves),
                        dtype=torch.uint8, device=dev)
 
     def e2e_step():
@@ -276,8 +273,7 @@ def run_cuda(args):
         # rows of the result back to the host
         for (b0, b1, kh, vh), ev_ in zip(parts, arrived):
             stream.wait_event(ev_)
-            nsnq.nsnq_encode(k[b0:b1], cb, kh, workspace=ws_h)
-            nsnq.nsnq_encode(v[b0:b1], cb, vh, workspace=ws_h)
+            nsnq.nsnq_encode_kv(k[b0:b1], v[b0:b1], cb, kh, vh, workspace=ws_h)
             nsnq.nsnq_attn_decode(q[b0:b1], kh, vh, cb, cb, seq[b0:b1], T, Hkv=H, out=out[b0:b1],
                                   workspace=ws_a)
             res_host[b0:b1].copy_(out[b0:b1], non_blocking=True)
@@ -304,14 +300,14 @@ def run_cuda(args):
 
     # ---- roofline of the dominant call (encode), algorithmic bytes ----
     hbm, peak_kind = peaks()
-    enc_bytes = B * H * T * encode_bytes_per_token_head(w.sub_dim)
+    enc_bytes = 2 * B * H * T * encode_bytes_per_token_head(w.sub_dim)  # K and V
     enc_avg_ms = sum(enc_ms) / len(enc_ms)
     enc_gbs = enc_bytes / (enc_avg_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(enc_gbs, 1), "peak": hbm, "unit": "GB/s",
                 "frac": round(enc_gbs / hbm, 4), "frac_vs_8tbs": round(enc_gbs / NOMINAL_HBM_GBS, 4), "peak_kind": peak_kind,
-                "kernel": "nsnq_encode (nsn_stats + nsn_encode_pruned, one tensor)",
+                "kernel": "nsnq_encode_kv (nsn_stats + nsn_encode_pruned over K and V, one call)",
                 "algorithmic_bytes_per_launch": enc_bytes,
-                "traffic": args.traffic if args.traffic is not None else measured_traffic("nsnq_encode")}
+                "traffic": args.traffic if args.traffic is not None else measured_traffic("nsnq_encode_kv")}
 
     # ---- decode attention alone at the 32k workload ----
     attention = run_attention_bench(args, nsnq, dev, world, barrier, hbm, peak_kind)
@@ -331,7 +327,7 @@ def run_cuda(args):
                                "T 4096, d 128, 2 bit/coord)",
                    "global_batch": B * world, "seq_len": T, "parallelism": f"replicas x{world}",
                    "l2": "flushed (256 MB write) before every timed step"},
-        "stages_ms": {"encode_per_tensor": round(enc_avg_ms, 4),
+        "stages_ms": {"encode_kv": round(enc_avg_ms, 4),
                       "attention_4k": round(sum(att_small_ms) / len(att_small_ms), 4)},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "roofline": roofline, "attention": attention, "attention_variants": attention_variants,
@@ -570,7 +566,7 @@ def run_long_context_bench(args, nsnq, dev, world, barrier, hbm):
     cap = T + n_dec
     kc = nsnq.Cache.empty(B, H, cap, w.sub_dim, device=dev)
     vc = nsnq.Cache.empty(B, H, cap, w.sub_dim, device=dev)
-    ws_e = torch.empty(nsnq.nsnq_encode_workspace(B, H, T), dtype=torch.uint8, device=dev)
+    ws_e = torch.empty(nsnq.nsnq_encode_kv_workspace(B, H, T), dtype=torch.uint8, device=dev)
     ws_a = torch.empty(nsnq.nsnq_attn_workspace(B, Hq, H, cap), dtype=torch.uint8, device=dev)
     out = torch.empty(B, Hq, 128, dtype=torch.bfloat16, device=dev)
     seqs = [torch.full((B,), T + i + 1, dtype=torch.int32, device=dev) for i in range(n_dec)]
@@ -579,8 +575,7 @@ def run_long_context_bench(args, nsnq, dev, world, barrier, hbm):
     ev = lambda: torch.cuda.Event(enable_timing=True)
 
     def prompt():
-        nsnq.nsnq_encode(k, cb, kc, workspace=ws_e)
-        nsnq.nsnq_encode(v, cb, vc, workspace=ws_e)
+        nsnq.nsnq_encode_kv(k, v, cb, kc, vc, workspace=ws_e)
 
     for _ in range(max(1, args.warmup // 2)):
         prompt()
@@ -600,10 +595,8 @@ def run_long_context_bench(args, nsnq, dev, world, barrier, hbm):
         flush.zero_()
         e0, e1, e2 = ev(), ev(), ev()
         e0.record(stream)
-        nsnq.nsnq_encode(kn[:, :, i:i + 1], cb, kc, t_offset=T + i, shift_mode=nsnq.SHIFT_GIVEN,
-                         workspace=ws_e)
-        nsnq.nsnq_encode(vn[:, :, i:i + 1], cb, vc, t_offset=T + i, shift_mode=nsnq.SHIFT_GIVEN,
-                         workspace=ws_e)
+        nsnq.nsnq_encode_kv(kn[:, :, i:i + 1], vn[:, :, i:i + 1], cb, kc, vc, t_offset=T + i,
+                            shift_mode=nsnq.SHIFT_GIVEN, workspace=ws_e)
         e1.record(stream)
         nsnq.nsnq_attn_decode(q[i], kc, vc, cb, cb, seqs[i], cap, Hkv=H, out=out, workspace=ws_a)
         e2.record(stream)
@@ -614,10 +607,8 @@ def run_long_context_bench(args, nsnq, dev, world, barrier, hbm):
     # device-side step latency without the per-call host overhead
     def decode_steps():
         for i in range(n_dec):
-            nsnq.nsnq_encode(kn[:, :, i:i + 1], cb, kc, t_offset=T + i,
-                             shift_mode=nsnq.SHIFT_GIVEN, workspace=ws_e)
-            nsnq.nsnq_encode(vn[:, :, i:i + 1], cb, vc, t_offset=T + i,
-                             shift_mode=nsnq.SHIFT_GIVEN, workspace=ws_e)
+            nsnq.nsnq_encode_kv(kn[:, :, i:i + 1], vn[:, :, i:i + 1], cb, kc, vc, t_offset=T + i,
+                                shift_mode=nsnq.SHIFT_GIVEN, workspace=ws_e)
             nsnq.nsnq_attn_decode(q[i], kc, vc, cb, cb, seqs[i], cap, Hkv=H, out=out,
                                   workspace=ws_a)
     side = torch.cuda.Stream(device=dev)
@@ -679,16 +670,16 @@ def run_serving_bench(args, nsnq, dev, world, barrier, hbm):
     kc = nsnq.Cache.empty(B + P, H, T, w.sub_dim, device=dev)
     vc = nsnq.Cache.empty(B + P, H, T, w.sub_dim, device=dev)
     view = lambda c, b0, b1: nsnq.Cache(c.codes[b0:b1], c.scales[b0:b1], c.shift[b0:b1])
-    ws_r = torch.empty(nsnq.nsnq_encode_workspace(1, H, T), dtype=torch.uint8, device=dev)
+    ws_r = torch.empty(nsnq.nsnq_encode_kv_workspace(1, H, T), dtype=torch.uint8, device=dev)
     for b in range(B):  # resident sequences, one at a time
-        nsnq.nsnq_encode(_device_kv(w, gen, dev, 1, T, "k"), cb, view(kc, b, b + 1), workspace=ws_r)
-        nsnq.nsnq_encode(_device_kv(w, gen, dev, 1, T, "v"), cb, view(vc, b, b + 1), workspace=ws_r)
+        nsnq.nsnq_encode_kv(_device_kv(w, gen, dev, 1, T, "k"), _device_kv(w, gen, dev, 1, T, "v"),
+                            cb, view(kc, b, b + 1), view(vc, b, b + 1), workspace=ws_r)
     kp = _device_kv(w, gen, dev, P, Tp, "k")
     vp = _device_kv(w, gen, dev, P, Tp, "v")
     q = torch.randn(B, Hq, 128, generator=gen, device=dev).to(torch.bfloat16)
     seq = torch.full((B,), T, dtype=torch.int32, device=dev)
     out = torch.empty(B, Hq, 128, dtype=torch.bfloat16, device=dev)
-    ws_e = torch.empty(nsnq.nsnq_encode_workspace(P, H, Tp), dtype=torch.uint8, device=dev)
+    ws_e = torch.empty(nsnq.nsnq_encode_kv_workspace(P, H, Tp), dtype=torch.uint8, device=dev)
     ws_a = torch.empty(nsnq.nsnq_attn_workspace(B, Hq, H, T), dtype=torch.uint8, device=dev)
     kres, vres = view(kc, 0, B), view(vc, 0, B)
     kspare, vspare = view(kc, B, B + P), view(vc, B, B + P)
@@ -697,8 +688,7 @@ def run_serving_bench(args, nsnq, dev, world, barrier, hbm):
 
     def step(evs=None):
         if evs: evs[0].record(stream)
-        nsnq.nsnq_encode(kp, cb, kspare, workspace=ws_e)
-        nsnq.nsnq_encode(vp, cb, vspare, workspace=ws_e)
+        nsnq.nsnq_encode_kv(kp, vp, cb, kspare, vspare, workspace=ws_e)
         if evs: evs[1].record(stream)
         nsnq.nsnq_attn_decode(q, kres, vres, cb, cb, seq, T, Hkv=H, out=out, workspace=ws_a)
         if evs: evs[2].record(stream)

@@ -225,6 +225,30 @@ nsnq_status nsnq_encode(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t
                         void* workspace, size_t workspace_bytes, nsnq_stream stream);
 
 /*
+ * nsnq_encode_kv -- nsnq_encode of a layer's keys and values in one call.
+ * NSNQuant quantizes both caches with one global codebook (Methodology §3),
+ * so the two tensors can share every launch of the call: one index staging,
+ * one work queue over the token-heads of both, and no idle tail between
+ * them. Each argument means what it means for nsnq_encode, applied to
+ * (x_k, cache_k) and to (x_v, cache_v); the two tensors share dtype, shape,
+ * strides, t_offset, mode, flags and the codebook, and the caches must agree
+ * in cap and form (both packed or neither). Codes, s1, s2 and o carry the
+ * guarantees of nsnq_encode for each tensor; the fp64 channel sums behind o
+ * are grouped by this call's chunk plan, so o can differ in its last fp32
+ * bit from a separate nsnq_encode of the same tensor. The workspace counters
+ * count both tensors.
+ *   workspace  >= nsnq_encode_kv_workspace(B, H, T, D) bytes (that of
+ *              nsnq_encode at batch 2B), 256-byte aligned.
+ * B <= 32767 (NSNQ_ERR_UNSUPPORTED above); T = 0 is a no-op.
+ */
+size_t nsnq_encode_kv_workspace(int B, int H, int64_t T, int D);
+nsnq_status nsnq_encode_kv(const void* x_k, const void* x_v, nsnq_dtype x_dtype, int B, int H,
+                           int64_t T, int D, int64_t stride_b, int64_t stride_h, int64_t stride_t,
+                           int64_t t_offset, nsnq_shift_mode mode, unsigned flags, nsnq_codebook cb,
+                           nsnq_cache cache_k, nsnq_cache cache_v, void* workspace,
+                           size_t workspace_bytes, nsnq_stream stream);
+
+/*
  * nsnq_dequant -- reconstruct tokens [t0, t0+T) of every (batch, head):
  * out = s1 * (s2 * H w_hat + o), w_hat the concatenated codewords
  * (Methodology §1: the byproducts reconstruct the tensor).

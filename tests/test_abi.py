@@ -93,6 +93,40 @@ def test_encode_validation(lib):
     assert lib.nsnq_last_error() == b""
 
 
+def _encode_kv(lib, **kw):
+    a = dict(xk=FAKE, xv=FAKE + 0x1000, dt=nsnq.NSNQ_BF16, B=1, H=1, T=10, D=128, sb=128 * 10,
+             sh=128 * 10, st=128, off=0, mode=0, flags=0, cb=_cb(), ck=_cache(), cv=_cache(),
+             ws=FAKE, wsb=1 << 20, stream=None)
+    a.update(kw)
+    return lib.nsnq_encode_kv(a["xk"], a["xv"], a["dt"], a["B"], a["H"], a["T"], a["D"], a["sb"],
+                              a["sh"], a["st"], a["off"], a["mode"], a["flags"], a["cb"], a["ck"],
+                              a["cv"], a["ws"], a["wsb"], a["stream"])
+
+
+def test_encode_kv_validation(lib):
+    assert _encode_kv(lib, D=64) == nsnq.NSNQ_ERR_UNSUPPORTED
+    assert _encode_kv(lib, xv=None) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert _encode_kv(lib, xv=FAKE + 2) == nsnq.NSNQ_ERR_INVALID_ARG     # misaligned
+    assert _encode_kv(lib, cv=_cache(cap=99)) == nsnq.NSNQ_ERR_INVALID_ARG  # caps differ
+    assert b"cap" in lib.nsnq_last_error()
+    assert _encode_kv(lib, cv=nsnq._Cache(FAKE, None, FAKE, 100)) == nsnq.NSNQ_ERR_INVALID_ARG
+    assert b"cache_v" in lib.nsnq_last_error()
+    packed = nsnq._Cache(FAKE, FAKE, FAKE, 100, FAKE, FAKE)
+    plain_dq = nsnq._Cache(FAKE, FAKE, FAKE, 100, FAKE, None)
+    assert _encode_kv(lib, ck=packed, cv=plain_dq, flags=nsnq.ENCODE_DOUBLE_QUANT) == \
+        nsnq.NSNQ_ERR_INVALID_ARG                                       # one packed, one not
+    assert b"packed" in lib.nsnq_last_error()
+    assert _encode_kv(lib, B=32768) == nsnq.NSNQ_ERR_UNSUPPORTED          # grid batch 2B
+    # the workspace is that of a 2B-batch encode
+    need = lib.nsnq_encode_kv_workspace(1, 1, 10, 128)
+    assert need == lib.nsnq_encode_workspace(2, 1, 10, 128) > 0
+    assert lib.nsnq_encode_kv_workspace(8, 8, 4096, 128) == lib.nsnq_encode_workspace(16, 8, 4096, 128)
+    assert lib.nsnq_encode_kv_workspace(32768, 1, 10, 128) == 0
+    assert _encode_kv(lib, wsb=need - 1) == nsnq.NSNQ_ERR_WORKSPACE
+    assert _encode_kv(lib, T=0) == nsnq.NSNQ_OK                          # no-op, no launch
+    assert lib.nsnq_last_error() == b""
+
+
 def test_index_build_validation(lib):
     assert lib.nsnq_codebook_index_bytes(4) > 0 and lib.nsnq_codebook_index_bytes(8) == 0
     need = lib.nsnq_codebook_index_bytes(4)
