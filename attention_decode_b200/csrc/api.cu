@@ -213,6 +213,10 @@ nsnq_status encode_impl(const void* x, const void* x2, nsnq_dtype x_dtype, int B
     if (stride_b < 0 || stride_h < 0 || stride_t < D)
         return fail(NSNQ_ERR_INVALID_ARG, "strides must be non-negative with stride_t >= D");
     const int Bg = pair ? 2 * B : B;  // batches of the grid
+    // work indices are 32-bit (2^31 token-heads of bf16 input are 550 GB)
+    if ((int64_t)Bg * H * T >= (int64_t)1 << 31)
+        return fail(NSNQ_ERR_UNSUPPORTED, "%lld token-heads in one call (limit 2^31)",
+                    (long long)Bg * H * T);
     const nsnq::EncodePlan plan = nsnq::plan_encode(Bg, H, T);
     if (!workspace || workspace_bytes < plan.total)
         return fail(NSNQ_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", plan.total,

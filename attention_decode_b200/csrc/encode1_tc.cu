@@ -317,10 +317,14 @@ __global__ void __launch_bounds__(kTcThreads) nsn_encode_tc_kernel(EncodeArgs a)
         const int64_t pi = 4 * tile + warp;
         const bool wvalid = pi < npairs;
         const int64_t pic = wvalid ? pi : 0;
-        const int64_t bh = pic / pairs_per_head;
-        const int64_t t0 = 2 * (pic - bh * pairs_per_head);
+        // pic < npairs < 2^31: 32-bit divisions by the launch's invariants
+        const uint32_t pic32 = (uint32_t)pic;
+        const uint32_t bh32 = fdiv(pic32, a.div_items);  // pairs_per_head
+        const int64_t bh = bh32;
+        const int64_t t0 = 2 * (int64_t)(pic32 - bh32 * a.div_items.d);
         const int64_t t = t0 + half;
-        const int b = (int)(bh / a.H), h = (int)(bh - (int64_t)b * a.H);
+        const uint32_t b32 = fdiv(bh32, a.div_H);
+        const int b = (int)b32, h = (int)(bh32 - b32 * (uint32_t)a.H);
         const bool valid = wvalid && t < a.T;
         const XT* xhead = enc_head<XT>(a, b, h);
         float v[8];
@@ -587,8 +591,11 @@ cudaError_t launch_tc(const EncodeArgs& a, cudaStream_t s) {
     const int64_t ntiles = (npairs + 3) / 4;
     const int64_t cap = (int64_t)sms * 4;  // four CTAs per SM: all resident, 512 TMEM columns
     const int grid = (int)(ntiles < cap ? ntiles : cap);
+    EncodeArgs k = a;
+    k.div_items = make_fastdiv((uint32_t)((a.T + 1) / 2));
+    k.div_H = make_fastdiv((uint32_t)a.H);
     return launch_smem_pdl(nsn_encode_tc_kernel<XT, ADAPT, DQ, SUB>, ready, dim3(grid), dim3(kTcThreads),
-                           (size_t)kTcSmem, s, a);
+                           (size_t)kTcSmem, s, k);
 }
 
 template <int SUB>

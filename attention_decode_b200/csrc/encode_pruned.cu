@@ -285,9 +285,13 @@ __global__ void __launch_bounds__(kPrunedThreads, 1) nsn_encode_pruned_kernel(En
         if (lane == 0) tl = atomicAdd(&a.stats[3], 1ull);
         const int64_t tile = (int64_t)__shfl_sync(kFull, tl, 0);
         if (tile >= ntiles) break;
-        const int64_t bh = tile / tiles_per_bh;
-        const int64_t t = (tile - bh * tiles_per_bh) * kWarpTile + (lane >> 1);
-        const int b = (int)(bh / a.H), h = (int)(bh - (int64_t)b * a.H);
+        // tile < ntiles < 2^31: 32-bit divisions by the launch's invariants
+        const uint32_t tile32 = (uint32_t)tile;
+        const uint32_t bh32 = fdiv(tile32, a.div_items);  // tiles_per_bh
+        const int64_t bh = bh32;
+        const int64_t t = (int64_t)(tile32 - bh32 * a.div_items.d) * kWarpTile + (lane >> 1);
+        const uint32_t b32 = fdiv(bh32, a.div_H);
+        const int b = (int)b32, h = (int)(bh32 - b32 * (uint32_t)a.H);
         if (bh != cur_bh) {  // warp-uniform
             __syncwarp();
             const float4 o =
@@ -471,8 +475,11 @@ static cudaError_t launch_pruned_t(const EncodeArgs& a, cudaStream_t s) {
     const int64_t ntiles = (int64_t)a.B * a.H * ((a.T + kWarpTile - 1) / kWarpTile);
     const int64_t ctas = (ntiles + kWarps - 1) / kWarps;
     const int grid = (int)(ctas < sms ? ctas : sms);
+    EncodeArgs k = a;
+    k.div_items = make_fastdiv((uint32_t)((a.T + kWarpTile - 1) / kWarpTile));
+    k.div_H = make_fastdiv((uint32_t)a.H);
     return launch_smem_pdl(nsn_encode_pruned_kernel<XT, ADAPT, DQ>, ready, dim3(grid),
-                           dim3(kPrunedThreads), kSmBytes, s, a);
+                           dim3(kPrunedThreads), kSmBytes, s, k);
 }
 
 cudaError_t launch_encode_pruned(const EncodeArgs& a, cudaStream_t s) {

@@ -41,8 +41,11 @@ __global__ void __launch_bounds__(kSmallThreads) nsn_encode_small_kernel(EncodeA
     const int lane = lane_id();
     const int64_t th = (int64_t)blockIdx.x * (kSmallThreads / 32) + (threadIdx.x >> 5);
     if (th >= (int64_t)a.B * a.H * a.T) return;  // warp-uniform
-    const int64_t bh = th / a.T, t = th - bh * a.T;
-    const int b = (int)(bh / a.H), h = (int)(bh - (int64_t)b * a.H);
+    // th < B H T <= kSmallEncode: 32-bit divisions by the launch's invariants
+    const uint32_t bh32 = fdiv((uint32_t)th, a.div_items);  // T
+    const int64_t bh = bh32, t = th - bh * a.T;
+    const uint32_t b32 = fdiv(bh32, a.div_H);
+    const int b = (int)b32, h = (int)(bh32 - b32 * (uint32_t)a.H);
     const bool sec = enc_second(a, bh);
     const int64_t cbh = enc_cbh(a, bh);
     const XT* xtok = enc_head<XT>(a, b, h) + t * a.st;
@@ -191,9 +194,12 @@ __global__ void __launch_bounds__(kSmallThreads) nsn_encode_small_kernel(EncodeA
 }
 
 template <typename XT, int G>
-cudaError_t launch_small_t(const EncodeArgs& a, cudaStream_t s) {
-    const int64_t n = (int64_t)a.B * a.H * a.T;
+cudaError_t launch_small_t(const EncodeArgs& args, cudaStream_t s) {
+    const int64_t n = (int64_t)args.B * args.H * args.T;
     const int grid = (int)((n + kSmallThreads / 32 - 1) / (kSmallThreads / 32));
+    EncodeArgs a = args;
+    a.div_items = make_fastdiv((uint32_t)args.T);
+    a.div_H = make_fastdiv((uint32_t)args.H);
     if (a.dq) {
         if (a.adaptive) nsn_encode_small_kernel<XT, G, true, true><<<grid, kSmallThreads, 0, s>>>(a);
         else nsn_encode_small_kernel<XT, G, false, true><<<grid, kSmallThreads, 0, s>>>(a);

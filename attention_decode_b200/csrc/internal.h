@@ -85,6 +85,29 @@ cudaError_t launch_smem_pdl(void (*kern)(P...), std::atomic<unsigned long long>&
     return e;
 }
 
+// ------------------------------------------------ division by an invariant --
+// n / d for 32-bit n and a divisor d >= 1 fixed per launch, as a multiply-high,
+// a subtract, an add and two shifts (T. Granlund and P. Montgomery, "Division
+// by Invariant Integers using Multiplication", PLDI 1994, section 4): with
+// l = ceil(log2 d) and m = floor(2^32 (2^l - d) / d) + 1,
+// q = (t + ((n - t) >> min(l, 1))) >> max(l - 1, 0), t = mulhi(m, n), exact
+// for every 32-bit n.
+struct FastDiv {
+    uint32_t d, m, s1, s2;
+};
+inline FastDiv make_fastdiv(uint32_t d) {
+    uint32_t l = 0;
+    while (l < 32 && (1ull << l) < d) ++l;
+    const uint64_t m = (((1ull << 32) * ((1ull << l) - d)) / d) + 1;
+    return {d, (uint32_t)m, l < 1 ? l : 1u, l > 0 ? l - 1 : 0u};
+}
+#ifdef __CUDACC__
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
+    const uint32_t t = __umulhi(n, f.m);
+    return (t + ((n - t) >> f.s1)) >> f.s2;
+}
+#endif
+
 // ------------------------------------------------------------------ encode --
 struct EncodeArgs {
     const void* x;
@@ -126,6 +149,10 @@ struct EncodeArgs {
     float* shift2;
     uint32_t* s1_levels2;
     float* s1_grid2;
+    // Set by the pass-2 launchers: the divisions of the work decomposition
+    // (work items per head, heads per batch); every index is below 2^31.
+    FastDiv div_items;
+    FastDiv div_H;
 };
 
 #ifdef __CUDACC__

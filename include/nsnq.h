@@ -217,7 +217,8 @@ size_t nsnq_encode_workspace(int B, int H, int64_t T, int D);
  * best and second best, and an fp64 re-scan of the sub-vectors inside the
  * near-tie band; the index is not read and the workspace counters stay 0.
  * Stored s1, s2, o are fp32 roundings. A zero-norm token (or a zero residual after the shift) maps to
- * the zero vector with s = 0. T = 0 is a no-op.
+ * the zero vector with s = 0. T = 0 is a no-op. At most 2^31 - 1 token-heads
+ * (B*H*T) per call: NSNQ_ERR_UNSUPPORTED above.
  */
 nsnq_status nsnq_encode(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t T, int D,
                         int64_t stride_b, int64_t stride_h, int64_t stride_t, int64_t t_offset,
@@ -239,7 +240,8 @@ nsnq_status nsnq_encode(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t
  * count both tensors.
  *   workspace  >= nsnq_encode_kv_workspace(B, H, T, D) bytes (that of
  *              nsnq_encode at batch 2B), 256-byte aligned.
- * B <= 32767 (NSNQ_ERR_UNSUPPORTED above); T = 0 is a no-op.
+ * B <= 32767 and 2*B*H*T < 2^31 (NSNQ_ERR_UNSUPPORTED above); T = 0 is a
+ * no-op.
  */
 size_t nsnq_encode_kv_workspace(int B, int H, int64_t T, int D);
 nsnq_status nsnq_encode_kv(const void* x_k, const void* x_v, nsnq_dtype x_dtype, int B, int H,
