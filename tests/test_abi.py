@@ -127,6 +127,18 @@ def test_encode_kv_validation(lib):
     assert lib.nsnq_last_error() == b""
 
 
+def test_binding_encode_kv_checks_the_pair_layout():
+    """The binding rejects keys and values of different shape, dtype or
+    strides before it touches the library (the C ABI takes one layout)."""
+    import torch
+    k = torch.empty(1, 2, 10, 128, dtype=torch.bfloat16)
+    for v in (torch.empty(1, 2, 11, 128, dtype=torch.bfloat16),
+              torch.empty(1, 2, 10, 128, dtype=torch.float32),
+              torch.empty(1, 2, 10, 256, dtype=torch.bfloat16)[..., :128]):
+        with pytest.raises(ValueError):
+            nsnq.nsnq_encode_kv(k, v, None, None, None)
+
+
 def test_index_build_validation(lib):
     assert lib.nsnq_codebook_index_bytes(4) > 0 and lib.nsnq_codebook_index_bytes(8) == 0
     need = lib.nsnq_codebook_index_bytes(4)
