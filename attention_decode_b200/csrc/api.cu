@@ -203,6 +203,10 @@ nsnq_status encode_impl(const void* x, const void* x2, nsnq_dtype x_dtype, int B
                         (long long)cache.cap, (long long)cache2->cap);
         if ((cache2->s1_levels != nullptr) != (cache.s1_levels != nullptr))
             return fail(NSNQ_ERR_INVALID_ARG, "cache_k and cache_v must both be packed or both not");
+        if (cache2->codes == cache.codes || cache2->scales == cache.scales || cache2->shift == cache.shift ||
+            (cache.s1_levels && cache2->s1_levels == cache.s1_levels) ||
+            (cache.s1_grid && cache2->s1_grid == cache.s1_grid))
+            return fail(NSNQ_ERR_INVALID_ARG, "cache_k and cache_v share a buffer");
     }
     if (B == 0 || H == 0 || T == 0) return ok();
     if (!x || (pair && !x2)) return fail(NSNQ_ERR_INVALID_ARG, "%s is NULL", pair ? "x_k or x_v" : "x");

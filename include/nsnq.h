@@ -233,7 +233,9 @@ nsnq_status nsnq_encode(const void* x, nsnq_dtype x_dtype, int B, int H, int64_t
  * them. Each argument means what it means for nsnq_encode, applied to
  * (x_k, cache_k) and to (x_v, cache_v); the two tensors share dtype, shape,
  * strides, t_offset, mode, flags and the codebook, and the caches must agree
- * in cap and form (both packed or neither). Codes, s1, s2 and o carry the
+ * in cap and form (both packed or neither) and share no buffer (the same
+ * codes, scales, shift, s1_levels or s1_grid pointer: NSNQ_ERR_INVALID_ARG;
+ * overlapping views of one allocation are the caller's to avoid). Codes, s1, s2 and o carry the
  * guarantees of nsnq_encode for each tensor; the fp64 channel sums behind o
  * are grouped by this call's chunk plan, so o can differ in its last fp32
  * bit from a separate nsnq_encode of the same tensor. The workspace counters

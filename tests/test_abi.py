@@ -93,9 +93,13 @@ def test_encode_validation(lib):
     assert lib.nsnq_last_error() == b""
 
 
+def _cache_v(cap=100):  # buffers distinct from _cache()'s
+    return nsnq._Cache(0x20000, 0x21000, 0x22000, cap)
+
+
 def _encode_kv(lib, **kw):
     a = dict(xk=FAKE, xv=FAKE + 0x1000, dt=nsnq.NSNQ_BF16, B=1, H=1, T=10, D=128, sb=128 * 10,
-             sh=128 * 10, st=128, off=0, mode=0, flags=0, cb=_cb(), ck=_cache(), cv=_cache(),
+             sh=128 * 10, st=128, off=0, mode=0, flags=0, cb=_cb(), ck=_cache(), cv=_cache_v(),
              ws=FAKE, wsb=1 << 20, stream=None)
     a.update(kw)
     return lib.nsnq_encode_kv(a["xk"], a["xv"], a["dt"], a["B"], a["H"], a["T"], a["D"], a["sb"],
@@ -107,16 +111,20 @@ def test_encode_kv_validation(lib):
     assert _encode_kv(lib, D=64) == nsnq.NSNQ_ERR_UNSUPPORTED
     assert _encode_kv(lib, xv=None) == nsnq.NSNQ_ERR_INVALID_ARG
     assert _encode_kv(lib, xv=FAKE + 2) == nsnq.NSNQ_ERR_INVALID_ARG     # misaligned
-    assert _encode_kv(lib, cv=_cache(cap=99)) == nsnq.NSNQ_ERR_INVALID_ARG  # caps differ
+    assert _encode_kv(lib, cv=_cache_v(cap=99)) == nsnq.NSNQ_ERR_INVALID_ARG  # caps differ
     assert b"cap" in lib.nsnq_last_error()
     assert _encode_kv(lib, cv=nsnq._Cache(FAKE, None, FAKE, 100)) == nsnq.NSNQ_ERR_INVALID_ARG
     assert b"cache_v" in lib.nsnq_last_error()
     packed = nsnq._Cache(FAKE, FAKE, FAKE, 100, FAKE, FAKE)
-    plain_dq = nsnq._Cache(FAKE, FAKE, FAKE, 100, FAKE, None)
+    plain_dq = nsnq._Cache(0x20000, 0x21000, 0x22000, 100, 0x23000, None)
     assert _encode_kv(lib, ck=packed, cv=plain_dq, flags=nsnq.ENCODE_DOUBLE_QUANT) == \
         nsnq.NSNQ_ERR_INVALID_ARG                                       # one packed, one not
     assert b"packed" in lib.nsnq_last_error()
     assert _encode_kv(lib, B=32768) == nsnq.NSNQ_ERR_UNSUPPORTED          # grid batch 2B
+    same = _cache()
+    assert _encode_kv(lib, ck=same, cv=same) == nsnq.NSNQ_ERR_INVALID_ARG  # one cache for both
+    assert b"share" in lib.nsnq_last_error()
+    assert _encode_kv(lib, B=1 << 14, H=1 << 10, T=1 << 6) == nsnq.NSNQ_ERR_UNSUPPORTED  # 2^31
     # the workspace is that of a 2B-batch encode
     need = lib.nsnq_encode_kv_workspace(1, 1, 10, 128)
     assert need == lib.nsnq_encode_workspace(2, 1, 10, 128) > 0
